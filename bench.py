@@ -1,0 +1,452 @@
+"""Benchmark of the DSA hot path: query-tokens/s per layer and % of HBM roofline.
+
+One step = one pass of the whole path over one batch of synthetic inputs already
+resident in HBM: dsa_index_scores -> dsa_topk -> sparse MLA for every layer of
+the workload (through the C ABI).  The step is captured once in a CUDA graph with
+CUDA events between the calls, so per-kernel device times come from the same
+timed replays; L2 is flushed (256 MB write) before every timed step.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_32k]
+    python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
+
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch of the
+workload (independent sequences, no collective on the data path: weak scaling);
+the time is the max over ranks and `value` counts every rank's queries.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+from dsa_indexer_top_b200 import binding as B
+from dsa_indexer_top_b200 import workloads as wl
+
+METRIC = "query-tokens/s per layer (indexer+top-k+sparse MLA); % of HBM roofline"
+UNIT = "qtok/s/layer"
+ROOT = os.path.dirname(os.path.abspath(__file__))
+DECODE_MAX_QUERIES = 256    # the MLA decode (split-K) schedule up to this many queries
+L2_FLUSH_BYTES = 256 << 20
+
+# dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch, from the ncu
+# capture summarised under profiles/ (None until captured for the current kernel).
+NCU_INDEXER_TRAFFIC = {}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+# ------------------------------------------------------------------ algorithmic bytes
+def path_bytes(w: wl.Workload, seq_run: int):
+    """Algorithmic HBM bytes of one step (each input byte once, outputs once)."""
+    vis = np.array(w.q_pos, dtype=np.int64) + 1
+    seqs = {}
+    for s, t in zip(w.q_seq, w.q_pos):
+        key = 0 if w.shared_cache else s
+        seqs[key] = max(seqs.get(key, 0), t + 1)
+    key_rows = sum(seqs.values())
+    eb = w.elem_bytes
+    idx_in = key_rows * w.idx_dim * eb + w.n_q * w.idx_heads * (w.idx_dim * eb + 4)
+    idx_out = int(vis.sum()) * 4
+    cnt = np.minimum(vis, w.topk)
+    rows = int(cnt.sum()) * (w.d_lat + w.d_rope) * eb
+    q_out = w.n_q * w.mla_heads * ((w.d_lat + w.d_rope) * eb + w.d_lat * eb + 4)
+    return {
+        "indexer": idx_in + idx_out,
+        "topk": idx_out + w.n_q * (w.topk + 1) * 4,
+        "mla_per_layer": rows + q_out,
+        # the path's roofline bytes: indexer keys + gathered rows + q/out
+        "path": key_rows * w.idx_dim * eb + w.n_layers * (rows + q_out) + w.n_q * w.idx_heads * (w.idx_dim * eb + 4),
+    }
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.proc = None
+        sel = str(device_index)
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else f"GPU-{uuid}"
+        except Exception:
+            pass
+        self.cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                    "-i", sel]
+        self.active = False
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                self.samples.append((time.time(), parts))
+
+    def mark(self, on: bool):
+        self.active = on
+        if on:
+            self.t_on = time.time()
+        else:
+            self.t_off = time.time()
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        t0, t1 = getattr(self, "t_on", 0), getattr(self, "t_off", time.time())
+        inside = [p for t, p in self.samples if t0 - 0.06 <= t <= t1 + 0.06] or [p for _, p in self.samples]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for p in inside for j in range(4) if p[3 + j].lower() == "active"})
+        sm = [float(p[0]) for p in inside if p[0].replace(".", "").isdigit()]
+        mx = [float(p[1]) for p in inside if p[1].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(inside)}
+
+
+# ------------------------------------------------------------------ the step
+class Step:
+    """Device buffers, descriptors and the captured CUDA graph of one step."""
+
+    def __init__(self, w: wl.Workload, dev, seed_offset: int = 0):
+        self.w = w
+        self.dev = dev
+        w = wl.scaled(w, seed=w.seed + seed_offset) if seed_offset else w
+        self.x = wl.make_inputs(w, device=dev)
+        self.seq_run = w.n_q if len(set(w.q_seq)) == 1 else 1
+        x = self.x
+        self.q = B.Queries(x["q_seq"], x["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=self.seq_run)
+        self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"])
+        self.mlas = []
+        for layer in range(w.n_layers):
+            out = torch.empty((w.n_q, w.mla_heads, w.d_lat), dtype=w.torch_dtype, device=dev)
+            lse = torch.empty((w.n_q, w.mla_heads), dtype=torch.float32, device=dev)
+            kv = x["kv"][layer][0] if w.shared_cache else x["kv"][layer]
+            self.mlas.append(B.Mla(x["q_mla"][layer], kv, out, w.d_lat, w.scale, lse))
+        self.ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, self.q, w.topk, w.n_layers, dev)
+        self.scores = B.scores_buffer(w.n_q, w.L, dev)
+        self.idx = torch.empty((w.n_q, w.topk), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((w.n_q,), dtype=torch.int32, device=dev)
+        self.decode = w.n_q <= DECODE_MAX_QUERIES
+        self.mla_fn = B.dsa_sparse_mla_decode if self.decode else B.dsa_sparse_mla_prefill
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        self.graph = None
+
+    def launches_per_step(self) -> int:
+        w = self.w
+        n_chunks = (w.topk + 127) // 128
+        mla = 2 if (self.decode and n_chunks > 1) else 1
+        return 2 + w.n_layers * mla
+
+    def run(self, events: bool):
+        if events:
+            self.ev[0].record()
+        B.dsa_index_scores(self.q, self.ix, self.scores, self.ws)
+        if events:
+            self.ev[1].record()
+        B.dsa_topk(self.q, self.scores, self.w.topk, self.idx, self.cnt, self.ws)
+        if events:
+            self.ev[2].record()
+        for m in self.mlas:
+            self.mla_fn(self.q, m, self.idx, self.cnt, self.w.topk, self.ws)
+        if events:
+            self.ev[3].record()
+
+    def capture(self):
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            self.run(events=False)      # one eager pass: one-time kernel attribute setup
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
+            self.run(events=True)
+        torch.cuda.synchronize()
+
+    def times_ms(self):
+        e = self.ev
+        return (e[0].elapsed_time(e[3]), e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]))
+
+
+class E2EStep:
+    """The same step through the public API with host buffers: copy the step's
+    query inputs from pinned host memory, run, copy the outputs back."""
+
+    def __init__(self, step: Step):
+        self.s = step
+        x = step.x
+        self.h_in = {k: x[k].cpu().pin_memory() for k in ("q_idx", "w", "q_seq", "q_pos")}
+        self.h_qmla = [t.cpu().pin_memory() for t in x["q_mla"]]
+        self.h_out = [torch.empty(m.out.shape, dtype=m.out.dtype).pin_memory() for m in step.mlas]
+        self.h_idx = torch.empty(step.idx.shape, dtype=torch.int32).pin_memory()
+        self.h2d = sum(t.numel() * t.element_size() for t in list(self.h_in.values()) + self.h_qmla)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out) + self.h_idx.numel() * 4
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        self.graph = None
+
+    def run(self):
+        s, x = self.s, self.s.x
+        self.ev[0].record()
+        for k, h in self.h_in.items():
+            x[k].copy_(h, non_blocking=True)
+        for d, h in zip(x["q_mla"], self.h_qmla):
+            d.copy_(h, non_blocking=True)
+        s.run(events=False)
+        for h, m in zip(self.h_out, s.mlas):
+            h.copy_(m.out, non_blocking=True)
+        self.h_idx.copy_(s.idx, non_blocking=True)
+        self.ev[1].record()
+
+    def capture(self):
+        torch.cuda.synchronize()
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
+            self.run()
+        torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------------ CPU oracle timing
+def host_copies(w: wl.Workload, dev_x: dict, queries) -> dict:
+    """Host copies of what the sampled queries read (their sequences only)."""
+    seqs = sorted({0 if w.shared_cache else w.q_seq[i] for i in queries})
+    return {"q_idx": dev_x["q_idx"].cpu(), "w": dev_x["w"].cpu(), "q_mla": [t.cpu() for t in dev_x["q_mla"]],
+            "k": {b: dev_x["k_idx"][b].cpu() for b in seqs},
+            "kv": {b: [t[b].cpu() for t in dev_x["kv"]] for b in seqs}}
+
+
+def oracle_sample_time(w: wl.Workload, h: dict, queries) -> float:
+    """Seconds the fp64 oracle takes for the whole path (scores over every visible
+    key -> top-k -> MLA of every layer) of the given queries."""
+    import oracle
+    t0 = time.perf_counter()
+    for i in queries:
+        b = 0 if w.shared_cache else w.q_seq[i]
+        k = h["k"][b].float().numpy()[None]
+        sc = oracle.index_scores(h["q_idx"][i:i + 1].float().numpy(), h["w"][i:i + 1].numpy(), k, [0],
+                                 [w.q_pos[i]])
+        idx, cnt = oracle.topk(sc, [w.q_pos[i]], w.topk)
+        sel = idx[0, : cnt[0]]
+        for layer in range(w.n_layers):
+            rows = h["kv"][b][layer][torch.from_numpy(sel.astype(np.int64))].float().numpy()[None]
+            oracle.sparse_mla(h["q_mla"][layer][i:i + 1].float().numpy(), rows, [0],
+                              np.arange(len(sel), dtype=np.int32)[None], cnt, w.d_lat, w.scale)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w: wl.Workload, dev_x: dict, budget_s: float = 12.0):
+    import oracle
+    oracle.build()
+    order = list(range(w.n_q))
+    h = host_copies(w, dev_x, order[:1])
+    t1 = oracle_sample_time(w, h, order[:1])
+    n = max(1, min(w.n_q, int(budget_s / max(t1, 1e-6))))
+    if n > 1:
+        h = host_copies(w, dev_x, order[:n])
+        t = oracle_sample_time(w, h, order[:n])
+    else:
+        t = t1
+    return {"value": n * w.n_layers / t, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n} of {w.n_q} queries of {w.name}, all {w.n_layers} layer(s), full path "
+                      f"(fp64 scores over all visible keys, full sort, sparse MLA)"}
+
+
+# ------------------------------------------------------------------ main
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, dev) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def run_reference(args, w: wl.Workload, world: int, rank: int):
+    """The oracle as it stands on host cores: each step one query's full path."""
+    if rank != 0:
+        return
+    import oracle
+    oracle.build()
+    x = wl.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    order = list(range(w.n_q))
+    h = host_copies(w, x, order)
+    for s in range(args.warmup):
+        oracle_sample_time(w, h, [order[s % w.n_q]])
+    t = 0.0
+    for s in range(args.steps):
+        t += oracle_sample_time(w, h, [order[s % w.n_q]])
+    value = args.steps * w.n_layers / t
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {**w.describe(), "sample_per_step": "1 query, all layers"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
+                             "sample": "each step: one query of the workload, full path, all layers"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="decode_32k", choices=list(wl.NAMED))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    w = wl.NAMED[args.workload]
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, w, world, rank)
+        return
+    assert args.warmup >= 3, "at least 3 warm-up steps"
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    B.lib()
+
+    step = Step(w, dev, seed_offset=rank)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    step.capture()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step.graph.replay()
+    torch.cuda.synchronize()
+    st = B.dsa_check_status(step.ws)
+    if st != B.DSA_OK:
+        raise SystemExit(f"device status {B.status_str(st)}")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.mark(True)
+    tot = idx_t = topk_t = mla_t = 0.0
+    for _ in range(args.steps):
+        flush.fill_(1)
+        step.graph.replay()
+        torch.cuda.synchronize()
+        a, b, c, d = step.times_ms()
+        tot += a
+        idx_t += b
+        topk_t += c
+        mla_t += d
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks.mark(False)
+    time.sleep(0.1)
+    clocks.stop()
+    tot_max = max_over_ranks(tot, world, dev)
+
+    ms_per_step = tot_max / args.steps
+    value = world * w.n_q * w.n_layers * args.steps / (tot_max * 1e-3)
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    by = path_bytes(w, step.seq_run)
+    idx_ms = idx_t / args.steps
+    idx_gbs = by["indexer"] / (idx_ms * 1e-3) / 1e9
+    t_roof_us = by["path"] / (hbm_peak * 1e9) * 1e6
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {**w.describe(), "parallelism": f"dp{world} (independent batches per GPU)",
+                   "l2": "flushed before every timed step (256 MB write)", "graph": "CUDA graph per step"},
+        "roofline": {"bound": "hbm", "kernel": "idx_score_tc (dsa_index_scores)", "achieved": idx_gbs,
+                     "peak": hbm_peak, "unit": "GB/s", "frac": idx_gbs / hbm_peak,
+                     "traffic": NCU_INDEXER_TRAFFIC.get(w.name), "peak_kind": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes": by["indexer"], "avg_launch_us": idx_ms * 1e3},
+        "path_roofline": {"bytes": by["path"], "t_roof_us": t_roof_us,
+                          "frac": t_roof_us / (ms_per_step * 1e3), "peak_kind": f"{peak_kind} hbm_gbs"},
+        "breakdown_us": {"index_scores": idx_ms * 1e3, "topk": topk_t / args.steps * 1e3,
+                         "sparse_mla": mla_t / args.steps * 1e3},
+        "gpu_launches": step.launches_per_step() * args.steps,
+        "clocks": clocks.summary(),
+    }
+
+    if not args.no_e2e:
+        e2e = E2EStep(step)
+        e2e.capture()
+        for _ in range(3):
+            e2e.graph.replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        te = 0.0
+        n_e2e = max(10, min(args.steps, 500))
+        for _ in range(n_e2e):
+            flush.fill_(1)
+            e2e.graph.replay()
+            torch.cuda.synchronize()
+            te += e2e.ev[0].elapsed_time(e2e.ev[1])
+        te = max_over_ranks(te, world, dev)
+        line["e2e"] = {"value": world * w.n_q * w.n_layers * n_e2e / (te * 1e-3), "unit": UNIT,
+                       "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "steps": n_e2e}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, step.x)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        step.graph = None
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,223 @@
+"""ctypes binding of libdsa.so (include/dsa.h): argument marshalling only.
+
+Every function here has the name of the C entry point it calls and does nothing
+but turn torch tensors into plain pointers and sizes, call the library on the
+current CUDA stream, and raise DsaError on a non-OK status.  All arithmetic runs
+in the library's CUDA kernels; there is no other code path.  If libdsa.so is
+missing the first call raises (build it with `python -m dsa_indexer_top_b200.build`).
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+
+DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT = range(6)
+DSA_BF16, DSA_F32 = 0, 1
+DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_MLA_DECODE, DSA_OP_MLA_PREFILL, DSA_OP_INDEXSHARE_GROUP = range(5)
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_str(status)} ({status})")
+
+
+class _Queries(ctypes.Structure):
+    _fields_ = [("n_q", ctypes.c_int32), ("n_seq", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
+                ("seq_run", ctypes.c_int32), ("q_seq", ctypes.c_void_p), ("q_pos", ctypes.c_void_p)]
+
+
+class _Indexer(ctypes.Structure):
+    _fields_ = [("heads", ctypes.c_int32), ("dim", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("q", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("k", ctypes.c_void_p), ("k_seq_stride", ctypes.c_int64), ("k_row_stride", ctypes.c_int64)]
+
+
+class _Mla(ctypes.Structure):
+    _fields_ = [("heads", ctypes.c_int32), ("d_latent", ctypes.c_int32), ("d_rope", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("scale", ctypes.c_float), ("reserved", ctypes.c_int32),
+                ("q", ctypes.c_void_p), ("kv", ctypes.c_void_p), ("kv_seq_stride", ctypes.c_int64),
+                ("kv_row_stride", ctypes.c_int64), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
+
+
+_lib_handle = None
+
+
+def lib():
+    """Load libdsa.so once (raises OSError when it has not been built)."""
+    global _lib_handle
+    if _lib_handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"{LIB_PATH} is missing: build it with `python -m dsa_indexer_top_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        st = ctypes.c_int
+        h.dsa_index_scores.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Indexer), P, I64, P, SZ, P]
+        h.dsa_topk.argtypes = [ctypes.POINTER(_Queries), P, I64, I32, P, P, P, SZ, P]
+        for name in ("dsa_sparse_mla_decode", "dsa_sparse_mla_prefill"):
+            getattr(h, name).argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Mla), P, P, I32, P, SZ, P]
+        h.dsa_indexshare_group.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Indexer),
+                                           ctypes.POINTER(_Mla), I32, I32, P, P, P, SZ, P]
+        h.dsa_workspace_bytes.argtypes = [I32, ctypes.POINTER(_Queries), I32, I32, I32, I32]
+        h.dsa_workspace_bytes.restype = SZ
+        h.dsa_workspace_init.argtypes = [P, SZ, P]
+        h.dsa_check_status.argtypes = [P, P]
+        h.dsa_status_str.argtypes = [st]
+        h.dsa_status_str.restype = ctypes.c_char_p
+        for name in ("dsa_index_scores", "dsa_topk", "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill",
+                     "dsa_indexshare_group", "dsa_workspace_init", "dsa_check_status"):
+            getattr(h, name).restype = st
+        _lib_handle = h
+    return _lib_handle
+
+
+def status_str(status: int) -> str:
+    return lib().dsa_status_str(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != DSA_OK:
+        raise DsaError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DSA_BF16
+    if t.dtype == torch.float32:
+        return DSA_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------ descriptors
+@dataclass
+class Queries:
+    q_seq: torch.Tensor          # int32 [n_q]
+    q_pos: torch.Tensor          # int32 [n_q]
+    n_seq: int
+    max_ctx: int
+    seq_run: int = 1
+
+    def c(self) -> _Queries:
+        return _Queries(self.q_pos.numel(), self.n_seq, self.max_ctx, self.seq_run,
+                        self.q_seq.data_ptr() if self.q_seq.numel() else None,
+                        self.q_pos.data_ptr() if self.q_pos.numel() else None)
+
+
+@dataclass
+class Indexer:
+    q: torch.Tensor              # [n_q, heads, dim]
+    w: torch.Tensor              # float32 [n_q, heads]
+    k: torch.Tensor              # [n_seq, L, dim] or [L, dim] (shared cache)
+
+    def c(self) -> _Indexer:
+        shared = self.k.dim() == 2
+        seq_stride = 0 if shared else self.k.stride(0)
+        return _Indexer(self.q.shape[1], self.q.shape[2], _dtype_code(self.q), 0, self.q.data_ptr(),
+                        self.w.data_ptr(), self.k.data_ptr(), seq_stride, self.k.stride(-2))
+
+
+@dataclass
+class Mla:
+    q: torch.Tensor              # [n_q, heads, d_latent + d_rope]
+    kv: torch.Tensor             # [n_seq, L, d_latent + d_rope] or [L, ...] (shared)
+    out: torch.Tensor            # [n_q, heads, d_latent]
+    d_latent: int
+    scale: float
+    lse: Optional[torch.Tensor] = None   # float32 [n_q, heads]
+
+    def c(self) -> _Mla:
+        shared = self.kv.dim() == 2
+        seq_stride = 0 if shared else self.kv.stride(0)
+        heads, dk = self.q.shape[1], self.q.shape[2]
+        return _Mla(heads, self.d_latent, dk - self.d_latent, _dtype_code(self.q), float(self.scale), 0,
+                    self.q.data_ptr(), self.kv.data_ptr(), seq_stride, self.kv.stride(-2),
+                    self.out.data_ptr(), self.lse.data_ptr() if self.lse is not None else None)
+
+
+# ------------------------------------------------------------------ entry points
+def dsa_workspace_bytes(op: int, queries: Queries, topk: int = 1, mla_heads: int = 64, d_latent: int = 512,
+                        n_layers: int = 1) -> int:
+    return int(lib().dsa_workspace_bytes(op, ctypes.byref(queries.c()), topk, mla_heads, d_latent, n_layers))
+
+
+def dsa_workspace_init(ws: torch.Tensor, stream=None):
+    _check(lib().dsa_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_workspace_init")
+
+
+def dsa_check_status(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise, read and clear the workspace status word (returns the code)."""
+    return int(lib().dsa_check_status(_ptr(ws), _stream(stream)))
+
+
+def dsa_index_scores(queries: Queries, indexer: Indexer, scores: torch.Tensor, ws: torch.Tensor, stream=None):
+    qc, ic = queries.c(), indexer.c()
+    _check(lib().dsa_index_scores(ctypes.byref(qc), ctypes.byref(ic), _ptr(scores), scores.stride(0), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _stream(stream)), "dsa_index_scores")
+
+
+def dsa_topk(queries: Queries, scores: torch.Tensor, topk: int, idx: torch.Tensor, cnt: torch.Tensor,
+             ws: torch.Tensor, stream=None):
+    qc = queries.c()
+    _check(lib().dsa_topk(ctypes.byref(qc), _ptr(scores), scores.stride(0), topk, _ptr(idx), _ptr(cnt), _ptr(ws),
+                          ws.numel() * ws.element_size(), _stream(stream)), "dsa_topk")
+
+
+def dsa_sparse_mla_decode(queries: Queries, mla: Mla, idx: torch.Tensor, cnt: torch.Tensor, topk: int,
+                          ws: torch.Tensor, stream=None):
+    qc, mc = queries.c(), mla.c()
+    _check(lib().dsa_sparse_mla_decode(ctypes.byref(qc), ctypes.byref(mc), _ptr(idx), _ptr(cnt), topk, _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)), "dsa_sparse_mla_decode")
+
+
+def dsa_sparse_mla_prefill(queries: Queries, mla: Mla, idx: torch.Tensor, cnt: torch.Tensor, topk: int,
+                           ws: torch.Tensor, stream=None):
+    qc, mc = queries.c(), mla.c()
+    _check(lib().dsa_sparse_mla_prefill(ctypes.byref(qc), ctypes.byref(mc), _ptr(idx), _ptr(cnt), topk, _ptr(ws),
+                                        ws.numel() * ws.element_size(), _stream(stream)), "dsa_sparse_mla_prefill")
+
+
+def dsa_indexshare_group(queries: Queries, indexer: Indexer, layers: Sequence[Mla], topk: int, idx: torch.Tensor,
+                         cnt: torch.Tensor, ws: torch.Tensor, stream=None):
+    qc, ic = queries.c(), indexer.c()
+    arr = (_Mla * len(layers))(*[m.c() for m in layers])
+    _check(lib().dsa_indexshare_group(ctypes.byref(qc), ctypes.byref(ic), arr, len(layers), topk, _ptr(idx),
+                                      _ptr(cnt), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_indexshare_group")
+
+
+# ------------------------------------------------------------------ conveniences
+def workspace(op: int, queries: Queries, topk: int = 1, n_layers: int = 1, device="cuda", stream=None):
+    """Allocate (torch) and zero-initialise a workspace for `op`."""
+    n = dsa_workspace_bytes(op, queries, topk, 64, 512, n_layers)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    dsa_workspace_init(ws, stream)
+    return ws
+
+
+def scores_buffer(n_q: int, max_ctx: int, device="cuda") -> torch.Tensor:
+    """float32 [n_q, ld] with ld = max_ctx rounded up to a multiple of 4."""
+    ld = (max_ctx + 3) // 4 * 4
+    return torch.empty((n_q, ld), dtype=torch.float32, device=device)
+
+
+def default_scale(d_nope: int = 192, d_rope: int = 64) -> float:
+    return 1.0 / math.sqrt(d_nope + d_rope)

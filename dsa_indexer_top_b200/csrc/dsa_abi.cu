@@ -1,0 +1,382 @@
+// dsa_abi.cu -- the extern "C" entry points declared in include/dsa.h:
+// argument validation, workspace layout, TMA descriptor encoding and dispatch to
+// the kernels.  No allocation, no synchronisation (except dsa_check_status).
+#include <cstring>
+#include <mutex>
+
+#include "dsa.h"
+#include "kernels.cuh"
+
+using namespace dsa;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+constexpr int kTopkCacheCap = 40960;  // elements of a top-k chunk kept in shared memory
+constexpr int kDecodeMaxQueries = 256;  // IndexShare group: split-K MLA up to this many queries
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round4(int64_t x) { return (x + 3) & ~static_cast<int64_t>(3); }
+
+int num_sms_current() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+bool valid_queries(const dsa_queries *qs) {
+    if (!qs) return false;
+    if (qs->n_q < 0 || qs->n_seq < 1 || qs->max_ctx < 1 || qs->seq_run < 1) return false;
+    if (qs->n_q > 0 && (!qs->q_seq || !qs->q_pos)) return false;
+    return true;
+}
+
+uint32_t *status_word(void *ws) { return static_cast<uint32_t *>(ws); }
+
+bool ws_ok(void *ws, size_t ws_bytes, size_t need) {
+    return ws && (reinterpret_cast<uintptr_t>(ws) & 255u) == 0 && ws_bytes >= need;
+}
+
+bool indexer_tc_ok(const dsa_indexer *ix) {
+    return ix->dtype == DSA_BF16 && ix->heads == kIdxHeads && ix->dim == kIdxDim && aligned16(ix->q) &&
+           aligned16(ix->k) && ix->k_row_stride % 8 == 0 && ix->k_seq_stride % 8 == 0 &&
+           ix->k_row_stride >= kIdxDim;
+}
+
+bool mla_tc_ok(const dsa_mla *m) {
+    return m->dtype == DSA_BF16 && m->heads == kMlaHeads && m->d_latent == kLatent && m->d_rope == kRope &&
+           aligned16(m->q) && aligned16(m->kv) && aligned16(m->out) && m->kv_row_stride % 8 == 0 &&
+           m->kv_seq_stride % 8 == 0 && m->kv_row_stride >= kRow;
+}
+
+size_t ws_index_scores() { return kStatusBytes; }
+size_t ws_topk() { return kStatusBytes; }
+int decode_splits(int topk) { return (topk + kRowsPerChunk - 1) / kRowsPerChunk; }
+size_t ws_mla_decode(int n_q, int topk, int n_layers) {
+    const int ns = decode_splits(topk);
+    return kStatusBytes + (ns > 1 ? align256(mla_partial_bytes(n_layers, n_q, ns)) : 0);
+}
+size_t ws_scores(int n_q, int max_ctx) {
+    return align256(static_cast<size_t>(n_q) * round4(max_ctx) * sizeof(float));
+}
+bool group_uses_decode(int n_q) { return n_q <= kDecodeMaxQueries; }
+size_t ws_group(int n_q, int max_ctx, int topk, int n_layers) {
+    size_t b = kStatusBytes + ws_scores(n_q, max_ctx);
+    if (group_uses_decode(n_q)) b += ws_mla_decode(n_q, topk, n_layers) - kStatusBytes;
+    return b;
+}
+
+// ------------------------------------------------------------------ indexer
+dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *scores, int64_t ld,
+                           uint32_t *status, cudaStream_t st) {
+    const int n_cache = ix->k_seq_stride == 0 ? 1 : qs->n_seq;
+    if (indexer_tc_ok(ix)) {
+        EncodeTiledFn enc = encode_fn();
+        if (!enc) return DSA_ERR_CUDA;
+        CUtensorMap tk, tq;
+        {
+            cuuint64_t dims[3] = {static_cast<cuuint64_t>(kIdxDim), static_cast<cuuint64_t>(qs->max_ctx),
+                                  static_cast<cuuint64_t>(n_cache)};
+            const int64_t seq_stride = ix->k_seq_stride == 0 ? ix->k_row_stride * qs->max_ctx : ix->k_seq_stride;
+            cuuint64_t strides[2] = {static_cast<cuuint64_t>(ix->k_row_stride * 2),
+                                     static_cast<cuuint64_t>(seq_stride * 2)};
+            cuuint32_t box[3] = {64, 128, 1};
+            cuuint32_t es[3] = {1, 1, 1};
+            if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ix->k), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return DSA_ERR_INVALID;
+        }
+        int G = 1;
+        while (G < 8 && qs->seq_run % (G * 2) == 0) G *= 2;
+        {
+            cuuint64_t dims[2] = {static_cast<cuuint64_t>(kIdxDim), static_cast<cuuint64_t>(qs->n_q) * kIdxHeads};
+            cuuint64_t strides[1] = {static_cast<cuuint64_t>(kIdxDim * 2)};
+            cuuint32_t box[2] = {64, static_cast<cuuint32_t>(32 * G)};
+            cuuint32_t es[2] = {1, 1};
+            if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ix->q), dims, strides, box, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return DSA_ERR_INVALID;
+        }
+        IdxTcArgs a;
+        a.w = ix->w;
+        a.q_seq = qs->q_seq;
+        a.q_pos = qs->q_pos;
+        a.scores = scores;
+        a.ld = ld;
+        a.status = status;
+        a.n_q = qs->n_q;
+        a.n_seq = qs->n_seq;
+        a.L = qs->max_ctx;
+        a.k_shared = ix->k_seq_stride == 0 ? 1 : 0;
+        a.tiles_per_group = (qs->max_ctx + 127) / 128;
+        const long long groups = (qs->n_q + G - 1) / G;
+        a.total_items = groups * a.tiles_per_group;
+        const int sms = num_sms_current();
+        const int grid = static_cast<int>(a.total_items < sms ? a.total_items : sms);
+        return launch_idx_score_tc(G, tk, tq, a, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    }
+    const size_t smem = sizeof(float) * (static_cast<size_t>(ix->heads) * ix->dim + ix->heads);
+    if (smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
+    IdxGenericArgs g;
+    g.q = ix->q;
+    g.w = ix->w;
+    g.k = ix->k;
+    g.k_seq_stride = ix->k_seq_stride;
+    g.k_row_stride = ix->k_row_stride;
+    g.q_seq = qs->q_seq;
+    g.q_pos = qs->q_pos;
+    g.scores = scores;
+    g.ld = ld;
+    g.status = status;
+    g.n_q = qs->n_q;
+    g.n_seq = qs->n_seq;
+    g.L = qs->max_ctx;
+    g.heads = ix->heads;
+    g.dim = ix->dim;
+    g.is_bf16 = ix->dtype == DSA_BF16;
+    return launch_idx_score_generic(g, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status check_indexer(const dsa_queries *qs, const dsa_indexer *ix) {
+    if (!ix || !ix->q || !ix->w || !ix->k) return DSA_ERR_INVALID;
+    if (ix->heads < 1 || ix->dim < 1 || (ix->dtype != DSA_BF16 && ix->dtype != DSA_F32)) return DSA_ERR_INVALID;
+    if (ix->k_row_stride < ix->dim || ix->k_seq_stride < 0) return DSA_ERR_INVALID;
+    if (ix->k_seq_stride != 0 && ix->k_seq_stride < ix->k_row_stride * qs->max_ctx) return DSA_ERR_INVALID;
+    return DSA_OK;
+}
+
+// ------------------------------------------------------------------ top-k
+dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int topk, int32_t *idx,
+                   int32_t *cnt, uint32_t *status, cudaStream_t st) {
+    TopkArgs a;
+    a.scores = scores;
+    a.ld = ld;
+    a.q_pos = qs->q_pos;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.status = status;
+    a.n_q = qs->n_q;
+    a.L = qs->max_ctx;
+    a.topk = topk;
+    a.cache_cap = kTopkCacheCap;
+    return launch_topk(a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+bool scores_ok(const float *scores, int64_t ld, int max_ctx) {
+    return scores && aligned16(scores) && ld >= max_ctx && ld % 4 == 0;
+}
+
+// ------------------------------------------------------------------ MLA
+dsa_status check_mla_layers(const dsa_mla *layers, int n_layers) {
+    if (!layers || n_layers < 1 || n_layers > kMaxLayers) return DSA_ERR_INVALID;
+    const dsa_mla &m0 = layers[0];
+    for (int l = 0; l < n_layers; ++l) {
+        const dsa_mla &m = layers[l];
+        if (!m.q || !m.kv || !m.out) return DSA_ERR_INVALID;
+        if (m.heads < 1 || m.d_latent < 1 || m.d_rope < 0 || (m.dtype != DSA_BF16 && m.dtype != DSA_F32))
+            return DSA_ERR_INVALID;
+        if (m.kv_row_stride < m.d_latent + m.d_rope || m.kv_seq_stride < 0) return DSA_ERR_INVALID;
+        if (m.heads != m0.heads || m.d_latent != m0.d_latent || m.d_rope != m0.d_rope || m.dtype != m0.dtype ||
+            m.scale != m0.scale || m.kv_row_stride != m0.kv_row_stride || m.kv_seq_stride != m0.kv_seq_stride)
+            return DSA_ERR_INVALID;
+    }
+    return DSA_OK;
+}
+
+dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, const int32_t *idx,
+                  const int32_t *cnt, int topk, bool decode, uint8_t *scratch, uint32_t *status,
+                  cudaStream_t st) {
+    MlaArgs a;
+    std::memset(&a, 0, sizeof(a));
+    for (int l = 0; l < n_layers; ++l) {
+        a.layer[l].q = layers[l].q;
+        a.layer[l].kv = layers[l].kv;
+        a.layer[l].out = layers[l].out;
+        a.layer[l].lse = layers[l].lse;
+    }
+    const dsa_mla &m = layers[0];
+    a.n_layers = n_layers;
+    a.kv_seq_stride = m.kv_seq_stride;
+    a.kv_row_stride = m.kv_row_stride;
+    a.q_seq = qs->q_seq;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.topk = topk;
+    a.n_q = qs->n_q;
+    a.n_seq = qs->n_seq;
+    a.L = qs->max_ctx;
+    a.heads = m.heads;
+    a.d_lat = m.d_latent;
+    a.d_rope = m.d_rope;
+    a.scale = m.scale;
+    a.is_bf16 = m.dtype == DSA_BF16;
+    a.status = status;
+    bool tc = true;
+    for (int l = 0; l < n_layers; ++l) tc = tc && mla_tc_ok(&layers[l]);
+    if (tc) {
+        const int nch = decode_splits(topk);
+        if (decode && nch > 1) {
+            a.n_splits = nch;
+            a.chunks_per_cta = 1;
+            a.part_o = reinterpret_cast<float *>(scratch);
+            const size_t rows = static_cast<size_t>(n_layers) * qs->n_q * nch * kMlaHeads;
+            a.part_ml = reinterpret_cast<float *>(scratch + rows * kLatent * sizeof(float));
+            if (launch_mla_tc(a, st) != cudaSuccess) return DSA_ERR_CUDA;
+            return launch_mla_combine(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+        }
+        a.n_splits = 1;
+        a.chunks_per_cta = nch;
+        return launch_mla_tc(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    }
+    const size_t smem = sizeof(float) * (static_cast<size_t>(m.d_latent + m.d_rope) + topk);
+    if (smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
+    return launch_mla_generic(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *dsa_status_str(dsa_status s) {
+    switch (s) {
+        case DSA_OK: return "DSA_OK";
+        case DSA_ERR_INVALID: return "DSA_ERR_INVALID";
+        case DSA_ERR_UNSUPPORTED: return "DSA_ERR_UNSUPPORTED";
+        case DSA_ERR_WORKSPACE: return "DSA_ERR_WORKSPACE";
+        case DSA_ERR_CUDA: return "DSA_ERR_CUDA";
+        case DSA_ERR_TIMEOUT: return "DSA_ERR_TIMEOUT";
+    }
+    return "DSA_ERR_UNKNOWN";
+}
+
+size_t dsa_workspace_bytes(int32_t op, const dsa_queries *qs, int32_t topk, int32_t mla_heads, int32_t d_latent,
+                           int32_t n_layers) {
+    (void)mla_heads;
+    (void)d_latent;
+    if (!qs) return 0;
+    const int n_q = qs->n_q > 0 ? qs->n_q : 0;
+    switch (op) {
+        case DSA_OP_INDEX_SCORES: return ws_index_scores();
+        case DSA_OP_TOPK: return ws_topk();
+        case DSA_OP_MLA_DECODE: return ws_mla_decode(n_q, topk > 0 ? topk : 1, 1);
+        case DSA_OP_MLA_PREFILL: return kStatusBytes;
+        case DSA_OP_INDEXSHARE_GROUP:
+            return ws_group(n_q, qs->max_ctx > 0 ? qs->max_ctx : 1, topk > 0 ? topk : 1,
+                            n_layers > 0 ? n_layers : 1);
+    }
+    return 0;
+}
+
+dsa_status dsa_workspace_init(void *ws, size_t ws_bytes, void *stream) {
+    if (!ws_ok(ws, ws_bytes, kStatusBytes)) return DSA_ERR_WORKSPACE;
+    return cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSA_OK
+                                                                                                   : DSA_ERR_CUDA;
+}
+
+dsa_status dsa_check_status(void *ws, void *stream) {
+    if (!ws) return DSA_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (v != 0 && cudaMemsetAsync(ws, 0, sizeof(v), st) != cudaSuccess) return DSA_ERR_CUDA;
+    return static_cast<dsa_status>(v);
+}
+
+dsa_status dsa_index_scores(const dsa_queries *queries, const dsa_indexer *indexer, float *scores,
+                            int64_t ld_scores, void *ws, size_t ws_bytes, void *stream) {
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (!ws_ok(ws, ws_bytes, ws_index_scores())) return DSA_ERR_WORKSPACE;
+    dsa_status s = check_indexer(queries, indexer);
+    if (s != DSA_OK) return s;
+    if (!scores_ok(scores, ld_scores, queries->max_ctx)) return DSA_ERR_INVALID;
+    if (queries->n_q == 0) return DSA_OK;
+    return do_index_scores(queries, indexer, scores, ld_scores, status_word(ws), static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_scores, int32_t topk, int32_t *idx,
+                    int32_t *cnt, void *ws, size_t ws_bytes, void *stream) {
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (!ws_ok(ws, ws_bytes, ws_topk())) return DSA_ERR_WORKSPACE;
+    if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
+    if (!scores_ok(scores, ld_scores, queries->max_ctx)) return DSA_ERR_INVALID;
+    if (queries->n_q == 0) return DSA_OK;
+    return do_topk(queries, scores, ld_scores, topk, idx, cnt, status_word(ws), static_cast<cudaStream_t>(stream));
+}
+
+static dsa_status mla_entry(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx, const int32_t *cnt,
+                            int32_t topk, void *ws, size_t ws_bytes, void *stream, bool decode) {
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
+    dsa_status s = check_mla_layers(mla, 1);
+    if (s != DSA_OK) return s;
+    const size_t need = decode ? ws_mla_decode(queries->n_q, topk, 1) : kStatusBytes;
+    if (!ws_ok(ws, ws_bytes, need)) return DSA_ERR_WORKSPACE;
+    if (queries->n_q == 0) return DSA_OK;
+    return do_mla(queries, mla, 1, idx, cnt, topk, decode, static_cast<uint8_t *>(ws) + kStatusBytes,
+                  status_word(ws), static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_sparse_mla_decode(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,
+                                 const int32_t *cnt, int32_t topk, void *ws, size_t ws_bytes, void *stream) {
+    return mla_entry(queries, mla, idx, cnt, topk, ws, ws_bytes, stream, true);
+}
+
+dsa_status dsa_sparse_mla_prefill(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,
+                                  const int32_t *cnt, int32_t topk, void *ws, size_t ws_bytes, void *stream) {
+    return mla_entry(queries, mla, idx, cnt, topk, ws, ws_bytes, stream, false);
+}
+
+dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *indexer, const dsa_mla *layers,
+                                int32_t n_layers, int32_t topk, int32_t *idx, int32_t *cnt, void *ws,
+                                size_t ws_bytes, void *stream) {
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
+    dsa_status s = check_indexer(queries, indexer);
+    if (s != DSA_OK) return s;
+    s = check_mla_layers(layers, n_layers);
+    if (s != DSA_OK) return s;
+    if (!ws_ok(ws, ws_bytes, ws_group(queries->n_q, queries->max_ctx, topk, n_layers))) return DSA_ERR_WORKSPACE;
+    if (queries->n_q == 0) return DSA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *scores = reinterpret_cast<float *>(base + kStatusBytes);
+    const int64_t ld = round4(queries->max_ctx);
+    uint8_t *scratch = base + kStatusBytes + ws_scores(queries->n_q, queries->max_ctx);
+    s = do_index_scores(queries, indexer, scores, ld, status_word(ws), st);
+    if (s != DSA_OK) return s;
+    s = do_topk(queries, scores, ld, topk, idx, cnt, status_word(ws), st);
+    if (s != DSA_OK) return s;
+    return do_mla(queries, layers, n_layers, idx, cnt, topk, group_uses_decode(queries->n_q), scratch,
+                  status_word(ws), st);
+}
+
+}  // extern "C"

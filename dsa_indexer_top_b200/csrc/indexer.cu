@@ -1,0 +1,363 @@
+// indexer.cu -- lightning-indexer scores.
+//
+// score(t,s) = sum_h w[t,h] * max(0, q_idx[t,h] . k_idx[s]) for s <= t
+// ("GLM-5.2 -- Model techniques map", "Checked in its code", Indexer-selected
+// sparse attention: the indexer scores past tokens per head, index_n_heads = 32,
+// index_head_dim = 128; row "QK normalization": one key per token, [B,S,1,D]).
+//
+// Tensor-core path (bf16, 32 x 128): a persistent, warp-specialised kernel.
+//   warp 0      TMA producer: 128-key x 128-dim tiles (32 KB, two 64-dim boxes,
+//               128-byte swizzle) into a ring of shared-memory stages; the
+//               query tile (G queries x 32 heads x 128 dims) once per group.
+//   warp 1      tcgen05.mma issuer: D[128 keys][32G] = K_tile (M=128, K-major)
+//               x Q^T (N = 32G, K-major), K = 128 in eight K=16 steps, fp32
+//               accumulators in TMEM, double-buffered.
+//   warps 2-5   epilogue: tcgen05.ld of its 32 TMEM lanes (one key per lane),
+//               ReLU, multiply by w and sum the 32 heads inside the thread, causal
+//               mask, coalesced fp32 store of one score per key per query.
+// Work items are (query group, key tile) pairs split evenly over a grid of at
+// most one CTA per SM; tiles past the group's last visible key are skipped.
+#include <algorithm>
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kTileKeys = 128;
+constexpr int kATileBytes = kTileKeys * kIdxDim * 2;  // 32 KB
+constexpr int kIdxThreads = 192;
+
+template <int G>
+struct IdxCfg {
+    static constexpr int N = 32 * G;
+    static constexpr int kStages = (G == 8) ? 4 : 6;
+    static constexpr int kBBytes = N * kIdxDim * 2;
+    static constexpr int kTmemCols = (2 * N < 32) ? 32 : 2 * N;
+    static constexpr int kSmem = kStages * kATileBytes + kBBytes + 1024;
+    static constexpr uint32_t kIdesc = idesc_bf16(128, N, false, false);
+};
+
+// Sequence and last visible position of a query group; every role calls this
+// with the same arguments and so skips the same tiles.
+template <int G>
+__device__ __forceinline__ void group_info(const IdxTcArgs &a, int g, int &seq, int &max_pos) {
+    int q0 = g * G;
+    int nq = min(G, a.n_q - q0);
+    seq = a.k_shared ? 0 : __ldg(a.q_seq + q0);
+    max_pos = -1;
+    if (seq < 0 || seq >= a.n_seq) {
+        seq = -1;
+        return;
+    }
+    for (int i = 0; i < nq; ++i) {
+        int p = __ldg(a.q_pos + q0 + i);
+        if (p >= 0 && p < a.L) max_pos = max(max_pos, p);
+    }
+}
+
+template <int G>
+__global__ void __launch_bounds__(kIdxThreads, 1)
+    idx_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_q, const IdxTcArgs a) {
+    using Cfg = IdxCfg<G>;
+    constexpr int N = Cfg::N;
+    constexpr int S = Cfg::kStages;
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                ~uintptr_t(1023));
+    uint8_t *a_tiles = smem;                      // S x 32 KB
+    uint8_t *b_tile = smem + S * kATileBytes;     // N rows x 256 B
+
+    __shared__ uint64_t full_bar[S], empty_bar[S];
+    __shared__ uint64_t tmem_full[2], tmem_empty[2];
+    __shared__ uint64_t b_full, b_empty, mma_done;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
+    __shared__ float w_sh[4][N];  // one private copy per epilogue warp
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&tmem_full[s], 1);
+            mbar_init(&tmem_empty[s], 4);
+        }
+        mbar_init(&b_full, 1);
+        mbar_init(&b_empty, 1);
+        mbar_init(&mma_done, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_q);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = tmem_base_sh;
+
+    const long long total = a.total_items;
+    const long long begin = total * blockIdx.x / gridDim.x;
+    const long long end = total * (blockIdx.x + 1) / gridDim.x;
+    const int tpg = a.tiles_per_group;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int cur_g = -1, seq = -1, max_pos = -1;
+            bool group_loaded = false;
+            int b_uses = 0;
+            long long k_tiles = 0;
+            int last_use[S];
+            for (int s = 0; s < S; ++s) last_use[s] = -1;
+            for (long long it = begin; it < end; ++it) {
+                const int g = static_cast<int>(it / tpg);
+                const int j = static_cast<int>(it % tpg);
+                if (g != cur_g) {
+                    group_info<G>(a, g, seq, max_pos);
+                    cur_g = g;
+                    group_loaded = false;
+                }
+                if (seq < 0 || j * kTileKeys > max_pos) continue;
+                if (!group_loaded) {
+                    if (b_uses > 0 &&
+                        !mbar_wait(&b_empty, (b_uses - 1) & 1, a.status, &abort_flag))
+                        break;
+                    mbar_arrive_expect_tx(&b_full, Cfg::kBBytes);
+                    tma_load_2d(b_tile, &tmap_q, &b_full, 0, g * N);
+                    tma_load_2d(b_tile + N * 128, &tmap_q, &b_full, 64, g * N);
+                    ++b_uses;
+                    group_loaded = true;
+                }
+                const int stage = static_cast<int>(k_tiles % S);
+                const int use = static_cast<int>(k_tiles / S);
+                if (!mbar_wait(&empty_bar[stage], (use & 1) ^ 1, a.status, &abort_flag)) break;
+                uint8_t *dst = a_tiles + stage * kATileBytes;
+                mbar_arrive_expect_tx(&full_bar[stage], kATileBytes);
+                tma_load_3d(dst, &tmap_k, &full_bar[stage], 0, j * kTileKeys, seq);
+                tma_load_3d(dst + kATileBytes / 2, &tmap_k, &full_bar[stage], 64, j * kTileKeys,
+                            seq);
+                last_use[stage] = use;
+                ++k_tiles;
+            }
+            // Drain: every copy this thread issued has landed before the CTA exits.
+            for (int s = 0; s < S; ++s)
+                if (last_use[s] >= 0) mbar_wait(&full_bar[s], last_use[s] & 1, a.status, nullptr);
+            if (b_uses > 0) mbar_wait(&b_full, (b_uses - 1) & 1, a.status, nullptr);
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int cur_g = -1, seq = -1, max_pos = -1;
+            bool group_ready = false;
+            int b_uses = 0;
+            long long k_tiles = 0;
+            for (long long it = begin; it < end; ++it) {
+                const int g = static_cast<int>(it / tpg);
+                const int j = static_cast<int>(it % tpg);
+                if (g != cur_g) {
+                    group_info<G>(a, g, seq, max_pos);
+                    cur_g = g;
+                    group_ready = false;
+                }
+                if (seq < 0 || j * kTileKeys > max_pos) continue;
+                if (!group_ready) {
+                    if (b_uses > 0) umma_commit(&b_empty);  // previous group's MMAs release B
+                    if (!mbar_wait(&b_full, b_uses & 1, a.status, &abort_flag)) break;
+                    tc_fence_after();
+                    ++b_uses;
+                    group_ready = true;
+                }
+                const int stage = static_cast<int>(k_tiles % S);
+                const int use = static_cast<int>(k_tiles / S);
+                const int acc = static_cast<int>(k_tiles & 1);
+                const int acc_use = static_cast<int>(k_tiles >> 1);
+                if (!mbar_wait(&tmem_empty[acc], (acc_use & 1) ^ 1, a.status, &abort_flag)) break;
+                tc_fence_after();
+                if (!mbar_wait(&full_bar[stage], use & 1, a.status, &abort_flag)) break;
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(a_tiles + stage * kATileBytes);
+                const uint32_t b_addr = smem_u32(b_tile);
+                const uint32_t d_tmem = tmem_base + acc * N;
+#pragma unroll
+                for (int kk = 0; kk < kIdxDim / 16; ++kk) {
+                    const uint32_t koff = (kk & 3) * 32u;
+                    const uint64_t adesc =
+                        sdesc_sw128(a_addr + (kk >> 2) * (kATileBytes / 2) + koff, 16, 1024);
+                    const uint64_t bdesc = sdesc_sw128(b_addr + (kk >> 2) * (N * 128) + koff, 16, 1024);
+                    umma_bf16(d_tmem, adesc, bdesc, Cfg::kIdesc, kk > 0 ? 1u : 0u);
+                }
+                umma_commit(&empty_bar[stage]);
+                umma_commit(&tmem_full[acc]);
+                ++k_tiles;
+            }
+            umma_commit(&mma_done);
+            mbar_wait(&mma_done, 0, a.status, nullptr);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        float *w_mine = w_sh[warp - 2];
+        int cur_g = -1, seq = -1, max_pos = -1;
+        int qpos[G];
+        bool qok[G];
+        long long k_tiles = 0;
+        for (long long it = begin; it < end; ++it) {
+            const int g = static_cast<int>(it / tpg);
+            const int j = static_cast<int>(it % tpg);
+            if (g != cur_g) {
+                group_info<G>(a, g, seq, max_pos);
+                cur_g = g;
+                const int q0 = g * G;
+                __syncwarp();  // this warp no longer reads the previous group's w
+                for (int e = lane; e < N; e += 32) {
+                    const int qi = q0 + e / 32;
+                    w_mine[e] = qi < a.n_q ? __ldg(a.w + static_cast<int64_t>(qi) * kIdxHeads + (e & 31)) : 0.f;
+                }
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < G; ++i) {
+                    const int qi = q0 + i;
+                    qpos[i] = -1;
+                    qok[i] = false;
+                    if (qi < a.n_q) {
+                        const int p = __ldg(a.q_pos + qi);
+                        const int sq = __ldg(a.q_seq + qi);
+                        const bool seq_ok = a.k_shared ? (sq >= 0 && sq < a.n_seq) : (sq == seq);
+                        qok[i] = p >= 0 && p < a.L && seq_ok && seq >= 0;
+                        qpos[i] = p;
+                        if (!qok[i] && lane == 0) report_status(a.status, DSA_ERR_INVALID);
+                    }
+                }
+            }
+            if (seq < 0 || j * kTileKeys > max_pos) continue;
+            const int acc = static_cast<int>(k_tiles & 1);
+            const int acc_use = static_cast<int>(k_tiles >> 1);
+            if (!mbar_wait(&tmem_full[acc], acc_use & 1, a.status, &abort_flag)) break;
+            tc_fence_after();
+            const int s = j * kTileKeys + quad * 32 + lane;
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * N;
+#pragma unroll
+            for (int i = 0; i < G; ++i) {
+                uint32_t r[32];
+                tmem_ld32(taddr + i * 32, r);
+                tmem_ld_wait();
+                float score = 0.f;
+#pragma unroll
+                for (int h = 0; h < 32; ++h) score = fmaf(w_mine[i * 32 + h], fmaxf(u2f(r[h]), 0.f), score);
+                if (qok[i] && s <= qpos[i])
+                    a.scores[static_cast<int64_t>(g * G + i) * a.ld + s] = score;
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tmem_empty[acc]);
+            ++k_tiles;
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, Cfg::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------- generic path
+// One thread per (query, key); the query's heads x dims and weights sit in
+// shared memory.  Any head count / dim, bf16 or fp32 inputs.
+template <typename T>
+__device__ __forceinline__ float to_f(T v);
+template <>
+__device__ __forceinline__ float to_f<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__global__ void __launch_bounds__(256) idx_score_generic_kernel(const IdxGenericArgs a) {
+    extern __shared__ float sq[];  // heads*dim query values, then heads weights
+    const int i = blockIdx.y;
+    const T *q = static_cast<const T *>(a.q) + static_cast<int64_t>(i) * a.heads * a.dim;
+    for (int e = threadIdx.x; e < a.heads * a.dim; e += blockDim.x) sq[e] = to_f<T>(q[e]);
+    for (int e = threadIdx.x; e < a.heads; e += blockDim.x)
+        sq[a.heads * a.dim + e] = a.w[static_cast<int64_t>(i) * a.heads + e];
+    __syncthreads();
+    const int pos = a.q_pos[i];
+    const int seq = a.q_seq[i];
+    const bool ok = pos >= 0 && pos < a.L && seq >= 0 && seq < a.n_seq;
+    if (!ok) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) report_status(a.status, DSA_ERR_INVALID);
+        return;
+    }
+    const T *kb = static_cast<const T *>(a.k) + (a.k_seq_stride ? static_cast<int64_t>(seq) * a.k_seq_stride : 0);
+    const float *wv = sq + a.heads * a.dim;
+    for (int s = blockIdx.x * blockDim.x + threadIdx.x; s <= pos; s += gridDim.x * blockDim.x) {
+        const T *kr = kb + static_cast<int64_t>(s) * a.k_row_stride;
+        float score = 0.f;
+        for (int h = 0; h < a.heads; ++h) {
+            const float *qh = sq + h * a.dim;
+            float dot = 0.f;
+            for (int d = 0; d < a.dim; ++d) dot = fmaf(qh[d], to_f<T>(kr[d]), dot);
+            score = fmaf(wv[h], fmaxf(dot, 0.f), score);
+        }
+        a.scores[static_cast<int64_t>(i) * a.ld + s] = score;
+    }
+}
+
+template <int G>
+cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcArgs &a, int grid,
+                      cudaStream_t st) {
+    using Cfg = IdxCfg<G>;
+    cudaError_t e = cudaFuncSetAttribute(idx_score_tc_kernel<G>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    if (e != cudaSuccess) return e;
+    idx_score_tc_kernel<G><<<grid, kIdxThreads, Cfg::kSmem, st>>>(tk, tq, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_idx_score_tc(int G, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
+                                const IdxTcArgs &a, int grid, cudaStream_t st) {
+    switch (G) {
+        case 1: return launch_tc<1>(tmap_k, tmap_q, a, grid, st);
+        case 2: return launch_tc<2>(tmap_k, tmap_q, a, grid, st);
+        case 4: return launch_tc<4>(tmap_k, tmap_q, a, grid, st);
+        case 8: return launch_tc<8>(tmap_k, tmap_q, a, grid, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_idx_score_generic(const IdxGenericArgs &a, cudaStream_t st) {
+    const size_t smem = sizeof(float) * (static_cast<size_t>(a.heads) * a.dim + a.heads);
+    const int bx = std::min((a.L + 255) / 256, 1024);
+    dim3 grid(bx, a.n_q);
+    if (a.is_bf16) {
+        cudaError_t e = cudaFuncSetAttribute(idx_score_generic_kernel<__nv_bfloat16>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        idx_score_generic_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(a);
+    } else {
+        cudaError_t e = cudaFuncSetAttribute(idx_score_generic_kernel<float>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        idx_score_generic_kernel<float><<<grid, 256, smem, st>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace dsa

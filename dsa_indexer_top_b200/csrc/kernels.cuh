@@ -1,0 +1,110 @@
+// kernels.cuh -- internal launch interface between the C ABI (dsa_abi.cu) and
+// the kernels (indexer.cu, topk.cu, mla.cu).  Not part of the public header.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace dsa {
+
+constexpr int kIdxHeads = 32;   // index_n_heads of GLM-5.2
+constexpr int kIdxDim = 128;    // index_head_dim of GLM-5.2
+constexpr int kMlaHeads = 64;   // num_attention_heads of GLM-5.2
+constexpr int kLatent = 512;    // kv_lora_rank
+constexpr int kRope = 64;       // qk_rope_head_dim
+constexpr int kRow = kLatent + kRope;
+constexpr int kRowsPerChunk = 128;  // selected rows per tensor-core chunk
+constexpr int kMaxTopk = 4096;
+constexpr int kMaxLayers = 4;
+
+// ------------------------------------------------------------------ indexer
+struct IdxTcArgs {
+    const float *w;
+    const int32_t *q_seq;
+    const int32_t *q_pos;
+    float *scores;
+    int64_t ld;
+    uint32_t *status;
+    int n_q, n_seq, L;
+    int k_shared;         // 1: every query reads cache 0
+    int tiles_per_group;  // ceil(L / 128)
+    long long total_items;
+};
+
+// G = queries per tensor-core tile (1, 2, 4 or 8).  Tensor maps: keys 3-D
+// {128, L, n_cache} bf16, box {64, 128, 1}; queries 2-D {128, n_q*32}, box
+// {64, 32*G}; both 128-byte swizzled.
+cudaError_t launch_idx_score_tc(int G, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
+                                const IdxTcArgs &a, int grid, cudaStream_t st);
+
+struct IdxGenericArgs {
+    const void *q;
+    const float *w;
+    const void *k;
+    int64_t k_seq_stride, k_row_stride;
+    const int32_t *q_seq;
+    const int32_t *q_pos;
+    float *scores;
+    int64_t ld;
+    uint32_t *status;
+    int n_q, n_seq, L, heads, dim;
+    int is_bf16;
+};
+cudaError_t launch_idx_score_generic(const IdxGenericArgs &a, cudaStream_t st);
+
+// ------------------------------------------------------------------ top-k
+struct TopkArgs {
+    const float *scores;
+    int64_t ld;
+    const int32_t *q_pos;
+    int32_t *idx;
+    int32_t *cnt;
+    uint32_t *status;
+    int n_q, L, topk;
+    int cache_cap;  // elements of a CTA's chunk kept in shared memory
+};
+cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st);
+
+// ------------------------------------------------------------------ sparse MLA
+struct MlaLayerPtrs {
+    const void *q;
+    const void *kv;
+    void *out;
+    float *lse;
+};
+
+struct MlaArgs {
+    MlaLayerPtrs layer[kMaxLayers];
+    int n_layers;
+    int64_t kv_seq_stride, kv_row_stride;
+    const int32_t *q_seq;
+    const int32_t *idx;
+    const int32_t *cnt;
+    int topk;
+    int n_q, n_seq, L;
+    int heads, d_lat, d_rope;
+    float scale;
+    int is_bf16;
+    uint32_t *status;
+    // split-K schedule (tensor-core path)
+    int n_splits;        // CTAs per query
+    int chunks_per_cta;  // 128-row chunks walked by one CTA
+    float *part_o;       // [layers][n_q][n_splits][64][512] unnormalised
+    float *part_ml;      // [layers][n_q][n_splits][64][2] (max, sum) in log2 units
+};
+
+// Tensor-core sparse MLA (bf16, 64 heads, 512 + 64).  n_splits == 1 writes the
+// final output; otherwise partials followed by launch_mla_combine.
+cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st);
+cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st);
+cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st);
+
+// Bytes of split-K partials for the tensor-core decode schedule.
+inline size_t mla_partial_bytes(int n_layers, int n_q, int n_splits) {
+    size_t rows = static_cast<size_t>(n_layers) * n_q * n_splits * kMlaHeads;
+    return rows * kLatent * sizeof(float) + rows * 2 * sizeof(float);
+}
+
+}  // namespace dsa

@@ -1,0 +1,255 @@
+/*
+ * dsa.h -- C ABI of libdsa.so: the DeepSeek-Sparse-Attention hot path of GLM-5.2
+ * (lightning indexer -> causal top-k -> absorbed sparse MLA, with IndexShare
+ * reuse), as hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title, section) for what each call computes:
+ *  [TM] "GLM-5.2 -- Model techniques map", section "Checked in its code":
+ *       row "Indexer-selected sparse attention (DeepSeek Sparse Attention)" --
+ *       an indexer scores past tokens per head, each query attends only to the
+ *       index_topk = 2048 selected tokens; index_n_heads = 32, index_head_dim =
+ *       128; the selection is min(index_topk, n) indices as int32 [B, S, topk];
+ *       row "QK normalization" -- one indexer key per token, [B, S, 1, D];
+ *       row "Multi-head latent attention" -- a 512-dim kv latent plus a 64-dim
+ *       RoPE key per token; row "Learnable attention sink" -- plain float32
+ *       softmax, no sink; row "Partial RoPE" -- 192 nope + 64 rope dims.
+ *  [HA] "GLM 5.2 -- Hermosa AI", section "MLA + DSA with IndexShare" -- a full
+ *       layer selects the top 2048 cached tokens per query, the next three
+ *       layers reuse that selection; section "78 layers, IndexShare pattern".
+ *  [AE] "GLM-5.2 -- LLM architectures explained", section "Modelled costs" --
+ *       93 KiB of BF16 cache per token pins the per-layer row of 576 bf16 and the
+ *       128-bf16 indexer key on full layers.
+ *
+ * Details the pages leave open, fixed here:
+ *  - score(t,s) = sum_h w[t,h] * max(0, q_idx[t,h] . k_idx[s]) (post-RoPE
+ *    inputs, no extra scale), w float32;
+ *  - query t sees cache rows s = 0..t;
+ *  - top-k keeps min(topk, t+1) rows, ties go to the lower position, the kept
+ *    positions are written in ascending order and padded with -1;
+ *  - absorbed MLA: per head the query is [q_lat (d_latent) | q_rope (d_rope)],
+ *    logit = scale * (q_lat . c_s + q_rope . r_s) with cache rows [c_s | r_s],
+ *    output o = sum_j softmax_j * c_{s_j} (d_latent values per head); the W_UV
+ *    up-projection is applied by the caller.
+ *
+ * Conventions for every call:
+ *  - Memory: the caller owns every buffer.  All tensor pointers are DEVICE
+ *    pointers unless stated otherwise; the library never allocates, frees or
+ *    synchronises inside a compute call.  `stream` is a cudaStream_t (NULL =
+ *    legacy default stream); work is enqueued on it and results are valid in
+ *    stream order.
+ *  - Workspace: `ws` is a device buffer of at least dsa_workspace_bytes(...)
+ *    bytes, 256-byte aligned.  Its first 256 bytes hold a status word that
+ *    kernels set on device-detected errors (out-of-range positions or indices,
+ *    a bounded wait that ran out).  Zero it once with dsa_workspace_init();
+ *    read (and clear) it with dsa_check_status().
+ *  - Errors: invalid arguments are rejected synchronously, before any launch,
+ *    with DSA_ERR_INVALID (null pointer, bad size, misaligned row, workspace too
+ *    small -> DSA_ERR_WORKSPACE); a launch failure returns DSA_ERR_CUDA.  A call
+ *    with n_q == 0 does nothing and returns DSA_OK.
+ *  - Fast paths: bf16 indexers with 32 heads x 128 dims run on tcgen05 tensor
+ *    cores fed by TMA; bf16 MLA with 64 heads x (512 + 64) runs on tcgen05 with
+ *    TMEM accumulators.  Other shapes and float32 inputs run generic CUDA-core
+ *    kernels.  There is no CPU path.
+ *  - Thread safety: calls are re-entrant; the only global state is one-time
+ *    per-device kernel attribute setup.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID = 1,     /* bad argument (host) or bad position/index (device) */
+    DSA_ERR_UNSUPPORTED = 2, /* valid but unsupported shape/dtype combination */
+    DSA_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+    DSA_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+    DSA_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (device) */
+} dsa_status;
+
+typedef enum { DSA_BF16 = 0, DSA_F32 = 1 } dsa_dtype;
+
+/* Operation ids for dsa_workspace_bytes. */
+typedef enum {
+    DSA_OP_INDEX_SCORES = 0,
+    DSA_OP_TOPK = 1,
+    DSA_OP_MLA_DECODE = 2,
+    DSA_OP_MLA_PREFILL = 3,
+    DSA_OP_INDEXSHARE_GROUP = 4
+} dsa_op;
+
+/*
+ * The query tokens of one call.
+ *   n_q      number of query tokens (>= 0)
+ *   n_seq    number of sequences (caches), >= 1
+ *   max_ctx  L: rows in every cache; each q_pos must be < L
+ *   seq_run  a promise that queries come in runs of `seq_run` consecutive
+ *            queries sharing one sequence (run r = queries r*seq_run ...); 1 makes
+ *            no promise.  The indexer tiles up to gcd(seq_run, 8) queries that
+ *            share a cache into one tensor-core tile.  A broken promise is
+ *            reported as DSA_ERR_INVALID in the status word.
+ *   q_seq    device int32 [n_q]: sequence of each query, in [0, n_seq)
+ *   q_pos    device int32 [n_q]: position t of each query, in [0, L); the query
+ *            sees rows 0..t of its sequence
+ */
+typedef struct {
+    int32_t n_q;
+    int32_t n_seq;
+    int32_t max_ctx;
+    int32_t seq_run;
+    const int32_t *q_seq;
+    const int32_t *q_pos;
+} dsa_queries;
+
+/*
+ * Lightning indexer of one full layer [TM, Indexer-selected sparse attention].
+ *   heads, dim    32 and 128 for GLM-5.2 (any positive values on the generic path)
+ *   dtype         DSA_BF16 or DSA_F32, for q and k
+ *   q             [n_q][heads][dim], contiguous, post-RoPE
+ *   w             float32 [n_q][heads], contiguous
+ *   k             row s of sequence b at k + b*k_seq_stride + s*k_row_stride
+ *                 (strides in elements; k_seq_stride 0 = all sequences share one
+ *                 cache).  Tensor-core path: row and sequence strides multiple of
+ *                 8 elements, k and q 16-byte aligned.
+ */
+typedef struct {
+    int32_t heads;
+    int32_t dim;
+    int32_t dtype;
+    int32_t reserved;
+    const void *q;
+    const float *w;
+    const void *k;
+    int64_t k_seq_stride;
+    int64_t k_row_stride;
+} dsa_indexer;
+
+/*
+ * Absorbed MLA of one layer [TM, Multi-head latent attention; Partial RoPE].
+ *   heads              64 for GLM-5.2
+ *   d_latent, d_rope   512 and 64 for GLM-5.2
+ *   dtype              DSA_BF16 or DSA_F32 for q, kv and out
+ *   scale              softmax scale (1/sqrt(192 + 64) for GLM-5.2)
+ *   q                  [n_q][heads][d_latent + d_rope], contiguous
+ *   kv                 cache row s of sequence b at kv + b*kv_seq_stride +
+ *                      s*kv_row_stride, laid out [c (d_latent) | r (d_rope)];
+ *                      tensor-core path: strides multiple of 8 elements, 16-byte
+ *                      aligned base
+ *   out                [n_q][heads][d_latent], dtype `dtype`
+ *   lse                float32 [n_q][heads] (natural log of the softmax
+ *                      normaliser of the scaled logits), or NULL
+ */
+typedef struct {
+    int32_t heads;
+    int32_t d_latent;
+    int32_t d_rope;
+    int32_t dtype;
+    float scale;
+    int32_t reserved;
+    const void *q;
+    const void *kv;
+    int64_t kv_seq_stride;
+    int64_t kv_row_stride;
+    void *out;
+    float *lse;
+} dsa_mla;
+
+/*
+ * Indexer scores [TM, Indexer-selected sparse attention; QK normalization]:
+ *   scores[i*ld_scores + s] = sum_h w[i,h] * max(0, q[i,h,:] . k[q_seq[i], s, :])
+ * for s <= q_pos[i]; entries s > q_pos[i] are left unspecified.
+ *   scores     float32 [n_q][ld_scores], ld_scores >= max_ctx, multiple of 4,
+ *              16-byte aligned base
+ *   ws         workspace of dsa_workspace_bytes(DSA_OP_INDEX_SCORES, ...) bytes
+ * On integer-valued inputs (see the test recipe) every score is exact in float32.
+ */
+dsa_status dsa_index_scores(const dsa_queries *queries, const dsa_indexer *indexer, float *scores,
+                            int64_t ld_scores, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Causal top-k [TM, Indexer-selected sparse attention: min(index_topk, n)
+ * largest scores, int32 indices]: for query i with n = q_pos[i] + 1 visible
+ * rows keep k = min(topk, n) positions with the largest scores (ties -> lower
+ * position; -0.0 == +0.0), written ascending to idx[i*topk + 0..k-1], the rest
+ * of the row set to -1, cnt[i] = k.  Scores must not be NaN.
+ *   scores     float32 [n_q][ld_scores] (only s <= q_pos[i] is read),
+ *              ld_scores >= max_ctx, multiple of 4, 16-byte aligned base
+ *   topk       1 .. 4096
+ *   idx        int32 [n_q][topk];  cnt  int32 [n_q]
+ */
+dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_scores,
+                    int32_t topk, int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
+                    void *stream);
+
+/*
+ * Sparse absorbed MLA, decode schedule [TM, Indexer-selected sparse attention;
+ * Multi-head latent attention; Learnable attention sink]: for each query i and
+ * head h, attention over the rows idx[i*topk + 0..cnt[i]-1] of its sequence:
+ *   l_j = scale * (q_lat[i,h] . c_{s_j} + q_rope[i,h] . r_{s_j}),
+ *   out[i,h,:] = sum_j softmax(l)_j c_{s_j},  lse[i,h] = log sum_j exp(l_j).
+ * The selected rows are split over several CTAs per query (split-K over rows,
+ * partial results in the workspace, then a log-sum-exp merge): the schedule for
+ * few queries.  Entries of idx must lie in [0, max_ctx).
+ */
+dsa_status dsa_sparse_mla_decode(const dsa_queries *queries, const dsa_mla *mla,
+                                 const int32_t *idx, const int32_t *cnt, int32_t topk, void *ws,
+                                 size_t ws_bytes, void *stream);
+
+/*
+ * Same result as dsa_sparse_mla_decode, prefill schedule: one CTA per query
+ * walks all of its selected rows with an online softmax (no partials), the
+ * schedule for many queries.
+ */
+dsa_status dsa_sparse_mla_prefill(const dsa_queries *queries, const dsa_mla *mla,
+                                  const int32_t *idx, const int32_t *cnt, int32_t topk, void *ws,
+                                  size_t ws_bytes, void *stream);
+
+/*
+ * IndexShare group [HA, MLA + DSA with IndexShare]: layer 0 (the full layer)
+ * runs dsa_index_scores -> dsa_topk -> sparse MLA; layers 1..n_layers-1 run
+ * sparse MLA with layer 0's idx/cnt on their own queries and caches, without
+ * re-scoring.  The scores live in the workspace.
+ *   indexer   the full layer's indexer
+ *   layers    host array of n_layers (1..4) dsa_mla descriptions (same heads,
+ *             dims, dtype and scale)
+ *   idx, cnt  outputs as in dsa_topk
+ * The decode or prefill MLA schedule is chosen from n_q.
+ */
+dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *indexer,
+                                const dsa_mla *layers, int32_t n_layers, int32_t topk,
+                                int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
+                                void *stream);
+
+/*
+ * Upper bound of the workspace bytes an operation needs (host only).
+ *   op         a dsa_op value
+ *   queries    n_q and max_ctx are read (pointers are not)
+ *   topk       selection size (ignored for DSA_OP_INDEX_SCORES)
+ *   mla_heads, d_latent, n_layers   MLA shape (ignored where no MLA runs)
+ * Returns 0 for an unknown op.
+ */
+size_t dsa_workspace_bytes(int32_t op, const dsa_queries *queries, int32_t topk, int32_t mla_heads,
+                           int32_t d_latent, int32_t n_layers);
+
+/* Zero the status word of a workspace (async on `stream`). */
+dsa_status dsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronise `stream`, read the workspace status word, clear it, and return
+ * it (DSA_OK when no kernel reported an error).  The one synchronising call.
+ */
+dsa_status dsa_check_status(void *ws, void *stream);
+
+/* Human-readable name of a status code (static string). */
+const char *dsa_status_str(dsa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,149 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point include/dsa.h declares, rejects bad arguments synchronously
+before any launch, and sizes workspaces as documented."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from dsa_indexer_top_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    syms = set()
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        if name.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", name)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            syms |= set(re.findall(r"\b(dsa_[a-z0-9_]+)\s*\(", text))
+    return syms
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.lib()
+    syms = declared_symbols()
+    assert {"dsa_index_scores", "dsa_topk", "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill",
+            "dsa_indexshare_group", "dsa_workspace_bytes"} <= syms
+    for s in sorted(syms):
+        assert hasattr(lib, s), f"{s} not exported"
+
+
+def test_status_strings():
+    assert B.status_str(B.DSA_OK) == "DSA_OK"
+    assert B.status_str(B.DSA_ERR_TIMEOUT) == "DSA_ERR_TIMEOUT"
+    assert B.status_str(99) == "DSA_ERR_UNKNOWN"
+
+
+def _q(n_q=4, n_seq=4, L=1000, seq_run=1):
+    return B._Queries(n_q, n_seq, L, seq_run, 0x1000, 0x2000)
+
+
+def test_workspace_bytes():
+    lib = B.lib()
+    q = _q(n_q=8, L=32768)
+    assert lib.dsa_workspace_bytes(B.DSA_OP_INDEX_SCORES, ctypes.byref(q), 2048, 64, 512, 1) == 256
+    assert lib.dsa_workspace_bytes(B.DSA_OP_TOPK, ctypes.byref(q), 2048, 64, 512, 1) == 256
+    dec = lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 2048, 64, 512, 1)
+    # 16 splits x 8 queries x 64 heads x (512 + 2) floats, 256-aligned, + status
+    assert dec == 256 + ((8 * 16 * 64 * 514 * 4 + 255) // 256) * 256
+    assert lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 128, 64, 512, 1) == 256
+    grp = lib.dsa_workspace_bytes(B.DSA_OP_INDEXSHARE_GROUP, ctypes.byref(q), 2048, 64, 512, 4)
+    scores = 8 * 32768 * 4
+    assert grp == 256 + scores + ((4 * 8 * 16 * 64 * 514 * 4 + 255) // 256) * 256
+    assert lib.dsa_workspace_bytes(77, ctypes.byref(q), 2048, 64, 512, 1) == 0
+
+
+class _FakeWs:
+    """An aligned host address standing in for a workspace: validation runs
+    before any use of it, so nothing dereferences it."""
+    ptr = 0x10000
+    size = 1 << 30
+
+
+def _idx(heads=32, dim=128, dtype=0, q=0x3000, w=0x4000, k=0x5000, kss=1000 * 128, krs=128):
+    return B._Indexer(heads, dim, dtype, 0, q, w, k, kss, krs)
+
+
+def _mla(heads=64, dl=512, dr=64, dtype=0, q=0x6000, kv=0x7000, out=0x8000, kss=1000 * 576, krs=576):
+    return B._Mla(heads, dl, dr, dtype, 0.0625, 0, q, kv, kss, krs, out, None)
+
+
+@pytest.mark.parametrize("case", [
+    "null_queries", "neg_nq", "zero_ctx", "bad_seq_run", "null_pos", "bad_dim", "bad_dtype", "row_stride",
+    "seq_stride", "ld_small", "ld_unaligned", "scores_null"])
+def test_index_scores_rejects(case):
+    lib = B.lib()
+    q = _q()
+    ix = _idx()
+    ld = 1000
+    scores = 0x9000
+    if case == "neg_nq": q.n_q = -1
+    if case == "zero_ctx": q.max_ctx = 0
+    if case == "bad_seq_run": q.seq_run = 0
+    if case == "null_pos": q.q_pos = None
+    if case == "bad_dim": ix.dim = 0
+    if case == "bad_dtype": ix.dtype = 5
+    if case == "row_stride": ix.k_row_stride = 64
+    if case == "seq_stride": ix.k_seq_stride = 999 * 128
+    if case == "ld_small": ld = 996
+    if case == "ld_unaligned": ld = 1002
+    if case == "scores_null": scores = 0
+    qp = None if case == "null_queries" else ctypes.byref(q)
+    st = lib.dsa_index_scores(qp, ctypes.byref(ix), scores, ld, _FakeWs.ptr, _FakeWs.size, None)
+    assert st == B.DSA_ERR_INVALID
+
+
+def test_workspace_checks():
+    lib = B.lib()
+    q, ix = _q(), _idx()
+    assert lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(ix), 0x9000, 1000, 0, 1 << 20, None) == B.DSA_ERR_WORKSPACE
+    assert lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(ix), 0x9000, 1000, 0x10010, 1 << 20, None) == B.DSA_ERR_WORKSPACE
+    assert lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(ix), 0x9000, 1000, 0x10000, 128, None) == B.DSA_ERR_WORKSPACE
+    m = _mla()
+    need = lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 2048, 64, 512, 1)
+    assert lib.dsa_sparse_mla_decode(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, 0x10000, need - 1,
+                                     None) == B.DSA_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("topk", [0, -3, 4097])
+def test_topk_rejects_bad_k(topk):
+    lib = B.lib()
+    q = _q()
+    assert lib.dsa_topk(ctypes.byref(q), 0x9000, 1000, topk, 0xA000, 0xB000, _FakeWs.ptr, _FakeWs.size,
+                        None) == B.DSA_ERR_INVALID
+
+
+def test_mla_rejects():
+    lib = B.lib()
+    q = _q()
+    for kw in [dict(q=0), dict(kv=0), dict(out=0), dict(heads=0), dict(dtype=3), dict(krs=500),
+               dict(dl=0)]:
+        m = _mla(**kw)
+        st = lib.dsa_sparse_mla_prefill(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, _FakeWs.ptr,
+                                        _FakeWs.size, None)
+        assert st == B.DSA_ERR_INVALID, kw
+    m = _mla()
+    assert lib.dsa_sparse_mla_prefill(ctypes.byref(q), ctypes.byref(m), 0, 0xB000, 2048, _FakeWs.ptr,
+                                      _FakeWs.size, None) == B.DSA_ERR_INVALID
+
+
+def test_group_rejects_layer_mismatch_and_count():
+    lib = B.lib()
+    q, ix = _q(), _idx()
+    arr = (B._Mla * 2)(_mla(), _mla(dl=256, krs=576))
+    assert lib.dsa_indexshare_group(ctypes.byref(q), ctypes.byref(ix), arr, 2, 2048, 0xA000, 0xB000, _FakeWs.ptr,
+                                    _FakeWs.size, None) == B.DSA_ERR_INVALID
+    arr5 = (B._Mla * 5)(*[_mla() for _ in range(5)])
+    assert lib.dsa_indexshare_group(ctypes.byref(q), ctypes.byref(ix), arr5, 5, 2048, 0xA000, 0xB000, _FakeWs.ptr,
+                                    _FakeWs.size, None) == B.DSA_ERR_INVALID
+
+
+def test_zero_queries_is_a_noop():
+    lib = B.lib()
+    q = _q(n_q=0)
+    assert lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(_idx()), 0x9000, 1000, _FakeWs.ptr, _FakeWs.size,
+                                None) == B.DSA_OK

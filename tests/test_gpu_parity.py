@@ -1,0 +1,164 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle on
+the same seeded inputs.  Indices are compared bit for bit (the input recipe
+makes every score exact in float32); attention outputs within max-abs 2e-2 and
+mean-abs 2e-3 on bf16 outputs (tighter on the fp32 path)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from dsa_indexer_top_b200 import binding as B
+from dsa_indexer_top_b200 import workloads as wl
+from tests import common as C
+
+pytestmark = pytest.mark.gpu
+
+D32 = wl.NAMED["decode_32k"]
+
+SMALL = {
+    "tiny": wl.NAMED["tiny"],
+    # n > topk, n < topk, n == topk, n == topk + 1 in one batch
+    "decode_edges": wl.scaled(D32, n_seq=4, L=3000, q_pos=(2999, 1500, 2047, 2048), q_seq=(0, 1, 2, 3)),
+    # context not a multiple of the 128-key tile, queries on a ragged tail
+    "decode_ragged": wl.scaled(D32, n_seq=2, L=5037, q_pos=(5036, 4100), q_seq=(0, 1), seed=7),
+    # several queries of one sequence share a tensor-core tile (seq_run = 40 -> 8 per tile)
+    "prefill_small": wl.scaled(D32, n_seq=1, L=4173, q_pos=tuple(range(3000, 3040)), q_seq=(0,) * 40, seed=8),
+    # causal start: positions 0..63 (every query keeps all visible rows)
+    "prefill_start": wl.scaled(D32, n_seq=1, L=4096, q_pos=tuple(range(64)), q_seq=(0,) * 64, seed=9),
+    # every sequence reads one shared cache (sequence stride 0)
+    "shared_cache": wl.scaled(D32, n_seq=3, L=2600, q_pos=(2599, 2400, 2100), q_seq=(0, 1, 2),
+                              shared_cache=True, seed=10),
+    # heavy ties: indexer values in {-1, 0, 1}
+    "ties": wl.scaled(D32, n_seq=2, L=6000, q_pos=(5999, 4444), q_seq=(0, 1), int_range=1, seed=11),
+    # IndexShare group of 4 layers
+    "indexshare_small": wl.scaled(D32, n_seq=2, L=3000, q_pos=(2999, 2500), q_seq=(0, 1), n_layers=4, seed=12),
+}
+
+
+def seq_run_of(w):
+    runs = [w.n_q] if len(set(w.q_seq)) == 1 else [1]
+    return runs[0]
+
+
+@pytest.fixture(scope="module")
+def dev(cuda_ok):
+    B.lib()
+    return torch.device("cuda")
+
+
+def _run_steps(w, x, decode=True):
+    """The three-call chain (as timed by the benchmark): scores -> top-k -> MLA."""
+    q, ix, mlas = C.descriptors(w, x, seq_run=seq_run_of(w))
+    dev = x["q_pos"].device
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, w.n_layers, dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    B.dsa_index_scores(q, ix, scores, ws)
+    idx = torch.full((w.n_q, w.topk), -7, dtype=torch.int32, device=dev)
+    cnt = torch.full((w.n_q,), -7, dtype=torch.int32, device=dev)
+    B.dsa_topk(q, scores, w.topk, idx, cnt, ws)
+    for m in mlas:
+        (B.dsa_sparse_mla_decode if decode else B.dsa_sparse_mla_prefill)(q, m, idx, cnt, w.topk, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    return scores, idx, cnt, mlas
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_index_scores_bit_exact(dev, name):
+    w = SMALL[name]
+    xh = wl.make_inputs(w, layers=[])
+    x = C.to_device(xh)
+    q, ix, _ = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ws = B.workspace(B.DSA_OP_INDEX_SCORES, q, device=dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    scores.fill_(float("nan"))
+    B.dsa_index_scores(q, ix, scores, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    ref, _, _ = C.oracle_selection(w, xh)
+    got = scores[:, : w.L].cpu().double().numpy()
+    for i, t in enumerate(w.q_pos):
+        np.testing.assert_array_equal(got[i, : t + 1], ref[i, : t + 1], err_msg=f"query {i}")
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+@pytest.mark.parametrize("decode", [True, False])
+def test_chain_matches_oracle(dev, name, decode):
+    w = SMALL[name]
+    xh = wl.make_inputs(w)
+    x = C.to_device(xh)
+    _, idx, cnt, mlas = _run_steps(w, x, decode=decode)
+    _, ridx, rcnt = C.oracle_selection(w, xh)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+    for layer, m in enumerate(mlas):
+        out, lse = C.oracle_mla(w, xh, layer, ridx, rcnt)
+        C.assert_attention_close(m.out, out, w.dtype, f"layer {layer} out")
+        C.assert_lse_close(m.lse, lse, w.dtype)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode_edges", "indexshare_small", "prefill_small", "shared_cache"])
+def test_indexshare_group_call(dev, name):
+    w = SMALL[name]
+    xh = wl.make_inputs(w)
+    x = C.to_device(xh)
+    q, ix, mlas = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, w.n_layers, dev)
+    idx = torch.empty((w.n_q, w.topk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.n_q,), dtype=torch.int32, device=dev)
+    B.dsa_indexshare_group(q, ix, mlas, w.topk, idx, cnt, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    ridx, rcnt, outs, lses = oracle.indexshare_group(
+        C.host_f32(xh["q_idx"]), C.host_f32(xh["w"]), C.host_f32(xh["k_idx"]),
+        np.zeros(w.n_q, np.int32) if w.shared_cache else xh["q_seq"].numpy(), xh["q_pos"].numpy(), w.topk,
+        [C.host_f32(t) for t in xh["q_mla"]], [C.host_f32(t) for t in xh["kv"]], w.d_lat, w.scale)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    for layer, m in enumerate(mlas):
+        C.assert_attention_close(m.out, outs[layer], w.dtype, f"layer {layer}")
+        C.assert_lse_close(m.lse, lses[layer], w.dtype)
+
+
+@pytest.mark.parametrize("mode", ["ties", "normal", "equal"])
+@pytest.mark.parametrize("L,topk", [(300, 64), (5000, 2048), (70000, 2048), (200000, 512), (700001, 2048)])
+def test_topk_alone(dev, mode, L, topk):
+    n_q = 5
+    s = wl.random_scores(n_q, L, seed=L + topk, mode=mode)
+    q_pos = torch.tensor([L - 1, L // 2, min(topk, L) - 1, min(topk, L - 1), 0], dtype=torch.int32)
+    q = B.Queries(torch.zeros(n_q, dtype=torch.int32, device=dev), q_pos.to(dev), n_seq=1, max_ctx=L)
+    scores = B.scores_buffer(n_q, L, dev)
+    scores[:, :L] = s.to(dev)
+    ws = B.workspace(B.DSA_OP_TOPK, q, topk, device=dev)
+    idx = torch.full((n_q, topk), -7, dtype=torch.int32, device=dev)
+    cnt = torch.full((n_q,), -7, dtype=torch.int32, device=dev)
+    B.dsa_topk(q, scores, topk, idx, cnt, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    ridx, rcnt = oracle.topk(s.double().numpy(), q_pos.numpy(), topk)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
+@pytest.mark.parametrize("decode", [True, False])
+@pytest.mark.parametrize("topk,L", [(2048, 3000), (300, 1000), (100, 500), (4096, 5000)])
+def test_sparse_mla_alone(dev, decode, topk, L):
+    w = wl.scaled(D32, n_seq=3, L=L, q_pos=(L - 1, L // 3, 5), q_seq=(2, 0, 1), topk=topk, seed=topk)
+    xh = wl.make_inputs(w)
+    x = C.to_device(xh)
+    q, _, mlas = C.descriptors(w, x)
+    idx, cnt = C.random_selection(w, seed=L)
+    ws = B.workspace(B.DSA_OP_MLA_DECODE, q, topk, device=dev)
+    (B.dsa_sparse_mla_decode if decode else B.dsa_sparse_mla_prefill)(q, mlas[0], idx.to(dev), cnt.to(dev), topk, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    out, lse = C.oracle_mla(w, xh, 0, idx.numpy(), cnt.numpy())
+    C.assert_attention_close(mlas[0].out, out, "bf16")
+    C.assert_lse_close(mlas[0].lse, lse, "bf16")
+
+
+def test_device_detects_bad_positions(dev):
+    w = wl.scaled(D32, n_seq=2, L=1000, q_pos=(999, 500), q_seq=(0, 1))
+    x = C.to_device(wl.make_inputs(w, layers=[]))
+    x["q_pos"][1] = 5000  # beyond the cache
+    q, ix, _ = C.descriptors(w, x)
+    ws = B.workspace(B.DSA_OP_INDEX_SCORES, q, device=dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    B.dsa_index_scores(q, ix, scores, ws)
+    assert B.dsa_check_status(ws) == B.DSA_ERR_INVALID
+    assert B.dsa_check_status(ws) == B.DSA_OK      # reading clears it
