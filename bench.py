@@ -161,7 +161,7 @@ class Step:
         self.cnt = torch.empty((w.n_q,), dtype=torch.int32, device=dev)
         self.decode = w.n_q <= DECODE_MAX_QUERIES
         self.mla_fn = B.dsa_sparse_mla_decode if self.decode else B.dsa_sparse_mla_prefill
-        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
         self.graph = None
 
     def launches_per_step(self) -> int:
@@ -214,7 +214,7 @@ class E2EStep:
         self.h_idx = torch.empty(step.idx.shape, dtype=torch.int32).pin_memory()
         self.h2d = sum(t.numel() * t.element_size() for t in list(self.h_in.values()) + self.h_qmla)
         self.d2h = sum(t.numel() * t.element_size() for t in self.h_out) + self.h_idx.numel() * 4
-        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
         self.graph = None
 
     def run(self):
@@ -346,8 +346,13 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--n-seq", type=int, default=0,
+                    help="decode workloads: override the batch (a smaller case for profiling; not a bench line)")
     args = ap.parse_args()
     w = wl.NAMED[args.workload]
+    if args.n_seq and len(set(w.q_seq)) == w.n_q:
+        w = wl.scaled(w, n_seq=args.n_seq, q_pos=w.q_pos[:1] * args.n_seq, q_seq=tuple(range(args.n_seq)),
+                      name=f"{w.name}_b{args.n_seq}")
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))

@@ -12,7 +12,6 @@ using namespace dsa;
 namespace {
 
 constexpr size_t kStatusBytes = 256;
-constexpr int kTopkCacheCap = 40960;  // elements of a top-k chunk kept in shared memory
 constexpr int kDecodeMaxQueries = 256;  // IndexShare group: split-K MLA up to this many queries
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -76,7 +75,7 @@ bool mla_tc_ok(const dsa_mla *m) {
 }
 
 size_t ws_index_scores() { return kStatusBytes; }
-size_t ws_topk() { return kStatusBytes; }
+size_t ws_topk(int n_q, int max_ctx) { return kStatusBytes + align256(topk_scratch_bytes(n_q, max_ctx)); }
 int decode_splits(int topk) { return (topk + kRowsPerChunk - 1) / kRowsPerChunk; }
 size_t ws_mla_decode(int n_q, int topk, int n_layers) {
     const int ns = decode_splits(topk);
@@ -87,7 +86,7 @@ size_t ws_scores(int n_q, int max_ctx) {
 }
 bool group_uses_decode(int n_q) { return n_q <= kDecodeMaxQueries; }
 size_t ws_group(int n_q, int max_ctx, int topk, int n_layers) {
-    size_t b = kStatusBytes + ws_scores(n_q, max_ctx);
+    size_t b = kStatusBytes + ws_scores(n_q, max_ctx) + align256(topk_scratch_bytes(n_q, max_ctx));
     if (group_uses_decode(n_q)) b += ws_mla_decode(n_q, topk, n_layers) - kStatusBytes;
     return b;
 }
@@ -175,7 +174,7 @@ dsa_status check_indexer(const dsa_queries *qs, const dsa_indexer *ix) {
 
 // ------------------------------------------------------------------ top-k
 dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int topk, int32_t *idx,
-                   int32_t *cnt, uint32_t *status, cudaStream_t st) {
+                   int32_t *cnt, uint32_t *status, void *scratch, cudaStream_t st) {
     TopkArgs a;
     a.scores = scores;
     a.ld = ld;
@@ -186,7 +185,10 @@ dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int t
     a.n_q = qs->n_q;
     a.L = qs->max_ctx;
     a.topk = topk;
-    a.cache_cap = kTopkCacheCap;
+    a.ghist = nullptr;
+    a.gcount = nullptr;
+    a.gcand = nullptr;
+    if (topk_uses_split(qs->n_q, qs->max_ctx)) topk_bind_scratch(a, scratch);
     return launch_topk(a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -285,7 +287,7 @@ size_t dsa_workspace_bytes(int32_t op, const dsa_queries *qs, int32_t topk, int3
     const int n_q = qs->n_q > 0 ? qs->n_q : 0;
     switch (op) {
         case DSA_OP_INDEX_SCORES: return ws_index_scores();
-        case DSA_OP_TOPK: return ws_topk();
+        case DSA_OP_TOPK: return ws_topk(n_q, qs->max_ctx > 0 ? qs->max_ctx : 1);
         case DSA_OP_MLA_DECODE: return ws_mla_decode(n_q, topk > 0 ? topk : 1, 1);
         case DSA_OP_MLA_PREFILL: return kStatusBytes;
         case DSA_OP_INDEXSHARE_GROUP:
@@ -325,11 +327,12 @@ dsa_status dsa_index_scores(const dsa_queries *queries, const dsa_indexer *index
 dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_scores, int32_t topk, int32_t *idx,
                     int32_t *cnt, void *ws, size_t ws_bytes, void *stream) {
     if (!valid_queries(queries)) return DSA_ERR_INVALID;
-    if (!ws_ok(ws, ws_bytes, ws_topk())) return DSA_ERR_WORKSPACE;
+    if (!ws_ok(ws, ws_bytes, ws_topk(queries->n_q, queries->max_ctx))) return DSA_ERR_WORKSPACE;
     if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
     if (!scores_ok(scores, ld_scores, queries->max_ctx)) return DSA_ERR_INVALID;
     if (queries->n_q == 0) return DSA_OK;
-    return do_topk(queries, scores, ld_scores, topk, idx, cnt, status_word(ws), static_cast<cudaStream_t>(stream));
+    return do_topk(queries, scores, ld_scores, topk, idx, cnt, status_word(ws), static_cast<uint8_t *>(ws) + kStatusBytes,
+                   static_cast<cudaStream_t>(stream));
 }
 
 static dsa_status mla_entry(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx, const int32_t *cnt,
@@ -370,10 +373,11 @@ dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *i
     uint8_t *base = static_cast<uint8_t *>(ws);
     float *scores = reinterpret_cast<float *>(base + kStatusBytes);
     const int64_t ld = round4(queries->max_ctx);
-    uint8_t *scratch = base + kStatusBytes + ws_scores(queries->n_q, queries->max_ctx);
+    uint8_t *topk_scratch = base + kStatusBytes + ws_scores(queries->n_q, queries->max_ctx);
+    uint8_t *scratch = topk_scratch + align256(topk_scratch_bytes(queries->n_q, queries->max_ctx));
     s = do_index_scores(queries, indexer, scores, ld, status_word(ws), st);
     if (s != DSA_OK) return s;
-    s = do_topk(queries, scores, ld, topk, idx, cnt, status_word(ws), st);
+    s = do_topk(queries, scores, ld, topk, idx, cnt, status_word(ws), topk_scratch, st);
     if (s != DSA_OK) return s;
     return do_mla(queries, layers, n_layers, idx, cnt, topk, group_uses_decode(queries->n_q), scratch,
                   status_word(ws), st);

@@ -55,6 +55,11 @@ struct IdxGenericArgs {
 cudaError_t launch_idx_score_generic(const IdxGenericArgs &a, cudaStream_t st);
 
 // ------------------------------------------------------------------ top-k
+constexpr int kTopkRowMaxCtx = 65536;      // contexts up to this use one CTA per query
+constexpr int kTopkSplitMaxQueries = 64;   // longer contexts with at most this many queries split rows
+constexpr int kSplitMax = 64;              // chunks per query (split schedule)
+constexpr int kSplitCap = 1024;            // candidates stored per chunk
+
 struct TopkArgs {
     const float *scores;
     int64_t ld;
@@ -63,8 +68,14 @@ struct TopkArgs {
     int32_t *cnt;
     uint32_t *status;
     int n_q, L, topk;
-    int cache_cap;  // elements of a CTA's chunk kept in shared memory
+    // split-schedule scratch (workspace)
+    uint32_t *ghist;   // [n_q][4096] first-digit histogram
+    uint32_t *gcount;  // [n_q][kSplitMax] candidates per chunk
+    uint2 *gcand;      // [n_q][kSplitMax][kSplitCap] (key, position)
 };
+bool topk_uses_split(int n_q, int max_ctx);
+size_t topk_scratch_bytes(int n_q, int max_ctx);
+void topk_bind_scratch(TopkArgs &a, void *scratch);
 cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st);
 
 // ------------------------------------------------------------------ sparse MLA

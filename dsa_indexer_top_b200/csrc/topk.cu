@@ -5,273 +5,481 @@
 // order and padded with -1 ("GLM-5.2 -- Model techniques map", "Checked in its
 // code", Indexer-selected sparse attention: min(index_topk, n) largest, int32).
 //
-// One thread-block cluster (1..16 CTAs) per query; CTA r owns a contiguous chunk
-// of positions.  No sort: a most-significant-digit radix select over the
-// order-preserving 32-bit image of the float scores, three digits (11, 11, 10
-// bits).  Each pass builds a shared-memory histogram of the next digit among the
-// rows that still match the threshold prefix (warp-aggregated atomics), the
-// cluster's histograms are summed through distributed shared memory, and the
-// digit holding the k-th largest key is found with a block-wide suffix scan.
-// After three passes the threshold key T is exact and `need_eq` rows equal to T
-// must be taken.  An ordered compaction follows: per-CTA counts of rows > T and
-// == T are exchanged through distributed shared memory, and each CTA writes its
-// kept positions at the right slots (rows == T kept first-come in position
-// order, which is the lower-position tie rule).  All cross-CTA synchronisation is
-// the hardware cluster barrier; nothing spins.  A CTA keeps its chunk of keys in
-// shared memory when it fits, else re-reads the scores (L2) every pass.
-#include <cooperative_groups.h>
+// No sort.  Scores are mapped to order-preserving 32-bit keys and the k-th
+// largest key T is found by a most-significant-digit radix select with digits of
+// 12, 12 and 8 bits.  Only the first digit is taken over the whole row: every
+// row whose first digit is >= the threshold digit is copied, in position order,
+// into a candidate list (a few thousand rows), and the last two digits are
+// resolved on that list in shared memory.  The output is an ordered filter of the
+// candidates: keys > T, then the first `need_eq` keys == T in position order (the
+// lower-position tie rule), written at their exclusive-scan slots.  When ties
+// make the candidate list too long the same digits are resolved by streaming the
+// row again (correct for any input, slower).
+//
+// Two schedules:
+//   row    one CTA per query (contexts up to 64K): histogram pass, candidate
+//          pass (L2-hot), refine + write -- a single launch.
+//   split  long contexts with few queries: P CTAs per query build a global
+//          first-digit histogram (atomics), then collect their chunk's
+//          candidates into the workspace, then one CTA per query merges the
+//          chunks (in position order) and finishes as above.
+#include <cstdint>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
 
-namespace cg = cooperative_groups;
-
 namespace dsa {
 namespace {
 
-constexpr int kTkThreads = 512;
-constexpr int kTkWarps = kTkThreads / 32;
-constexpr int kBins = 2048;
-constexpr int kPerThread = 8;  // consecutive rows per thread in the ordered write
+constexpr int kT = 512;                // threads per CTA
+constexpr int kWarps = kT / 32;
+constexpr int kBins = 4096;            // first and second digit (12 bits)
+constexpr int kBins3 = 256;            // third digit (8 bits)
+constexpr int kCap = 10240;            // candidates kept in shared memory
+constexpr int kV = 4;                  // consecutive rows per thread per tile
 
-// Order-preserving map float -> uint32 (larger float -> larger key); -0.0 is
-// folded onto +0.0 so the two compare equal.
+struct TopkSmem {
+    uint32_t hist[kBins];
+    uint32_t cand_key[kCap];
+    int32_t cand_pos[kCap];
+    uint64_t scan[kWarps];
+    uint32_t sel[4];
+};
+
 __device__ __forceinline__ uint32_t order_key(float f) {
     uint32_t b = __float_as_uint(f);
-    if (b == 0x80000000u) b = 0u;
+    if (b == 0x80000000u) b = 0u;  // -0.0 == +0.0
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Exclusive block-wide scan of a 64-bit value (two packed 32-bit counters);
-// also returns the block total.  Every thread of the block must call it.
-__device__ __forceinline__ uint64_t block_excl_scan(uint64_t v, uint64_t *buf, uint64_t &total) {
+// Exclusive block-wide scan (64-bit); returns the block total in `total`.
+__device__ __forceinline__ uint64_t block_scan(uint64_t v, uint64_t *buf, uint64_t &total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     uint64_t x = v;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
     }
     if (lane == 31) buf[warp] = x;
     __syncthreads();
     if (warp == 0) {
-        uint64_t t = lane < kTkWarps ? buf[lane] : 0;
+        uint64_t t = lane < kWarps ? buf[lane] : 0;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            uint64_t y = __shfl_up_sync(0xffffffffu, t, o);
+            const uint64_t y = __shfl_up_sync(0xffffffffu, t, o);
             if (lane >= o) t += y;
         }
-        if (lane < kTkWarps) buf[lane] = t;
+        if (lane < kWarps) buf[lane] = t;
     }
     __syncthreads();
     const uint64_t before = warp == 0 ? 0 : buf[warp - 1];
-    total = buf[kTkWarps - 1];
+    total = buf[kWarps - 1];
     __syncthreads();
     return before + x - v;
 }
 
-__global__ void __launch_bounds__(kTkThreads, 1) topk_cluster_kernel(const TopkArgs a) {
-    cg::cluster_group cluster = cg::this_cluster();
-    const int C = static_cast<int>(cluster.num_blocks());
-    const int rank = static_cast<int>(cluster.block_rank());
-    const int i = blockIdx.x / C;
-    const int tid = threadIdx.x, lane = tid & 31;
+// Add one to hist[d] for every lane with d != ~0u (warp-aggregated).
+__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t d) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+    if (d != 0xFFFFFFFFu && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+}
 
-    __shared__ uint32_t hist[2][kBins];
-    __shared__ uint64_t scan_buf[32];
-    __shared__ uint32_t sel_digit, sel_above;
-    __shared__ uint32_t cta_counts[2];  // rows > T, rows == T in this CTA's chunk
-    __shared__ int32_t cta_plan[2];     // first output slot, quota of rows == T
-    extern __shared__ uint32_t cache[];
+__device__ __forceinline__ void zero_hist(uint32_t *hist, int nbins) {
+    for (int b = threadIdx.x; b < nbins; b += kT) hist[b] = 0;
+}
 
-    int pos = a.q_pos[i];
-    if (pos < 0 || pos >= a.L) {
-        if (rank == 0 && tid == 0) report_status(a.status, DSA_ERR_INVALID);
-        pos = -1;
-    }
-    const int n = pos + 1;
-    int32_t *out = a.idx + static_cast<int64_t>(i) * a.topk;
-    if (n <= a.topk) {
-        // every visible row is kept (every CTA of the cluster takes this branch)
-        for (int p = rank * kTkThreads + tid; p < a.topk; p += C * kTkThreads) out[p] = p < n ? p : -1;
-        if (rank == 0 && tid == 0) a.cnt[i] = n;
-        return;
-    }
-    const int k = a.topk;
-    const int chunk = (((n + C - 1) / C) + 3) & ~3;
-    const int lo = min(n, rank * chunk);
-    const int hi = min(n, lo + chunk);
-    const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
-    const bool cached = chunk <= a.cache_cap;
-    if (cached) {
-        for (int e = lo + tid * 4; e < hi; e += kTkThreads * 4) {
-            if (e + 3 < hi) {
-                const float4 v = __ldg(reinterpret_cast<const float4 *>(row + e));
-                cache[e - lo] = order_key(v.x);
-                cache[e - lo + 1] = order_key(v.y);
-                cache[e - lo + 2] = order_key(v.z);
-                cache[e - lo + 3] = order_key(v.w);
-            } else {
-                for (int x = e; x < hi; ++x) cache[x - lo] = order_key(__ldg(row + x));
-            }
+// The digit holding the r-th largest key: sel[0] = digit, sel[1] = rows in
+// higher bins.  Requires sum(hist) >= r >= 1.
+__device__ __forceinline__ void find_digit(const uint32_t *hist, int nbins, uint32_t r, uint64_t *scan,
+                                           uint32_t *sel) {
+    const int per = nbins / kT > 0 ? nbins / kT : 1;
+    const int b0 = threadIdx.x * per;
+    uint32_t mine = 0;
+    for (int j = 0; j < per; ++j)
+        if (b0 + j < nbins) mine += hist[b0 + j];
+    uint64_t all;
+    const uint64_t before = block_scan(mine, scan, all);
+    uint32_t above = static_cast<uint32_t>(all - before - mine);
+    for (int j = per - 1; j >= 0; --j) {
+        if (b0 + j >= nbins) continue;
+        const uint32_t upto = above + hist[b0 + j];
+        if (upto >= r && above < r) {
+            sel[0] = b0 + j;
+            sel[1] = above;
         }
-        __syncthreads();
+        above = upto;
     }
+    __syncthreads();
+}
 
-    uint32_t prefix = 0, pmask = 0;
-    int remaining = k;
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
-        const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
-        uint32_t *h = hist[pass & 1];
-        for (int b = tid; b < kBins; b += kTkThreads) h[b] = 0;
-        __syncthreads();
-        for (int base = lo; base < hi; base += kTkThreads) {
-            const int e = base + tid;
-            uint32_t d = 0xFFFFFFFFu;
-            if (e < hi) {
-                const uint32_t u = cached ? cache[e - lo] : order_key(__ldg(row + e));
-                if ((u & pmask) == prefix) d = (u >> shift) & dmask;
-            }
-            const uint32_t peers = __match_any_sync(0xffffffffu, d);
-            if (d != 0xFFFFFFFFu && lane == __ffs(peers) - 1) atomicAdd(&h[d], __popc(peers));
-        }
-        cluster.sync();  // every CTA's histogram of this pass is complete
-        uint32_t tot[4];
-        uint32_t mine = 0;
+// Histogram of digit (u >> shift) & dmask over rows [lo, hi) of a score row
+// whose key matches `prefix` under `pmask`.
+__device__ __forceinline__ void stream_hist(const float *row, int lo, int hi, uint32_t prefix, uint32_t pmask,
+                                            int shift, uint32_t dmask, uint32_t *hist) {
+    for (int base = lo; base < hi; base += kT * kV) {
+        const int e0 = base + threadIdx.x * kV;
+        float v[kV];
+        if (e0 + kV <= hi) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(row + e0));
+            v[0] = f.x, v[1] = f.y, v[2] = f.z, v[3] = f.w;
+        } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            uint32_t t = 0;
-            for (int r = 0; r < C; ++r) t += cluster.map_shared_rank(h, r)[tid * 4 + j];
-            tot[j] = t;
-            mine += t;
+            for (int x = 0; x < kV; ++x) v[x] = e0 + x < hi ? __ldg(row + e0 + x) : 0.f;
         }
-        uint64_t all;
-        const uint64_t before = block_excl_scan(mine, scan_buf, all);
-        // rows in bins above this thread's four bins
-        uint32_t above = static_cast<uint32_t>(all - before - mine);
 #pragma unroll
-        for (int j = 3; j >= 0; --j) {
-            const uint32_t upto = above + tot[j];  // rows in bins >= tid*4 + j
-            if (upto >= static_cast<uint32_t>(remaining) && above < static_cast<uint32_t>(remaining)) {
-                sel_digit = tid * 4 + j;
-                sel_above = above;
-            }
-            above = upto;
+        for (int x = 0; x < kV; ++x) {
+            const uint32_t u = order_key(v[x]);
+            const bool in = e0 + x < hi && (u & pmask) == prefix;
+            hist_add(hist, in ? (u >> shift) & dmask : 0xFFFFFFFFu);
         }
-        __syncthreads();
-        remaining -= static_cast<int>(sel_above);
-        prefix |= sel_digit << shift;
-        pmask |= dmask << shift;
-        __syncthreads();  // sel_digit / sel_above are rewritten next pass
     }
-    const uint32_t T = prefix;
-    const int need_eq = remaining;  // rows equal to T that are kept (>= 1)
+    __syncthreads();
+}
 
-    // ----------------------------------------------------------- ordered write
-    uint32_t gt = 0, eq = 0;
-    for (int e = lo + tid; e < hi; e += kTkThreads) {
-        const uint32_t u = cached ? cache[e - lo] : order_key(__ldg(row + e));
-        gt += u > T;
-        eq += u == T;
-    }
-    uint64_t tot_pair;
-    block_excl_scan((static_cast<uint64_t>(eq) << 32) | gt, scan_buf, tot_pair);
-    if (tid == 0) {
-        cta_counts[0] = static_cast<uint32_t>(tot_pair & 0xFFFFFFFFu);
-        cta_counts[1] = static_cast<uint32_t>(tot_pair >> 32);
-    }
-    cluster.sync();
-    if (tid == 0) {
-        int eq_before = 0, sel_before = 0;
-        for (int r = 0; r < rank; ++r) {
-            const uint32_t *rc = cluster.map_shared_rank(cta_counts, r);
-            const int g_r = static_cast<int>(rc[0]), e_r = static_cast<int>(rc[1]);
-            sel_before += g_r + max(0, min(need_eq - eq_before, e_r));
-            eq_before += e_r;
+// Resolve the last two digits on a candidate list (keys in shared memory):
+// returns T and the number of rows equal to T to keep.
+__device__ __forceinline__ void refine_candidates(TopkSmem &sm, int m, uint32_t d1, uint32_t r2, uint32_t &T,
+                                                  uint32_t &need_eq) {
+    zero_hist(sm.hist, kBins);
+    __syncthreads();
+    for (int base = 0; base < m; base += kT) {
+        const int c = base + threadIdx.x;
+        uint32_t d = 0xFFFFFFFFu;
+        if (c < m) {
+            const uint32_t u = sm.cand_key[c];
+            if ((u >> 20) == d1) d = (u >> 8) & 0xFFFu;
         }
-        cta_plan[0] = sel_before;
-        cta_plan[1] = max(0, min(need_eq - eq_before, static_cast<int>(cta_counts[1])));
+        hist_add(sm.hist, d);
     }
-    cluster.sync();  // remote reads done: shared memory of every CTA may be released
-    const int sel_before = cta_plan[0];
-    const int quota = cta_plan[1];
+    __syncthreads();
+    find_digit(sm.hist, kBins, r2, sm.scan, sm.sel);
+    const uint32_t d2 = sm.sel[0];
+    const uint32_t r3 = r2 - sm.sel[1];
+    __syncthreads();
+    zero_hist(sm.hist, kBins3);
+    __syncthreads();
+    const uint32_t p24 = (d1 << 12) | d2;
+    for (int base = 0; base < m; base += kT) {
+        const int c = base + threadIdx.x;
+        uint32_t d = 0xFFFFFFFFu;
+        if (c < m) {
+            const uint32_t u = sm.cand_key[c];
+            if ((u >> 8) == p24) d = u & 0xFFu;
+        }
+        hist_add(sm.hist, d);
+    }
+    __syncthreads();
+    find_digit(sm.hist, kBins3, r3, sm.scan, sm.sel);
+    T = (p24 << 8) | sm.sel[0];
+    need_eq = r3 - sm.sel[1];
+    __syncthreads();
+}
+
+// Resolve the last two digits by streaming the whole row (tie-heavy fallback).
+__device__ __forceinline__ void refine_stream(TopkSmem &sm, const float *row, int n, uint32_t d1, uint32_t r2,
+                                              uint32_t &T, uint32_t &need_eq) {
+    zero_hist(sm.hist, kBins);
+    __syncthreads();
+    stream_hist(row, 0, n, d1 << 20, 0xFFF00000u, 8, 0xFFFu, sm.hist);
+    find_digit(sm.hist, kBins, r2, sm.scan, sm.sel);
+    const uint32_t d2 = sm.sel[0];
+    const uint32_t r3 = r2 - sm.sel[1];
+    __syncthreads();
+    zero_hist(sm.hist, kBins3);
+    __syncthreads();
+    const uint32_t p24 = (d1 << 12) | d2;
+    stream_hist(row, 0, n, p24 << 8, 0xFFFFFF00u, 0, 0xFFu, sm.hist);
+    find_digit(sm.hist, kBins3, r3, sm.scan, sm.sel);
+    T = (p24 << 8) | sm.sel[0];
+    need_eq = r3 - sm.sel[1];
+    __syncthreads();
+}
+
+// Ordered filter: keep keys > T and the first need_eq keys == T (in list
+// order), writing their positions to out[] at exclusive-scan slots.  The list is
+// either the candidates in shared memory or the row itself.
+template <bool kFromCandidates>
+__device__ __forceinline__ void ordered_write(TopkSmem &sm, const float *row, int m, uint32_t T,
+                                              uint32_t need_eq, int32_t *out) {
     uint32_t g_run = 0, e_run = 0;
-    for (int base = lo; base < hi; base += kTkThreads * kPerThread) {
-        const int e0 = base + tid * kPerThread;
-        uint32_t u[kPerThread];
+    for (int base = 0; base < m; base += kT * kV) {
+        const int e0 = base + threadIdx.x * kV;
+        uint32_t u[kV];
+        int32_t p[kV];
         uint32_t tg = 0, te = 0;
 #pragma unroll
-        for (int x = 0; x < kPerThread; ++x) {
+        for (int x = 0; x < kV; ++x) {
             const int e = e0 + x;
-            u[x] = 0u;
-            if (e < hi) u[x] = cached ? cache[e - lo] : order_key(__ldg(row + e));
-            tg += (e < hi) && u[x] > T;
-            te += (e < hi) && u[x] == T;
+            u[x] = 0;
+            p[x] = -1;
+            if (e < m) {
+                if (kFromCandidates) {
+                    u[x] = sm.cand_key[e];
+                    p[x] = sm.cand_pos[e];
+                } else {
+                    u[x] = order_key(__ldg(row + e));
+                    p[x] = e;
+                }
+                tg += u[x] > T;
+                te += u[x] == T;
+            }
         }
-        uint64_t tile_tot;
-        const uint64_t ex = block_excl_scan((static_cast<uint64_t>(te) << 32) | tg, scan_buf, tile_tot);
+        uint64_t tot;
+        const uint64_t ex = block_scan((static_cast<uint64_t>(te) << 32) | tg, sm.scan, tot);
         uint32_t g = g_run + static_cast<uint32_t>(ex & 0xFFFFFFFFu);
         uint32_t q = e_run + static_cast<uint32_t>(ex >> 32);
 #pragma unroll
-        for (int x = 0; x < kPerThread; ++x) {
-            const int e = e0 + x;
-            if (e >= hi) break;
+        for (int x = 0; x < kV; ++x) {
+            if (p[x] < 0) continue;
             if (u[x] > T) {
-                out[sel_before + g + min(q, static_cast<uint32_t>(quota))] = e;
+                out[g + min(q, need_eq)] = p[x];
                 ++g;
             } else if (u[x] == T) {
-                if (q < static_cast<uint32_t>(quota)) out[sel_before + g + q] = e;
+                if (q < need_eq) out[g + q] = p[x];
                 ++q;
             }
         }
-        g_run += static_cast<uint32_t>(tile_tot & 0xFFFFFFFFu);
-        e_run += static_cast<uint32_t>(tile_tot >> 32);
+        g_run += static_cast<uint32_t>(tot & 0xFFFFFFFFu);
+        e_run += static_cast<uint32_t>(tot >> 32);
     }
-    if (rank == C - 1) {
-        for (int p = k + tid; p < a.topk; p += kTkThreads) out[p] = -1;
+}
+
+// Copy rows [lo, hi) whose first digit is >= d1 into dst (position order).
+// Returns the number of such rows (may exceed cap; only cap are stored).
+template <bool kToShared>
+__device__ __forceinline__ uint32_t collect(const float *row, int lo, int hi, uint32_t d1, TopkSmem &sm,
+                                            uint2 *gdst, uint32_t cap) {
+    uint32_t run = 0;
+    for (int base = lo; base < hi; base += kT * kV) {
+        const int e0 = base + threadIdx.x * kV;
+        float v[kV];
+        if (e0 + kV <= hi) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(row + e0));
+            v[0] = f.x, v[1] = f.y, v[2] = f.z, v[3] = f.w;
+        } else {
+#pragma unroll
+            for (int x = 0; x < kV; ++x) v[x] = e0 + x < hi ? __ldg(row + e0 + x) : 0.f;
+        }
+        uint32_t u[kV];
+        uint32_t c = 0;
+#pragma unroll
+        for (int x = 0; x < kV; ++x) {
+            u[x] = order_key(v[x]);
+            c += (e0 + x < hi) && (u[x] >> 20) >= d1;
+        }
+        uint64_t tot;
+        uint32_t off = run + static_cast<uint32_t>(block_scan(c, sm.scan, tot));
+#pragma unroll
+        for (int x = 0; x < kV; ++x) {
+            if (e0 + x < hi && (u[x] >> 20) >= d1) {
+                if (off < cap) {
+                    if (kToShared) {
+                        sm.cand_key[off] = u[x];
+                        sm.cand_pos[off] = e0 + x;
+                    } else {
+                        gdst[off] = make_uint2(u[x], static_cast<uint32_t>(e0 + x));
+                    }
+                }
+                ++off;
+            }
+        }
+        run += static_cast<uint32_t>(tot);
     }
-    if (rank == 0 && tid == 0) a.cnt[i] = k;
+    __syncthreads();
+    return run;
+}
+
+__device__ __forceinline__ int visible_rows(const TopkArgs &a, int i) {
+    const int pos = a.q_pos[i];
+    if (pos < 0 || pos >= a.L) {
+        if (threadIdx.x == 0 && blockIdx.x == 0) report_status(a.status, DSA_ERR_INVALID);
+        return 0;
+    }
+    return pos + 1;
+}
+
+// Every visible row is kept (n <= topk).
+__device__ __forceinline__ void write_all(const TopkArgs &a, int i, int n) {
+    int32_t *out = a.idx + static_cast<int64_t>(i) * a.topk;
+    for (int p = threadIdx.x; p < a.topk; p += kT) out[p] = p < n ? p : -1;
+    if (threadIdx.x == 0) a.cnt[i] = n;
+}
+
+// Shared tail: given the first digit d1 (with `above1` rows above it) and a
+// candidate list of m rows in shared memory (or overflow), finish the query.
+__device__ __forceinline__ void finish(const TopkArgs &a, TopkSmem &sm, const float *row, int i, int n,
+                                       uint32_t d1, uint32_t above1, int m, bool overflow) {
+    const uint32_t k = static_cast<uint32_t>(a.topk);
+    uint32_t T, need_eq;
+    int32_t *out = a.idx + static_cast<int64_t>(i) * a.topk;
+    if (!overflow) {
+        refine_candidates(sm, m, d1, k - above1, T, need_eq);
+        ordered_write<true>(sm, row, m, T, need_eq, out);
+    } else {
+        refine_stream(sm, row, n, d1, k - above1, T, need_eq);
+        ordered_write<false>(sm, row, n, T, need_eq, out);
+    }
+    if (threadIdx.x == 0) a.cnt[i] = a.topk;
+}
+
+// ---------------------------------------------------------------- row schedule
+__global__ void __launch_bounds__(kT, 1) topk_row_kernel(const TopkArgs a) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    const int i = blockIdx.x;
+    const int n = visible_rows(a, i);
+    if (n <= a.topk) {
+        write_all(a, i, n);
+        return;
+    }
+    const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
+    zero_hist(sm.hist, kBins);
+    __syncthreads();
+    stream_hist(row, 0, n, 0u, 0u, 20, 0xFFFu, sm.hist);
+    find_digit(sm.hist, kBins, static_cast<uint32_t>(a.topk), sm.scan, sm.sel);
+    const uint32_t d1 = sm.sel[0], above1 = sm.sel[1];
+    const uint32_t m_est = above1 + sm.hist[d1];
+    __syncthreads();
+    bool overflow = m_est > static_cast<uint32_t>(kCap);
+    uint32_t m = 0;
+    if (!overflow) m = collect<true>(row, 0, n, d1, sm, nullptr, kCap);
+    finish(a, sm, row, i, n, d1, above1, static_cast<int>(m), overflow);
+}
+
+// ---------------------------------------------------------------- split schedule
+// (1) first-digit histogram of a chunk, added into the query's global histogram.
+__global__ void __launch_bounds__(kT, 2) topk_hist_kernel(const TopkArgs a, int chunk) {
+    __shared__ uint32_t hist[kBins];
+    const int i = blockIdx.y, p = blockIdx.x;
+    const int n = visible_rows(a, i);
+    if (n <= a.topk) return;
+    const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
+    if (lo >= hi) return;
+    zero_hist(hist, kBins);
+    __syncthreads();
+    stream_hist(a.scores + static_cast<int64_t>(i) * a.ld, lo, hi, 0u, 0u, 20, 0xFFFu, hist);
+    uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+    for (int b = threadIdx.x; b < kBins; b += kT)
+        if (hist[b]) atomicAdd(&g[b], hist[b]);
+}
+
+// (2) the chunk's candidates (first digit >= the threshold digit), in order.
+__global__ void __launch_bounds__(kT, 1) topk_collect_kernel(const TopkArgs a, int chunk) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    const int i = blockIdx.y, p = blockIdx.x;
+    const int n = visible_rows(a, i);
+    if (n <= a.topk) return;
+    const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
+    const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+    for (int b = threadIdx.x; b < kBins; b += kT) sm.hist[b] = g[b];
+    __syncthreads();
+    find_digit(sm.hist, kBins, static_cast<uint32_t>(a.topk), sm.scan, sm.sel);
+    const uint32_t d1 = sm.sel[0];
+    __syncthreads();
+    uint2 *dst = a.gcand + (static_cast<int64_t>(i) * kSplitMax + p) * kSplitCap;
+    const uint32_t c = collect<false>(a.scores + static_cast<int64_t>(i) * a.ld, lo, hi, d1, sm, dst, kSplitCap);
+    if (threadIdx.x == 0) a.gcount[static_cast<int64_t>(i) * kSplitMax + p] = c;
+}
+
+// (3) merge the chunks' candidates in position order and finish the query.
+__global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int n_chunks) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
+    __shared__ uint32_t offs[kSplitMax + 1];
+    __shared__ int bad;
+    const int i = blockIdx.x;
+    const int n = visible_rows(a, i);
+    if (n <= a.topk) {
+        write_all(a, i, n);
+        return;
+    }
+    const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+    for (int b = threadIdx.x; b < kBins; b += kT) sm.hist[b] = g[b];
+    __syncthreads();
+    find_digit(sm.hist, kBins, static_cast<uint32_t>(a.topk), sm.scan, sm.sel);
+    const uint32_t d1 = sm.sel[0], above1 = sm.sel[1];
+    if (threadIdx.x == 0) {
+        uint32_t o = 0;
+        int ov = 0;
+        for (int p = 0; p < n_chunks; ++p) {
+            const uint32_t c = a.gcount[static_cast<int64_t>(i) * kSplitMax + p];
+            offs[p] = o;
+            o += c;
+            ov |= c > static_cast<uint32_t>(kSplitCap);
+        }
+        offs[n_chunks] = o;
+        bad = ov || o > static_cast<uint32_t>(kCap);
+    }
+    __syncthreads();
+    const bool overflow = bad != 0;
+    const int m = overflow ? 0 : static_cast<int>(offs[n_chunks]);
+    if (!overflow) {
+        for (int p = 0; p < n_chunks; ++p) {
+            const uint2 *src = a.gcand + (static_cast<int64_t>(i) * kSplitMax + p) * kSplitCap;
+            const int c = static_cast<int>(offs[p + 1] - offs[p]);
+            for (int j = threadIdx.x; j < c; j += kT) {
+                const uint2 v = src[j];
+                sm.cand_key[offs[p] + j] = v.x;
+                sm.cand_pos[offs[p] + j] = static_cast<int32_t>(v.y);
+            }
+        }
+        __syncthreads();
+    }
+    finish(a, sm, a.scores + static_cast<int64_t>(i) * a.ld, i, n, d1, above1, m, overflow);
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+    return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
 }
 
 }  // namespace
 
+bool topk_uses_split(int n_q, int max_ctx) { return max_ctx > kTopkRowMaxCtx && n_q <= kTopkSplitMaxQueries; }
+
 cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
-    // Cluster size: enough CTAs to cover the SMs for small batches, and small
-    // enough chunks to stay in shared memory where possible.
-    int C = 1;
-    while (C < 16 && ((a.L + C - 1) / C > a.cache_cap || static_cast<long long>(a.n_q) * C < 2LL * num_sms))
-        C *= 2;
-    cudaError_t e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    cfg.blockDim = dim3(kTkThreads, 1, 1);
-    cfg.stream = st;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    // Shrink the cluster until the hardware can co-schedule one.
-    for (;; C /= 2) {
-        const int chunk = (((a.L + C - 1) / C) + 3) & ~3;
-        const size_t smem = chunk <= a.cache_cap ? static_cast<size_t>(chunk) * sizeof(uint32_t) : 0;
-        e = cudaFuncSetAttribute(topk_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        cfg.gridDim = dim3(static_cast<unsigned>(a.n_q) * C, 1, 1);
-        cfg.dynamicSmemBytes = smem;
-        attr[0].val.clusterDim.x = C;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        int clusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&clusters, topk_cluster_kernel, &cfg);
-        if ((e == cudaSuccess && clusters > 0) || C == 1) break;
-        (void)cudaGetLastError();
+    const size_t smem = sizeof(TopkSmem);
+    cudaError_t e;
+    if (!topk_uses_split(a.n_q, a.L)) {
+        if ((e = set_smem(topk_row_kernel, smem)) != cudaSuccess) return e;
+        topk_row_kernel<<<a.n_q, kT, smem, st>>>(a);
+        return cudaGetLastError();
     }
-    TopkArgs b = a;
-    if ((((a.L + C - 1) / C) + 3 & ~3) > a.cache_cap) b.cache_cap = 0;
-    return cudaLaunchKernelEx(&cfg, topk_cluster_kernel, b);
+    int P = (2 * num_sms + a.n_q - 1) / a.n_q;
+    P = P < 1 ? 1 : (P > kSplitMax ? kSplitMax : P);
+    int chunk = (a.L + P - 1) / P;
+    chunk = (chunk + kT * kV - 1) / (kT * kV) * (kT * kV);
+    P = (a.L + chunk - 1) / chunk;
+    if ((e = cudaMemsetAsync(a.ghist, 0, sizeof(uint32_t) * kBins * a.n_q, st)) != cudaSuccess) return e;
+    topk_hist_kernel<<<dim3(P, a.n_q), kT, 0, st>>>(a, chunk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = set_smem(topk_collect_kernel, smem)) != cudaSuccess) return e;
+    topk_collect_kernel<<<dim3(P, a.n_q), kT, smem, st>>>(a, chunk);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = set_smem(topk_merge_kernel, smem)) != cudaSuccess) return e;
+    topk_merge_kernel<<<a.n_q, kT, smem, st>>>(a, P);
+    return cudaGetLastError();
+}
+
+size_t topk_scratch_bytes(int n_q, int max_ctx) {
+    if (!topk_uses_split(n_q, max_ctx)) return 0;
+    const size_t hist = sizeof(uint32_t) * kBins * n_q;
+    const size_t counts = sizeof(uint32_t) * kSplitMax * n_q;
+    const size_t cand = sizeof(uint2) * static_cast<size_t>(kSplitCap) * kSplitMax * n_q;
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    return al(hist) + al(counts) + al(cand);
+}
+
+void topk_bind_scratch(TopkArgs &a, void *scratch) {
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    uint8_t *p = static_cast<uint8_t *>(scratch);
+    a.ghist = reinterpret_cast<uint32_t *>(p);
+    p += al(sizeof(uint32_t) * kBins * a.n_q);
+    a.gcount = reinterpret_cast<uint32_t *>(p);
+    p += al(sizeof(uint32_t) * kSplitMax * a.n_q);
+    a.gcand = reinterpret_cast<uint2 *>(p);
 }
 
 }  // namespace dsa
