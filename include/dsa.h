@@ -210,6 +210,32 @@ dsa_status dsa_sparse_mla_prefill(const dsa_queries *queries, const dsa_mla *mla
                                   size_t ws_bytes, void *stream);
 
 /*
+ * dsa_sparse_mla_decode without a workspace.  The pages have no counterpart to
+ * this call: it exists for callers that cannot allocate device memory where
+ * they run attention (a runtime or plugin that hands over only its input and
+ * output tensors, or memory that was planned and fixed up front), so they have
+ * no workspace to pass.  Same arguments and result as dsa_sparse_mla_decode
+ * (tensor-core shape only: bf16, 64 heads, 512 + 64; other shapes return
+ * DSA_ERR_UNSUPPORTED), minus `ws`.
+ *  - Scratch: a fixed 32 MiB device array inside the library (status word +
+ *    split-K partials), held by every GPU that loads the library until the
+ *    process exits.  Calls that need more -- 256 + ceil(topk/128) * n_q *
+ *    131,584 bytes, e.g. more than 15 queries at topk = 2048 -- are rejected
+ *    with DSA_ERR_WORKSPACE before any launch.
+ *  - Set-up: the first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the one array, so calls that overlap on the
+ *    GPU (other streams, other host threads) race; serialise them.
+ *  - Device-side checks (indices out of range) are applied -- such rows are
+ *    skipped -- but not reported: there is no workspace status word to read.
+ *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
+ */
+dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, const dsa_mla *mla,
+                                         const int32_t *idx, const int32_t *cnt, int32_t topk,
+                                         void *stream);
+
+/*
  * IndexShare group [HA, MLA + DSA with IndexShare]: layer 0 (the full layer)
  * runs dsa_index_scores -> dsa_topk -> sparse MLA; layers 1..n_layers-1 run
  * sparse MLA with layer 0's idx/cnt on their own queries and caches, without
