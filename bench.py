@@ -148,7 +148,9 @@ class Step:
         self.seq_run = w.n_q if len(set(w.q_seq)) == 1 else 1
         x = self.x
         self.q = B.Queries(x["q_seq"], x["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=self.seq_run)
-        self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"])
+        # the indexer leaves the top-k's first-digit histograms in the workspace
+        self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"],
+                            flags=B.DSA_INDEXER_TOPK_HIST)
         self.mlas = []
         for layer in range(w.n_layers):
             out = torch.empty((w.n_q, w.mla_heads, w.d_lat), dtype=w.torch_dtype, device=dev)
@@ -176,7 +178,7 @@ class Step:
         B.dsa_index_scores(self.q, self.ix, self.scores, self.ws)
         if events:
             self.ev[1].record()
-        B.dsa_topk(self.q, self.scores, self.w.topk, self.idx, self.cnt, self.ws)
+        B.dsa_topk(self.q, self.scores, self.w.topk, self.idx, self.cnt, self.ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
         if events:
             self.ev[2].record()
         for m in self.mlas:

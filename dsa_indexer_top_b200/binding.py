@@ -22,6 +22,8 @@ LIB_PATH = os.path.join(_HERE, "libdsa.so")
 DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT = range(6)
 DSA_BF16, DSA_F32 = 0, 1
 DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_MLA_DECODE, DSA_OP_MLA_PREFILL, DSA_OP_INDEXSHARE_GROUP = range(5)
+DSA_INDEXER_TOPK_HIST = 1
+DSA_TOPK_HIST_FROM_INDEXER = 1
 
 
 class DsaError(RuntimeError):
@@ -37,7 +39,7 @@ class _Queries(ctypes.Structure):
 
 class _Indexer(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("dim", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("q", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("flags", ctypes.c_int32), ("q", ctypes.c_void_p), ("w", ctypes.c_void_p),
                 ("k", ctypes.c_void_p), ("k_seq_stride", ctypes.c_int64), ("k_row_stride", ctypes.c_int64)]
 
 
@@ -61,7 +63,7 @@ def lib():
         P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
         st = ctypes.c_int
         h.dsa_index_scores.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Indexer), P, I64, P, SZ, P]
-        h.dsa_topk.argtypes = [ctypes.POINTER(_Queries), P, I64, I32, P, P, P, SZ, P]
+        h.dsa_topk.argtypes = [ctypes.POINTER(_Queries), P, I64, I32, I32, P, P, P, SZ, P]
         for name in ("dsa_sparse_mla_decode", "dsa_sparse_mla_prefill"):
             getattr(h, name).argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Mla), P, P, I32, P, SZ, P]
         h.dsa_indexshare_group.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Indexer),
@@ -126,11 +128,12 @@ class Indexer:
     q: torch.Tensor              # [n_q, heads, dim]
     w: torch.Tensor              # float32 [n_q, heads]
     k: torch.Tensor              # [n_seq, L, dim] or [L, dim] (shared cache)
+    flags: int = 0               # DSA_INDEXER_TOPK_HIST or 0
 
     def c(self) -> _Indexer:
         shared = self.k.dim() == 2
         seq_stride = 0 if shared else self.k.stride(0)
-        return _Indexer(self.q.shape[1], self.q.shape[2], _dtype_code(self.q), 0, self.q.data_ptr(),
+        return _Indexer(self.q.shape[1], self.q.shape[2], _dtype_code(self.q), self.flags, self.q.data_ptr(),
                         self.w.data_ptr(), self.k.data_ptr(), seq_stride, self.k.stride(-2))
 
 
@@ -175,9 +178,9 @@ def dsa_index_scores(queries: Queries, indexer: Indexer, scores: torch.Tensor, w
 
 
 def dsa_topk(queries: Queries, scores: torch.Tensor, topk: int, idx: torch.Tensor, cnt: torch.Tensor,
-             ws: torch.Tensor, stream=None):
+             ws: torch.Tensor, stream=None, flags: int = 0):
     qc = queries.c()
-    _check(lib().dsa_topk(ctypes.byref(qc), _ptr(scores), scores.stride(0), topk, _ptr(idx), _ptr(cnt), _ptr(ws),
+    _check(lib().dsa_topk(ctypes.byref(qc), _ptr(scores), scores.stride(0), topk, flags, _ptr(idx), _ptr(cnt), _ptr(ws),
                           ws.numel() * ws.element_size(), _stream(stream)), "dsa_topk")
 
 

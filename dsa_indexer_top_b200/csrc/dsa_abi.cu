@@ -92,8 +92,19 @@ size_t ws_group(int n_q, int max_ctx, int topk, int n_layers) {
 }
 
 // ------------------------------------------------------------------ indexer
+dsa_status do_index_generic(const dsa_queries *qs, const dsa_indexer *ix, float *scores, int64_t ld,
+                            uint32_t *status, cudaStream_t st);
+
+// ghist: non-null to leave the top-k first-digit histograms there.
 dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *scores, int64_t ld,
-                           uint32_t *status, cudaStream_t st) {
+                           uint32_t *status, uint32_t *ghist, cudaStream_t st) {
+    // the histograms are left only when queries are not tiled together (odd
+    // seq_run: one query per tensor-core tile, where the epilogue builds them)
+    if ((qs->seq_run & 1) == 0) ghist = nullptr;
+    if (ghist && cudaMemsetAsync(ghist, 0, sizeof(uint32_t) * kTopkBins * qs->n_q, st) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    bool hist_done = false;
+    dsa_status s = DSA_OK;
     const int n_cache = ix->k_seq_stride == 0 ? 1 : qs->n_seq;
     if (indexer_tc_ok(ix)) {
         EncodeTiledFn enc = encode_fn();
@@ -138,10 +149,30 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
         a.tiles_per_group = (qs->max_ctx + 127) / 128;
         const long long groups = (qs->n_q + G - 1) / G;
         a.total_items = groups * a.tiles_per_group;
+        a.ghist = (ghist && G == 1) ? ghist : nullptr;  // fused into the epilogue
+        hist_done = a.ghist != nullptr;
         const int sms = num_sms_current();
         const int grid = static_cast<int>(a.total_items < sms ? a.total_items : sms);
-        return launch_idx_score_tc(G, tk, tq, a, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+        s = launch_idx_score_tc(G, tk, tq, a, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    } else {
+        s = do_index_generic(qs, ix, scores, ld, status, st);
     }
+    if (s != DSA_OK || !ghist || hist_done) return s;
+    // histogram pass over the scores just written (generic CUDA-core path)
+    TopkArgs t = {};
+    t.scores = scores;
+    t.ld = ld;
+    t.q_pos = qs->q_pos;
+    t.status = status;
+    t.n_q = qs->n_q;
+    t.L = qs->max_ctx;
+    t.topk = 0;
+    t.ghist = ghist;
+    return launch_topk_hist(t, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status do_index_generic(const dsa_queries *qs, const dsa_indexer *ix, float *scores, int64_t ld,
+                            uint32_t *status, cudaStream_t st) {
     const size_t smem = sizeof(float) * (static_cast<size_t>(ix->heads) * ix->dim + ix->heads);
     if (smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;
     IdxGenericArgs g;
@@ -174,7 +205,7 @@ dsa_status check_indexer(const dsa_queries *qs, const dsa_indexer *ix) {
 
 // ------------------------------------------------------------------ top-k
 dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int topk, int32_t *idx,
-                   int32_t *cnt, uint32_t *status, void *scratch, cudaStream_t st) {
+                   int32_t *cnt, uint32_t *status, void *scratch, bool hist_ready, cudaStream_t st) {
     TopkArgs a;
     a.scores = scores;
     a.ld = ld;
@@ -185,10 +216,11 @@ dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int t
     a.n_q = qs->n_q;
     a.L = qs->max_ctx;
     a.topk = topk;
+    a.hist_ready = (hist_ready && (qs->seq_run & 1)) ? 1 : 0;
     a.ghist = nullptr;
     a.gcount = nullptr;
     a.gcand = nullptr;
-    if (topk_uses_split(qs->n_q, qs->max_ctx)) topk_bind_scratch(a, scratch);
+    topk_bind_scratch(a, scratch);
     return launch_topk(a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
@@ -320,19 +352,25 @@ dsa_status dsa_index_scores(const dsa_queries *queries, const dsa_indexer *index
     dsa_status s = check_indexer(queries, indexer);
     if (s != DSA_OK) return s;
     if (!scores_ok(scores, ld_scores, queries->max_ctx)) return DSA_ERR_INVALID;
+    const bool hist = (indexer->flags & DSA_INDEXER_TOPK_HIST) != 0;
+    if (indexer->flags & ~DSA_INDEXER_TOPK_HIST) return DSA_ERR_INVALID;
+    if (hist && !ws_ok(ws, ws_bytes, ws_topk(queries->n_q, queries->max_ctx))) return DSA_ERR_WORKSPACE;
     if (queries->n_q == 0) return DSA_OK;
-    return do_index_scores(queries, indexer, scores, ld_scores, status_word(ws), static_cast<cudaStream_t>(stream));
+    uint32_t *ghist = hist ? reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(ws) + kStatusBytes) : nullptr;
+    return do_index_scores(queries, indexer, scores, ld_scores, status_word(ws), ghist,
+                           static_cast<cudaStream_t>(stream));
 }
 
-dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_scores, int32_t topk, int32_t *idx,
-                    int32_t *cnt, void *ws, size_t ws_bytes, void *stream) {
+dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_scores, int32_t topk, int32_t flags,
+                    int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes, void *stream) {
     if (!valid_queries(queries)) return DSA_ERR_INVALID;
     if (!ws_ok(ws, ws_bytes, ws_topk(queries->n_q, queries->max_ctx))) return DSA_ERR_WORKSPACE;
     if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
+    if (flags & ~DSA_TOPK_HIST_FROM_INDEXER) return DSA_ERR_INVALID;
     if (!scores_ok(scores, ld_scores, queries->max_ctx)) return DSA_ERR_INVALID;
     if (queries->n_q == 0) return DSA_OK;
     return do_topk(queries, scores, ld_scores, topk, idx, cnt, status_word(ws), static_cast<uint8_t *>(ws) + kStatusBytes,
-                   static_cast<cudaStream_t>(stream));
+                   (flags & DSA_TOPK_HIST_FROM_INDEXER) != 0, static_cast<cudaStream_t>(stream));
 }
 
 static dsa_status mla_entry(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx, const int32_t *cnt,
@@ -375,9 +413,10 @@ dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *i
     const int64_t ld = round4(queries->max_ctx);
     uint8_t *topk_scratch = base + kStatusBytes + ws_scores(queries->n_q, queries->max_ctx);
     uint8_t *scratch = topk_scratch + align256(topk_scratch_bytes(queries->n_q, queries->max_ctx));
-    s = do_index_scores(queries, indexer, scores, ld, status_word(ws), st);
+    // the first-digit histograms of top-k come out of the indexer (ghist heads the top-k scratch)
+    s = do_index_scores(queries, indexer, scores, ld, status_word(ws), reinterpret_cast<uint32_t *>(topk_scratch), st);
     if (s != DSA_OK) return s;
-    s = do_topk(queries, scores, ld, topk, idx, cnt, status_word(ws), topk_scratch, st);
+    s = do_topk(queries, scores, ld, topk, idx, cnt, status_word(ws), topk_scratch, true, st);
     if (s != DSA_OK) return s;
     return do_mla(queries, layers, n_layers, idx, cnt, topk, group_uses_decode(queries->n_q), scratch,
                   status_word(ws), st);

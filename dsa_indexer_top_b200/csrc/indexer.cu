@@ -28,7 +28,6 @@ namespace {
 
 constexpr int kTileKeys = 128;
 constexpr int kATileBytes = kTileKeys * kIdxDim * 2;  // 32 KB
-constexpr int kIdxThreads = 192;
 
 template <int G>
 struct IdxCfg {
@@ -38,6 +37,10 @@ struct IdxCfg {
     static constexpr int kTmemCols = (2 * N < 32) ? 32 : 2 * N;
     static constexpr int kSmem = kStages * kATileBytes + kBBytes + 1024;
     static constexpr uint32_t kIdesc = idesc_bf16(128, N, false, false);
+    // epilogue warps: two per TMEM lane quadrant when a tile holds several
+    // queries (each takes half of them), one otherwise
+    static constexpr int kEpiWarps = G >= 2 ? 8 : 4;
+    static constexpr int kThreads = (2 + kEpiWarps) * 32;
 };
 
 // Sequence and last visible position of a query group; every role calls this
@@ -59,7 +62,7 @@ __device__ __forceinline__ void group_info(const IdxTcArgs &a, int g, int &seq, 
 }
 
 template <int G>
-__global__ void __launch_bounds__(kIdxThreads, 1)
+__global__ void __launch_bounds__(IdxCfg<G>::kThreads, 1)
     idx_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_q, const IdxTcArgs a) {
     using Cfg = IdxCfg<G>;
@@ -77,7 +80,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     __shared__ uint64_t b_full, b_empty, mma_done;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
-    __shared__ float w_sh[4][N];  // one private copy per epilogue warp
+    constexpr int E = Cfg::kEpiWarps;
+    __shared__ __align__(16) float w_sh[E][N];  // one private copy per epilogue warp
+    // Fused top-k first-digit histogram of the current query (one query per
+    // tile only), flushed into a.ghist when the epilogue moves to another query.
+    __shared__ uint32_t ehist[G == 1 ? kTopkBins : 1];
+    __shared__ uint64_t epi_bar;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -89,11 +97,12 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&tmem_full[s], 1);
-            mbar_init(&tmem_empty[s], 4);
+            mbar_init(&tmem_empty[s], E);
         }
         mbar_init(&b_full, 1);
         mbar_init(&b_empty, 1);
         mbar_init(&mma_done, 1);
+        mbar_init(&epi_bar, 4);
         abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmap_k);
@@ -103,6 +112,9 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
         tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
         tmem_relinquish();
     }
+    const bool fuse_hist = (G == 1) && a.ghist != nullptr;
+    if (fuse_hist)
+        for (int b = threadIdx.x; b < kTopkBins; b += Cfg::kThreads) ehist[b] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -209,15 +221,44 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;  // TMEM lane quadrant this warp may access
+        // queries of the tile this warp handles
+        constexpr int kQPerWarp = E == 8 ? G / 2 : G;
+        const int qlo = E == 8 ? ((warp - 2) >> 2) * kQPerWarp : 0;
         float *w_mine = w_sh[warp - 2];
+        const int etid = threadIdx.x - 64;
         int cur_g = -1, seq = -1, max_pos = -1;
-        int qpos[G];
-        bool qok[G];
+        int qpos[kQPerWarp];   // this warp's queries of the current group
+        bool qok[kQPerWarp];
         long long k_tiles = 0;
+        uint32_t epi_phase = 0;
+        bool hist_dirty = false;
+        // all four epilogue warps meet (bounded wait on an mbarrier)
+        auto epi_sync = [&]() {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&epi_bar);
+            mbar_wait(&epi_bar, epi_phase, a.status, &abort_flag);
+            epi_phase ^= 1;
+        };
+        auto flush_hist = [&](int g) {
+            epi_sync();
+            uint32_t *dst = a.ghist + static_cast<int64_t>(g) * kTopkBins;
+            for (int b = etid; b < kTopkBins; b += 128) {
+                const uint32_t v = ehist[b];
+                if (v) {
+                    atomicAdd(dst + b, v);
+                    ehist[b] = 0;
+                }
+            }
+            epi_sync();
+        };
         for (long long it = begin; it < end; ++it) {
             const int g = static_cast<int>(it / tpg);
             const int j = static_cast<int>(it % tpg);
             if (g != cur_g) {
+                if (fuse_hist && hist_dirty) {
+                    flush_hist(cur_g);
+                    hist_dirty = false;
+                }
                 group_info<G>(a, g, seq, max_pos);
                 cur_g = g;
                 const int q0 = g * G;
@@ -228,17 +269,17 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
                 }
                 __syncwarp();
 #pragma unroll
-                for (int i = 0; i < G; ++i) {
-                    const int qi = q0 + i;
-                    qpos[i] = -1;
-                    qok[i] = false;
+                for (int ii = 0; ii < kQPerWarp; ++ii) {
+                    const int qi = q0 + qlo + ii;
+                    qpos[ii] = -1;
+                    qok[ii] = false;
                     if (qi < a.n_q) {
                         const int p = __ldg(a.q_pos + qi);
                         const int sq = __ldg(a.q_seq + qi);
                         const bool seq_ok = a.k_shared ? (sq >= 0 && sq < a.n_seq) : (sq == seq);
-                        qok[i] = p >= 0 && p < a.L && seq_ok && seq >= 0;
-                        qpos[i] = p;
-                        if (!qok[i] && lane == 0) report_status(a.status, DSA_ERR_INVALID);
+                        qok[ii] = p >= 0 && p < a.L && seq_ok && seq >= 0;
+                        qpos[ii] = p;
+                        if (!qok[ii] && lane == 0) report_status(a.status, DSA_ERR_INVALID);
                     }
                 }
             }
@@ -250,21 +291,32 @@ __global__ void __launch_bounds__(kIdxThreads, 1)
             const int s = j * kTileKeys + quad * 32 + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * N;
 #pragma unroll
-            for (int i = 0; i < G; ++i) {
+            for (int ii = 0; ii < kQPerWarp; ++ii) {
+                const int i = qlo + ii;
                 uint32_t r[32];
                 tmem_ld32(taddr + i * 32, r);
                 tmem_ld_wait();
                 float score = 0.f;
+                const float4 *w4 = reinterpret_cast<const float4 *>(w_mine + i * 32);
 #pragma unroll
-                for (int h = 0; h < 32; ++h) score = fmaf(w_mine[i * 32 + h], fmaxf(u2f(r[h]), 0.f), score);
-                if (qok[i] && s <= qpos[i])
-                    a.scores[static_cast<int64_t>(g * G + i) * a.ld + s] = score;
+                for (int h4 = 0; h4 < 8; ++h4) {
+                    const float4 wv = w4[h4];
+                    score = fmaf(wv.x, fmaxf(u2f(r[4 * h4]), 0.f), score);
+                    score = fmaf(wv.y, fmaxf(u2f(r[4 * h4 + 1]), 0.f), score);
+                    score = fmaf(wv.z, fmaxf(u2f(r[4 * h4 + 2]), 0.f), score);
+                    score = fmaf(wv.w, fmaxf(u2f(r[4 * h4 + 3]), 0.f), score);
+                }
+                const bool vis = qok[ii] && s <= qpos[ii];
+                if (vis) a.scores[static_cast<int64_t>(g * G + i) * a.ld + s] = score;
+                if (fuse_hist) hist_add_warp(ehist, vis ? first_digit(order_key(score)) : 0xFFFFFFFFu);
             }
+            hist_dirty = true;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tmem_empty[acc]);
             ++k_tiles;
         }
+        if (fuse_hist && hist_dirty && !abort_flag) flush_hist(cur_g);
     }
 
     tc_fence_before();
@@ -323,7 +375,7 @@ cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcA
     cudaError_t e = cudaFuncSetAttribute(idx_score_tc_kernel<G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     if (e != cudaSuccess) return e;
-    idx_score_tc_kernel<G><<<grid, kIdxThreads, Cfg::kSmem, st>>>(tk, tq, a);
+    idx_score_tc_kernel<G><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(tk, tq, a);
     return cudaGetLastError();
 }
 

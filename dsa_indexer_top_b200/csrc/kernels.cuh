@@ -7,6 +7,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include "dsa.h"
+
 namespace dsa {
 
 constexpr int kIdxHeads = 32;   // index_n_heads of GLM-5.2
@@ -31,6 +33,8 @@ struct IdxTcArgs {
     int k_shared;         // 1: every query reads cache 0
     int tiles_per_group;  // ceil(L / 128)
     long long total_items;
+    uint32_t *ghist;      // non-null (one query per tile only): accumulate the top-k
+                          // first-digit histogram [n_q][4096] of the scores written
 };
 
 // G = queries per tensor-core tile (1, 2, 4 or 8).  Tensor maps: keys 3-D
@@ -55,8 +59,9 @@ struct IdxGenericArgs {
 cudaError_t launch_idx_score_generic(const IdxGenericArgs &a, cudaStream_t st);
 
 // ------------------------------------------------------------------ top-k
-constexpr int kTopkRowMaxCtx = 65536;      // contexts up to this use one CTA per query
-constexpr int kTopkSplitMaxQueries = 64;   // longer contexts with at most this many queries split rows
+constexpr int kTopkBins = 4096;            // first radix digit: 12 bits
+constexpr int kTopkSplitMinCtx = 8192;     // contexts above this, with at most
+constexpr int kTopkSplitMaxQueries = 64;   // this many queries, split rows over CTAs
 constexpr int kSplitMax = 64;              // chunks per query (split schedule)
 constexpr int kSplitCap = 1024;            // candidates stored per chunk
 
@@ -68,7 +73,8 @@ struct TopkArgs {
     int32_t *cnt;
     uint32_t *status;
     int n_q, L, topk;
-    // split-schedule scratch (workspace)
+    int hist_ready;    // ghist already holds the first-digit histograms (indexer epilogue)
+    // scratch (workspace)
     uint32_t *ghist;   // [n_q][4096] first-digit histogram
     uint32_t *gcount;  // [n_q][kSplitMax] candidates per chunk
     uint2 *gcand;      // [n_q][kSplitMax][kSplitCap] (key, position)
@@ -77,6 +83,8 @@ bool topk_uses_split(int n_q, int max_ctx);
 size_t topk_scratch_bytes(int n_q, int max_ctx);
 void topk_bind_scratch(TopkArgs &a, void *scratch);
 cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st);
+// First-digit histograms only (into a.ghist, which must be zeroed), every query.
+cudaError_t launch_topk_hist(const TopkArgs &a, int num_sms, cudaStream_t st);
 
 // ------------------------------------------------------------------ sparse MLA
 struct MlaLayerPtrs {

@@ -42,7 +42,11 @@ constexpr int kCBytes = kBlocks * kCBlockBytes;        // 144 KB
 constexpr int kMlaSmem = kQBytes + kCBytes + 1024;
 constexpr int kTmemCols = 512;                          // S: 0..63, O: 64..319
 constexpr uint32_t kIdescS = idesc_bf16(128, 64, false, false);
-constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, false);
+constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, true);
+// A running maximum is kept until a head's chunk maximum exceeds it by more than
+// this many powers of two (probabilities stay below 2^8, exact in bf16 range);
+// only then is the accumulated O rescaled.
+constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -70,7 +74,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                                                 ~uintptr_t(1023));
     uint8_t *q_sm = smem;
     uint8_t *c_sm = smem + kQBytes;
-    uint8_t *p_sm = c_sm + 8 * kCBlockBytes;  // P^T reuses the RoPE block after the S-MMA
+    uint8_t *p_sm = c_sm + 8 * kCBlockBytes;  // P reuses the RoPE block after the S-MMA
 
     __shared__ uint64_t bar_s, bar_o;
     __shared__ uint32_t tmem_base_sh;
@@ -78,7 +82,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     __shared__ int need_rescale;
     __shared__ int row_idx[kRowsPerChunk];
     __shared__ float red[4][kMlaHeads];
-    __shared__ float m_run[kMlaHeads], l_run[kMlaHeads], alpha[kMlaHeads];
+    __shared__ float m_run[kMlaHeads], l_run[kMlaHeads], alpha[kMlaHeads], inv_l[kMlaHeads];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, i = blockIdx.y, layer = blockIdx.z;
@@ -121,32 +125,39 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(lp.q) + static_cast<int64_t>(i) * kMlaHeads * kRow;
     const uint32_t q_addr = smem_u32(q_sm), c_addr = smem_u32(c_sm), p_addr = smem_u32(p_sm);
 
+    // the query tile does not depend on the selection: start its copy first
+    if (c_begin < c_end) {
+        for (int f = tid; f < kMlaHeads * (kRow / 8); f += kMlaThreads) {
+            const int h = f / (kRow / 8), ch = f % (kRow / 8);
+            cp_async_16(q_addr + (ch >> 3) * kQBlockBytes + sw128_offset(h, ch & 7), q + h * kRow + ch * 8);
+        }
+        cp_async_commit();
+    }
+    // row index of selected slot j of this query (-1: none or out of range)
+    auto load_idx = [&](int c) -> int {
+        const int j = c * kRowsPerChunk + tid;
+        int r = -1;
+        if (j < cnt) {
+            r = a.idx[static_cast<int64_t>(i) * a.topk + j];
+            if (r < 0 || r >= a.L) {
+                report_status(a.status, DSA_ERR_INVALID);
+                r = -1;
+            }
+        }
+        return r;
+    };
+    int pending = (tid < kRowsPerChunk && c_begin < c_end) ? load_idx(c_begin) : -1;
+
     int done = 0;  // chunks whose O-MMA was issued
     for (int c = c_begin; c < c_end; ++c, ++done) {
         const bool first = (c == c_begin);
         // ---- 1. row indices of this chunk (previous O-MMA must be done with C)
         if (!first && !mbar_wait(&bar_o, (done - 1) & 1, a.status, &abort_flag)) break;
-        if (tid < kRowsPerChunk) {
-            const int j = c * kRowsPerChunk + tid;
-            int r = -1;
-            if (j < cnt) {
-                r = a.idx[static_cast<int64_t>(i) * a.topk + j];
-                if (r < 0 || r >= a.L) {
-                    report_status(a.status, DSA_ERR_INVALID);
-                    r = -1;
-                }
-            }
-            row_idx[tid] = r;
-        }
+        if (tid < kRowsPerChunk) row_idx[tid] = pending;
         __syncthreads();
-        // ---- 2. gather rows (and the query tile on the first chunk)
-        if (first) {
-            for (int f = tid; f < kMlaHeads * (kRow / 8); f += kMlaThreads) {
-                const int h = f / (kRow / 8), ch = f % (kRow / 8);
-                cp_async_16(q_addr + (ch >> 3) * kQBlockBytes + sw128_offset(h, ch & 7),
-                            q + h * kRow + ch * 8);
-            }
-        }
+        // the next chunk's indices load while this chunk is gathered and computed
+        if (tid < kRowsPerChunk && c + 1 < c_end) pending = load_idx(c + 1);
+        // ---- 2. gather the chunk's rows
         for (int f = tid; f < kRowsPerChunk * (kRow / 8); f += kMlaThreads) {
             const int r = f / (kRow / 8), ch = f % (kRow / 8);
             const uint32_t dst = c_addr + (ch >> 3) * kCBlockBytes + sw128_offset(r, ch & 7);
@@ -166,7 +177,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             tc_fence_after();
 #pragma unroll
             for (int kk = 0; kk < kRow / 16; ++kk) {
-                const uint32_t koff = (kk >> 2) * 0 + (kk & 3) * 32;
+                const uint32_t koff = (kk & 3) * 32;
                 const uint64_t ad = sdesc_sw128(c_addr + (kk >> 2) * kCBlockBytes + koff, 16, 1024);
                 const uint64_t bd = sdesc_sw128(q_addr + (kk >> 2) * kQBlockBytes + koff, 16, 1024);
                 umma_bf16(tbase, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
@@ -174,56 +185,66 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             umma_commit(&bar_s);
         }
         // ---- 4. softmax over the chunk's rows, per head
-        float v[64];
-        const int row = warp * 32 + lane;  // warps 0-3 only
+        const int row = warp * 32 + lane;  // warps 0-3: one selected row per thread
+        const uint32_t s_taddr = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
         if (warp < 4) {
-            if (!mbar_wait(&bar_s, done & 1, a.status, &abort_flag)) {
-                // fall through with masked values; the CTA aborts below
-            }
+            mbar_wait(&bar_s, done & 1, a.status, &abort_flag);  // on timeout the CTA aborts below
             tc_fence_after();
-            uint32_t r0[32], r1[32];
-            const uint32_t ta = tbase + (static_cast<uint32_t>(warp * 32) << 16);
-            tmem_ld32(ta, r0);
-            tmem_ld32(ta + 32, r1);
-            tmem_ld_wait();
-            const bool valid = row_idx[row] >= 0;
+            float v[64];
+            {
+                uint32_t r0[32], r1[32];
+                tmem_ld32(s_taddr, r0);
+                tmem_ld32(s_taddr + 32, r1);
+                tmem_ld_wait();
+                const bool valid = row_idx[row] >= 0;
 #pragma unroll
-            for (int h = 0; h < 32; ++h) {
-                v[h] = valid ? u2f(r0[h]) : -INFINITY;
-                v[h + 32] = valid ? u2f(r1[h]) : -INFINITY;
+                for (int h = 0; h < 32; ++h) {
+                    v[h] = valid ? u2f(r0[h]) : -INFINITY;
+                    v[h + 32] = valid ? u2f(r1[h]) : -INFINITY;
+                }
             }
-            float t[64];
-#pragma unroll
-            for (int h = 0; h < 64; ++h) t[h] = v[h];
-            warp_transpose_reduce<true>(t, lane);
-            red[warp][2 * lane] = t[0];
-            red[warp][2 * lane + 1] = t[1];
+            warp_transpose_reduce<true>(v, lane);
+            red[warp][2 * lane] = v[0];
+            red[warp][2 * lane + 1] = v[1];
         }
         __syncthreads();
         if (abort_flag) break;
         if (tid < kMlaHeads) {
             const float mc = fmaxf(fmaxf(red[0][tid], red[1][tid]), fmaxf(red[2][tid], red[3][tid]));
             const float m_old = m_run[tid];
-            const float m_new = fmaxf(m_old, mc);
             float al = 1.f;
-            if (m_new != -INFINITY && m_old != m_new) al = (m_old == -INFINITY) ? 0.f : exp2f((m_old - m_new) * c2);
+            if (mc != -INFINITY && (m_old == -INFINITY || (mc - m_old) * c2 > kRescaleLog2)) {
+                al = (m_old == -INFINITY) ? 0.f : exp2f((m_old - mc) * c2);
+                m_run[tid] = mc;
+                if (!first) need_rescale = 1;
+            }
             alpha[tid] = al;
-            m_run[tid] = m_new;
-            if (!first && al != 1.f) need_rescale = 1;
         }
         __syncthreads();
         if (warp < 4) {
-            const int kb = row >> 6;
-            const uint32_t sub = (row & 63) >> 3;
-            const uint32_t byte_in = (row & 7) * 2;
+            // P[row][head] (bf16, 128-byte swizzled rows: the MN-major B operand)
+            uint32_t r0[32], r1[32];
+            tmem_ld32(s_taddr, r0);
+            tmem_ld32(s_taddr + 32, r1);
+            tmem_ld_wait();
+            const bool valid = row_idx[row] >= 0;
+            float v[64];
 #pragma unroll
             for (int h = 0; h < 64; ++h) {
+                const float sv = u2f(h < 32 ? r0[h] : r1[h - 32]);
                 const float m = m_run[h];
-                float p = (v[h] == -INFINITY) ? 0.f : exp2f((v[h] - m) * c2);
-                const __nv_bfloat16 pb = __float2bfloat16_rn(p);
-                v[h] = __bfloat162float(pb);  // the sum uses the rounded value the MMA sees
-                const uint32_t off = kb * kQBlockBytes + sw128_offset(h, sub) + byte_in;
-                *reinterpret_cast<__nv_bfloat16 *>(p_sm + off) = pb;
+                const float pf = (!valid || m == -INFINITY) ? 0.f : exp2f((sv - m) * c2);
+                v[h] = pf;
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                __align__(16) __nv_bfloat16 pb[8];
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {
+                    pb[x] = __float2bfloat16_rn(v[8 * j + x]);
+                    v[8 * j + x] = __bfloat162float(pb[x]);  // the sum uses the value the MMA sees
+                }
+                *reinterpret_cast<uint4 *>(p_sm + sw128_offset(row, j)) = *reinterpret_cast<const uint4 *>(pb);
             }
             warp_transpose_reduce<false>(v, lane);
             red[warp][2 * lane] = v[0];
@@ -262,7 +283,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
 #pragma unroll
                 for (int kk = 0; kk < kRowsPerChunk / 16; ++kk) {
                     const uint64_t ad = sdesc_sw128(c_addr + 2 * mt * kCBlockBytes + kk * 2048, kCBlockBytes, 1024);
-                    const uint64_t bd = sdesc_sw128(p_addr + (kk >> 2) * kQBlockBytes + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = sdesc_sw128(p_addr + kk * 2048, kCBlockBytes, 1024);
                     umma_bf16(tbase + 64 + mt * 64, ad, bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
                 }
             }
@@ -270,9 +291,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
         }
     }
 
-    if (done > 0 && !abort_flag) {
+    __syncthreads();  // every thread has left the loop: `go` is uniform
+    const bool go = done > 0 && !abort_flag;
+    if (go) {
+        if (tid < kMlaHeads) inv_l[tid] = 1.f / l_run[tid];
         mbar_wait(&bar_o, (done - 1) & 1, a.status, &abort_flag);
         tc_fence_after();
+        __syncthreads();
         const int quad = warp & 3;
         const int mt0 = (warp < 4) ? 0 : 2;
         const bool final_out = (a.n_splits == 1);
@@ -288,7 +313,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
 #pragma unroll
                     for (int x = 0; x < 32; ++x) {
                         const int h = half * 32 + x;
-                        o[h * kLatent + d] = __float2bfloat16_rn(u2f(r[x]) / l_run[h]);
+                        o[h * kLatent + d] = __float2bfloat16_rn(u2f(r[x]) * inv_l[h]);
                     }
                 } else {
                     float *po = a.part_o + ((static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits + split) * kMlaHeads * kLatent;
@@ -326,19 +351,27 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
     const int nch = (cnt + kRowsPerChunk - 1) / kRowsPerChunk;
     const int ns = (nch + a.chunks_per_cta - 1) / a.chunks_per_cta;
     const int64_t base = (static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits;
-    if (threadIdx.x < 4) {
-        const int h = hg * 4 + threadIdx.x;
-        float M = -INFINITY;
-        for (int s = 0; s < ns; ++s) M = fmaxf(M, a.part_ml[((base + s) * kMlaHeads + h) * 2]);
-        float L = 0.f;
-        for (int s = 0; s < ns; ++s) {
-            const float *ml = a.part_ml + ((base + s) * kMlaHeads + h) * 2;
-            const float wv = (ml[0] == -INFINITY) ? 0.f : exp2f(ml[0] - M);
-            wgt[threadIdx.x][s] = wv;
-            L += wv * ml[1];
+    // (max, sum) of every split for the 4 heads: one thread per (head, split)
+    {
+        const int hl = threadIdx.x >> 5, s = threadIdx.x & 31;  // warps 0-3: one head each
+        if (hl < 4) {
+            const int h = hg * 4 + hl;
+            float m = -INFINITY, l = 0.f;
+            if (s < ns) {
+                const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + ((base + s) * kMlaHeads + h) * 2);
+                m = ml.x;
+                l = ml.y;
+            }
+            float M = m;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+            const float wv = (m == -INFINITY) ? 0.f : exp2f(m - M);
+            float L = wv * l;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+            if (s < ns) wgt[hl][s] = wv / L;
+            if (s == 0 && lp.lse) lp.lse[static_cast<int64_t>(i) * kMlaHeads + h] = (M + log2f(L)) * kLn2;
         }
-        for (int s = 0; s < ns; ++s) wgt[threadIdx.x][s] /= L;
-        if (lp.lse) lp.lse[static_cast<int64_t>(i) * kMlaHeads + h] = (M + log2f(L)) * kLn2;
     }
     __syncthreads();
     // 4 heads x 512 dims = 2048 outputs, 8 per thread
@@ -346,6 +379,7 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
     const int hl = e / kLatent, d = e % kLatent;
     const int h = hg * 4 + hl;
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 8
     for (int s = 0; s < ns; ++s) {
         const float *po = a.part_o + ((base + s) * kMlaHeads + h) * kLatent + d;
         const float4 x0 = *reinterpret_cast<const float4 *>(po);

@@ -226,4 +226,23 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
+// Order-preserving map float -> uint32 (a larger float gives a larger key);
+// -0.0 is folded onto +0.0 so the two compare equal.  The top-k radix select
+// and the indexer's fused first-digit histogram both use it.
+__device__ __forceinline__ uint32_t order_key(float f) {
+    uint32_t b = __float_as_uint(f);
+    if (b == 0x80000000u) b = 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// First radix digit of a key (12 bits; kTopkBins histogram bins).
+__device__ __forceinline__ uint32_t first_digit(uint32_t key) { return key >> 20; }
+
+// Add one to hist[d] for every lane with d != ~0u, one atomic per distinct
+// digit in the warp.  Every lane of the warp must call it.
+__device__ __forceinline__ void hist_add_warp(uint32_t *hist, uint32_t d) {
+    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+    if (d != 0xFFFFFFFFu && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+}
+
 }  // namespace dsa

@@ -74,6 +74,22 @@ typedef enum {
 
 typedef enum { DSA_BF16 = 0, DSA_F32 = 1 } dsa_dtype;
 
+/* Flags of dsa_indexer.flags and of dsa_topk. */
+enum {
+    /* dsa_indexer.flags: dsa_index_scores also leaves, in the workspace, the
+     * per-query histogram of the first radix digit of the scores it wrote (the
+     * first pass of dsa_topk; on the tensor-core path it is built in the
+     * epilogue at no extra pass).  The workspace must then be at least
+     * dsa_workspace_bytes(DSA_OP_TOPK, ...) bytes.  Honoured only when
+     * queries->seq_run is odd (queries not tiled together); ignored otherwise. */
+    DSA_INDEXER_TOPK_HIST = 1,
+    /* dsa_topk flags: the workspace holds that histogram for these scores (the
+     * preceding dsa_index_scores on the same scores, queries and workspace had
+     * DSA_INDEXER_TOPK_HIST), so the top-k skips its own histogram pass.
+     * Ignored, like the indexer flag, when queries->seq_run is even. */
+    DSA_TOPK_HIST_FROM_INDEXER = 1
+};
+
 /* Operation ids for dsa_workspace_bytes. */
 typedef enum {
     DSA_OP_INDEX_SCORES = 0,
@@ -121,7 +137,7 @@ typedef struct {
     int32_t heads;
     int32_t dim;
     int32_t dtype;
-    int32_t reserved;
+    int32_t flags; /* DSA_INDEXER_TOPK_HIST or 0 */
     const void *q;
     const float *w;
     const void *k;
@@ -180,11 +196,12 @@ dsa_status dsa_index_scores(const dsa_queries *queries, const dsa_indexer *index
  *   scores     float32 [n_q][ld_scores] (only s <= q_pos[i] is read),
  *              ld_scores >= max_ctx, multiple of 4, 16-byte aligned base
  *   topk       1 .. 4096
+ *   flags      0, or DSA_TOPK_HIST_FROM_INDEXER (see the flag)
  *   idx        int32 [n_q][topk];  cnt  int32 [n_q]
  */
 dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_scores,
-                    int32_t topk, int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
-                    void *stream);
+                    int32_t topk, int32_t flags, int32_t *idx, int32_t *cnt, void *ws,
+                    size_t ws_bytes, void *stream);
 
 /*
  * Sparse absorbed MLA, decode schedule [TM, Indexer-selected sparse attention;

@@ -46,14 +46,19 @@ def test_workspace_bytes():
     lib = B.lib()
     q = _q(n_q=8, L=32768)
     assert lib.dsa_workspace_bytes(B.DSA_OP_INDEX_SCORES, ctypes.byref(q), 2048, 64, 512, 1) == 256
-    assert lib.dsa_workspace_bytes(B.DSA_OP_TOPK, ctypes.byref(q), 2048, 64, 512, 1) == 256
+    # top-k: status + first-digit histograms + (split schedule: 8 queries, ctx > 8192) chunk candidates
+    hist = 8 * 4096 * 4
+    split = hist + 8 * 64 * 4 + 8 * 64 * 1024 * 8
+    assert lib.dsa_workspace_bytes(B.DSA_OP_TOPK, ctypes.byref(q), 2048, 64, 512, 1) == 256 + split
+    q2 = _q(n_q=8, L=8192)
+    assert lib.dsa_workspace_bytes(B.DSA_OP_TOPK, ctypes.byref(q2), 2048, 64, 512, 1) == 256 + hist
     dec = lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 2048, 64, 512, 1)
     # 16 splits x 8 queries x 64 heads x (512 + 2) floats, 256-aligned, + status
     assert dec == 256 + ((8 * 16 * 64 * 514 * 4 + 255) // 256) * 256
     assert lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 128, 64, 512, 1) == 256
     grp = lib.dsa_workspace_bytes(B.DSA_OP_INDEXSHARE_GROUP, ctypes.byref(q), 2048, 64, 512, 4)
     scores = 8 * 32768 * 4
-    assert grp == 256 + scores + ((4 * 8 * 16 * 64 * 514 * 4 + 255) // 256) * 256
+    assert grp == 256 + scores + split + ((4 * 8 * 16 * 64 * 514 * 4 + 255) // 256) * 256
     assert lib.dsa_workspace_bytes(77, ctypes.byref(q), 2048, 64, 512, 1) == 0
 
 
@@ -113,8 +118,22 @@ def test_workspace_checks():
 def test_topk_rejects_bad_k(topk):
     lib = B.lib()
     q = _q()
-    assert lib.dsa_topk(ctypes.byref(q), 0x9000, 1000, topk, 0xA000, 0xB000, _FakeWs.ptr, _FakeWs.size,
+    assert lib.dsa_topk(ctypes.byref(q), 0x9000, 1000, topk, 0, 0xA000, 0xB000, _FakeWs.ptr, _FakeWs.size,
                         None) == B.DSA_ERR_INVALID
+
+
+def test_flags_validated():
+    lib = B.lib()
+    q = _q()
+    assert lib.dsa_topk(ctypes.byref(q), 0x9000, 1000, 64, 6, 0xA000, 0xB000, _FakeWs.ptr, _FakeWs.size,
+                        None) == B.DSA_ERR_INVALID
+    ix = _idx()
+    ix.flags = 2
+    assert lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(ix), 0x9000, 1000, _FakeWs.ptr, _FakeWs.size,
+                                None) == B.DSA_ERR_INVALID
+    ix.flags = B.DSA_INDEXER_TOPK_HIST   # needs a top-k sized workspace
+    assert lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(ix), 0x9000, 1000, 0x10000, 256,
+                                None) == B.DSA_ERR_WORKSPACE
 
 
 def test_mla_rejects():

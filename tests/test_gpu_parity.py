@@ -46,16 +46,19 @@ def dev(cuda_ok):
     return torch.device("cuda")
 
 
-def _run_steps(w, x, decode=True):
-    """The three-call chain (as timed by the benchmark): scores -> top-k -> MLA."""
+def _run_steps(w, x, decode=True, fused=True):
+    """The three-call chain (as timed by the benchmark): scores -> top-k -> MLA;
+    `fused`: the indexer leaves the top-k's first-digit histograms."""
     q, ix, mlas = C.descriptors(w, x, seq_run=seq_run_of(w))
+    if fused:
+        ix.flags = B.DSA_INDEXER_TOPK_HIST
     dev = x["q_pos"].device
     ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, w.n_layers, dev)
     scores = B.scores_buffer(w.n_q, w.L, dev)
     B.dsa_index_scores(q, ix, scores, ws)
     idx = torch.full((w.n_q, w.topk), -7, dtype=torch.int32, device=dev)
     cnt = torch.full((w.n_q,), -7, dtype=torch.int32, device=dev)
-    B.dsa_topk(q, scores, w.topk, idx, cnt, ws)
+    B.dsa_topk(q, scores, w.topk, idx, cnt, ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER if fused else 0)
     for m in mlas:
         (B.dsa_sparse_mla_decode if decode else B.dsa_sparse_mla_prefill)(q, m, idx, cnt, w.topk, ws)
     assert B.dsa_check_status(ws) == B.DSA_OK
@@ -80,12 +83,12 @@ def test_index_scores_bit_exact(dev, name):
 
 
 @pytest.mark.parametrize("name", list(SMALL))
-@pytest.mark.parametrize("decode", [True, False])
-def test_chain_matches_oracle(dev, name, decode):
+@pytest.mark.parametrize("decode,fused", [(True, True), (False, True), (True, False)])
+def test_chain_matches_oracle(dev, name, decode, fused):
     w = SMALL[name]
     xh = wl.make_inputs(w)
     x = C.to_device(xh)
-    _, idx, cnt, mlas = _run_steps(w, x, decode=decode)
+    _, idx, cnt, mlas = _run_steps(w, x, decode=decode, fused=fused)
     _, ridx, rcnt = C.oracle_selection(w, xh)
     np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
     np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
