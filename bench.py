@@ -37,8 +37,10 @@ DECODE_MAX_QUERIES = 256    # the MLA decode (split-K) schedule up to this many 
 L2_FLUSH_BYTES = 256 << 20
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch, from the ncu
-# capture summarised under profiles/ (None until captured for the current kernel).
-NCU_INDEXER_TRAFFIC = {}
+# capture summarised in profiles/idx_score_tc_decode_1m.md (one sequence of 1M keys:
+# 276.2 MB; the 4-sequence launch streams 4 such caches, so traffic x 4).  Absent
+# workloads report null.
+NCU_INDEXER_TRAFFIC = {"decode_1m": 4 * 276.2e6}
 
 
 def measured_peaks():
@@ -308,6 +310,12 @@ def max_over_ranks(value: float, world: int, dev) -> float:
     return float(t.item())
 
 
+def weak_scaling_value(world: int, n_q: int, n_layers: int, steps: int, tot_ms_max: float) -> float:
+    """Whole-job query-tokens/s per layer: every rank processed its own batch of
+    n_q queries x n_layers layers per step; the time is the slowest rank's."""
+    return world * n_q * n_layers * steps / (tot_ms_max * 1e-3)
+
+
 def barrier(world):
     if world > 1:
         import torch.distributed as dist
@@ -401,7 +409,7 @@ def main():
     tot_max = max_over_ranks(tot, world, dev)
 
     ms_per_step = tot_max / args.steps
-    value = world * w.n_q * w.n_layers * args.steps / (tot_max * 1e-3)
+    value = weak_scaling_value(world, w.n_q, w.n_layers, args.steps, tot_max)
     hbm_peak, tc_peak, peak_kind = measured_peaks()
     by = path_bytes(w, step.seq_run)
     idx_ms = idx_t / args.steps
