@@ -276,18 +276,17 @@ dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, co
     bool tc = true;
     for (int l = 0; l < n_layers; ++l) tc = tc && mla_tc_ok(&layers[l]);
     if (tc) {
-        const int nch = decode_splits(topk);
-        if (decode && nch > 1) {
-            a.n_splits = nch;
-            a.chunks_per_cta = 1;
+        int n_splits, cpc;
+        mla_plan(qs->n_q, n_layers, topk, decode, num_sms_current(), n_splits, cpc);
+        a.n_splits = n_splits;
+        a.chunks_per_cta = cpc;
+        if (n_splits > 1) {
             a.part_o = reinterpret_cast<float *>(scratch);
-            const size_t rows = static_cast<size_t>(n_layers) * qs->n_q * nch * kMlaHeads;
+            const size_t rows = static_cast<size_t>(n_layers) * qs->n_q * n_splits * kMlaHeads;
             a.part_ml = reinterpret_cast<float *>(scratch + rows * kLatent * sizeof(float));
             if (launch_mla_tc(a, st) != cudaSuccess) return DSA_ERR_CUDA;
             return launch_mla_combine(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
         }
-        a.n_splits = 1;
-        a.chunks_per_cta = nch;
         return launch_mla_tc(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
     }
     const size_t smem = sizeof(float) * (static_cast<size_t>(m.d_latent + m.d_rope) + topk);

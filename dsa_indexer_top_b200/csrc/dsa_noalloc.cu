@@ -96,16 +96,20 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
     a.scale = m.scale;
     a.is_bf16 = 1;
     a.status = reinterpret_cast<uint32_t *>(scratch);
-    if (n_splits > 1) {
-        a.n_splits = n_splits;
-        a.chunks_per_cta = 1;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    int plan_splits, cpc;
+    mla_plan(queries->n_q, 1, topk, true, sms, plan_splits, cpc);
+    a.n_splits = plan_splits;
+    a.chunks_per_cta = cpc;
+    if (plan_splits > 1) {
         a.part_o = reinterpret_cast<float *>(scratch + kStatusBytes);
-        const size_t rows = static_cast<size_t>(queries->n_q) * n_splits * kMlaHeads;
+        const size_t rows = static_cast<size_t>(queries->n_q) * plan_splits * kMlaHeads;
         a.part_ml = reinterpret_cast<float *>(scratch + kStatusBytes + rows * kLatent * sizeof(float));
         if (launch_mla_tc(a, st) != cudaSuccess) return DSA_ERR_CUDA;
         return launch_mla_combine(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
     }
-    a.n_splits = 1;
-    a.chunks_per_cta = n_splits;
     return launch_mla_tc(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

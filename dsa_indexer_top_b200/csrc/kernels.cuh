@@ -17,7 +17,8 @@ constexpr int kMlaHeads = 64;   // num_attention_heads of GLM-5.2
 constexpr int kLatent = 512;    // kv_lora_rank
 constexpr int kRope = 64;       // qk_rope_head_dim
 constexpr int kRow = kLatent + kRope;
-constexpr int kRowsPerChunk = 128;  // selected rows per tensor-core chunk
+constexpr int kRowsPerChunk = 128;  // rows per split of the workspace bound (ceil(topk / 128) splits)
+constexpr int kMlaChunk = 64;       // selected rows per tensor-core pipeline chunk
 constexpr int kMaxTopk = 4096;
 constexpr int kMaxLayers = 4;
 
@@ -119,6 +120,24 @@ struct MlaArgs {
 cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st);
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st);
 cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st);
+
+// Split-K plan of the tensor-core MLA: n_splits CTAs per query, each walking
+// cpc chunks of 64 selected rows.  Decode spreads a query over up to 16 CTAs
+// (about one CTA per SM over the batch, at least two chunks each); prefill uses
+// one CTA per query (n_splits = 1: the final output is written directly).
+inline void mla_plan(int n_q, int n_layers, int topk, bool decode, int num_sms, int &n_splits, int &cpc) {
+    const int nch = (topk + kMlaChunk - 1) / kMlaChunk;
+    int s = 1;
+    if (decode) {
+        const int work = n_q * n_layers > 0 ? n_q * n_layers : 1;
+        s = num_sms / work;
+        s = s < 1 ? 1 : (s > 16 ? 16 : s);
+        const int half = nch / 2 > 0 ? nch / 2 : 1;
+        s = s > half ? half : s;
+    }
+    cpc = (nch + s - 1) / s;
+    n_splits = (nch + cpc - 1) / cpc;
+}
 
 // Bytes of split-K partials for the tensor-core decode schedule.
 inline size_t mla_partial_bytes(int n_layers, int n_q, int n_splits) {

@@ -8,23 +8,26 @@
 // Multi-head latent attention -- 512-dim latent + 64-dim RoPE key per token;
 // Learnable attention sink -- plain float32 softmax, no sink.)
 //
-// Tensor-core path (bf16, 64 heads, 512 + 64), one CTA of 8 warps per (query,
-// split, layer), 128 selected rows per chunk:
-//   gather   the chunk's 128 rows (1152 B each) are copied with 16-byte cp.async
-//            into nine 64-column blocks of 128-byte-swizzled shared memory; the
-//            query's 64 x 576 tile likewise, once per CTA.
-//   S-MMA    S^T[128 rows][64 heads] = C (M = 128, K-major) x Q^T (N = 64,
-//            K-major), K = 576: 36 tcgen05.mma, fp32 in TMEM columns 0..63.
-//   softmax  warps 0-3 read one row each from TMEM; per-head maxima and sums
-//            across the 128 rows by a shuffle transpose-reduction and a 4-warp
-//            combine; P (bf16) is written into the freed RoPE block.
-//   O-MMA    O^T[512 dims][64 heads] += C_lat^T (M = 4 x 128, MN-major view of
-//            the same tile) x P^T (N = 64, K-major), K = 128 rows: 32 MMAs into
-//            TMEM columns 64..319.  Several chunks per CTA use an online softmax
-//            (O rescaled in TMEM when a head's maximum grows).
-//   epilogue all 8 warps read O^T from TMEM; either the final bf16 output
-//            (one CTA per query) or fp32 partials + (max, sum) for a split-K
-//            merge (decode: several CTAs per query).
+// Tensor-core path (bf16, 64 heads, 512 + 64): one CTA per (query, split,
+// layer) walks its share of the selected rows in chunks of 64, software-pipelined
+// across warp roles with mbarriers (every wait bounded):
+//   producers (warps 4-7)  gather chunk c+1 -- 64 rows x 1152 B by 16-byte
+//            cp.async into nine 64-column blocks of 128-byte-swizzled shared
+//            memory -- into one of two 72 KB slots while chunk c is computed;
+//            the 64 x 576 query tile once per CTA.
+//   MMA issuer (warp 8)   S = Q . C^T (M = 64 heads, N = 64 rows, K = 576, both
+//            operands K-major): 36 tcgen05.mma into TMEM columns 64*slot; then
+//            O^T += C_lat^T . P^T (the row tile read MN-major: M = 4 x 128 latent
+//            dims, N = 64 heads, K = 64 rows) into columns 128..383.
+//   softmax (warps 0-3)   thread lane < 16 of warp w owns head 16w + lane (the
+//            M = 64 accumulator layout keeps rows 16w..16w+15 in lanes
+//            32w..32w+15): running max, exponentials and sum of its head over
+//            the chunk's 64 rows in registers; P (bf16) as one 128-byte line per
+//            head in the slot's freed RoPE block; the accumulated O is rescaled
+//            only when a head's maximum grows by more than 2^8.
+//   epilogue (warps 0-7)  reads O^T from TMEM: the final bf16 output (one CTA
+//            per query) or fp32 partials + (max, sum) per head for a split-K
+//            merge (decode with few queries).
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"
@@ -33,56 +36,38 @@
 namespace dsa {
 namespace {
 
-constexpr int kMlaThreads = 256;
-constexpr int kQBlockBytes = kMlaHeads * 128;          // 64 heads x 64 dims bf16 = 8 KB
-constexpr int kCBlockBytes = kRowsPerChunk * 128;      // 128 rows x 64 dims bf16 = 16 KB
-constexpr int kBlocks = kRow / 64;                     // 9 column blocks (8 latent + rope)
-constexpr int kQBytes = kBlocks * kQBlockBytes;        // 72 KB
-constexpr int kCBytes = kBlocks * kCBlockBytes;        // 144 KB
-constexpr int kMlaSmem = kQBytes + kCBytes + 1024;
-constexpr int kTmemCols = 512;                          // S: 0..63, O: 64..319
-constexpr uint32_t kIdescS = idesc_bf16(128, 64, false, false);
-constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, true);
+constexpr int kChunk = 64;                          // selected rows per pipeline chunk
+constexpr int kMlaThreads = 288;                    // 4 softmax + 4 producer + 1 MMA warp
+constexpr int kBlockBytes = kChunk * 128;           // 64 rows (or heads) x 64 dims bf16 = 8 KB
+constexpr int kBlocks = kRow / 64;                  // 9 column blocks (8 latent + rope)
+constexpr int kSlotBytes = kBlocks * kBlockBytes;   // 72 KB: one chunk of rows
+constexpr int kQBytes = kBlocks * kBlockBytes;      // 72 KB: 64 heads x 576
+constexpr int kMlaSmem = kQBytes + 2 * kSlotBytes + 1024;
+constexpr int kTmemCols = 512;                      // S slots: 0..127, O^T: 128..383
+constexpr int kOCol = 128;
+constexpr uint32_t kIdescS = idesc_bf16(64, 64, false, false);
+constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, false);
 // A running maximum is kept until a head's chunk maximum exceeds it by more than
-// this many powers of two (probabilities stay below 2^8, exact in bf16 range);
-// only then is the accumulated O rescaled.
+// this many powers of two (probabilities stay below 2^8); only then is the
+// accumulated O rescaled.
 constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-
-// Transpose-reduction inside a warp: on entry lane L holds v[0..63] (one value
-// per head for its row); on exit v[0], v[1] hold the reduction over the warp's
-// 32 rows for heads 2L and 2L+1.
-template <bool kMax>
-__device__ __forceinline__ void warp_transpose_reduce(float (&v)[64], int lane) {
-#pragma unroll
-    for (int o = 16, half = 32; o >= 1; o >>= 1, half >>= 1) {
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int j = 0; j < half; ++j) {
-            const float send = upper ? v[j] : v[j + half];
-            const float keep = upper ? v[j + half] : v[j];
-            const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-            v[j] = kMax ? fmaxf(keep, recv) : keep + recv;
-        }
-    }
-}
 
 __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint8_t *q_sm = smem;
-    uint8_t *c_sm = smem + kQBytes;
-    uint8_t *p_sm = c_sm + 8 * kCBlockBytes;  // P reuses the RoPE block after the S-MMA
+    uint8_t *slot_sm = smem + kQBytes;  // slot s at slot_sm + s * kSlotBytes
 
-    __shared__ uint64_t bar_s, bar_o;
+    // o_done[s]: the O-MMA of the chunk in slot s completed (the slot may be refilled)
+    __shared__ uint64_t q_full, slot_full[2], s_full[2], p_full[2], o_done[2], fin, sm_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
-    __shared__ int need_rescale;
-    __shared__ int row_idx[kRowsPerChunk];
-    __shared__ float red[4][kMlaHeads];
-    __shared__ float m_run[kMlaHeads], l_run[kMlaHeads], alpha[kMlaHeads], inv_l[kMlaHeads];
+    __shared__ int row_idx[2][kChunk];
+    __shared__ float alpha_sm[kMlaHeads], m_fin[kMlaHeads], l_fin[kMlaHeads], inv_l[kMlaHeads];
+    __shared__ int rescale_w[4];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int split = blockIdx.x, i = blockIdx.y, layer = blockIdx.z;
@@ -90,20 +75,21 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     const float c2 = a.scale * kLog2e;
 
     if (tid == 0) {
-        mbar_init(&bar_s, 1);
-        mbar_init(&bar_o, 1);
+        mbar_init(&q_full, 4);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&slot_full[s], 4);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&p_full[s], 4);
+            mbar_init(&o_done[s], 1);
+        }
+        mbar_init(&fin, 1);
+        mbar_init(&sm_bar, 4);
         abort_flag = 0;
-        need_rescale = 0;
         fence_barrier_init();
     }
-    if (warp == 0) {
+    if (warp == 8) {
         tmem_alloc(&tmem_base_sh, kTmemCols);
         tmem_relinquish();
-    }
-    if (tid < kMlaHeads) {
-        m_run[tid] = -INFINITY;
-        l_run[tid] = 0.f;
-        alpha[tid] = 1.f;
     }
     tc_fence_before();
     __syncthreads();
@@ -112,229 +98,269 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
 
     int seq = a.q_seq[i];
     int cnt = a.cnt[i];
-    bool ok = seq >= 0 && seq < a.n_seq && cnt >= 0 && cnt <= a.topk;
-    if (!ok) {
+    if (!(seq >= 0 && seq < a.n_seq && cnt >= 0 && cnt <= a.topk)) {
         if (tid == 0) report_status(a.status, DSA_ERR_INVALID);
         cnt = 0;
         seq = 0;
     }
-    const int nch = (cnt + kRowsPerChunk - 1) / kRowsPerChunk;
+    const int nch = (cnt + kChunk - 1) / kChunk;
     const int c_begin = split * a.chunks_per_cta;
-    const int c_end = min(c_begin + a.chunks_per_cta, nch);
+    const int nloc = max(0, min(c_begin + a.chunks_per_cta, nch) - c_begin);
     const __nv_bfloat16 *kv = static_cast<const __nv_bfloat16 *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(lp.q) + static_cast<int64_t>(i) * kMlaHeads * kRow;
-    const uint32_t q_addr = smem_u32(q_sm), c_addr = smem_u32(c_sm), p_addr = smem_u32(p_sm);
+    const uint32_t q_addr = smem_u32(q_sm);
 
-    // the query tile does not depend on the selection: start its copy first
-    if (c_begin < c_end) {
-        for (int f = tid; f < kMlaHeads * (kRow / 8); f += kMlaThreads) {
-            const int h = f / (kRow / 8), ch = f % (kRow / 8);
-            cp_async_16(q_addr + (ch >> 3) * kQBlockBytes + sw128_offset(h, ch & 7), q + h * kRow + ch * 8);
-        }
-        cp_async_commit();
-    }
-    // row index of selected slot j of this query (-1: none or out of range)
-    auto load_idx = [&](int c) -> int {
-        const int j = c * kRowsPerChunk + tid;
-        int r = -1;
-        if (j < cnt) {
-            r = a.idx[static_cast<int64_t>(i) * a.topk + j];
-            if (r < 0 || r >= a.L) {
-                report_status(a.status, DSA_ERR_INVALID);
-                r = -1;
+    if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------ producers
+        const int pw = warp - 4;  // rows (and, once, heads) 16*pw .. 16*pw+15
+        for (int t = 0; t < nloc; ++t) {
+            const int c = c_begin + t, s = t & 1, u = t >> 1;
+            if (t >= 2 && !mbar_wait(&o_done[s], (u - 1) & 1, a.status, &abort_flag)) break;
+            const int rl = 16 * pw + (lane & 15);
+            const int j = c * kChunk + rl;
+            int r = -1;
+            if (j < cnt) {
+                r = a.idx[static_cast<int64_t>(i) * a.topk + j];
+                if (r < 0 || r >= a.L) {
+                    report_status(a.status, DSA_ERR_INVALID);
+                    r = -1;
+                }
             }
-        }
-        return r;
-    };
-    int pending = (tid < kRowsPerChunk && c_begin < c_end) ? load_idx(c_begin) : -1;
-
-    int done = 0;  // chunks whose O-MMA was issued
-    for (int c = c_begin; c < c_end; ++c, ++done) {
-        const bool first = (c == c_begin);
-        // ---- 1. row indices of this chunk (previous O-MMA must be done with C)
-        if (!first && !mbar_wait(&bar_o, (done - 1) & 1, a.status, &abort_flag)) break;
-        if (tid < kRowsPerChunk) row_idx[tid] = pending;
-        __syncthreads();
-        // the next chunk's indices load while this chunk is gathered and computed
-        if (tid < kRowsPerChunk && c + 1 < c_end) pending = load_idx(c + 1);
-        // ---- 2. gather the chunk's rows
-        for (int f = tid; f < kRowsPerChunk * (kRow / 8); f += kMlaThreads) {
-            const int r = f / (kRow / 8), ch = f % (kRow / 8);
-            const uint32_t dst = c_addr + (ch >> 3) * kCBlockBytes + sw128_offset(r, ch & 7);
-            const int src_row = row_idx[r];
-            if (src_row >= 0) {
-                cp_async_16(dst, kv + static_cast<int64_t>(src_row) * a.kv_row_stride + ch * 8);
-            } else {
-                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
-            }
-        }
-        cp_async_commit();
-        cp_async_wait_all();
-        fence_proxy_async_smem();
-        __syncthreads();
-        // ---- 3. S^T = C . Q^T
-        if (tid == 0) {
-            tc_fence_after();
+            if (lane < 16) row_idx[s][rl] = r;
+            if (t == 0) {
+                for (int hh = 0; hh < 16; ++hh) {
+                    const int h = 16 * pw + hh;
 #pragma unroll
-            for (int kk = 0; kk < kRow / 16; ++kk) {
-                const uint32_t koff = (kk & 3) * 32;
-                const uint64_t ad = sdesc_sw128(c_addr + (kk >> 2) * kCBlockBytes + koff, 16, 1024);
-                const uint64_t bd = sdesc_sw128(q_addr + (kk >> 2) * kQBlockBytes + koff, 16, 1024);
-                umma_bf16(tbase, ad, bd, kIdescS, kk > 0 ? 1u : 0u);
+                    for (int tt = 0; tt < 3; ++tt) {
+                        const int ch = lane + 32 * tt;
+                        if (ch < kRow / 8)
+                            cp_async_16(q_addr + (ch >> 3) * kBlockBytes + sw128_offset(h, ch & 7), q + h * kRow + ch * 8);
+                    }
+                }
             }
-            umma_commit(&bar_s);
+            const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
+            for (int rr = 0; rr < 16; ++rr) {
+                const int row = 16 * pw + rr;
+                const int src = __shfl_sync(0xffffffffu, r, rr);
+#pragma unroll
+                for (int tt = 0; tt < 3; ++tt) {
+                    const int ch = lane + 32 * tt;
+                    if (ch < kRow / 8) {
+                        const uint32_t dst = sb + (ch >> 3) * kBlockBytes + sw128_offset(row, ch & 7);
+                        if (src >= 0)
+                            cp_async_16(dst, kv + static_cast<int64_t>(src) * a.kv_row_stride + ch * 8);
+                        else
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+                    }
+                }
+            }
+            cp_async_commit();
+            cp_async_wait_all();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                if (t == 0) mbar_arrive(&q_full);
+                mbar_arrive(&slot_full[s]);
+            }
         }
-        // ---- 4. softmax over the chunk's rows, per head
-        const int row = warp * 32 + lane;  // warps 0-3: one selected row per thread
-        const uint32_t s_taddr = tbase + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        if (warp < 4) {
-            mbar_wait(&bar_s, done & 1, a.status, &abort_flag);  // on timeout the CTA aborts below
+    } else if (warp == 8) {
+        // ------------------------------------------------------------ MMA issuer
+        // Issues S of chunk ts as soon as its rows are in, and O of chunk to as
+        // soon as its P is written, whichever comes first (ts <= to + 1: S of a
+        // slot is rewritten only after that slot's O was issued).  Bounded.
+        if (lane == 0 && nloc > 0) {
+            bool ok = mbar_wait(&q_full, 0, a.status, &abort_flag);
+            int ts = 0, to = 0;
+            uint64_t t0 = global_timer_ns();
+            uint32_t spin = 0;
+            while (ok && to < nloc) {
+                bool progressed = false;
+                if (ts < nloc && ts <= to + 1 && mbar_test_wait(&slot_full[ts & 1], (ts >> 1) & 1)) {
+                    tc_fence_after();
+                    const int s = ts & 1;
+                    const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
+#pragma unroll
+                    for (int kk = 0; kk < kRow / 16; ++kk) {
+                        const uint32_t koff = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+                        umma_bf16(tbase + 64 * s, sdesc_sw128(q_addr + koff, 16, 1024), sdesc_sw128(sb + koff, 16, 1024),
+                                  kIdescS, kk > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&s_full[s]);
+                    ++ts;
+                    progressed = true;
+                }
+                if (to < ts && mbar_test_wait(&p_full[to & 1], (to >> 1) & 1)) {
+                    tc_fence_after();
+                    const int sp = to & 1;
+                    const uint32_t sb = smem_u32(slot_sm + sp * kSlotBytes);
+                    const uint32_t pb = sb + 8 * kBlockBytes;  // P: the slot's RoPE block
+#pragma unroll
+                    for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+                        for (int kk = 0; kk < kChunk / 16; ++kk) {
+                            umma_bf16(tbase + kOCol + 64 * mt, sdesc_sw128(sb + 2 * mt * kBlockBytes + kk * 2048, kBlockBytes, 1024),
+                                      sdesc_sw128(pb + kk * 32, 16, 1024), kIdescO, (to > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                    umma_commit(&o_done[sp]);
+                    ++to;
+                    progressed = true;
+                }
+                if (progressed) {
+                    t0 = global_timer_ns();
+                    spin = 0;
+                } else if ((++spin & 63u) == 0) {
+                    if (abort_flag) break;
+                    if (global_timer_ns() - t0 > kWaitLimitNs) {
+                        report_status(a.status, DSA_ERR_TIMEOUT);
+                        abort_flag = 1;
+                        break;
+                    }
+                }
+            }
+            umma_commit(&fin);
+            mbar_wait(&fin, 0, a.status, nullptr);  // every MMA of this CTA has completed
+        }
+    } else {
+        // ------------------------------------------------------------ softmax
+        const bool owner = lane < 16;
+        const int h = 16 * warp + (lane & 15);
+        const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
+        float m = -INFINITY, l = 0.f;
+        uint32_t sm_phase = 0;
+        for (int t = 0; t < nloc; ++t) {
+            const int s = t & 1, u = t >> 1;
+            if (!mbar_wait(&slot_full[s], u & 1, a.status, &abort_flag)) break;  // row_idx of the chunk
+            if (!mbar_wait(&s_full[s], u & 1, a.status, &abort_flag)) break;
             tc_fence_after();
-            float v[64];
+            float mc = -INFINITY;
             {
                 uint32_t r0[32], r1[32];
-                tmem_ld32(s_taddr, r0);
-                tmem_ld32(s_taddr + 32, r1);
+                tmem_ld32(lane_base + 64 * s, r0);
+                tmem_ld32(lane_base + 64 * s + 32, r1);
                 tmem_ld_wait();
-                const bool valid = row_idx[row] >= 0;
 #pragma unroll
-                for (int h = 0; h < 32; ++h) {
-                    v[h] = valid ? u2f(r0[h]) : -INFINITY;
-                    v[h + 32] = valid ? u2f(r1[h]) : -INFINITY;
+                for (int x = 0; x < 64; ++x) {
+                    const float v = u2f(x < 32 ? r0[x] : r1[x - 32]);
+                    if (row_idx[s][x] >= 0) mc = fmaxf(mc, v);
                 }
             }
-            warp_transpose_reduce<true>(v, lane);
-            red[warp][2 * lane] = v[0];
-            red[warp][2 * lane + 1] = v[1];
-        }
-        __syncthreads();
-        if (abort_flag) break;
-        if (tid < kMlaHeads) {
-            const float mc = fmaxf(fmaxf(red[0][tid], red[1][tid]), fmaxf(red[2][tid], red[3][tid]));
-            const float m_old = m_run[tid];
             float al = 1.f;
-            if (mc != -INFINITY && (m_old == -INFINITY || (mc - m_old) * c2 > kRescaleLog2)) {
-                al = (m_old == -INFINITY) ? 0.f : exp2f((m_old - mc) * c2);
-                m_run[tid] = mc;
-                if (!first) need_rescale = 1;
+            if (owner && mc != -INFINITY && (m == -INFINITY || (mc - m) * c2 > kRescaleLog2)) {
+                al = (m == -INFINITY) ? 0.f : exp2f((m - mc) * c2);
+                m = mc;
             }
-            alpha[tid] = al;
-        }
-        __syncthreads();
-        if (warp < 4) {
-            // P[row][head] (bf16, 128-byte swizzled rows: the MN-major B operand)
-            uint32_t r0[32], r1[32];
-            tmem_ld32(s_taddr, r0);
-            tmem_ld32(s_taddr + 32, r1);
+            if (owner) alpha_sm[h] = al;
+            const bool need = __any_sync(0xffffffffu, owner && al != 1.f && t > 0);
+            if (lane == 0) rescale_w[warp] = need ? 1 : 0;
+            // the four softmax warps meet: every head's alpha is needed below
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm_bar);
+            if (!mbar_wait(&sm_bar, sm_phase, a.status, &abort_flag)) break;
+            sm_phase ^= 1;
+            const bool any_need = (rescale_w[0] | rescale_w[1] | rescale_w[2] | rescale_w[3]) != 0;
+            if (any_need) {
+                // O is rescaled only after the previous chunk's O-MMA completed.  The
+                // parity wait is exact although most chunks skip it: the producers
+                // observed this barrier's previous phase (chunk t-3) before gathering
+                // chunk t-1 into the same slot, and its next phase needs chunk t+1.
+                const int tp = t - 1;
+                if (!mbar_wait(&o_done[tp & 1], (tp >> 1) & 1, a.status, &abort_flag)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int mt = 0; mt < 4; ++mt) {
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const uint32_t ta = lane_base + kOCol + 64 * mt + 32 * half;
+                        uint32_t r[32];
+                        tmem_ld32(ta, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(u2f(r[x]) * alpha_sm[half * 32 + x]);
+                        tmem_st32(ta, r);
+                    }
+                }
+                tmem_st_wait();
+            }
+            uint32_t r0[32], r1[32];  // the chunk's logits again (cheaper than keeping them live)
+            tmem_ld32(lane_base + 64 * s, r0);
+            tmem_ld32(lane_base + 64 * s + 32, r1);
             tmem_ld_wait();
-            const bool valid = row_idx[row] >= 0;
-            float v[64];
+            if (owner) {
+                uint8_t *pl = slot_sm + s * kSlotBytes + 8 * kBlockBytes;  // this head's P line
+                float sum = 0.f;
 #pragma unroll
-            for (int h = 0; h < 64; ++h) {
-                const float sv = u2f(h < 32 ? r0[h] : r1[h - 32]);
-                const float m = m_run[h];
-                const float pf = (!valid || m == -INFINITY) ? 0.f : exp2f((sv - m) * c2);
-                v[h] = pf;
-            }
+                for (int jc = 0; jc < 8; ++jc) {
+                    __align__(16) __nv_bfloat16 pb[8];
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                __align__(16) __nv_bfloat16 pb[8];
-#pragma unroll
-                for (int x = 0; x < 8; ++x) {
-                    pb[x] = __float2bfloat16_rn(v[8 * j + x]);
-                    v[8 * j + x] = __bfloat162float(pb[x]);  // the sum uses the value the MMA sees
+                    for (int x = 0; x < 8; ++x) {
+                        const int row = 8 * jc + x;
+                        const float v = u2f(row < 32 ? r0[row] : r1[row - 32]);
+                        const float pf = (row_idx[s][row] >= 0) ? exp2f((v - m) * c2) : 0.f;
+                        pb[x] = __float2bfloat16_rn(pf);
+                        sum += __bfloat162float(pb[x]);  // the sum uses the value the MMA sees
+                    }
+                    *reinterpret_cast<uint4 *>(pl + sw128_offset(h, jc)) = *reinterpret_cast<const uint4 *>(pb);
                 }
-                *reinterpret_cast<uint4 *>(p_sm + sw128_offset(row, j)) = *reinterpret_cast<const uint4 *>(pb);
+                l = l * al + sum;
             }
-            warp_transpose_reduce<false>(v, lane);
-            red[warp][2 * lane] = v[0];
-            red[warp][2 * lane + 1] = v[1];
             fence_proxy_async_smem();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[s]);
         }
-        __syncthreads();
-        if (tid < kMlaHeads)
-            l_run[tid] = l_run[tid] * alpha[tid] + (red[0][tid] + red[1][tid]) + (red[2][tid] + red[3][tid]);
-        // ---- rescale the running O when a head's maximum grew
-        if (need_rescale) {
-            const int quad = warp & 3;
-            const int mt0 = (warp < 4) ? 0 : 2;
-            for (int mt = mt0; mt < mt0 + 2; ++mt) {
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    const uint32_t ta = tbase + (static_cast<uint32_t>(quad * 32) << 16) + 64 + mt * 64 + half * 32;
-                    uint32_t r[32];
-                    tmem_ld32(ta, r);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(u2f(r[x]) * alpha[half * 32 + x]);
-                    tmem_st32(ta, r);
-                }
-            }
-            tmem_st_wait();
-        }
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) need_rescale = 0;
-        // ---- 5. O^T += C_lat^T . P^T
-        if (tid == 0) {
-            tc_fence_after();
-#pragma unroll
-            for (int mt = 0; mt < 4; ++mt) {
-#pragma unroll
-                for (int kk = 0; kk < kRowsPerChunk / 16; ++kk) {
-                    const uint64_t ad = sdesc_sw128(c_addr + 2 * mt * kCBlockBytes + kk * 2048, kCBlockBytes, 1024);
-                    const uint64_t bd = sdesc_sw128(p_addr + kk * 2048, kCBlockBytes, 1024);
-                    umma_bf16(tbase + 64 + mt * 64, ad, bd, kIdescO, (!first || kk > 0) ? 1u : 0u);
-                }
-            }
-            umma_commit(&bar_o);
+        if (owner) {
+            m_fin[h] = m;
+            l_fin[h] = l;
         }
     }
 
-    __syncthreads();  // every thread has left the loop: `go` is uniform
-    const bool go = done > 0 && !abort_flag;
+    __syncthreads();  // every role has left its loop: `go` is uniform
+    const bool go = nloc > 0 && !abort_flag;
     if (go) {
-        if (tid < kMlaHeads) inv_l[tid] = 1.f / l_run[tid];
-        mbar_wait(&bar_o, (done - 1) & 1, a.status, &abort_flag);
+        mbar_wait(&fin, 0, a.status, &abort_flag);
         tc_fence_after();
+        if (tid < kMlaHeads) inv_l[tid] = 1.f / l_fin[tid];
         __syncthreads();
-        const int quad = warp & 3;
-        const int mt0 = (warp < 4) ? 0 : 2;
-        const bool final_out = (a.n_splits == 1);
-        for (int mt = mt0; mt < mt0 + 2; ++mt) {
-            const int d = mt * 128 + quad * 32 + lane;
+        if (warp < 8) {
+            const int quad = warp & 3;
+            const int mt0 = (warp < 4) ? 0 : 2;
+            const bool final_out = (a.n_splits == 1);
+            for (int mt = mt0; mt < mt0 + 2; ++mt) {
+                const int d = mt * 128 + quad * 32 + lane;
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                uint32_t r[32];
-                tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + 64 + mt * 64 + half * 32, r);
-                tmem_ld_wait();
-                if (final_out) {
-                    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(lp.out) + static_cast<int64_t>(i) * kMlaHeads * kLatent;
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r[32];
+                    tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + kOCol + mt * 64 + half * 32, r);
+                    tmem_ld_wait();
+                    if (final_out) {
+                        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(lp.out) + static_cast<int64_t>(i) * kMlaHeads * kLatent;
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        const int h = half * 32 + x;
-                        o[h * kLatent + d] = __float2bfloat16_rn(u2f(r[x]) * inv_l[h]);
+                        for (int x = 0; x < 32; ++x) {
+                            const int hh = half * 32 + x;
+                            o[hh * kLatent + d] = __float2bfloat16_rn(u2f(r[x]) * inv_l[hh]);
+                        }
+                    } else {
+                        float *po = a.part_o + ((static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits + split) * kMlaHeads * kLatent;
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) po[(half * 32 + x) * kLatent + d] = u2f(r[x]);
                     }
-                } else {
-                    float *po = a.part_o + ((static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits + split) * kMlaHeads * kLatent;
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) po[(half * 32 + x) * kLatent + d] = u2f(r[x]);
                 }
             }
         }
         if (tid < kMlaHeads) {
-            if (final_out) {
-                if (lp.lse) lp.lse[static_cast<int64_t>(i) * kMlaHeads + tid] = m_run[tid] * a.scale + logf(l_run[tid]);
+            if (a.n_splits == 1) {
+                if (lp.lse) lp.lse[static_cast<int64_t>(i) * kMlaHeads + tid] = m_fin[tid] * a.scale + logf(l_fin[tid]);
             } else {
                 float *ml = a.part_ml + (((static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits + split) * kMlaHeads + tid) * 2;
-                ml[0] = m_run[tid] * c2;  // log2 units
-                ml[1] = l_run[tid];
+                ml[0] = m_fin[tid] * c2;  // log2 units
+                ml[1] = l_fin[tid];
             }
         }
     }
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) {
+    if (warp == 8) {
         tc_fence_after();
         tmem_dealloc(tbase, kTmemCols);
     }
@@ -345,11 +371,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
 __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
     const int hg = blockIdx.x, i = blockIdx.y, layer = blockIdx.z;
     const MlaLayerPtrs lp = a.layer[layer];
-    __shared__ float wgt[4][kMaxTopk / kRowsPerChunk];
+    __shared__ float wgt[4][32];  // splits per query: at most 16 by the planner
     int cnt = a.cnt[i];
     if (cnt < 0 || cnt > a.topk) cnt = 0;
-    const int nch = (cnt + kRowsPerChunk - 1) / kRowsPerChunk;
-    const int ns = (nch + a.chunks_per_cta - 1) / a.chunks_per_cta;
+    const int nch = (cnt + kChunk - 1) / kChunk;
+    const int ns = min(32, (nch + a.chunks_per_cta - 1) / a.chunks_per_cta);
     const int64_t base = (static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits;
     // (max, sum) of every split for the 4 heads: one thread per (head, split)
     {

@@ -496,19 +496,12 @@ __global__ void __launch_bounds__(kT, 2) topk_collect_kernel(const TopkArgs a, i
     const int n = visible_rows(a, i);
     if (n <= a.topk) return;
     const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
-    const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
-    for (int b = threadIdx.x; b < kBins; b += kT) hist[b] = g[b];
-    __syncthreads();
-    find_digit(hist, kBins, static_cast<uint32_t>(a.topk), scan, sel);
-    const uint32_t d1 = sel[0];
     const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
     const int sub = ((hi - lo + kWarps - 1) / kWarps + 127) / 128 * 128;
     const int wlo = min(hi, lo + warp * sub), whi = min(hi, wlo + sub);
-    uint32_t cnt = 0;
-    for (int base0 = wlo; base0 < whi; base0 += 128 * kU) {
-        float v[kU][4];
+    auto load_batch = [&](int base0, float (&v)[kU][4]) {
 #pragma unroll
-        for (int j = 0; j < kU; ++j) {  // all loads of the batch first
+        for (int j = 0; j < kU; ++j) {
             const int e0 = base0 + j * 128 + lane * 4;
             if (e0 + 4 <= whi) {
                 const float4 f = __ldg(reinterpret_cast<const float4 *>(row + e0));
@@ -518,6 +511,17 @@ __global__ void __launch_bounds__(kT, 2) topk_collect_kernel(const TopkArgs a, i
                 for (int x = 0; x < 4; ++x) v[j][x] = e0 + x < whi ? __ldg(row + e0 + x) : 0.f;
             }
         }
+    };
+    float v[kU][4];
+    load_batch(wlo, v);  // in flight while the threshold digit is found
+    const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+    for (int b = threadIdx.x; b < kBins; b += kT) hist[b] = g[b];
+    __syncthreads();
+    find_digit(hist, kBins, static_cast<uint32_t>(a.topk), scan, sel);
+    const uint32_t d1 = sel[0];
+    uint32_t cnt = 0;
+    for (int base0 = wlo; base0 < whi; base0 += 128 * kU) {
+        if (base0 != wlo) load_batch(base0, v);
 #pragma unroll
         for (int j = 0; j < kU; ++j) {
             const int e0 = base0 + j * 128 + lane * 4;
@@ -632,8 +636,12 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int
         for (int p = threadIdx.x >> 5; p < n_chunks; p += kWarps) {
             const uint32_t c = sm.coff[p + 1] - sm.coff[p];
             for (uint32_t j = threadIdx.x & 31; j < c; j += 32)
-                sm.cand[sm.coff[p] + j] = src[static_cast<int64_t>(p) * kSplitCap + j];
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(&sm.cand[sm.coff[p] + j])),
+                             "l"(src + static_cast<int64_t>(p) * kSplitCap + j)
+                             : "memory");
         }
+        cp_async_commit();
+        cp_async_wait_all();
         __syncthreads();
         const StagedSegs sg{sm.cand, sm.coff, n_chunks};
         uint32_t T, need_eq;
