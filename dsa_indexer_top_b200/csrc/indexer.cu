@@ -200,16 +200,15 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, 1)
                 tc_fence_after();
                 if (!mbar_wait(&full_bar[stage], use & 1, a.status, &abort_flag)) break;
                 tc_fence_after();
-                const uint32_t a_addr = smem_u32(a_tiles + stage * kATileBytes);
-                const uint32_t b_addr = smem_u32(b_tile);
+                const uint64_t adesc = sdesc_sw128(smem_u32(a_tiles + stage * kATileBytes), 16, 1024);
+                const uint64_t bdesc = sdesc_sw128(smem_u32(b_tile), 16, 1024);
                 const uint32_t d_tmem = tmem_base + acc * N;
 #pragma unroll
                 for (int kk = 0; kk < kIdxDim / 16; ++kk) {
-                    const uint32_t koff = (kk & 3) * 32u;
-                    const uint64_t adesc =
-                        sdesc_sw128(a_addr + (kk >> 2) * (kATileBytes / 2) + koff, 16, 1024);
-                    const uint64_t bdesc = sdesc_sw128(b_addr + (kk >> 2) * (N * 128) + koff, 16, 1024);
-                    umma_bf16(d_tmem, adesc, bdesc, Cfg::kIdesc, kk > 0 ? 1u : 0u);
+                    // offsets in 16-byte units added to the descriptors' start-address field
+                    const uint64_t aoff = static_cast<uint64_t>(((kk >> 2) * (kATileBytes / 2) + (kk & 3) * 32) >> 4);
+                    const uint64_t boff = static_cast<uint64_t>(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
+                    umma_bf16(d_tmem, adesc + aoff, bdesc + boff, Cfg::kIdesc, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&empty_bar[stage]);
                 umma_commit(&tmem_full[acc]);

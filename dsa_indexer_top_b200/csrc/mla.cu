@@ -169,6 +169,14 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
         // soon as its P is written, whichever comes first (ts <= to + 1: S of a
         // slot is rewritten only after that slot's O was issued).  Bounded.
         if (lane == 0 && nloc > 0) {
+            // base descriptors; each MMA adds its (16-byte unit) offset to the
+            // start-address field, which never carries out of it
+            const uint32_t sb0 = smem_u32(slot_sm), sb1 = smem_u32(slot_sm + kSlotBytes);
+            const uint64_t qdesc = sdesc_sw128(q_addr, 16, 1024);
+            const uint64_t cdesc0 = sdesc_sw128(sb0, 16, 1024), cdesc1 = sdesc_sw128(sb1, 16, 1024);
+            const uint64_t odesc0 = sdesc_sw128(sb0, kBlockBytes, 1024), odesc1 = sdesc_sw128(sb1, kBlockBytes, 1024);
+            const uint64_t pdesc0 = sdesc_sw128(sb0 + 8 * kBlockBytes, 16, 1024);
+            const uint64_t pdesc1 = sdesc_sw128(sb1 + 8 * kBlockBytes, 16, 1024);
             bool ok = mbar_wait(&q_full, 0, a.status, &abort_flag);
             int ts = 0, to = 0;
             uint64_t t0 = global_timer_ns();
@@ -178,12 +186,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                 if (ts < nloc && ts <= to + 1 && mbar_test_wait(&slot_full[ts & 1], (ts >> 1) & 1)) {
                     tc_fence_after();
                     const int s = ts & 1;
-                    const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
+                    const uint64_t cdesc = s ? cdesc1 : cdesc0;
 #pragma unroll
                     for (int kk = 0; kk < kRow / 16; ++kk) {
-                        const uint32_t koff = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-                        umma_bf16(tbase + 64 * s, sdesc_sw128(q_addr + koff, 16, 1024), sdesc_sw128(sb + koff, 16, 1024),
-                                  kIdescS, kk > 0 ? 1u : 0u);
+                        const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                        umma_bf16(tbase + 64 * s, qdesc + koff, cdesc + koff, kIdescS, kk > 0 ? 1u : 0u);
                     }
                     umma_commit(&s_full[s]);
                     ++ts;
@@ -192,14 +199,15 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                 if (to < ts && mbar_test_wait(&p_full[to & 1], (to >> 1) & 1)) {
                     tc_fence_after();
                     const int sp = to & 1;
-                    const uint32_t sb = smem_u32(slot_sm + sp * kSlotBytes);
-                    const uint32_t pb = sb + 8 * kBlockBytes;  // P: the slot's RoPE block
+                    const uint64_t adesc = sp ? odesc1 : odesc0;  // latent blocks, MN-major
+                    const uint64_t bdesc = sp ? pdesc1 : pdesc0;  // P in the RoPE block
 #pragma unroll
                     for (int mt = 0; mt < 4; ++mt) {
 #pragma unroll
                         for (int kk = 0; kk < kChunk / 16; ++kk) {
-                            umma_bf16(tbase + kOCol + 64 * mt, sdesc_sw128(sb + 2 * mt * kBlockBytes + kk * 2048, kBlockBytes, 1024),
-                                      sdesc_sw128(pb + kk * 32, 16, 1024), kIdescO, (to > 0 || kk > 0) ? 1u : 0u);
+                            umma_bf16(tbase + kOCol + 64 * mt,
+                                      adesc + static_cast<uint64_t>((2 * mt * kBlockBytes + kk * 2048) >> 4),
+                                      bdesc + static_cast<uint64_t>((kk * 32) >> 4), kIdescO, (to > 0 || kk > 0) ? 1u : 0u);
                         }
                     }
                     umma_commit(&o_done[sp]);
