@@ -119,6 +119,7 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = tmem_base_sh;
+    griddep_wait();
 
     const long long total = a.total_items;
     const long long begin = total * blockIdx.x / gridDim.x;
@@ -128,6 +129,7 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            const uint64_t stream_policy = l2_evict_first_policy();  // keys are read once
             int cur_g = -1, seq = -1, max_pos = -1;
             bool group_loaded = false;
             int b_uses = 0;
@@ -158,9 +160,9 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, 1)
                 if (!mbar_wait(&empty_bar[stage], (use & 1) ^ 1, a.status, &abort_flag)) break;
                 uint8_t *dst = a_tiles + stage * kATileBytes;
                 mbar_arrive_expect_tx(&full_bar[stage], kATileBytes);
-                tma_load_3d(dst, &tmap_k, &full_bar[stage], 0, j * kTileKeys, seq);
-                tma_load_3d(dst + kATileBytes / 2, &tmap_k, &full_bar[stage], 64, j * kTileKeys,
-                            seq);
+                tma_load_3d_hint(dst, &tmap_k, &full_bar[stage], 0, j * kTileKeys, seq, stream_policy);
+                tma_load_3d_hint(dst + kATileBytes / 2, &tmap_k, &full_bar[stage], 64, j * kTileKeys, seq,
+                                 stream_policy);
                 last_use[stage] = use;
                 ++k_tiles;
             }
@@ -318,6 +320,7 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, 1)
         if (fuse_hist && hist_dirty && !abort_flag) flush_hist(cur_g);
     }
 
+    griddep_launch_dependents();
     tc_fence_before();
     __syncthreads();
     if (warp == 1) {
@@ -374,8 +377,7 @@ cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcA
     cudaError_t e = cudaFuncSetAttribute(idx_score_tc_kernel<G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     if (e != cudaSuccess) return e;
-    idx_score_tc_kernel<G><<<grid, Cfg::kThreads, Cfg::kSmem, st>>>(tk, tq, a);
-    return cudaGetLastError();
+    return launch_pdl(idx_score_tc_kernel<G>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmem, st, tk, tq, a);
 }
 
 }  // namespace

@@ -11,6 +11,24 @@
 
 namespace dsa {
 
+// Launch with programmatic stream serialisation (the kernel calls
+// griddep_wait() before it reads what earlier work in the stream wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
 constexpr int kIdxHeads = 32;   // index_n_heads of GLM-5.2
 constexpr int kIdxDim = 128;    // index_head_dim of GLM-5.2
 constexpr int kMlaHeads = 64;   // num_attention_heads of GLM-5.2

@@ -95,6 +95,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_base_sh;
+    griddep_wait();
 
     int seq = a.q_seq[i];
     int cnt = a.cnt[i];
@@ -323,6 +324,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
         }
     }
 
+    griddep_launch_dependents();
     __syncthreads();  // every role has left its loop: `go` is uniform
     const bool go = nloc > 0 && !abort_flag;
     if (go) {
@@ -379,7 +381,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
 __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
     const int hg = blockIdx.x, i = blockIdx.y, layer = blockIdx.z;
     const MlaLayerPtrs lp = a.layer[layer];
-    __shared__ float wgt[4][32];  // splits per query: at most 16 by the planner
+    __shared__ float wgt[4][32];
+    griddep_wait();  // splits per query: at most 16 by the planner
     int cnt = a.cnt[i];
     if (cnt < 0 || cnt > a.topk) cnt = 0;
     const int nch = (cnt + kChunk - 1) / kChunk;
@@ -525,14 +528,12 @@ cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_splits, a.n_q, a.n_layers);
-    mla_tc_kernel<<<grid, kMlaThreads, kMlaSmem, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(mla_tc_kernel, grid, dim3(kMlaThreads), kMlaSmem, st, a);
 }
 
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st) {
     dim3 grid(kMlaHeads / 4, a.n_q, a.n_layers);
-    mla_combine_kernel<<<grid, 256, 0, st>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(mla_combine_kernel, grid, dim3(256), 0, st, a);
 }
 
 cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st) {

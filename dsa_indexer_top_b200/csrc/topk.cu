@@ -327,6 +327,7 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
     RowSmem &sm = *reinterpret_cast<RowSmem *>(smem_raw);
     const int i = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_wait();
     const int n = visible_rows(a, i);
     if (n <= a.topk) {
         write_all(a, i, n);
@@ -469,6 +470,7 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
 __global__ void __launch_bounds__(kT, 2) topk_hist_kernel(const TopkArgs a, int chunk) {
     __shared__ uint32_t hist[kBins];
     const int i = blockIdx.y, p = blockIdx.x;
+    griddep_wait();
     const int n = visible_rows(a, i);
     if (n <= a.topk) return;
     const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
@@ -493,6 +495,7 @@ __global__ void __launch_bounds__(kT, 2) topk_collect_kernel(const TopkArgs a, i
     __shared__ uint32_t wcount[kWarps], woff[kWarps + 1];
     const int i = blockIdx.y, p = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_wait();
     const int n = visible_rows(a, i);
     if (n <= a.topk) return;
     const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
@@ -600,6 +603,7 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int
     extern __shared__ __align__(16) uint8_t smem_raw[];
     MergeSmem &sm = *reinterpret_cast<MergeSmem *>(smem_raw);
     const int i = blockIdx.x;
+    griddep_wait();
     const int n = visible_rows(a, i);
     if (n <= a.topk) {
         write_all(a, i, n);
@@ -668,8 +672,7 @@ bool topk_uses_split(int n_q, int max_ctx) { return max_ctx > kTopkSplitMinCtx &
 cudaError_t launch_topk_hist(const TopkArgs &a, int num_sms, cudaStream_t st) {
     int P, chunk;
     split_plan(a, num_sms, P, chunk);
-    topk_hist_kernel<<<dim3(P, a.n_q), kT, 0, st>>>(a, chunk);
-    return cudaGetLastError();
+    return launch_pdl(topk_hist_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk);
 }
 
 cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
@@ -679,23 +682,19 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
         if ((e = cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       static_cast<int>(smem))) != cudaSuccess)
             return e;
-        topk_row_kernel<<<a.n_q, kT, smem, st>>>(a);
-        return cudaGetLastError();
+        return launch_pdl(topk_row_kernel, dim3(a.n_q), dim3(kT), smem, st, a);
     }
     int P, chunk;
     split_plan(a, num_sms, P, chunk);
     if (!a.hist_ready) {
         if ((e = cudaMemsetAsync(a.ghist, 0, sizeof(uint32_t) * kBins * a.n_q, st)) != cudaSuccess) return e;
-        topk_hist_kernel<<<dim3(P, a.n_q), kT, 0, st>>>(a, chunk);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_pdl(topk_hist_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk)) != cudaSuccess) return e;
     }
-    topk_collect_kernel<<<dim3(P, a.n_q), kT, 0, st>>>(a, chunk);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(topk_collect_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(sizeof(MergeSmem)))) != cudaSuccess)
         return e;
-    topk_merge_kernel<<<a.n_q, kT, sizeof(MergeSmem), st>>>(a, P);
-    return cudaGetLastError();
+    return launch_pdl(topk_merge_kernel, dim3(a.n_q), dim3(kT), sizeof(MergeSmem), st, a, P);
 }
 
 size_t topk_scratch_bytes(int n_q, int max_ctx) {
