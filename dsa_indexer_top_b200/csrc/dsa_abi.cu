@@ -219,6 +219,7 @@ dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int t
     a.hist_ready = (hist_ready && (qs->seq_run & 1)) ? 1 : 0;
     a.ghist = nullptr;
     a.gcount = nullptr;
+    a.gdigit = nullptr;
     a.gcand = nullptr;
     topk_bind_scratch(a, scratch);
     return launch_topk(a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

@@ -96,6 +96,7 @@ struct TopkArgs {
     // scratch (workspace)
     uint32_t *ghist;   // [n_q][4096] first-digit histogram
     uint32_t *gcount;  // [n_q][kSplitMax] candidates per chunk
+    uint32_t *gdigit;  // [n_q][2] threshold first digit and rows above it
     uint2 *gcand;      // [n_q][kSplitMax][kSplitCap] (key, position)
 };
 bool topk_uses_split(int n_q, int max_ctx);

@@ -72,26 +72,51 @@ __device__ __forceinline__ uint64_t block_scan(uint64_t v, uint64_t *buf, uint64
     return before + x - v;
 }
 
+// Copy a query's first-digit histogram from global memory: every thread's
+// eight loads are issued before any is used.
+__device__ __forceinline__ void load_hist(uint32_t *hist, const uint32_t *g) {
+    uint32_t v[kBins / kT];
+#pragma unroll
+    for (int j = 0; j < kBins / kT; ++j) v[j] = __ldg(g + threadIdx.x + j * kT);
+#pragma unroll
+    for (int j = 0; j < kBins / kT; ++j) hist[threadIdx.x + j * kT] = v[j];
+}
+
 __device__ __forceinline__ void zero_hist(uint32_t *hist, int nbins) {
     for (int b = threadIdx.x; b < nbins; b += kT) hist[b] = 0;
 }
 
 // The digit holding the r-th largest key: sel[0] = digit, sel[1] = rows in
 // higher bins.  If the histogram holds fewer than r rows, sel = {0, total}.
+// Thread t owns bins [t*per, t*per + per); one barrier: warp totals, then the
+// rows above a thread = the warps above + a suffix scan inside its warp.
 __device__ __forceinline__ void find_digit(const uint32_t *hist, int nbins, uint32_t r, uint64_t *scan,
                                            uint32_t *sel) {
+    uint32_t *wsum = reinterpret_cast<uint32_t *>(scan);  // kWarps entries
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int per = nbins / kT > 0 ? nbins / kT : 1;
     const int b0 = threadIdx.x * per;
     uint32_t mine = 0;
     for (int j = 0; j < per; ++j)
         if (b0 + j < nbins) mine += hist[b0 + j];
-    uint64_t all;
-    const uint64_t before = block_scan(mine, scan, all);
-    if (threadIdx.x == 0 && all < r) {
-        sel[0] = 0;
-        sel[1] = static_cast<uint32_t>(all);
+    uint32_t suf = mine;  // rows in this lane's bins and every higher lane's
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += y;
     }
-    uint32_t above = static_cast<uint32_t>(all - before - mine);
+    if (lane == 0) wsum[warp] = suf;
+    __syncthreads();
+    uint32_t above = suf - mine, total = 0;
+    for (int w = 0; w < kWarps; ++w) {
+        const uint32_t x = wsum[w];
+        total += x;
+        if (w > warp) above += x;
+    }
+    if (threadIdx.x == 0 && total < r) {
+        sel[0] = 0;
+        sel[1] = total;
+    }
     for (int j = per - 1; j >= 0; --j) {
         if (b0 + j >= nbins) continue;
         const uint32_t upto = above + hist[b0 + j];
@@ -342,7 +367,7 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
     const bool exact = a.hist_ready != 0;
     if (exact) {
         const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
-        for (int b = threadIdx.x; b < kBins; b += kT) sm.hist[b] = g[b];
+        load_hist(sm.hist, g);
         __syncthreads();
         find_digit(sm.hist, kBins, k, sm.scan, sm.sel);
         d_lo = sm.sel[0];
@@ -518,10 +543,14 @@ __global__ void __launch_bounds__(kT, 2) topk_collect_kernel(const TopkArgs a, i
     float v[kU][4];
     load_batch(wlo, v);  // in flight while the threshold digit is found
     const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
-    for (int b = threadIdx.x; b < kBins; b += kT) hist[b] = g[b];
+    load_hist(hist, g);
     __syncthreads();
     find_digit(hist, kBins, static_cast<uint32_t>(a.topk), scan, sel);
     const uint32_t d1 = sel[0];
+    if (p == 0 && threadIdx.x == 0) {  // the merge reads the threshold digit from here
+        a.gdigit[2 * i] = d1;
+        a.gdigit[2 * i + 1] = sel[1];
+    }
     uint32_t cnt = 0;
     for (int base0 = wlo; base0 < whi; base0 += 128 * kU) {
         if (base0 != wlo) load_batch(base0, v);
@@ -612,8 +641,7 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int
     const uint32_t k = static_cast<uint32_t>(a.topk);
     const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
     int32_t *out = a.idx + static_cast<int64_t>(i) * a.topk;
-    const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
-    for (int b = threadIdx.x; b < kBins; b += kT) sm.hist[b] = g[b];
+    const uint32_t d1 = a.gdigit[2 * i], above1 = a.gdigit[2 * i + 1];  // from collect chunk 0
     const uint32_t *counts = a.gcount + static_cast<int64_t>(i) * kSplitMax;
     // chunk counts -> offsets (a block scan; count > cap marks an overflow)
     {
@@ -629,8 +657,6 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int
         }
     }
     __syncthreads();
-    find_digit(sm.hist, kBins, k, sm.scan, sm.sel);
-    const uint32_t d1 = sm.sel[0], above1 = sm.sel[1];
     const bool overflow = sm.sel[2] != 0;
     if (overflow) {
         finish_stream(row, n, k, d1, above1, sm.hist, sm.scan, sm.sel, out);
@@ -702,8 +728,9 @@ size_t topk_scratch_bytes(int n_q, int max_ctx) {
     auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     if (!topk_uses_split(n_q, max_ctx)) return al(hist);
     const size_t counts = sizeof(uint32_t) * kSplitMax * n_q;
+    const size_t digits = sizeof(uint32_t) * 2 * n_q;
     const size_t cand = sizeof(uint2) * static_cast<size_t>(kSplitCap) * kSplitMax * n_q;
-    return al(hist) + al(counts) + al(cand);
+    return al(hist) + al(counts) + al(digits) + al(cand);
 }
 
 void topk_bind_scratch(TopkArgs &a, void *scratch) {
@@ -714,6 +741,8 @@ void topk_bind_scratch(TopkArgs &a, void *scratch) {
     p += al(sizeof(uint32_t) * kBins * a.n_q);
     a.gcount = reinterpret_cast<uint32_t *>(p);
     p += al(sizeof(uint32_t) * kSplitMax * a.n_q);
+    a.gdigit = reinterpret_cast<uint32_t *>(p);
+    p += al(sizeof(uint32_t) * 2 * a.n_q);
     a.gcand = reinterpret_cast<uint2 *>(p);
 }
 
