@@ -76,7 +76,7 @@ bool mla_tc_ok(const dsa_mla *m) {
 
 size_t ws_index_scores() { return kStatusBytes; }
 size_t ws_topk(int n_q, int max_ctx) { return kStatusBytes + align256(topk_scratch_bytes(n_q, max_ctx)); }
-int decode_splits(int topk) { return (topk + kRowsPerChunk - 1) / kRowsPerChunk; }
+int decode_splits(int topk) { return mla_max_splits(topk); }
 size_t ws_mla_decode(int n_q, int topk, int n_layers) {
     const int ns = decode_splits(topk);
     return kStatusBytes + (ns > 1 ? align256(mla_partial_bytes(n_layers, n_q, ns)) : 0);
@@ -278,7 +278,7 @@ dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, co
     for (int l = 0; l < n_layers; ++l) tc = tc && mla_tc_ok(&layers[l]);
     if (tc) {
         int n_splits, cpc;
-        mla_plan(qs->n_q, n_layers, topk, decode, num_sms_current(), n_splits, cpc);
+        mla_plan(qs->n_q, n_layers, topk, decode, num_sms_current(), kMlaMaxSplits, n_splits, cpc);
         a.n_splits = n_splits;
         a.chunks_per_cta = cpc;
         if (n_splits > 1) {

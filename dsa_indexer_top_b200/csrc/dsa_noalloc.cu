@@ -101,7 +101,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
         sms = 148;
     int plan_splits, cpc;
-    mla_plan(queries->n_q, 1, topk, true, sms, plan_splits, cpc);
+    mla_plan(queries->n_q, 1, topk, true, sms, n_splits, plan_splits, cpc);  // at most the bound above
     a.n_splits = plan_splits;
     a.chunks_per_cta = cpc;
     if (plan_splits > 1) {

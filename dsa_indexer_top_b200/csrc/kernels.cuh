@@ -141,21 +141,32 @@ cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st);
 cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st);
 
 // Split-K plan of the tensor-core MLA: n_splits CTAs per query, each walking
-// cpc chunks of 64 selected rows.  Decode spreads a query over up to 16 CTAs
-// (about one CTA per SM over the batch, at least two chunks each); prefill uses
-// one CTA per query (n_splits = 1: the final output is written directly).
-inline void mla_plan(int n_q, int n_layers, int topk, bool decode, int num_sms, int &n_splits, int &cpc) {
+// cpc chunks of 64 selected rows.  Decode spreads each query over as many CTAs
+// as fill the SMs across the batch (at most max_splits, and at least two
+// chunks per CTA: measured on 4 x 1M decode, 16 splits x 2 chunks beat both
+// 32 x 1 and 8 x 4); prefill uses one CTA
+// per query (n_splits = 1: the final output is written directly).
+inline void mla_plan(int n_q, int n_layers, int topk, bool decode, int num_sms, int max_splits, int &n_splits,
+                     int &cpc) {
     const int nch = (topk + kMlaChunk - 1) / kMlaChunk;
     int s = 1;
     if (decode) {
         const int work = n_q * n_layers > 0 ? n_q * n_layers : 1;
         s = num_sms / work;
-        s = s < 1 ? 1 : (s > 16 ? 16 : s);
-        const int half = nch / 2 > 0 ? nch / 2 : 1;
+        s = s < 1 ? 1 : (s > max_splits ? max_splits : s);
+        const int half = nch / 2 > 0 ? nch / 2 : 1;  // at least two chunks per CTA
         s = s > half ? half : s;
     }
     cpc = (nch + s - 1) / s;
     n_splits = (nch + cpc - 1) / cpc;
+}
+
+// Upper bound of the decode splits per query the planner can pick with
+// max_splits = kMlaMaxSplits (sizes the workspace).
+constexpr int kMlaMaxSplits = 32;
+inline int mla_max_splits(int topk) {
+    const int nch = (topk + kMlaChunk - 1) / kMlaChunk;
+    return nch < kMlaMaxSplits ? nch : kMlaMaxSplits;
 }
 
 // Bytes of split-K partials for the tensor-core decode schedule.

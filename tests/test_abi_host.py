@@ -53,12 +53,12 @@ def test_workspace_bytes():
     q2 = _q(n_q=8, L=8192)
     assert lib.dsa_workspace_bytes(B.DSA_OP_TOPK, ctypes.byref(q2), 2048, 64, 512, 1) == 256 + hist
     dec = lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 2048, 64, 512, 1)
-    # 16 splits x 8 queries x 64 heads x (512 + 2) floats, 256-aligned, + status
-    assert dec == 256 + ((8 * 16 * 64 * 514 * 4 + 255) // 256) * 256
-    assert lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 128, 64, 512, 1) == 256
+    # up to 32 splits (64-row chunks) x 8 queries x 64 heads x (512 + 2) floats, 256-aligned, + status
+    assert dec == 256 + ((8 * 32 * 64 * 514 * 4 + 255) // 256) * 256
+    assert lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 64, 64, 512, 1) == 256
     grp = lib.dsa_workspace_bytes(B.DSA_OP_INDEXSHARE_GROUP, ctypes.byref(q), 2048, 64, 512, 4)
     scores = 8 * 32768 * 4
-    assert grp == 256 + scores + split + ((4 * 8 * 16 * 64 * 514 * 4 + 255) // 256) * 256
+    assert grp == 256 + scores + split + ((4 * 8 * 32 * 64 * 514 * 4 + 255) // 256) * 256
     assert lib.dsa_workspace_bytes(77, ctypes.byref(q), 2048, 64, 512, 1) == 0
 
 
