@@ -151,9 +151,7 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
         a.total_items = groups * a.tiles_per_group;
         a.ghist = (ghist && G == 1) ? ghist : nullptr;  // fused into the epilogue
         hist_done = a.ghist != nullptr;
-        const int sms = num_sms_current();
-        const int grid = static_cast<int>(a.total_items < sms ? a.total_items : sms);
-        s = launch_idx_score_tc(G, tk, tq, a, grid, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+        s = launch_idx_score_tc(G, tk, tq, a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
     } else {
         s = do_index_generic(qs, ix, scores, ld, status, st);
     }

@@ -15,8 +15,9 @@
 //   warps 2-5   epilogue: tcgen05.ld of its 32 TMEM lanes (one key per lane),
 //               ReLU, multiply by w and sum the 32 heads inside the thread, causal
 //               mask, coalesced fp32 store of one score per key per query.
-// Work items are (query group, key tile) pairs split evenly over a grid of at
-// most one CTA per SM; tiles past the group's last visible key are skipped.
+// Work items are (query group, key tile) pairs split into contiguous ranges over
+// a grid of at most two CTAs per SM (one query per tile) or one (several);
+// tiles past the group's last visible key are skipped.
 #include <algorithm>
 #include <cuda_bf16.h>
 
@@ -32,7 +33,13 @@ constexpr int kATileBytes = kTileKeys * kIdxDim * 2;  // 32 KB
 template <int G>
 struct IdxCfg {
     static constexpr int N = 32 * G;
-    static constexpr int kStages = (G == 8) ? 4 : 6;
+    // One query per tile: two CTAs per SM with two 32 KB stages each.  Two
+    // independent load -> MMA -> epilogue pipelines per SM keep the key stream
+    // at the rate of a plain TMA read stream, where one CTA with deeper
+    // buffering loses about 6% to the MMA turnaround of each stage; more than
+    // about 128 KB in flight per SM lowers the stream rate again.
+    static constexpr int kCtasPerSm = G == 1 ? 2 : 1;
+    static constexpr int kStages = G == 1 ? 2 : 4;
     static constexpr int kBBytes = N * kIdxDim * 2;
     static constexpr int kTmemCols = (2 * N < 32) ? 32 : 2 * N;
     static constexpr int kSmem = kStages * kATileBytes + kBBytes + 1024;
@@ -62,7 +69,7 @@ __device__ __forceinline__ void group_info(const IdxTcArgs &a, int g, int &seq, 
 }
 
 template <int G>
-__global__ void __launch_bounds__(IdxCfg<G>::kThreads, 1)
+__global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
     idx_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_q, const IdxTcArgs a) {
     using Cfg = IdxCfg<G>;
@@ -371,9 +378,11 @@ __global__ void __launch_bounds__(256) idx_score_generic_kernel(const IdxGeneric
 }
 
 template <int G>
-cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcArgs &a, int grid,
+cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcArgs &a, int num_sms,
                       cudaStream_t st) {
     using Cfg = IdxCfg<G>;
+    const long long slots = static_cast<long long>(num_sms) * Cfg::kCtasPerSm;
+    const int grid = static_cast<int>(a.total_items < slots ? a.total_items : slots);
     cudaError_t e = cudaFuncSetAttribute(idx_score_tc_kernel<G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     if (e != cudaSuccess) return e;
@@ -383,12 +392,12 @@ cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcA
 }  // namespace
 
 cudaError_t launch_idx_score_tc(int G, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
-                                const IdxTcArgs &a, int grid, cudaStream_t st) {
+                                const IdxTcArgs &a, int num_sms, cudaStream_t st) {
     switch (G) {
-        case 1: return launch_tc<1>(tmap_k, tmap_q, a, grid, st);
-        case 2: return launch_tc<2>(tmap_k, tmap_q, a, grid, st);
-        case 4: return launch_tc<4>(tmap_k, tmap_q, a, grid, st);
-        case 8: return launch_tc<8>(tmap_k, tmap_q, a, grid, st);
+        case 1: return launch_tc<1>(tmap_k, tmap_q, a, num_sms, st);
+        case 2: return launch_tc<2>(tmap_k, tmap_q, a, num_sms, st);
+        case 4: return launch_tc<4>(tmap_k, tmap_q, a, num_sms, st);
+        case 8: return launch_tc<8>(tmap_k, tmap_q, a, num_sms, st);
         default: return cudaErrorInvalidValue;
     }
 }

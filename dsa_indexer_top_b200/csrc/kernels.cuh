@@ -60,7 +60,7 @@ struct IdxTcArgs {
 // {128, L, n_cache} bf16, box {64, 128, 1}; queries 2-D {128, n_q*32}, box
 // {64, 32*G}; both 128-byte swizzled.
 cudaError_t launch_idx_score_tc(int G, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
-                                const IdxTcArgs &a, int grid, cudaStream_t st);
+                                const IdxTcArgs &a, int num_sms, cudaStream_t st);
 
 struct IdxGenericArgs {
     const void *q;
