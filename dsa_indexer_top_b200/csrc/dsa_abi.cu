@@ -101,7 +101,7 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
     // the histograms are left only when queries are not tiled together (odd
     // seq_run: one query per tensor-core tile, where the epilogue builds them)
     if ((qs->seq_run & 1) == 0) ghist = nullptr;
-    if (ghist && cudaMemsetAsync(ghist, 0, sizeof(uint32_t) * kTopkBins * qs->n_q, st) != cudaSuccess)
+    if (ghist && cudaMemsetAsync(ghist, 0, topk_zeroed_bytes(qs->n_q), st) != cudaSuccess)
         return DSA_ERR_CUDA;
     bool hist_done = false;
     dsa_status s = DSA_OK;
@@ -216,8 +216,8 @@ dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int t
     a.topk = topk;
     a.hist_ready = (hist_ready && (qs->seq_run & 1)) ? 1 : 0;
     a.ghist = nullptr;
+    a.gticket = nullptr;
     a.gcount = nullptr;
-    a.gdigit = nullptr;
     a.gcand = nullptr;
     topk_bind_scratch(a, scratch);
     return launch_topk(a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;

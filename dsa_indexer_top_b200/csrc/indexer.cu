@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
                 }
                 const bool vis = qok[ii] && s <= qpos[ii];
                 if (vis) a.scores[static_cast<int64_t>(g * G + i) * a.ld + s] = score;
-                if (fuse_hist) hist_add_warp(ehist, vis ? first_digit(order_key(score)) : 0xFFFFFFFFu);
+                if (fuse_hist) hist_add(ehist, vis ? first_digit(order_key(score)) : 0xFFFFFFFFu);
             }
             hist_dirty = true;
             tc_fence_before();

@@ -95,11 +95,14 @@ struct TopkArgs {
     int hist_ready;    // ghist already holds the first-digit histograms (indexer epilogue)
     // scratch (workspace)
     uint32_t *ghist;   // [n_q][4096] first-digit histogram
+    uint32_t *gticket; // [n_q] chunks of the query done (split schedule), after ghist
     uint32_t *gcount;  // [n_q][kSplitMax] candidates per chunk
-    uint32_t *gdigit;  // [n_q][2] threshold first digit and rows above it
     uint2 *gcand;      // [n_q][kSplitMax][kSplitCap] (key, position)
 };
 bool topk_uses_split(int n_q, int max_ctx);
+// Bytes at the head of the top-k scratch (histograms, then tickets) that must be
+// zero when a top-k launch starts.
+size_t topk_zeroed_bytes(int n_q);
 size_t topk_scratch_bytes(int n_q, int max_ctx);
 void topk_bind_scratch(TopkArgs &a, void *scratch);
 cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st);

@@ -279,11 +279,13 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // First radix digit of a key (12 bits; kTopkBins histogram bins).
 __device__ __forceinline__ uint32_t first_digit(uint32_t key) { return key >> 20; }
 
-// Add one to hist[d] for every lane with d != ~0u, one atomic per distinct
-// digit in the warp.  Every lane of the warp must call it.
-__device__ __forceinline__ void hist_add_warp(uint32_t *hist, uint32_t d) {
-    const uint32_t peers = __match_any_sync(0xffffffffu, d);
-    if (d != 0xFFFFFFFFu && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+// Add one to hist[d] unless d == ~0u.  A plain shared-memory atomic per lane:
+// lanes of a warp that hit the same bin are combined by the hardware, and on
+// sm_100a this is several times cheaper than grouping the lanes first with
+// __match_any_sync (measured: 16-170 cycles per warp instruction with 16 warps
+// resident, against 150-1080 for match + atomic).
+__device__ __forceinline__ void hist_add(uint32_t *hist, uint32_t d) {
+    if (d != 0xFFFFFFFFu) atomicAdd(&hist[d], 1u);
 }
 
 }  // namespace dsa

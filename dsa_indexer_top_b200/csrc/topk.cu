@@ -27,8 +27,9 @@
 //   row    one CTA per query: threshold digit, one streaming candidate pass,
 //          refine and write -- a single launch.
 //   split  long contexts with few queries: P CTAs per query collect their
-//          chunk's candidates (given the histogram), then one CTA per query
-//          walks the chunks' candidates in position order and finishes.
+//          chunk's candidates (given the histogram); the last of them to finish
+//          walks all the chunks' candidates in position order and writes the
+//          query's result -- one launch.
 #include <cstdint>
 
 #include "kernels.cuh"
@@ -72,33 +73,38 @@ __device__ __forceinline__ uint64_t block_scan(uint64_t v, uint64_t *buf, uint64
     return before + x - v;
 }
 
-// Copy a query's first-digit histogram from global memory: every thread's
-// eight loads are issued before any is used.
-__device__ __forceinline__ void load_hist(uint32_t *hist, const uint32_t *g) {
-    uint32_t v[kBins / kT];
-#pragma unroll
-    for (int j = 0; j < kBins / kT; ++j) v[j] = __ldg(g + threadIdx.x + j * kT);
-#pragma unroll
-    for (int j = 0; j < kBins / kT; ++j) hist[threadIdx.x + j * kT] = v[j];
-}
-
 __device__ __forceinline__ void zero_hist(uint32_t *hist, int nbins) {
     for (int b = threadIdx.x; b < nbins; b += kT) hist[b] = 0;
 }
 
 // The digit holding the r-th largest key: sel[0] = digit, sel[1] = rows in
 // higher bins.  If the histogram holds fewer than r rows, sel = {0, total}.
-// Thread t owns bins [t*per, t*per + per); one barrier: warp totals, then the
-// rows above a thread = the warps above + a suffix scan inside its warp.
+// nbins = 4096: thread t owns bins [8t, 8t + 8) (two 16-byte loads); nbins =
+// 256: threads t < 256 own bin t.  One barrier: each warp's suffix total goes to
+// shared memory, and every warp adds up the totals of the warps above it with
+// lane-parallel loads and four shuffles.
 __device__ __forceinline__ void find_digit(const uint32_t *hist, int nbins, uint32_t r, uint64_t *scan,
                                            uint32_t *sel) {
     uint32_t *wsum = reinterpret_cast<uint32_t *>(scan);  // kWarps entries
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int per = nbins / kT > 0 ? nbins / kT : 1;
-    const int b0 = threadIdx.x * per;
+    constexpr int kPer = kBins / kT;  // 8
+    uint32_t hb[kPer];
+    int b0;
+    if (nbins == kBins) {
+        b0 = threadIdx.x * kPer;
+        const uint4 x0 = reinterpret_cast<const uint4 *>(hist)[2 * threadIdx.x];
+        const uint4 x1 = reinterpret_cast<const uint4 *>(hist)[2 * threadIdx.x + 1];
+        hb[0] = x0.x, hb[1] = x0.y, hb[2] = x0.z, hb[3] = x0.w;
+        hb[4] = x1.x, hb[5] = x1.y, hb[6] = x1.z, hb[7] = x1.w;
+    } else {  // nbins <= kT: one bin per thread
+        b0 = threadIdx.x;
+        hb[0] = threadIdx.x < nbins ? hist[threadIdx.x] : 0u;
+#pragma unroll
+        for (int j = 1; j < kPer; ++j) hb[j] = 0u;
+    }
     uint32_t mine = 0;
-    for (int j = 0; j < per; ++j)
-        if (b0 + j < nbins) mine += hist[b0 + j];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) mine += hb[j];
     uint32_t suf = mine;  // rows in this lane's bins and every higher lane's
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -107,19 +113,23 @@ __device__ __forceinline__ void find_digit(const uint32_t *hist, int nbins, uint
     }
     if (lane == 0) wsum[warp] = suf;
     __syncthreads();
-    uint32_t above = suf - mine, total = 0;
-    for (int w = 0; w < kWarps; ++w) {
-        const uint32_t x = wsum[w];
-        total += x;
-        if (w > warp) above += x;
+    uint32_t ws = lane < kWarps ? wsum[lane] : 0u;  // suffix over warps, lane-parallel
+#pragma unroll
+    for (int o = 1; o < kWarps; o <<= 1) {
+        const uint32_t y = __shfl_down_sync(0xffffffffu, ws, o);
+        if (lane + o < 32) ws += y;
     }
+    const uint32_t total = __shfl_sync(0xffffffffu, ws, 0);
+    uint32_t above = suf - mine + __shfl_sync(0xffffffffu, ws, (warp + 1) & 31);
     if (threadIdx.x == 0 && total < r) {
         sel[0] = 0;
         sel[1] = total;
     }
-    for (int j = per - 1; j >= 0; --j) {
-        if (b0 + j >= nbins) continue;
-        const uint32_t upto = above + hist[b0 + j];
+    const int nb = nbins == kBins ? kPer : 1;
+#pragma unroll
+    for (int j = kPer - 1; j >= 0; --j) {
+        if (j >= nb) continue;
+        const uint32_t upto = above + hb[j];
         if (upto >= r && above < r) {
             sel[0] = b0 + j;
             sel[1] = above;
@@ -158,7 +168,7 @@ __device__ __forceinline__ void stream_hist(const float *row, int lo, int hi, ui
             for (int x = 0; x < 4; ++x) {
                 const uint32_t u = order_key(v[j][x]);
                 const bool in = e0 + x < hi && (u & pmask) == prefix;
-                hist_add_warp(hist, in ? (u >> shift) & dmask : 0xFFFFFFFFu);
+                hist_add(hist, in ? (u >> shift) & dmask : 0xFFFFFFFFu);
             }
         }
     }
@@ -167,8 +177,8 @@ __device__ __forceinline__ void stream_hist(const float *row, int lo, int hi, ui
 
 // Ordered filter by streaming the row (fallback): keep keys > T and the first
 // need_eq keys == T, at exclusive-scan slots.
-__device__ __forceinline__ void stream_write(const float *row, int n, uint32_t T, uint32_t need_eq, int32_t *out,
-                                             uint64_t *scan) {
+__device__ __forceinline__ void stream_write(const float *row, int n, uint32_t T, uint32_t need_eq, uint32_t k,
+                                             int32_t *out, uint64_t *scan) {
     uint32_t g_run = 0, e_run = 0;
     for (int base = 0; base < n; base += kT * 4) {
         const int e0 = base + threadIdx.x * 4;
@@ -188,10 +198,10 @@ __device__ __forceinline__ void stream_write(const float *row, int n, uint32_t T
         for (int x = 0; x < 4; ++x) {
             if (e0 + x >= n) continue;
             if (u[x] > T) {
-                out[g + min(q, need_eq)] = e0 + x;
+                if (g + min(q, need_eq) < k) out[g + min(q, need_eq)] = e0 + x;
                 ++g;
             } else if (u[x] == T) {
-                if (q < need_eq) out[g + q] = e0 + x;
+                if (q < need_eq && g + q < k) out[g + q] = e0 + x;
                 ++q;
             }
         }
@@ -219,7 +229,7 @@ __device__ __forceinline__ void finish_stream(const float *row, int n, uint32_t 
     const uint32_t T = (p24 << 8) | sel[0];
     const uint32_t need_eq = r3 - sel[1];
     __syncthreads();
-    stream_write(row, n, T, need_eq, out, scan);
+    stream_write(row, n, T, need_eq, k, out, scan);
 }
 
 // ------------------------------------------------------------ warp segments
@@ -241,13 +251,9 @@ __device__ __forceinline__ void seg_hist(const Segs &sg, uint32_t prefix, uint32
     for (int j = 0; j < sg.pieces(w); ++j) {
         const uint2 *p = sg.ptr(w, j);
         const uint32_t c = sg.count(w, j);
-        for (uint32_t b = 0; b < c; b += 32) {
-            uint32_t d = 0xFFFFFFFFu;
-            if (b + lane < c) {
-                const uint32_t u = p[b + lane].x;
-                if ((u & pmask) == prefix) d = (u >> shift) & dmask;
-            }
-            hist_add_warp(hist, d);
+        for (uint32_t b = lane; b < c; b += 32) {
+            const uint32_t u = p[b].x;
+            if ((u & pmask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1u);
         }
     }
     __syncthreads();
@@ -277,7 +283,7 @@ __device__ __forceinline__ void seg_refine(const Segs &sg, uint32_t d1, uint32_t
 // Ordered write of the kept candidates: per-warp counts, a 16-entry prefix,
 // then ballots inside each warp.
 template <class Segs>
-__device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t need_eq, int32_t *out,
+__device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t need_eq, uint32_t k, int32_t *out,
                                           uint32_t *wg, uint32_t *we) {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     uint32_t g = 0, e = 0;
@@ -313,12 +319,77 @@ __device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t n
             const bool isg = ok && v.x > T, ise = ok && v.x == T;
             const uint32_t mg = __ballot_sync(0xffffffffu, isg), me = __ballot_sync(0xffffffffu, ise);
             const uint32_t gb = gtb + g + __popc(mg & lt), eb = eqb + e + __popc(me & lt);
-            if (isg) out[gb + min(eb, need_eq)] = static_cast<int32_t>(v.y);
-            if (ise && eb < need_eq) out[gb + eb] = static_cast<int32_t>(v.y);
+            if (isg && gb + min(eb, need_eq) < k) out[gb + min(eb, need_eq)] = static_cast<int32_t>(v.y);
+            if (ise && eb < need_eq && gb + eb < k) out[gb + eb] = static_cast<int32_t>(v.y);
             g += __popc(mg);
             e += __popc(me);
         }
     }
+}
+
+// Refine and write in one go with the candidates in registers: lane l of warp
+// w owns a contiguous run of at most kOwn (odd) candidates of the warp's segment, so
+// (warp, lane, run index) is position order.  Digit 2 and digit 3 are counted
+// with per-lane shared atomics over the owned keys only; the kept rows' output
+// slots come from one block scan of (rows > T, rows == T) per thread.  Returns
+// false, having written nothing, when a segment holds more than 32 * kOwn
+// candidates (the caller then uses seg_refine + seg_write).  Output slots are
+// bounds-checked against k (they stay below k whenever the histogram the
+// threshold digit came from describes these scores).
+constexpr int kOwn = 9;
+template <class Segs>
+__device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t r2, uint32_t k, uint32_t *hist,
+                                           uint64_t *scan, uint32_t *sel, int32_t *out) {
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint2 *p = sg.ptr(w, 0);
+    const uint32_t c = sg.count(w, 0);
+    const uint32_t m = ((c + 31) / 32) | 1u;  // odd run length: the lanes' loads fall in distinct banks
+    zero_hist(hist, kBins);
+    if (__syncthreads_or(m > static_cast<uint32_t>(kOwn) || sg.pieces(w) != 1)) return false;
+    const uint32_t b0 = min(c, lane * m), b1 = min(c, b0 + m);
+    uint32_t key[kOwn];
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j) key[j] = b0 + j < b1 ? p[b0 + j].x : 0u;
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j)
+        if (b0 + j < b1 && first_digit(key[j]) == d1) atomicAdd(&hist[(key[j] >> 8) & 0xFFFu], 1u);
+    __syncthreads();
+    find_digit(hist, kBins, r2, scan, sel);
+    const uint32_t d2 = sel[0];
+    const uint32_t r3 = r2 - sel[1];
+    const uint32_t p24 = (d1 << 12) | d2;
+    __syncthreads();  // every thread has read sel and hist
+    if (threadIdx.x < kBins3) hist[threadIdx.x] = 0u;
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j)
+        if (b0 + j < b1 && (key[j] >> 8) == p24) atomicAdd(&hist[key[j] & 0xFFu], 1u);
+    __syncthreads();
+    find_digit(hist, kBins3, r3, scan, sel);
+    const uint32_t T = (p24 << 8) | sel[0];
+    const uint32_t need_eq = r3 - sel[1];
+    uint32_t tg = 0, te = 0;
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j) {
+        tg += (b0 + j < b1 && key[j] > T) ? 1u : 0u;
+        te += (b0 + j < b1 && key[j] == T) ? 1u : 0u;
+    }
+    uint64_t tot;
+    const uint64_t ex = block_scan((static_cast<uint64_t>(te) << 32) | tg, scan, tot);
+    uint32_t g = static_cast<uint32_t>(ex & 0xFFFFFFFFu), q = static_cast<uint32_t>(ex >> 32);
+#pragma unroll
+    for (int j = 0; j < kOwn; ++j) {
+        if (b0 + j >= b1) continue;
+        if (key[j] > T) {
+            const uint32_t slot = g + min(q, need_eq);
+            if (slot < k) out[slot] = static_cast<int32_t>(p[b0 + j].y);
+            ++g;
+        } else if (key[j] == T) {
+            if (q < need_eq && g + q < k) out[g + q] = static_cast<int32_t>(p[b0 + j].y);
+            ++q;
+        }
+    }
+    return true;
 }
 
 __device__ __forceinline__ int visible_rows(const TopkArgs &a, int i) {
@@ -339,7 +410,7 @@ __device__ __forceinline__ void write_all(const TopkArgs &a, int i, int n) {
 
 // ---------------------------------------------------------------- row schedule
 struct RowSmem {
-    uint32_t hist[kBins];
+    __align__(16) uint32_t hist[kBins];
     uint2 wbuf[kWarps * kWCap];
     uint32_t wcnt[kWarps], wg[kWarps], we[kWarps];
     uint64_t scan[kWarps];
@@ -347,12 +418,73 @@ struct RowSmem {
     int flag;
 };
 
+// Load kU float4 groups of a warp slice: element e = base + (j * 32 + lane) * 4 + x
+// (elements at or past `hi` read as 0 and are masked by the caller).
+__device__ __forceinline__ void load_warp_batch(const float *row, int base, int hi, float (&v)[kU][4]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < kU; ++j) {
+        const int e0 = base + (j * 32 + lane) * 4;
+        if (e0 + 4 <= hi) {
+            const float4 f = __ldg(reinterpret_cast<const float4 *>(row + e0));
+            v[j][0] = f.x, v[j][1] = f.y, v[j][2] = f.z, v[j][3] = f.w;
+        } else {
+#pragma unroll
+            for (int x = 0; x < 4; ++x) v[j][x] = e0 + x < hi ? __ldg(row + e0 + x) : 0.f;
+        }
+    }
+}
+
+// Append, in position order, the rows of a loaded batch whose first digit is at
+// least d_lo to a warp's (key, position) buffer of capacity cap; cnt counts every
+// such row, also past the capacity.  Groups of 128 rows without a candidate cost
+// one ballot.
+__device__ __forceinline__ void compact_batch(const float (&v)[kU][4], int base, int hi, uint32_t d_lo, uint2 *buf,
+                                              uint32_t cap, uint32_t &cnt) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int j = 0; j < kU; ++j) {
+        const int e0 = base + (j * 32 + lane) * 4;
+        uint32_t u[4], pick = 0;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            u[x] = order_key(v[j][x]);
+            if (e0 + x < hi && first_digit(u[x]) >= d_lo) pick |= 1u << x;
+        }
+        if (__ballot_sync(0xffffffffu, pick != 0u) == 0u) continue;
+        const uint32_t c = __popc(pick);
+        uint32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        uint32_t slot = cnt + incl - c;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            if (pick & (1u << x)) {
+                if (slot < cap) buf[slot] = make_uint2(u[x], static_cast<uint32_t>(e0 + x));
+                ++slot;
+            }
+        }
+        cnt += __shfl_sync(0xffffffffu, incl, 31);
+    }
+}
+
 __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     RowSmem &sm = *reinterpret_cast<RowSmem *>(smem_raw);
     const int i = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     griddep_wait();
+    const bool exact = a.hist_ready != 0;
+    // the histogram does not depend on the position: its loads go out first
+    uint32_t hv[kBins / kT];
+    if (exact) {
+        const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+#pragma unroll
+        for (int j = 0; j < kBins / kT; ++j) hv[j] = __ldg(g + threadIdx.x + j * kT);
+    }
     const int n = visible_rows(a, i);
     if (n <= a.topk) {
         write_all(a, i, n);
@@ -361,13 +493,18 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
     const uint32_t k = static_cast<uint32_t>(a.topk);
     const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
     int32_t *out = a.idx + static_cast<int64_t>(i) * a.topk;
+    // each warp streams a contiguous slice of the row; its first batch is in
+    // flight while the threshold digit is found
+    const int sub = ((n + kWarps - 1) / kWarps + 127) / 128 * 128;
+    const int wlo = min(n, warp * sub), whi = min(n, wlo + sub);
+    float v[kU][4];
+    if (exact) load_warp_batch(row, wlo, whi, v);
 
     // ---- 1. a threshold digit d_lo: rows with first digit >= d_lo are candidates
     uint32_t d_lo, above_exact = 0;
-    const bool exact = a.hist_ready != 0;
     if (exact) {
-        const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
-        load_hist(sm.hist, g);
+#pragma unroll
+        for (int j = 0; j < kBins / kT; ++j) sm.hist[threadIdx.x + j * kT] = hv[j];
         __syncthreads();
         find_digit(sm.hist, kBins, k, sm.scan, sm.sel);
         d_lo = sm.sel[0];
@@ -379,17 +516,17 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
         const int nblk = (n + 127) / 128;
         for (int bi = warp * kSampleEvery; bi < nblk; bi += kWarps * kSampleEvery) {
             const int e0 = bi * 128 + lane * 4;
-            float v[4];
+            float sv[4];
             if (e0 + 4 <= n) {
                 const float4 f = __ldg(reinterpret_cast<const float4 *>(row + e0));
-                v[0] = f.x, v[1] = f.y, v[2] = f.z, v[3] = f.w;
+                sv[0] = f.x, sv[1] = f.y, sv[2] = f.z, sv[3] = f.w;
             } else {
 #pragma unroll
-                for (int x = 0; x < 4; ++x) v[x] = e0 + x < n ? __ldg(row + e0 + x) : 0.f;
+                for (int x = 0; x < 4; ++x) sv[x] = e0 + x < n ? __ldg(row + e0 + x) : 0.f;
             }
 #pragma unroll
             for (int x = 0; x < 4; ++x)
-                hist_add_warp(sm.hist, e0 + x < n ? first_digit(order_key(v[x])) : 0xFFFFFFFFu);
+                hist_add(sm.hist, e0 + x < n ? first_digit(order_key(sv[x])) : 0xFFFFFFFFu);
         }
         __syncthreads();
         // sampled rows, and the rank to look for among them (k scaled, +25% and +64)
@@ -402,51 +539,13 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
     }
     __syncthreads();
 
-    // ---- 2. candidates: each warp streams a contiguous slice of the row
+    // ---- 2. candidates
     {
-        const int sub = ((n + kWarps - 1) / kWarps + 127) / 128 * 128;
-        const int wlo = min(n, warp * sub), whi = min(n, wlo + sub);
         uint2 *mine = sm.wbuf + warp * kWCap;
         uint32_t cnt = 0;
         for (int base = wlo; base < whi; base += 32 * 4 * kU) {
-            float v[kU][4];
-#pragma unroll
-            for (int j = 0; j < kU; ++j) {
-                const int e0 = base + (j * 32 + lane) * 4;
-                if (e0 + 4 <= whi) {
-                    const float4 f = __ldg(reinterpret_cast<const float4 *>(row + e0));
-                    v[j][0] = f.x, v[j][1] = f.y, v[j][2] = f.z, v[j][3] = f.w;
-                } else {
-#pragma unroll
-                    for (int x = 0; x < 4; ++x) v[j][x] = e0 + x < whi ? __ldg(row + e0 + x) : 0.f;
-                }
-            }
-#pragma unroll
-            for (int j = 0; j < kU; ++j) {
-                const int e0 = base + (j * 32 + lane) * 4;
-                uint32_t u[4], pick = 0;
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    u[x] = order_key(v[j][x]);
-                    if (e0 + x < whi && first_digit(u[x]) >= d_lo) pick |= 1u << x;
-                }
-                const uint32_t c = __popc(pick);
-                uint32_t incl = c;
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                    if (lane >= o) incl += y;
-                }
-                uint32_t slot = cnt + incl - c;
-#pragma unroll
-                for (int x = 0; x < 4; ++x) {
-                    if (pick & (1u << x)) {
-                        if (slot < kWCap) mine[slot] = make_uint2(u[x], static_cast<uint32_t>(e0 + x));
-                        ++slot;
-                    }
-                }
-                cnt += __shfl_sync(0xffffffffu, incl, 31);
-            }
+            if (!exact || base != wlo) load_warp_batch(row, base, whi, v);
+            compact_batch(v, base, whi, d_lo, mine, kWCap, cnt);
         }
         if (lane == 0) sm.wcnt[warp] = cnt;
     }
@@ -483,9 +582,11 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
         }
         finish_stream(row, n, k, d1, above1, sm.hist, sm.scan, sm.sel, out);
     } else {
-        uint32_t T, need_eq;
-        seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
-        seg_write(sg, T, need_eq, out, sm.wg, sm.we);
+        if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out)) {
+            uint32_t T, need_eq;
+            seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
+            seg_write(sg, T, need_eq, k, out, sm.wg, sm.we);
+        }
     }
     if (threadIdx.x == 0) a.cnt[i] = a.topk;
 }
@@ -508,113 +609,36 @@ __global__ void __launch_bounds__(kT, 2) topk_hist_kernel(const TopkArgs a, int 
         if (hist[b]) atomicAdd(&g[b], hist[b]);
 }
 
-// (2) the chunk's candidates (first digit >= the threshold digit), in order.
-// Each warp walks a contiguous slice of the chunk and compacts its candidates
-// (warp prefix sums, so position order is kept) into a private buffer; the 16
-// warp counts then place the slices in order.
-__global__ void __launch_bounds__(kT, 2) topk_collect_kernel(const TopkArgs a, int chunk) {
-    __shared__ uint32_t hist[kBins];
-    __shared__ uint64_t scan[kWarps];
-    __shared__ uint32_t sel[4];
-    __shared__ uint2 wbuf[kWarps][kWarpCap];
-    __shared__ uint32_t wcount[kWarps], woff[kWarps + 1];
-    const int i = blockIdx.y, p = blockIdx.x;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    griddep_wait();
-    const int n = visible_rows(a, i);
-    if (n <= a.topk) return;
-    const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
-    const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
-    const int sub = ((hi - lo + kWarps - 1) / kWarps + 127) / 128 * 128;
-    const int wlo = min(hi, lo + warp * sub), whi = min(hi, wlo + sub);
-    auto load_batch = [&](int base0, float (&v)[kU][4]) {
-#pragma unroll
-        for (int j = 0; j < kU; ++j) {
-            const int e0 = base0 + j * 128 + lane * 4;
-            if (e0 + 4 <= whi) {
-                const float4 f = __ldg(reinterpret_cast<const float4 *>(row + e0));
-                v[j][0] = f.x, v[j][1] = f.y, v[j][2] = f.z, v[j][3] = f.w;
-            } else {
-#pragma unroll
-                for (int x = 0; x < 4; ++x) v[j][x] = e0 + x < whi ? __ldg(row + e0 + x) : 0.f;
-            }
-        }
-    };
-    float v[kU][4];
-    load_batch(wlo, v);  // in flight while the threshold digit is found
-    const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
-    load_hist(hist, g);
-    __syncthreads();
-    find_digit(hist, kBins, static_cast<uint32_t>(a.topk), scan, sel);
-    const uint32_t d1 = sel[0];
-    if (p == 0 && threadIdx.x == 0) {  // the merge reads the threshold digit from here
-        a.gdigit[2 * i] = d1;
-        a.gdigit[2 * i + 1] = sel[1];
-    }
-    uint32_t cnt = 0;
-    for (int base0 = wlo; base0 < whi; base0 += 128 * kU) {
-        if (base0 != wlo) load_batch(base0, v);
-#pragma unroll
-        for (int j = 0; j < kU; ++j) {
-            const int e0 = base0 + j * 128 + lane * 4;
-            uint32_t u[4], pick = 0;
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                u[x] = order_key(v[j][x]);
-                if (e0 + x < whi && first_digit(u[x]) >= d1) pick |= 1u << x;
-            }
-            const uint32_t c = __popc(pick);
-            uint32_t incl = c;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (lane >= o) incl += y;
-            }
-            uint32_t slot = cnt + incl - c;
-#pragma unroll
-            for (int x = 0; x < 4; ++x) {
-                if (pick & (1u << x)) {
-                    if (slot < kWarpCap) wbuf[warp][slot] = make_uint2(u[x], static_cast<uint32_t>(e0 + x));
-                    ++slot;
-                }
-            }
-            cnt += __shfl_sync(0xffffffffu, incl, 31);
-        }
-    }
-    if (lane == 0) wcount[warp] = cnt;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        uint32_t o = 0;
-        bool over = false;
-        for (int w = 0; w < kWarps; ++w) {
-            woff[w] = o;
-            o += wcount[w];
-            over |= wcount[w] > static_cast<uint32_t>(kWarpCap);
-        }
-        // a warp buffer that overflowed makes the chunk report more than the
-        // per-chunk capacity, which sends the query down the streaming path
-        woff[kWarps] = over ? static_cast<uint32_t>(kSplitCap) + 1u : o;
-    }
-    __syncthreads();
-    const uint32_t total = woff[kWarps];
-    uint2 *dst = a.gcand + (static_cast<int64_t>(i) * kSplitMax + p) * kSplitCap;
-    if (total <= static_cast<uint32_t>(kSplitCap)) {
-        const uint32_t c = wcount[warp];
-        for (uint32_t j = lane; j < c; j += 32) dst[woff[warp] + j] = wbuf[warp][j];
-    }
-    if (threadIdx.x == 0) a.gcount[static_cast<int64_t>(i) * kSplitMax + p] = total;
-}
+// (2) one launch per query set: every CTA collects its chunk's candidates (first
+// digit >= the threshold digit) in position order -- each warp compacts a
+// contiguous slice into a private buffer, the 16 warp counts place the slices --
+// and the last CTA of a query to finish (a ticket in global memory) walks all the
+// chunks' candidates in position order and writes the query's result.
+struct CollectSmem {
+    __align__(16) uint32_t hist[kBins];
+    uint64_t scan[kWarps];
+    uint32_t sel[4];
+    uint2 wbuf[kWarps][kWarpCap];
+    uint32_t wcount[kWarps], woff[kWarps + 1];
+};
 
-// (3) walk the chunks' candidates in position order and finish the query.
-// The candidates are first staged in shared memory (independent loads), laid
-// out as warp segments: warp w's chunks, in order, at a running offset.
+// The finishing CTA: candidates staged in shared memory as warp segments (warp
+// w's chunks, in order, at a running offset).
 struct MergeSmem {
-    uint32_t hist[kBins];
+    __align__(16) uint32_t hist[kBins];
     uint2 cand[kWarps * kWCap];
     uint32_t coff[kSplitMax + 1];
     uint32_t wcnt[kWarps], wg[kWarps], we[kWarps];
     uint64_t scan[kWarps];
     uint32_t sel[4];
+};
+
+struct SplitSmem {
+    union {
+        CollectSmem c;
+        MergeSmem m;
+    } u;
+    int last;
 };
 
 struct StagedSegs {  // warp w: candidates [wbeg[w], wbeg[w] + wcnt[w]) of one array
@@ -628,24 +652,17 @@ struct StagedSegs {  // warp w: candidates [wbeg[w], wbeg[w] + wcnt[w]) of one a
     }
 };
 
-__global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int n_chunks) {
-    extern __shared__ __align__(16) uint8_t smem_raw[];
-    MergeSmem &sm = *reinterpret_cast<MergeSmem *>(smem_raw);
-    const int i = blockIdx.x;
-    griddep_wait();
-    const int n = visible_rows(a, i);
-    if (n <= a.topk) {
-        write_all(a, i, n);
-        return;
-    }
+// Finish query i from the chunks' candidates (written by other CTAs of this
+// launch: read through L2).
+__device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int n_chunks, uint32_t d1,
+                                            uint32_t above1, MergeSmem &sm) {
     const uint32_t k = static_cast<uint32_t>(a.topk);
     const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
     int32_t *out = a.idx + static_cast<int64_t>(i) * a.topk;
-    const uint32_t d1 = a.gdigit[2 * i], above1 = a.gdigit[2 * i + 1];  // from collect chunk 0
     const uint32_t *counts = a.gcount + static_cast<int64_t>(i) * kSplitMax;
     // chunk counts -> offsets (a block scan; count > cap marks an overflow)
     {
-        const uint32_t c = threadIdx.x < n_chunks ? counts[threadIdx.x] : 0u;
+        const uint32_t c = threadIdx.x < n_chunks ? __ldcg(counts + threadIdx.x) : 0u;
         const uint64_t ov = c > static_cast<uint32_t>(kSplitCap) ? 1ull : 0ull;
         uint64_t tot;
         const uint64_t ex = block_scan((ov << 32) | c, sm.scan, tot);
@@ -661,7 +678,10 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int
     if (overflow) {
         finish_stream(row, n, k, d1, above1, sm.hist, sm.scan, sm.sel, out);
     } else {
-        // stage: warp w copies chunks w, w + 16, ... (all loads independent)
+        // stage: warp w copies chunks w, w + 16, ... with asynchronous copies
+        // (all in flight at once).  The L1-allocating form is safe here: this
+        // CTA is the only reader of these lines in this launch, after every
+        // writer's fence, so no earlier copy of them can sit in this SM's L1.
         const uint2 *src = a.gcand + static_cast<int64_t>(i) * kSplitMax * kSplitCap;
         for (int p = threadIdx.x >> 5; p < n_chunks; p += kWarps) {
             const uint32_t c = sm.coff[p + 1] - sm.coff[p];
@@ -674,11 +694,85 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkArgs a, int
         cp_async_wait_all();
         __syncthreads();
         const StagedSegs sg{sm.cand, sm.coff, n_chunks};
-        uint32_t T, need_eq;
-        seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
-        seg_write(sg, T, need_eq, out, sm.wg, sm.we);
+        if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out)) {
+            uint32_t T, need_eq;
+            seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
+            seg_write(sg, T, need_eq, k, out, sm.wg, sm.we);
+        }
     }
     if (threadIdx.x == 0) a.cnt[i] = a.topk;
+}
+
+__global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int chunk, int n_chunks) {
+    extern __shared__ __align__(16) uint8_t smem_raw[];
+    SplitSmem &ss = *reinterpret_cast<SplitSmem *>(smem_raw);
+    CollectSmem &cs = ss.u.c;
+    const int i = blockIdx.y, p = blockIdx.x;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_wait();
+    // the histogram does not depend on the position: its loads go out first
+    uint32_t hv[kBins / kT];
+    {
+        const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+#pragma unroll
+        for (int j = 0; j < kBins / kT; ++j) hv[j] = __ldg(g + threadIdx.x + j * kT);
+    }
+    const int n = visible_rows(a, i);
+    if (n <= a.topk) {  // every chunk of the query sees the same n
+        if (p == 0) write_all(a, i, n);
+        return;
+    }
+    const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
+    const float *row = a.scores + static_cast<int64_t>(i) * a.ld;
+    const int sub = ((hi - lo + kWarps - 1) / kWarps + 127) / 128 * 128;
+    const int wlo = min(hi, lo + warp * sub), whi = min(hi, wlo + sub);
+    float v[kU][4];
+    load_warp_batch(row, wlo, whi, v);  // in flight while the threshold digit is found
+#pragma unroll
+    for (int j = 0; j < kBins / kT; ++j) cs.hist[threadIdx.x + j * kT] = hv[j];
+    __syncthreads();
+    find_digit(cs.hist, kBins, static_cast<uint32_t>(a.topk), cs.scan, cs.sel);
+    const uint32_t d1 = cs.sel[0], above1 = cs.sel[1];
+    uint32_t cnt = 0;
+    for (int base0 = wlo; base0 < whi; base0 += 128 * kU) {
+        if (base0 != wlo) load_warp_batch(row, base0, whi, v);
+        compact_batch(v, base0, whi, d1, cs.wbuf[warp], kWarpCap, cnt);
+    }
+    if (lane == 0) cs.wcount[warp] = cnt;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        uint32_t o = 0;
+        bool over = false;
+        for (int w = 0; w < kWarps; ++w) {
+            cs.woff[w] = o;
+            o += cs.wcount[w];
+            over |= cs.wcount[w] > static_cast<uint32_t>(kWarpCap);
+        }
+        // a warp buffer that overflowed makes the chunk report more than the
+        // per-chunk capacity, which sends the query down the streaming path
+        cs.woff[kWarps] = over ? static_cast<uint32_t>(kSplitCap) + 1u : o;
+    }
+    __syncthreads();
+    const uint32_t total = cs.woff[kWarps];
+    uint2 *dst = a.gcand + (static_cast<int64_t>(i) * kSplitMax + p) * kSplitCap;
+    if (total <= static_cast<uint32_t>(kSplitCap)) {
+        const uint32_t c = cs.wcount[warp];
+        for (uint32_t j = lane; j < c; j += 32) dst[cs.woff[warp] + j] = cs.wbuf[warp][j];
+    }
+    if (threadIdx.x == 0) a.gcount[static_cast<int64_t>(i) * kSplitMax + p] = total;
+
+    // ---- publish; the last CTA of the query finishes it
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const uint32_t prev = atomicAdd(a.gticket + i, 1u);
+        ss.last = prev == static_cast<uint32_t>(n_chunks - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!ss.last) return;
+    __threadfence();
+    merge_query(a, i, n, n_chunks, d1, above1, ss.u.m);
+    if (threadIdx.x == 0) a.gticket[i] = 0;  // every chunk has arrived: ready for the next launch
 }
 
 // P chunks per query so that about two CTAs per SM take part; chunks are
@@ -713,36 +807,38 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
     int P, chunk;
     split_plan(a, num_sms, P, chunk);
     if (!a.hist_ready) {
-        if ((e = cudaMemsetAsync(a.ghist, 0, sizeof(uint32_t) * kBins * a.n_q, st)) != cudaSuccess) return e;
+        if ((e = cudaMemsetAsync(a.ghist, 0, topk_zeroed_bytes(a.n_q), st)) != cudaSuccess) return e;
         if ((e = launch_pdl(topk_hist_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk)) != cudaSuccess) return e;
     }
-    if ((e = launch_pdl(topk_collect_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(sizeof(MergeSmem)))) != cudaSuccess)
+    if ((e = cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(sizeof(SplitSmem)))) != cudaSuccess)
         return e;
-    return launch_pdl(topk_merge_kernel, dim3(a.n_q), dim3(kT), sizeof(MergeSmem), st, a, P);
+    return launch_pdl(topk_split_kernel, dim3(P, a.n_q), dim3(kT), sizeof(SplitSmem), st, a, chunk, P);
 }
 
+size_t topk_zeroed_bytes(int n_q) { return sizeof(uint32_t) * (static_cast<size_t>(kBins) + 1) * n_q; }
+
+// Scratch: [n_q][4096] first-digit histograms, then [n_q] tickets (both zeroed
+// before every launch by the call that fills the histograms); the split
+// schedule adds [n_q][kSplitMax] candidate counts and the candidates.
 size_t topk_scratch_bytes(int n_q, int max_ctx) {
-    const size_t hist = sizeof(uint32_t) * kBins * n_q;
     auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    if (!topk_uses_split(n_q, max_ctx)) return al(hist);
+    const size_t hist = al(topk_zeroed_bytes(n_q));
+    if (!topk_uses_split(n_q, max_ctx)) return hist;
     const size_t counts = sizeof(uint32_t) * kSplitMax * n_q;
-    const size_t digits = sizeof(uint32_t) * 2 * n_q;
     const size_t cand = sizeof(uint2) * static_cast<size_t>(kSplitCap) * kSplitMax * n_q;
-    return al(hist) + al(counts) + al(digits) + al(cand);
+    return hist + al(counts) + al(cand);
 }
 
 void topk_bind_scratch(TopkArgs &a, void *scratch) {
     auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     uint8_t *p = static_cast<uint8_t *>(scratch);
     a.ghist = reinterpret_cast<uint32_t *>(p);
+    a.gticket = a.ghist + static_cast<size_t>(kBins) * a.n_q;
     if (!topk_uses_split(a.n_q, a.L)) return;
-    p += al(sizeof(uint32_t) * kBins * a.n_q);
+    p += al(topk_zeroed_bytes(a.n_q));
     a.gcount = reinterpret_cast<uint32_t *>(p);
     p += al(sizeof(uint32_t) * kSplitMax * a.n_q);
-    a.gdigit = reinterpret_cast<uint32_t *>(p);
-    p += al(sizeof(uint32_t) * 2 * a.n_q);
     a.gcand = reinterpret_cast<uint2 *>(p);
 }
 
