@@ -37,10 +37,10 @@ DECODE_MAX_QUERIES = 256    # the MLA decode (split-K) schedule up to this many 
 L2_FLUSH_BYTES = 256 << 20
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch, from the ncu
-# capture summarised in profiles/idx_score_tc_decode_1m.md (one sequence of 1M keys:
-# 276.2 MB; the 4-sequence launch streams 4 such caches, so traffic x 4).  Absent
-# workloads report null.
-NCU_INDEXER_TRAFFIC = {"decode_1m": 4 * 276.2e6}
+# captures summarised in profiles/idx_score_tc_decode.md: 8 x 32K keys captured at
+# full size (67.61 MB); one sequence of 1M keys (275.13 MB), whose 4-sequence
+# launch streams 4 such caches (traffic x 4).  Absent workloads report null.
+NCU_INDEXER_TRAFFIC = {"decode_32k": 67.61e6, "decode_1m": 4 * 275.13e6}
 
 
 def measured_peaks():

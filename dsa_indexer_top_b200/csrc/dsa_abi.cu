@@ -100,9 +100,8 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
                            uint32_t *status, uint32_t *ghist, cudaStream_t st) {
     // the histograms are left only when queries are not tiled together (odd
     // seq_run: one query per tensor-core tile, where the epilogue builds them)
+    // (the histograms are zero on entry: see topk_scratch_bytes)
     if ((qs->seq_run & 1) == 0) ghist = nullptr;
-    if (ghist && cudaMemsetAsync(ghist, 0, topk_zeroed_bytes(qs->n_q), st) != cudaSuccess)
-        return DSA_ERR_CUDA;
     bool hist_done = false;
     dsa_status s = DSA_OK;
     const int n_cache = ix->k_seq_stride == 0 ? 1 : qs->n_seq;
@@ -329,8 +328,8 @@ size_t dsa_workspace_bytes(int32_t op, const dsa_queries *qs, int32_t topk, int3
 
 dsa_status dsa_workspace_init(void *ws, size_t ws_bytes, void *stream) {
     if (!ws_ok(ws, ws_bytes, kStatusBytes)) return DSA_ERR_WORKSPACE;
-    return cudaMemsetAsync(ws, 0, kStatusBytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSA_OK
-                                                                                                   : DSA_ERR_CUDA;
+    return cudaMemsetAsync(ws, 0, ws_bytes, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSA_OK
+                                                                                               : DSA_ERR_CUDA;
 }
 
 dsa_status dsa_check_status(void *ws, void *stream) {

@@ -377,25 +377,40 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
 }
 
 // Merge split-K partials: o = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s.
-// One CTA per (4 heads, query, layer).
+// One CTA per (2 heads, query, layer), 256 threads: thread t owns 4 dims of
+// head 2 * blockIdx.x + t / 128.  The partials of the first 16 splits are loaded
+// (16-byte loads, all in flight) before the split weights are known: the merge
+// is one round trip to L2 plus the weight shuffles.
+constexpr int kCombineHeads = 2;
+constexpr int kCombineBatch = 16;  // splits whose partials are held in registers at once
+
 __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
-    const int hg = blockIdx.x, i = blockIdx.y, layer = blockIdx.z;
+    const int hp = blockIdx.x, i = blockIdx.y, layer = blockIdx.z;
     const MlaLayerPtrs lp = a.layer[layer];
-    __shared__ float wgt[4][32];
-    griddep_wait();  // splits per query: at most 16 by the planner
+    __shared__ float wgt[kCombineHeads][32];
+    griddep_wait();  // splits per query: at most 32 by the planner
     int cnt = a.cnt[i];
     if (cnt < 0 || cnt > a.topk) cnt = 0;
     const int nch = (cnt + kChunk - 1) / kChunk;
     const int ns = min(32, (nch + a.chunks_per_cta - 1) / a.chunks_per_cta);
     const int64_t base = (static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits;
-    // (max, sum) of every split for the 4 heads: one thread per (head, split)
+    const int hl = threadIdx.x >> 7;
+    const int h = hp * kCombineHeads + hl;
+    const int d = (threadIdx.x & 127) * 4;
+    const float *po = a.part_o + (base * kMlaHeads + h) * kLatent + d;  // split s at + s * kMlaHeads * kLatent
+    float4 x[kCombineBatch];
+#pragma unroll
+    for (int s = 0; s < kCombineBatch; ++s)
+        x[s] = s < ns ? *reinterpret_cast<const float4 *>(po + static_cast<int64_t>(s) * kMlaHeads * kLatent)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+    // (max, sum) of every split: warp w < 2 handles head 2 * hp + w, lane = split
     {
-        const int hl = threadIdx.x >> 5, s = threadIdx.x & 31;  // warps 0-3: one head each
-        if (hl < 4) {
-            const int h = hg * 4 + hl;
+        const int wl = threadIdx.x >> 5, s = threadIdx.x & 31;
+        if (wl < kCombineHeads) {
+            const int hh = hp * kCombineHeads + wl;
             float m = -INFINITY, l = 0.f;
             if (s < ns) {
-                const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + ((base + s) * kMlaHeads + h) * 2);
+                const float2 ml = *reinterpret_cast<const float2 *>(a.part_ml + ((base + s) * kMlaHeads + hh) * 2);
                 m = ml.x;
                 l = ml.y;
             }
@@ -406,30 +421,26 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
             float L = wv * l;
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-            if (s < ns) wgt[hl][s] = wv / L;
-            if (s == 0 && lp.lse) lp.lse[static_cast<int64_t>(i) * kMlaHeads + h] = (M + log2f(L)) * kLn2;
+            wgt[wl][s] = s < ns ? wv / L : 0.f;
+            if (s == 0 && lp.lse) lp.lse[static_cast<int64_t>(i) * kMlaHeads + hh] = (M + log2f(L)) * kLn2;
         }
     }
     __syncthreads();
-    // 4 heads x 512 dims = 2048 outputs, 8 per thread
-    const int e = threadIdx.x * 8;
-    const int hl = e / kLatent, d = e % kLatent;
-    const int h = hg * 4 + hl;
-    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll 8
-    for (int s = 0; s < ns; ++s) {
-        const float *po = a.part_o + ((base + s) * kMlaHeads + h) * kLatent + d;
-        const float4 x0 = *reinterpret_cast<const float4 *>(po);
-        const float4 x1 = *reinterpret_cast<const float4 *>(po + 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int s = 0; s < kCombineBatch; ++s) {
         const float wv = wgt[hl][s];
-        acc[0] += wv * x0.x; acc[1] += wv * x0.y; acc[2] += wv * x0.z; acc[3] += wv * x0.w;
-        acc[4] += wv * x1.x; acc[5] += wv * x1.y; acc[6] += wv * x1.z; acc[7] += wv * x1.w;
+        acc.x += wv * x[s].x, acc.y += wv * x[s].y, acc.z += wv * x[s].z, acc.w += wv * x[s].w;
+    }
+    for (int s = kCombineBatch; s < ns; ++s) {  // more than 16 splits (long contexts, few queries)
+        const float4 y = *reinterpret_cast<const float4 *>(po + static_cast<int64_t>(s) * kMlaHeads * kLatent);
+        const float wv = wgt[hl][s];
+        acc.x += wv * y.x, acc.y += wv * y.y, acc.z += wv * y.z, acc.w += wv * y.w;
     }
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(lp.out) + (static_cast<int64_t>(i) * kMlaHeads + h) * kLatent + d;
-    __align__(16) __nv_bfloat16 ob[8];
-#pragma unroll
-    for (int x = 0; x < 8; ++x) ob[x] = __float2bfloat16_rn(acc[x]);
-    *reinterpret_cast<uint4 *>(o) = *reinterpret_cast<const uint4 *>(ob);
+    __align__(8) __nv_bfloat16 ob[4] = {__float2bfloat16_rn(acc.x), __float2bfloat16_rn(acc.y),
+                                        __float2bfloat16_rn(acc.z), __float2bfloat16_rn(acc.w)};
+    *reinterpret_cast<uint2 *>(o) = *reinterpret_cast<const uint2 *>(ob);
 }
 
 // ---------------------------------------------------------------- generic path
@@ -532,7 +543,7 @@ cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st) {
 }
 
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st) {
-    dim3 grid(kMlaHeads / 4, a.n_q, a.n_layers);
+    dim3 grid(kMlaHeads / kCombineHeads, a.n_q, a.n_layers);
     return launch_pdl(mla_combine_kernel, grid, dim3(256), 0, st, a);
 }
 

@@ -486,6 +486,11 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
         for (int j = 0; j < kBins / kT; ++j) hv[j] = __ldg(g + threadIdx.x + j * kT);
     }
     const int n = visible_rows(a, i);
+    if (exact) {  // leave the histogram zero for the next indexer launch
+        uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+#pragma unroll
+        for (int j = 0; j < kBins / kT; ++j) g[threadIdx.x + j * kT] = 0u;
+    }
     if (n <= a.topk) {
         write_all(a, i, n);
         return;
@@ -719,7 +724,11 @@ __global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int
     }
     const int n = visible_rows(a, i);
     if (n <= a.topk) {  // every chunk of the query sees the same n
-        if (p == 0) write_all(a, i, n);
+        if (p == 0) {
+            write_all(a, i, n);
+            uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;  // zero for the next launch
+            for (int b = threadIdx.x; b < kBins; b += kT) g[b] = 0u;
+        }
         return;
     }
     const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
@@ -771,8 +780,14 @@ __global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int
     __syncthreads();
     if (!ss.last) return;
     __threadfence();
+    // every chunk has read the histogram and taken its ticket: leave both zero
+    // for the next launch
+    {
+        uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
+        for (int b = threadIdx.x; b < kBins; b += kT) g[b] = 0u;
+        if (threadIdx.x == 0) a.gticket[i] = 0;
+    }
     merge_query(a, i, n, n_chunks, d1, above1, ss.u.m);
-    if (threadIdx.x == 0) a.gticket[i] = 0;  // every chunk has arrived: ready for the next launch
 }
 
 // P chunks per query so that about two CTAs per SM take part; chunks are
@@ -818,9 +833,11 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
 
 size_t topk_zeroed_bytes(int n_q) { return sizeof(uint32_t) * (static_cast<size_t>(kBins) + 1) * n_q; }
 
-// Scratch: [n_q][4096] first-digit histograms, then [n_q] tickets (both zeroed
-// before every launch by the call that fills the histograms); the split
-// schedule adds [n_q][kSplitMax] candidate counts and the candidates.
+// Scratch: [n_q][4096] first-digit histograms, then [n_q] tickets.  Both are
+// zero between calls: dsa_workspace_init zeroes them, a top-k launch zeroes
+// each query's histogram and ticket once it has used them, and the one launch
+// that builds histograms without an indexer (hist_ready == 0) zeroes them first.
+// The split schedule adds [n_q][kSplitMax] candidate counts and the candidates.
 size_t topk_scratch_bytes(int n_q, int max_ctx) {
     auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
     const size_t hist = al(topk_zeroed_bytes(n_q));

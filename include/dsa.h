@@ -40,8 +40,8 @@
  *  - Workspace: `ws` is a device buffer of at least dsa_workspace_bytes(...)
  *    bytes, 256-byte aligned.  Its first 256 bytes hold a status word that
  *    kernels set on device-detected errors (out-of-range positions or indices,
- *    a bounded wait that ran out).  Zero it once with dsa_workspace_init();
- *    read (and clear) it with dsa_check_status().
+ *    a bounded wait that ran out).  Zero the workspace once with
+ *    dsa_workspace_init(); read (and clear) the status with dsa_check_status().
  *  - Errors: invalid arguments are rejected synchronously, before any launch,
  *    with DSA_ERR_INVALID (null pointer, bad size, misaligned row, workspace too
  *    small -> DSA_ERR_WORKSPACE); a launch failure returns DSA_ERR_CUDA.  A call
@@ -81,7 +81,12 @@ enum {
      * first pass of dsa_topk; on the tensor-core path it is built in the
      * epilogue at no extra pass).  The workspace must then be at least
      * dsa_workspace_bytes(DSA_OP_TOPK, ...) bytes.  Honoured only when
-     * queries->seq_run is odd (queries not tiled together); ignored otherwise. */
+     * queries->seq_run is odd (queries not tiled together); ignored otherwise.
+     * The histogram region is expected to be zero on entry (no memset per
+     * call): dsa_workspace_init zeroes it and dsa_topk zeroes it again once it
+     * has used it, so every dsa_index_scores with this flag must be followed by
+     * a dsa_topk on the same workspace before the next one (as
+     * dsa_indexshare_group does), or the workspace re-initialised. */
     DSA_INDEXER_TOPK_HIST = 1,
     /* dsa_topk flags: the workspace holds that histogram for these scores (the
      * preceding dsa_index_scores on the same scores, queries and workspace had
@@ -279,7 +284,9 @@ dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *i
 size_t dsa_workspace_bytes(int32_t op, const dsa_queries *queries, int32_t topk, int32_t mla_heads,
                            int32_t d_latent, int32_t n_layers);
 
-/* Zero the status word of a workspace (async on `stream`). */
+/* Zero a whole workspace, status word included (async on `stream`).  Call
+ * once after allocating it (and after any failed call that may have left it
+ * half-updated). */
 dsa_status dsa_workspace_init(void *ws, size_t ws_bytes, void *stream);
 
 /*

@@ -65,6 +65,32 @@ def _run_steps(w, x, decode=True, fused=True):
     return scores, idx, cnt, mlas
 
 
+@pytest.mark.parametrize("name", ["decode_edges", "decode_ragged", "ties"])
+@pytest.mark.parametrize("L_long", [False, True])
+def test_repeated_steps_one_workspace(dev, name, L_long):
+    """Several fused indexer -> top-k steps on one workspace: the top-k leaves the
+    histograms and tickets zero for the next indexer launch, so every step
+    matches the oracle (L_long: a context above the split-schedule threshold)."""
+    w = SMALL[name]
+    if L_long:
+        w = wl.scaled(w, L=20000, q_pos=tuple(min(19999, p + 15000) for p in w.q_pos))
+    xh = wl.make_inputs(w, layers=[])
+    x = C.to_device(xh)
+    q, ix, _ = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ix.flags = B.DSA_INDEXER_TOPK_HIST
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, 1, dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    _, ridx, rcnt = C.oracle_selection(w, xh)
+    for step in range(3):
+        idx = torch.full((w.n_q, w.topk), -7, dtype=torch.int32, device=dev)
+        cnt = torch.full((w.n_q,), -7, dtype=torch.int32, device=dev)
+        B.dsa_index_scores(q, ix, scores, ws)
+        B.dsa_topk(q, scores, w.topk, idx, cnt, ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+        assert B.dsa_check_status(ws) == B.DSA_OK
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt, err_msg=f"step {step}")
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 def test_index_scores_bit_exact(dev, name):
     w = SMALL[name]
