@@ -19,12 +19,13 @@
 //            operands K-major): 36 tcgen05.mma into TMEM columns 64*slot; then
 //            O^T += C_lat^T . P^T (the row tile read MN-major: M = 4 x 128 latent
 //            dims, N = 64 heads, K = 64 rows) into columns 128..383.
-//   softmax (warps 0-3)   thread lane < 16 of warp w owns head 16w + lane (the
-//            M = 64 accumulator layout keeps rows 16w..16w+15 in lanes
-//            32w..32w+15): running max, exponentials and sum of its head over
-//            the chunk's 64 rows in registers; P (bf16) as one 128-byte line per
-//            head in the slot's freed RoPE block; the accumulated O is rescaled
-//            only when a head's maximum grows by more than 2^8.
+//   softmax (warps 0-3)   the M = 64 accumulator keeps heads 16w..16w+15 in
+//            lanes 32w..32w+15; lanes l and l + 16 of warp w share head 16w + l
+//            (rows 0..31 and 32..63 of the chunk, one 16x32bx2 TMEM load):
+//            running max, exponentials and sum in registers, combined with one
+//            shuffle; P (bf16) as one 128-byte line per head in the slot's freed
+//            RoPE block; the accumulated O is rescaled only when a head's maximum
+//            grows by more than 2^8.
 //   epilogue (warps 0-7)  reads O^T from TMEM: the final bf16 output (one CTA
 //            per query) or fp32 partials + (max, sum) per head for a split-K
 //            merge (decode with few queries).
@@ -232,8 +233,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
         }
     } else {
         // ------------------------------------------------------------ softmax
-        const bool owner = lane < 16;
+        // Head 16w + (lane & 15) is held by two lanes: lane < 16 takes the chunk's
+        // rows 0..31, lane + 16 rows 32..63 (one tcgen05.ld of shape 16x32bx2);
+        // the two combine their maximum and their sum with one shuffle each and
+        // keep identical running (m, l).
         const int h = 16 * warp + (lane & 15);
+        const int rbase = 32 * (lane >> 4);  // first chunk row of this lane
         const uint32_t lane_base = tbase + (static_cast<uint32_t>(warp * 32) << 16);
         float m = -INFINITY, l = 0.f;
         uint32_t sm_phase = 0;
@@ -244,23 +249,21 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             tc_fence_after();
             float mc = -INFINITY;
             {
-                uint32_t r0[32], r1[32];
-                tmem_ld32(lane_base + 64 * s, r0);
-                tmem_ld32(lane_base + 64 * s + 32, r1);
+                uint32_t r[32];
+                tmem_ld16x2_32<32>(lane_base + 64 * s, r);
                 tmem_ld_wait();
 #pragma unroll
-                for (int x = 0; x < 64; ++x) {
-                    const float v = u2f(x < 32 ? r0[x] : r1[x - 32]);
-                    if (row_idx[s][x] >= 0) mc = fmaxf(mc, v);
-                }
+                for (int x = 0; x < 32; ++x)
+                    if (row_idx[s][rbase + x] >= 0) mc = fmaxf(mc, u2f(r[x]));
             }
+            mc = fmaxf(mc, __shfl_xor_sync(0xffffffffu, mc, 16));
             float al = 1.f;
-            if (owner && mc != -INFINITY && (m == -INFINITY || (mc - m) * c2 > kRescaleLog2)) {
+            if (mc != -INFINITY && (m == -INFINITY || (mc - m) * c2 > kRescaleLog2)) {
                 al = (m == -INFINITY) ? 0.f : exp2f((m - mc) * c2);
                 m = mc;
             }
-            if (owner) alpha_sm[h] = al;
-            const bool need = __any_sync(0xffffffffu, owner && al != 1.f && t > 0);
+            if (lane < 16) alpha_sm[h] = al;
+            const bool need = __any_sync(0xffffffffu, al != 1.f && t > 0);
             if (lane == 0) rescale_w[warp] = need ? 1 : 0;
             // the four softmax warps meet: every head's alpha is needed below
             __syncwarp();
@@ -291,26 +294,26 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                 }
                 tmem_st_wait();
             }
-            uint32_t r0[32], r1[32];  // the chunk's logits again (cheaper than keeping them live)
-            tmem_ld32(lane_base + 64 * s, r0);
-            tmem_ld32(lane_base + 64 * s + 32, r1);
+            uint32_t r[32];  // the chunk's logits again (cheaper than keeping them live)
+            tmem_ld16x2_32<32>(lane_base + 64 * s, r);
             tmem_ld_wait();
-            if (owner) {
-                uint8_t *pl = slot_sm + s * kSlotBytes + 8 * kBlockBytes;  // this head's P line
+            {
+                uint8_t *pl = slot_sm + s * kSlotBytes + 8 * kBlockBytes;  // head h's P line
                 float sum = 0.f;
 #pragma unroll
-                for (int jc = 0; jc < 8; ++jc) {
+                for (int jc = 0; jc < 4; ++jc) {
                     __align__(16) __nv_bfloat16 pb[8];
 #pragma unroll
                     for (int x = 0; x < 8; ++x) {
-                        const int row = 8 * jc + x;
-                        const float v = u2f(row < 32 ? r0[row] : r1[row - 32]);
-                        const float pf = (row_idx[s][row] >= 0) ? exp2f((v - m) * c2) : 0.f;
+                        const int xr = 8 * jc + x;
+                        const float pf = (row_idx[s][rbase + xr] >= 0) ? exp2f((u2f(r[xr]) - m) * c2) : 0.f;
                         pb[x] = __float2bfloat16_rn(pf);
                         sum += __bfloat162float(pb[x]);  // the sum uses the value the MMA sees
                     }
-                    *reinterpret_cast<uint4 *>(pl + sw128_offset(h, jc)) = *reinterpret_cast<const uint4 *>(pb);
+                    *reinterpret_cast<uint4 *>(pl + sw128_offset(h, (rbase >> 3) + jc)) =
+                        *reinterpret_cast<const uint4 *>(pb);
                 }
+                sum += __shfl_xor_sync(0xffffffffu, sum, 16);
                 l = l * al + sum;
             }
             fence_proxy_async_smem();
@@ -318,7 +321,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[s]);
         }
-        if (owner) {
+        if (lane < 16) {
             m_fin[h] = m;
             l_fin[h] = l;
         }
