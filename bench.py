@@ -218,35 +218,85 @@ class Step:
 
 
 class E2EStep:
-    """The same step through the public API with host buffers: copy the step's
-    query inputs from pinned host memory, run, copy the outputs back."""
+    """The same step through the public API with host buffers: the step's query
+    inputs are copied from pinned host memory, the library calls run, and the
+    outputs (attention output of every layer, the selected indices) are copied
+    back.  Inputs and outputs are packed into 256-byte aligned views of a few
+    device buffers, as a caller batching its per-step host traffic would, and
+    the copies overlap the work that does not need them: the MLA queries (most
+    of the input bytes) travel on a side stream while the indexer runs, and the
+    indices go back while the MLA runs."""
 
     def __init__(self, step: Step):
         self.s = step
-        x = step.x
-        self.h_in = {k: x[k].cpu().pin_memory() for k in ("q_idx", "w", "q_seq", "q_pos")}
-        self.h_qmla = [t.cpu().pin_memory() for t in x["q_mla"]]
-        self.h_out = [torch.empty(m.out.shape, dtype=m.out.dtype).pin_memory() for m in step.mlas]
-        self.h_idx = torch.empty(step.idx.shape, dtype=torch.int32).pin_memory()
-        self.h2d = sum(t.numel() * t.element_size() for t in list(self.h_in.values()) + self.h_qmla)
-        self.d2h = sum(t.numel() * t.element_size() for t in self.h_out) + self.h_idx.numel() * 4
+        w, x = step.w, step.x
+        dev = step.dev
+        self.d_in_ix, self.h_in_ix, vix = self._pack(
+            [("q_idx", x["q_idx"]), ("w", x["w"]), ("q_seq", x["q_seq"]), ("q_pos", x["q_pos"])], dev, fill=True)
+        self.d_in_mla, self.h_in_mla, vmla = self._pack(
+            [(f"q_mla{l}", t) for l, t in enumerate(x["q_mla"])], dev, fill=True)
+        self.d_out, self.h_out, vout = self._pack([(f"out{l}", m.out) for l, m in enumerate(step.mlas)], dev,
+                                                  fill=False)
+        self.d_idx, self.h_idx, vidx = self._pack([("idx", step.idx)], dev, fill=False)
+        self.h2d = self.h_in_ix.numel() + self.h_in_mla.numel()
+        self.d2h = self.h_out.numel() + self.h_idx.numel()
+        # descriptors over the packed views (caches, scores, counts and workspace are the step's)
+        self.q = B.Queries(vix["q_seq"], vix["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=step.seq_run)
+        self.ix = B.Indexer(vix["q_idx"], vix["w"], step.ix.k, flags=B.DSA_INDEXER_TOPK_HIST)
+        self.mlas = [B.Mla(vmla[f"q_mla{l}"], m.kv, vout[f"out{l}"], m.d_latent, m.scale, m.lse)
+                     for l, m in enumerate(step.mlas)]
+        self.idx = vidx["idx"]
+        self.side = torch.cuda.Stream(device=dev)
         self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
+        self.ev_mla_in = torch.cuda.Event()
+        self.ev_topk = torch.cuda.Event()
+        self.ev_idx_out = torch.cuda.Event()
         self.graph = None
 
+    @staticmethod
+    def _pack(items, dev, fill):
+        offs, tot = [], 0
+        for _, t in items:
+            offs.append(tot)
+            tot += (t.numel() * t.element_size() + 255) // 256 * 256
+        d = torch.empty(tot, dtype=torch.uint8, device=dev)
+        h = torch.zeros(tot, dtype=torch.uint8).pin_memory()
+        views = {}
+        for (name, t), o in zip(items, offs):
+            nb = t.numel() * t.element_size()
+            v = d[o:o + nb].view(t.dtype).view(t.shape)
+            if fill:
+                v.copy_(t)
+                h[o:o + nb].copy_(t.cpu().contiguous().view(-1).view(torch.uint8))
+            views[name] = v
+        return d, h, views
+
     def run(self):
-        s, x = self.s, self.s.x
+        s = self.s
+        main = torch.cuda.current_stream()
         self.ev[0].record()
-        for k, h in self.h_in.items():
-            x[k].copy_(h, non_blocking=True)
-        for d, h in zip(x["q_mla"], self.h_qmla):
-            d.copy_(h, non_blocking=True)
-        s.run(events=False)
-        for h, m in zip(self.h_out, s.mlas):
-            h.copy_(m.out, non_blocking=True)
-        self.h_idx.copy_(s.idx, non_blocking=True)
+        self.side.wait_stream(main)
+        with torch.cuda.stream(self.side):
+            self.d_in_mla.copy_(self.h_in_mla, non_blocking=True)
+            self.ev_mla_in.record()
+        self.d_in_ix.copy_(self.h_in_ix, non_blocking=True)
+        B.dsa_index_scores(self.q, self.ix, s.scores, s.ws)
+        main.wait_event(self.ev_mla_in)
+        B.dsa_topk(self.q, s.scores, s.w.topk, self.idx, s.cnt, s.ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+        self.ev_topk.record()
+        for m in self.mlas:
+            s.mla_fn(self.q, m, self.idx, s.cnt, s.w.topk, s.ws)
+        with torch.cuda.stream(self.side):
+            self.side.wait_event(self.ev_topk)
+            self.h_idx.copy_(self.d_idx, non_blocking=True)
+            self.ev_idx_out.record()
+        self.h_out.copy_(self.d_out, non_blocking=True)
+        main.wait_event(self.ev_idx_out)
         self.ev[1].record()
 
     def capture(self):
+        torch.cuda.synchronize()
+        self.run()  # one eager pass
         torch.cuda.synchronize()
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
