@@ -34,6 +34,7 @@ _lib = None
 _f32p = np.ctypeslib.ndpointer(dtype=np.float32, flags="C_CONTIGUOUS")
 _f64p = np.ctypeslib.ndpointer(dtype=np.float64, flags="C_CONTIGUOUS")
 _i32p = np.ctypeslib.ndpointer(dtype=np.int32, flags="C_CONTIGUOUS")
+_u8p = np.ctypeslib.ndpointer(dtype=np.uint8, flags="C_CONTIGUOUS")
 
 
 def build(force: bool = False) -> str:
@@ -57,6 +58,10 @@ def _load():
     lib.oracle_max_threads.restype = ci
     lib.oracle_index_scores.argtypes = [ci, ci, ci, _f32p, _f32p, _f32p, i64, i64, _i32p, _i32p, ci, _f64p]
     lib.oracle_topk.argtypes = [ci, ci, _f64p, _i32p, ci, _i32p, _i32p]
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+    lib.oracle_e4m3_to_double.restype = ctypes.c_double
+    lib.oracle_index_scores_e4m3.argtypes = [ci, ci, ci, _u8p, ctypes.c_void_p, _f32p, _u8p, ctypes.c_void_p, i64,
+                                             i64, i64, _i32p, _i32p, ci, _f64p]
     lib.oracle_sparse_mla.argtypes = [ci, ci, ci, ci, ctypes.c_double, _f32p, _f32p, i64, i64,
                                       _i32p, _i32p, _i32p, ci, _f64p, ctypes.c_void_p]
     lib.oracle_dense_mla.argtypes = [ci, ci, ci, ci, ctypes.c_double, _f32p, _f32p, i64, i64,
@@ -87,6 +92,35 @@ def index_scores(q, w, k, q_seq, q_pos):
     assert np.all((q_pos >= 0) & (q_pos < L)) and np.all((q_seq >= 0) & (q_seq < n_seq))
     out = np.empty((n_q, L), dtype=np.float64)
     _load().oracle_index_scores(n_q, heads, dim, q, w, k, L * dim, dim, q_seq, q_pos, L, out)
+    return out
+
+
+def e4m3_to_double(code: int) -> float:
+    """Value of one E4M3 code (0..255), decoded from the format definition."""
+    return float(_load().oracle_e4m3_to_double(int(code) & 0xFF))
+
+
+def index_scores_e4m3(q8, q_scale, w, k8, k_scale, q_seq, q_pos):
+    """FP8 variant: q8 [n_q,H,D] and k8 [n_seq,L,D] uint8 E4M3 codes, q_scale [n_q,H]
+    and k_scale [n_seq,L] float32 (or None = 1), w [n_q,H] -> scores [n_q,L] (NaN where
+    s > q_pos), on the exact operands e4m3(code) * scale."""
+    q8 = np.ascontiguousarray(np.asarray(q8, dtype=np.uint8))
+    k8 = np.ascontiguousarray(np.asarray(k8, dtype=np.uint8))
+    w = _f32(w)
+    q_seq, q_pos = _i32(q_seq), _i32(q_pos)
+    n_q, heads, dim = q8.shape
+    n_seq, L, kd = k8.shape
+    assert kd == dim and w.shape == (n_q, heads)
+    assert np.all((q_pos >= 0) & (q_pos < L)) and np.all((q_seq >= 0) & (q_seq < n_seq))
+    qs = None if q_scale is None else _f32(q_scale)
+    ks = None if k_scale is None else _f32(k_scale)
+    if qs is not None:
+        assert qs.shape == (n_q, heads)
+    if ks is not None:
+        assert ks.shape == (n_seq, L)
+    out = np.empty((n_q, L), dtype=np.float64)
+    _load().oracle_index_scores_e4m3(n_q, heads, dim, q8, None if qs is None else qs.ctypes.data, w, k8,
+                                     None if ks is None else ks.ctypes.data, L * dim, dim, L, q_seq, q_pos, L, out)
     return out
 
 

@@ -89,6 +89,58 @@ void oracle_index_scores(int n_q, int heads, int dim, const float *q, const floa
     }
 }
 
+/*
+ * One OCP 8-bit floating-point E4M3 value (the variant without infinities),
+ * decoded from the format's definition: a sign bit, a 4-bit exponent with bias
+ * 7 and a 3-bit mantissa; exponent field 0 is subnormal (m/8 * 2^-6); exponent
+ * and mantissa all ones (0x7F, 0xFF) is NaN.  Largest finite magnitude 448.
+ */
+double oracle_e4m3_to_double(uint8_t c) {
+    int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    if (e == 15 && m == 7) return NAN;
+    double mag = (e == 0) ? ldexp((double)m / 8.0, -6) : ldexp(1.0 + (double)m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+/*
+ * Lightning-indexer scores with 8-bit E4M3 queries and keys, each scaled per
+ * row (the FP8 variant; same definition as oracle_index_scores on the exact
+ * operand values):
+ *   q[i][h][d] = e4m3(q8[i][h][d]) * q_scale[i*heads + h]        (q_scale NULL = 1)
+ *   k[s][d]    = e4m3(k8[q_seq[i]*k_seq_stride + s*k_row_stride + d])
+ *                * k_scale[q_seq[i]*ks_seq_stride + s]           (k_scale NULL = 1)
+ * Every product and sum in double precision.
+ */
+void oracle_index_scores_e4m3(int n_q, int heads, int dim, const uint8_t *q8, const float *q_scale,
+                              const float *w, const uint8_t *k8, const float *k_scale, int64_t k_seq_stride,
+                              int64_t k_row_stride, int64_t ks_seq_stride, const int32_t *q_seq,
+                              const int32_t *q_pos, int L, double *scores) {
+    double lut[256];
+    for (int c = 0; c < 256; c++) lut[c] = oracle_e4m3_to_double((uint8_t)c);
+    int64_t total = (int64_t)n_q * L;
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < total; e++) {
+        int i = (int)(e / L);
+        int s = (int)(e % L);
+        if (s > q_pos[i]) {
+            scores[e] = NAN;
+            continue;
+        }
+        const uint8_t *key = k8 + (int64_t)q_seq[i] * k_seq_stride + (int64_t)s * k_row_stride;
+        double ks = k_scale ? (double)k_scale[(int64_t)q_seq[i] * ks_seq_stride + s] : 1.0;
+        double score = 0.0;
+        for (int h = 0; h < heads; h++) {
+            const uint8_t *qh = q8 + ((int64_t)i * heads + h) * dim;
+            double qs = q_scale ? (double)q_scale[(int64_t)i * heads + h] : 1.0;
+            double dot = 0.0;
+            for (int d = 0; d < dim; d++) dot += (lut[qh[d]] * qs) * (lut[key[d]] * ks);
+            double relu = dot > 0.0 ? dot : 0.0;
+            score += (double)w[(int64_t)i * heads + h] * relu;
+        }
+        scores[e] = score;
+    }
+}
+
 /* Candidate for the top-k ordering: larger score first, then lower position. */
 typedef struct {
     double score;

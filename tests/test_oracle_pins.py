@@ -11,7 +11,10 @@ transposed operand -- breaks at least one):
     masked-sparse attention;
   * the non-absorbed MLA form (per-head up-projections W_UK, W_UV) against the
     absorbed form the oracle computes;
-  * closed forms: constant rows, a single row, q = 0 (uniform weights).
+  * closed forms: constant rows, a single row, q = 0 (uniform weights);
+  * the E4M3 8-bit float format's defining values and torch's float8_e4m3fn
+    decoding, for the FP8 indexer variant, and the positive homogeneity of ReLU
+    (a per-row scale of the keys or of a head's query factors out).
 """
 import json
 import math
@@ -348,3 +351,72 @@ def test_integer_recipe_scores_exact_in_float32():
     vis = sc[np.isfinite(sc)]
     assert np.all(vis.astype(np.float32).astype(np.float64) == vis)
     assert np.all(vis * 8 == np.round(vis * 8)) and vis.max() < 2 ** 17
+
+
+# --------------------------------------------------------------------------- FP8 (E4M3) indexer variant
+@pytest.mark.parametrize("code,value", [
+    (0x00, 0.0), (0x38, 1.0), (0x40, 2.0), (0x44, 3.0), (0x48, 4.0), (0x30, 0.5), (0x3C, 1.5),
+    (0x7E, 448.0), (0xFE, -448.0), (0x08, 2.0 ** -6), (0x01, 2.0 ** -9), (0x07, 7 * 2.0 ** -9), (0xB8, -1.0),
+])
+def test_e4m3_defining_values(code, value):
+    # sign | 4-bit exponent (bias 7) | 3-bit mantissa; exponent 0 is subnormal (m/8 * 2^-6)
+    assert oracle.e4m3_to_double(code) == value
+
+
+def test_e4m3_nan_and_signed_zero():
+    assert math.isnan(oracle.e4m3_to_double(0x7F)) and math.isnan(oracle.e4m3_to_double(0xFF))
+    z = oracle.e4m3_to_double(0x80)
+    assert z == 0.0 and math.copysign(1.0, z) == -1.0
+
+
+def test_e4m3_matches_torch_for_every_code():
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    ref = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([oracle.e4m3_to_double(c) for c in range(256)])
+    nan = np.isnan(ref)
+    assert np.array_equal(np.isnan(got), nan)
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+
+
+def _fp8_case(seed, n_q=3, n_seq=2, L=37, heads=4, dim=16):
+    g = torch.Generator().manual_seed(seed)
+    qv = torch.randint(-4, 5, (n_q, heads, dim), generator=g).float()
+    kv = torch.randint(-4, 5, (n_seq, L, dim), generator=g).float()
+    q8 = qv.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    k8 = kv.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    w = torch.pow(2.0, torch.randint(-3, 2, (n_q, heads), generator=g).float()).numpy()
+    q_seq = np.array([0, 1, 1][:n_q], dtype=np.int32)
+    q_pos = np.array([L - 1, L - 5, 11][:n_q], dtype=np.int32)
+    return qv.numpy(), kv.numpy(), q8, k8, w, q_seq, q_pos
+
+
+def test_fp8_scores_with_unit_scales_equal_the_float_definition():
+    qv, kv, q8, k8, w, q_seq, q_pos = _fp8_case(1)
+    got = oracle.index_scores_e4m3(q8, None, w, k8, None, q_seq, q_pos)
+    # the same integers as float32 through relu(x) = (x + |x|) / 2 and a plain matmul
+    for i in range(qv.shape[0]):
+        dots = np.einsum("hd,sd->hs", qv[i].astype(np.float64), kv[q_seq[i]].astype(np.float64))
+        ref = (w[i][:, None] * (dots + np.abs(dots)) / 2).sum(0)
+        t = q_pos[i]
+        np.testing.assert_array_equal(got[i, : t + 1], ref[: t + 1])
+        assert np.all(np.isnan(got[i, t + 1:]))
+
+
+def test_fp8_scales_factor_out_of_relu():
+    qv, kv, q8, k8, w, q_seq, q_pos = _fp8_case(2)
+    g = np.random.default_rng(3)
+    n_q, heads, _ = q8.shape
+    n_seq, L, _ = k8.shape
+    q_scale = g.uniform(0.25, 3.0, size=(n_q, heads)).astype(np.float32)
+    k_scale = g.uniform(0.25, 3.0, size=(n_seq, L)).astype(np.float32)
+    base = oracle.index_scores_e4m3(q8, None, w, k8, None, q_seq, q_pos)
+    # a positive per-key scale multiplies that key's score
+    with_k = oracle.index_scores_e4m3(q8, None, w, k8, k_scale, q_seq, q_pos)
+    # a positive per-(query, head) scale acts as a factor on that head's weight
+    with_q = oracle.index_scores_e4m3(q8, q_scale, w, k8, None, q_seq, q_pos)
+    for i in range(n_q):
+        t = q_pos[i]
+        np.testing.assert_allclose(with_k[i, : t + 1], base[i, : t + 1] * k_scale[q_seq[i], : t + 1], rtol=1e-12)
+        dots = np.einsum("hd,sd->hs", qv[i].astype(np.float64), kv[q_seq[i], : t + 1].astype(np.float64))
+        ref_q = ((w[i].astype(np.float64) * q_scale[i].astype(np.float64))[:, None] * np.maximum(dots, 0)).sum(0)
+        np.testing.assert_allclose(with_q[i, : t + 1], ref_q, rtol=1e-12)
