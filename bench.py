@@ -53,8 +53,10 @@ def measured_peaks():
 
 
 # ------------------------------------------------------------------ algorithmic bytes
-def path_bytes(w: wl.Workload, seq_run: int):
-    """Algorithmic HBM bytes of one step (each input byte once, outputs once)."""
+def path_bytes(w: wl.Workload, seq_run: int, indexer_fp8: bool = False):
+    """Algorithmic HBM bytes of one step (each input byte once, outputs once).
+    indexer_fp8: E4M3 indexer keys and queries (1 byte per value) plus a float32
+    scale per key and per (query, head)."""
     vis = np.array(w.q_pos, dtype=np.int64) + 1
     seqs = {}
     for s, t in zip(w.q_seq, w.q_pos):
@@ -62,7 +64,9 @@ def path_bytes(w: wl.Workload, seq_run: int):
         seqs[key] = max(seqs.get(key, 0), t + 1)
     key_rows = sum(seqs.values())
     eb = w.elem_bytes
-    idx_in = key_rows * w.idx_dim * eb + w.n_q * w.idx_heads * (w.idx_dim * eb + 4)
+    key_b = w.idx_dim + 4 if indexer_fp8 else w.idx_dim * eb             # per key row
+    qry_b = w.idx_dim + 8 if indexer_fp8 else w.idx_dim * eb + 4         # per (query, head): q, w (+ scale)
+    idx_in = key_rows * key_b + w.n_q * w.idx_heads * qry_b
     idx_out = int(vis.sum()) * 4
     cnt = np.minimum(vis, w.topk)
     rows = int(cnt.sum()) * (w.d_lat + w.d_rope) * eb
@@ -72,7 +76,7 @@ def path_bytes(w: wl.Workload, seq_run: int):
         "topk": idx_out + w.n_q * (w.topk + 1) * 4,
         "mla_per_layer": rows + q_out,
         # the path's roofline bytes: indexer keys + gathered rows + q/out
-        "path": key_rows * w.idx_dim * eb + w.n_layers * (rows + q_out) + w.n_q * w.idx_heads * (w.idx_dim * eb + 4),
+        "path": key_rows * key_b + w.n_layers * (rows + q_out) + w.n_q * w.idx_heads * qry_b,
     }
 
 
@@ -142,7 +146,7 @@ class ClockSampler:
 class Step:
     """Device buffers, descriptors and the captured CUDA graph of one step."""
 
-    def __init__(self, w: wl.Workload, dev, seed_offset: int = 0):
+    def __init__(self, w: wl.Workload, dev, seed_offset: int = 0, indexer_fp8: bool = False):
         self.w = w
         self.dev = dev
         w = wl.scaled(w, seed=w.seed + seed_offset) if seed_offset else w
@@ -151,8 +155,17 @@ class Step:
         x = self.x
         self.q = B.Queries(x["q_seq"], x["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=self.seq_run)
         # the indexer leaves the top-k's first-digit histograms in the workspace
-        self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"],
-                            flags=B.DSA_INDEXER_TOPK_HIST)
+        self.f8 = None
+        if indexer_fp8:  # the FP8 variant: E4M3 indexer queries and keys with per-row scales
+            self.f8 = wl.fp8_indexer_inputs(w, x, device=dev)
+            f8 = self.f8
+            self.ix = B.Indexer(f8["q8"], x["w"], f8["k8"][0] if w.shared_cache else f8["k8"],
+                                flags=B.DSA_INDEXER_TOPK_HIST, q_scale=f8["q_scale"],
+                                k_scale=f8["k_scale"][0] if w.shared_cache else f8["k_scale"])
+            x["k_idx"] = None  # the bf16 keys are not read
+        else:
+            self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"],
+                                flags=B.DSA_INDEXER_TOPK_HIST)
         self.mlas = []
         for layer in range(w.n_layers):
             out = torch.empty((w.n_q, w.mla_heads, w.d_lat), dtype=w.torch_dtype, device=dev)
@@ -231,8 +244,10 @@ class E2EStep:
         self.s = step
         w, x = step.w, step.x
         dev = step.dev
-        self.d_in_ix, self.h_in_ix, vix = self._pack(
-            [("q_idx", x["q_idx"]), ("w", x["w"]), ("q_seq", x["q_seq"]), ("q_pos", x["q_pos"])], dev, fill=True)
+        ix_in = [("q_idx", step.ix.q), ("w", x["w"]), ("q_seq", x["q_seq"]), ("q_pos", x["q_pos"])]
+        if step.f8 is not None:
+            ix_in.append(("q_scale", step.ix.q_scale))
+        self.d_in_ix, self.h_in_ix, vix = self._pack(ix_in, dev, fill=True)
         self.d_in_mla, self.h_in_mla, vmla = self._pack(
             [(f"q_mla{l}", t) for l, t in enumerate(x["q_mla"])], dev, fill=True)
         self.d_out, self.h_out, vout = self._pack([(f"out{l}", m.out) for l, m in enumerate(step.mlas)], dev,
@@ -242,7 +257,8 @@ class E2EStep:
         self.d2h = self.h_out.numel() + self.h_idx.numel()
         # descriptors over the packed views (caches, scores, counts and workspace are the step's)
         self.q = B.Queries(vix["q_seq"], vix["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=step.seq_run)
-        self.ix = B.Indexer(vix["q_idx"], vix["w"], step.ix.k, flags=B.DSA_INDEXER_TOPK_HIST)
+        self.ix = B.Indexer(vix["q_idx"], vix["w"], step.ix.k, flags=B.DSA_INDEXER_TOPK_HIST,
+                            q_scale=vix.get("q_scale"), k_scale=step.ix.k_scale)
         self.mlas = [B.Mla(vmla[f"q_mla{l}"], m.kv, vout[f"out{l}"], m.d_latent, m.scale, m.lse)
                      for l, m in enumerate(step.mlas)]
         self.idx = vidx["idx"]
@@ -267,7 +283,7 @@ class E2EStep:
             v = d[o:o + nb].view(t.dtype).view(t.shape)
             if fill:
                 v.copy_(t)
-                h[o:o + nb].copy_(t.cpu().contiguous().view(-1).view(torch.uint8))
+                h[o:o + nb].copy_(t.detach().cpu().contiguous().view(-1).view(torch.uint8))
             views[name] = v
         return d, h, views
 
@@ -418,6 +434,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--indexer-fp8", action="store_true",
+                    help="the FP8 variant: E4M3 indexer queries/keys with per-row scales (a separate line, "
+                         "not the bf16 headline)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="decode workloads: override the batch (a smaller case for profiling; not a bench line)")
     args = ap.parse_args()
@@ -436,7 +455,7 @@ def main():
     torch.cuda.set_device(dev)
     B.lib()
 
-    step = Step(w, dev, seed_offset=rank)
+    step = Step(w, dev, seed_offset=rank, indexer_fp8=args.indexer_fp8)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     step.capture()
     for _ in range(args.warmup):
@@ -480,7 +499,8 @@ def main():
     ms_per_step = tot_max / args.steps
     value = weak_scaling_value(world, w.n_q, w.n_layers, args.steps, tot_max)
     hbm_peak, tc_peak, peak_kind = measured_peaks()
-    by = path_bytes(w, step.seq_run)
+    fp8 = args.indexer_fp8
+    by = path_bytes(w, step.seq_run, indexer_fp8=fp8)
     idx_ms = idx_t / n_bd
     idx_gbs = by["indexer"] / (idx_ms * 1e-3) / 1e9
     t_roof_us = by["path"] / (hbm_peak * 1e9) * 1e6
@@ -488,12 +508,13 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {**w.describe(), "parallelism": f"dp{world} (independent batches per GPU)",
+        "vs_baseline": None, "dtype": ("e4m3 indexer, " + w.dtype + " MLA") if fp8 else w.dtype, "data": "synthetic",
+        "config": {**w.describe(), **({"indexer_dtype": "e4m3 + per-row fp32 scales (FP8 variant)"} if fp8 else {}),
+                   "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": "flushed before every timed step (256 MB write)", "graph": "CUDA graph per step"},
         "roofline": {"bound": "hbm", "kernel": "idx_score_tc (dsa_index_scores)", "achieved": idx_gbs,
                      "peak": hbm_peak, "unit": "GB/s", "frac": idx_gbs / hbm_peak,
-                     "traffic": NCU_INDEXER_TRAFFIC.get(w.name), "peak_kind": f"{peak_kind} hbm_gbs",
+                     "traffic": None if fp8 else NCU_INDEXER_TRAFFIC.get(w.name), "peak_kind": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes": by["indexer"], "avg_launch_us": idx_ms * 1e3},
         "path_roofline": {"bytes": by["path"], "t_roof_us": t_roof_us,
                           "frac": t_roof_us / (ms_per_step * 1e3), "peak_kind": f"{peak_kind} hbm_gbs"},
@@ -522,7 +543,7 @@ def main():
                        "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "steps": n_e2e}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, step.x)
+        line["cpu_baseline"] = None if fp8 else cpu_baseline(w, step.x)
 
     if rank == 0:
         print(json.dumps(line), flush=True)

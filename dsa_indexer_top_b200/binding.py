@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT = range(6)
-DSA_BF16, DSA_F32 = 0, 1
+DSA_BF16, DSA_F32, DSA_FP8_E4M3 = 0, 1, 2
 DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_MLA_DECODE, DSA_OP_MLA_PREFILL, DSA_OP_INDEXSHARE_GROUP = range(5)
 DSA_INDEXER_TOPK_HIST = 1
 DSA_TOPK_HIST_FROM_INDEXER = 1
@@ -40,7 +40,8 @@ class _Queries(ctypes.Structure):
 class _Indexer(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("dim", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("flags", ctypes.c_int32), ("q", ctypes.c_void_p), ("w", ctypes.c_void_p),
-                ("k", ctypes.c_void_p), ("k_seq_stride", ctypes.c_int64), ("k_row_stride", ctypes.c_int64)]
+                ("k", ctypes.c_void_p), ("k_seq_stride", ctypes.c_int64), ("k_row_stride", ctypes.c_int64),
+                ("q_scale", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("ks_seq_stride", ctypes.c_int64)]
 
 
 class _Mla(ctypes.Structure):
@@ -105,6 +106,8 @@ def _dtype_code(t: torch.Tensor) -> int:
         return DSA_BF16
     if t.dtype == torch.float32:
         return DSA_F32
+    if t.dtype == torch.float8_e4m3fn:
+        return DSA_FP8_E4M3
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
@@ -125,16 +128,22 @@ class Queries:
 
 @dataclass
 class Indexer:
-    q: torch.Tensor              # [n_q, heads, dim]
+    q: torch.Tensor              # [n_q, heads, dim] (bf16, fp32 or float8_e4m3fn)
     w: torch.Tensor              # float32 [n_q, heads]
-    k: torch.Tensor              # [n_seq, L, dim] or [L, dim] (shared cache)
+    k: torch.Tensor              # [n_seq, L, dim] or [L, dim] (shared cache), q's dtype
     flags: int = 0               # DSA_INDEXER_TOPK_HIST or 0
+    q_scale: Optional[torch.Tensor] = None   # FP8 only: float32 [n_q, heads], positive
+    k_scale: Optional[torch.Tensor] = None   # FP8 only: float32 [n_seq, L] or [L] (shared), positive
 
     def c(self) -> _Indexer:
         shared = self.k.dim() == 2
         seq_stride = 0 if shared else self.k.stride(0)
+        ks = self.k_scale
+        ks_stride = 0 if ks is None or ks.dim() == 1 else ks.stride(0)
         return _Indexer(self.q.shape[1], self.q.shape[2], _dtype_code(self.q), self.flags, self.q.data_ptr(),
-                        self.w.data_ptr(), self.k.data_ptr(), seq_stride, self.k.stride(-2))
+                        self.w.data_ptr(), self.k.data_ptr(), seq_stride, self.k.stride(-2),
+                        None if self.q_scale is None else self.q_scale.data_ptr(),
+                        None if ks is None else ks.data_ptr(), ks_stride)
 
 
 @dataclass

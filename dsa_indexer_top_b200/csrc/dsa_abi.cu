@@ -63,8 +63,10 @@ bool ws_ok(void *ws, size_t ws_bytes, size_t need) {
 }
 
 bool indexer_tc_ok(const dsa_indexer *ix) {
-    return ix->dtype == DSA_BF16 && ix->heads == kIdxHeads && ix->dim == kIdxDim && aligned16(ix->q) &&
-           aligned16(ix->k) && ix->k_row_stride % 8 == 0 && ix->k_seq_stride % 8 == 0 &&
+    // TMA strides are multiples of 16 bytes: 8 bf16 or 16 FP8 elements
+    const int64_t al = ix->dtype == DSA_FP8_E4M3 ? 16 : 8;
+    return (ix->dtype == DSA_BF16 || ix->dtype == DSA_FP8_E4M3) && ix->heads == kIdxHeads && ix->dim == kIdxDim &&
+           aligned16(ix->q) && aligned16(ix->k) && ix->k_row_stride % al == 0 && ix->k_seq_stride % al == 0 &&
            ix->k_row_stride >= kIdxDim;
 }
 
@@ -109,15 +111,20 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
         EncodeTiledFn enc = encode_fn();
         if (!enc) return DSA_ERR_CUDA;
         CUtensorMap tk, tq;
+        // bf16: boxes of 64 values; FP8 (E4M3 bytes, mapped as uint8): boxes of 128
+        const bool f8 = ix->dtype == DSA_FP8_E4M3;
+        const int esz = f8 ? 1 : 2;
+        const CUtensorMapDataType dt = f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        const cuuint32_t box_x = f8 ? 128 : 64;
         {
             cuuint64_t dims[3] = {static_cast<cuuint64_t>(kIdxDim), static_cast<cuuint64_t>(qs->max_ctx),
                                   static_cast<cuuint64_t>(n_cache)};
             const int64_t seq_stride = ix->k_seq_stride == 0 ? ix->k_row_stride * qs->max_ctx : ix->k_seq_stride;
-            cuuint64_t strides[2] = {static_cast<cuuint64_t>(ix->k_row_stride * 2),
-                                     static_cast<cuuint64_t>(seq_stride * 2)};
-            cuuint32_t box[3] = {64, 128, 1};
+            cuuint64_t strides[2] = {static_cast<cuuint64_t>(ix->k_row_stride * esz),
+                                     static_cast<cuuint64_t>(seq_stride * esz)};
+            cuuint32_t box[3] = {box_x, 128, 1};
             cuuint32_t es[3] = {1, 1, 1};
-            if (enc(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ix->k), dims, strides, box, es,
+            if (enc(&tk, dt, 3, const_cast<void *>(ix->k), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
                 return DSA_ERR_INVALID;
@@ -126,10 +133,10 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
         while (G < 8 && qs->seq_run % (G * 2) == 0) G *= 2;
         {
             cuuint64_t dims[2] = {static_cast<cuuint64_t>(kIdxDim), static_cast<cuuint64_t>(qs->n_q) * kIdxHeads};
-            cuuint64_t strides[1] = {static_cast<cuuint64_t>(kIdxDim * 2)};
-            cuuint32_t box[2] = {64, static_cast<cuuint32_t>(32 * G)};
+            cuuint64_t strides[1] = {static_cast<cuuint64_t>(kIdxDim * esz)};
+            cuuint32_t box[2] = {box_x, static_cast<cuuint32_t>(32 * G)};
             cuuint32_t es[2] = {1, 1};
-            if (enc(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(ix->q), dims, strides, box, es,
+            if (enc(&tq, dt, 2, const_cast<void *>(ix->q), dims, strides, box, es,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
                 return DSA_ERR_INVALID;
@@ -149,8 +156,13 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
         const long long groups = (qs->n_q + G - 1) / G;
         a.total_items = groups * a.tiles_per_group;
         a.ghist = (ghist && G == 1) ? ghist : nullptr;  // fused into the epilogue
+        a.q_scale = f8 ? ix->q_scale : nullptr;
+        a.k_scale = f8 ? ix->k_scale : nullptr;
+        a.ks_seq_stride = f8 ? ix->ks_seq_stride : 0;
         hist_done = a.ghist != nullptr;
-        s = launch_idx_score_tc(G, tk, tq, a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+        s = launch_idx_score_tc(G, f8, tk, tq, a, num_sms_current(), st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    } else if (ix->dtype == DSA_FP8_E4M3) {
+        s = DSA_ERR_UNSUPPORTED;  // FP8 runs on the tensor-core path only
     } else {
         s = do_index_generic(qs, ix, scores, ld, status, st);
     }
@@ -194,8 +206,15 @@ dsa_status do_index_generic(const dsa_queries *qs, const dsa_indexer *ix, float 
 
 dsa_status check_indexer(const dsa_queries *qs, const dsa_indexer *ix) {
     if (!ix || !ix->q || !ix->w || !ix->k) return DSA_ERR_INVALID;
-    if (ix->heads < 1 || ix->dim < 1 || (ix->dtype != DSA_BF16 && ix->dtype != DSA_F32)) return DSA_ERR_INVALID;
+    if (ix->heads < 1 || ix->dim < 1 ||
+        (ix->dtype != DSA_BF16 && ix->dtype != DSA_F32 && ix->dtype != DSA_FP8_E4M3))
+        return DSA_ERR_INVALID;
     if (ix->k_row_stride < ix->dim || ix->k_seq_stride < 0) return DSA_ERR_INVALID;
+    if (ix->dtype == DSA_FP8_E4M3) {
+        if (ix->ks_seq_stride < 0 || (ix->k_scale && ix->ks_seq_stride != 0 && ix->ks_seq_stride < qs->max_ctx))
+            return DSA_ERR_INVALID;
+        if (!indexer_tc_ok(ix)) return DSA_ERR_UNSUPPORTED;  // 32 heads x 128 dims, aligned, TMA strides
+    }
     if (ix->k_seq_stride != 0 && ix->k_seq_stride < ix->k_row_stride * qs->max_ctx) return DSA_ERR_INVALID;
     return DSA_OK;
 }

@@ -28,22 +28,26 @@ namespace dsa {
 namespace {
 
 constexpr int kTileKeys = 128;
-constexpr int kATileBytes = kTileKeys * kIdxDim * 2;  // 32 KB
 
-template <int G>
+// F8: queries and keys are E4M3 bytes (the FP8 variant) instead of bf16.
+template <int G, bool F8>
 struct IdxCfg {
     static constexpr int N = 32 * G;
-    // One query per tile: two CTAs per SM with two 32 KB stages each.  Two
+    static constexpr int kElem = F8 ? 1 : 2;                     // bytes per value
+    static constexpr int kTileBytes = kTileKeys * kIdxDim * kElem;  // 32 KB bf16, 16 KB FP8
+    static constexpr int kBoxes = kElem;                          // 128-byte-wide boxes per row
+    static constexpr int kKSteps = F8 ? kIdxDim / 32 : kIdxDim / 16;  // MMA K = 32 (8-bit) or 16
+    // One query per tile: two CTAs per SM, 64 KB of key stages each.  Two
     // independent load -> MMA -> epilogue pipelines per SM keep the key stream
     // at the rate of a plain TMA read stream, where one CTA with deeper
     // buffering loses about 6% to the MMA turnaround of each stage; more than
     // about 128 KB in flight per SM lowers the stream rate again.
     static constexpr int kCtasPerSm = G == 1 ? 2 : 1;
-    static constexpr int kStages = G == 1 ? 2 : 4;
-    static constexpr int kBBytes = N * kIdxDim * 2;
+    static constexpr int kStages = G == 1 ? (F8 ? 4 : 2) : 4;
+    static constexpr int kBBytes = N * kIdxDim * kElem;
     static constexpr int kTmemCols = (2 * N < 32) ? 32 : 2 * N;
-    static constexpr int kSmem = kStages * kATileBytes + kBBytes + 1024;
-    static constexpr uint32_t kIdesc = idesc_bf16(128, N, false, false);
+    static constexpr int kSmem = kStages * kTileBytes + kBBytes + 1024;
+    static constexpr uint32_t kIdesc = F8 ? idesc_e4m3(128, N) : idesc_bf16(128, N, false, false);
     // epilogue warps: two per TMEM lane quadrant when a tile holds several
     // queries (each takes half of them), one otherwise
     static constexpr int kEpiWarps = G >= 2 ? 8 : 4;
@@ -68,11 +72,12 @@ __device__ __forceinline__ void group_info(const IdxTcArgs &a, int g, int &seq, 
     }
 }
 
-template <int G>
-__global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
+template <int G, bool F8>
+__global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasPerSm)
     idx_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_q, const IdxTcArgs a) {
-    using Cfg = IdxCfg<G>;
+    using Cfg = IdxCfg<G, F8>;
+    constexpr int kATileBytes = Cfg::kTileBytes;
     constexpr int N = Cfg::N;
     constexpr int S = Cfg::kStages;
 
@@ -80,7 +85,7 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
     uint8_t *a_tiles = smem;                      // S x 32 KB
-    uint8_t *b_tile = smem + S * kATileBytes;     // N rows x 256 B
+    uint8_t *b_tile = smem + S * kATileBytes;     // N rows x 128 dims
 
     __shared__ uint64_t full_bar[S], empty_bar[S];
     __shared__ uint64_t tmem_full[2], tmem_empty[2];
@@ -157,8 +162,10 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
                         !mbar_wait(&b_empty, (b_uses - 1) & 1, a.status, &abort_flag))
                         break;
                     mbar_arrive_expect_tx(&b_full, Cfg::kBBytes);
-                    tma_load_2d(b_tile, &tmap_q, &b_full, 0, g * N);
-                    tma_load_2d(b_tile + N * 128, &tmap_q, &b_full, 64, g * N);
+                    // box x = 64 bf16 or 128 FP8 values: 128 bytes
+#pragma unroll
+                    for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+                        tma_load_2d(b_tile + bx * N * 128, &tmap_q, &b_full, bx * 64, g * N);
                     ++b_uses;
                     group_loaded = true;
                 }
@@ -167,9 +174,10 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
                 if (!mbar_wait(&empty_bar[stage], (use & 1) ^ 1, a.status, &abort_flag)) break;
                 uint8_t *dst = a_tiles + stage * kATileBytes;
                 mbar_arrive_expect_tx(&full_bar[stage], kATileBytes);
-                tma_load_3d_hint(dst, &tmap_k, &full_bar[stage], 0, j * kTileKeys, seq, stream_policy);
-                tma_load_3d_hint(dst + kATileBytes / 2, &tmap_k, &full_bar[stage], 64, j * kTileKeys, seq,
-                                 stream_policy);
+#pragma unroll
+                for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+                    tma_load_3d_hint(dst + bx * (kTileKeys * 128), &tmap_k, &full_bar[stage], bx * 64, j * kTileKeys,
+                                     seq, stream_policy);
                 last_use[stage] = use;
                 ++k_tiles;
             }
@@ -213,11 +221,15 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
                 const uint64_t bdesc = sdesc_sw128(smem_u32(b_tile), 16, 1024);
                 const uint32_t d_tmem = tmem_base + acc * N;
 #pragma unroll
-                for (int kk = 0; kk < kIdxDim / 16; ++kk) {
-                    // offsets in 16-byte units added to the descriptors' start-address field
-                    const uint64_t aoff = static_cast<uint64_t>(((kk >> 2) * (kATileBytes / 2) + (kk & 3) * 32) >> 4);
+                for (int kk = 0; kk < Cfg::kKSteps; ++kk) {
+                    // offsets in 16-byte units added to the descriptors' start-address field:
+                    // each K step covers 32 bytes of a 128-byte row; bf16 rows span two boxes
+                    const uint64_t aoff = static_cast<uint64_t>(((kk >> 2) * (kTileKeys * 128) + (kk & 3) * 32) >> 4);
                     const uint64_t boff = static_cast<uint64_t>(((kk >> 2) * (N * 128) + (kk & 3) * 32) >> 4);
-                    umma_bf16(d_tmem, adesc + aoff, bdesc + boff, Cfg::kIdesc, kk > 0 ? 1u : 0u);
+                    if constexpr (F8)
+                        umma_e4m3(d_tmem, adesc + aoff, bdesc + boff, Cfg::kIdesc, kk > 0 ? 1u : 0u);
+                    else
+                        umma_bf16(d_tmem, adesc + aoff, bdesc + boff, Cfg::kIdesc, kk > 0 ? 1u : 0u);
                 }
                 umma_commit(&empty_bar[stage]);
                 umma_commit(&tmem_full[acc]);
@@ -273,7 +285,10 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
                 __syncwarp();  // this warp no longer reads the previous group's w
                 for (int e = lane; e < N; e += 32) {
                     const int qi = q0 + e / 32;
-                    w_mine[e] = qi < a.n_q ? __ldg(a.w + static_cast<int64_t>(qi) * kIdxHeads + (e & 31)) : 0.f;
+                    float wv = qi < a.n_q ? __ldg(a.w + static_cast<int64_t>(qi) * kIdxHeads + (e & 31)) : 0.f;
+                    // FP8: a positive per-(query, head) scale factors out of the ReLU onto w
+                    if (F8 && a.q_scale && qi < a.n_q) wv *= __ldg(a.q_scale + static_cast<int64_t>(qi) * kIdxHeads + (e & 31));
+                    w_mine[e] = wv;
                 }
                 __syncwarp();
 #pragma unroll
@@ -298,6 +313,9 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
             tc_fence_after();
             const int s = j * kTileKeys + quad * 32 + lane;
             const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * N;
+            // FP8: the key's positive scale factors out of every head's ReLU
+            const float ks = (F8 && a.k_scale && s < a.L) ? __ldg(a.k_scale + static_cast<int64_t>(seq) * a.ks_seq_stride + s)
+                                                         : 1.f;
 #pragma unroll
             for (int ii = 0; ii < kQPerWarp; ++ii) {
                 const int i = qlo + ii;
@@ -314,6 +332,7 @@ __global__ void __launch_bounds__(IdxCfg<G>::kThreads, IdxCfg<G>::kCtasPerSm)
                     score = fmaf(wv.z, fmaxf(u2f(r[4 * h4 + 2]), 0.f), score);
                     score = fmaf(wv.w, fmaxf(u2f(r[4 * h4 + 3]), 0.f), score);
                 }
+                if (F8) score *= ks;
                 const bool vis = qok[ii] && s <= qpos[ii];
                 if (vis) a.scores[static_cast<int64_t>(g * G + i) * a.ld + s] = score;
                 if (fuse_hist) hist_add(ehist, vis ? first_digit(order_key(score)) : 0xFFFFFFFFu);
@@ -377,29 +396,36 @@ __global__ void __launch_bounds__(256) idx_score_generic_kernel(const IdxGeneric
     }
 }
 
-template <int G>
+template <int G, bool F8>
 cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcArgs &a, int num_sms,
                       cudaStream_t st) {
-    using Cfg = IdxCfg<G>;
+    using Cfg = IdxCfg<G, F8>;
     const long long slots = static_cast<long long>(num_sms) * Cfg::kCtasPerSm;
     const int grid = static_cast<int>(a.total_items < slots ? a.total_items : slots);
-    cudaError_t e = cudaFuncSetAttribute(idx_score_tc_kernel<G>,
+    cudaError_t e = cudaFuncSetAttribute(idx_score_tc_kernel<G, F8>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(idx_score_tc_kernel<G>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmem, st, tk, tq, a);
+    return launch_pdl(idx_score_tc_kernel<G, F8>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmem, st, tk, tq, a);
+}
+
+template <bool F8>
+cudaError_t launch_tc_g(int G, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q, const IdxTcArgs &a,
+                        int num_sms, cudaStream_t st) {
+    switch (G) {
+        case 1: return launch_tc<1, F8>(tmap_k, tmap_q, a, num_sms, st);
+        case 2: return launch_tc<2, F8>(tmap_k, tmap_q, a, num_sms, st);
+        case 4: return launch_tc<4, F8>(tmap_k, tmap_q, a, num_sms, st);
+        case 8: return launch_tc<8, F8>(tmap_k, tmap_q, a, num_sms, st);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
 
-cudaError_t launch_idx_score_tc(int G, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
+cudaError_t launch_idx_score_tc(int G, bool fp8, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
                                 const IdxTcArgs &a, int num_sms, cudaStream_t st) {
-    switch (G) {
-        case 1: return launch_tc<1>(tmap_k, tmap_q, a, num_sms, st);
-        case 2: return launch_tc<2>(tmap_k, tmap_q, a, num_sms, st);
-        case 4: return launch_tc<4>(tmap_k, tmap_q, a, num_sms, st);
-        case 8: return launch_tc<8>(tmap_k, tmap_q, a, num_sms, st);
-        default: return cudaErrorInvalidValue;
-    }
+    return fp8 ? launch_tc_g<true>(G, tmap_k, tmap_q, a, num_sms, st)
+               : launch_tc_g<false>(G, tmap_k, tmap_q, a, num_sms, st);
 }
 
 cudaError_t launch_idx_score_generic(const IdxGenericArgs &a, cudaStream_t st) {

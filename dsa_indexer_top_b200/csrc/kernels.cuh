@@ -54,12 +54,17 @@ struct IdxTcArgs {
     long long total_items;
     uint32_t *ghist;      // non-null (one query per tile only): accumulate the top-k
                           // first-digit histogram [n_q][4096] of the scores written
+    // FP8 (E4M3) operands only: positive per-(query, head) and per-key scales, or null
+    const float *q_scale;    // [n_q][32]
+    const float *k_scale;    // sequence b's key s at k_scale[b * ks_seq_stride + s]
+    int64_t ks_seq_stride;
 };
 
 // G = queries per tensor-core tile (1, 2, 4 or 8).  Tensor maps: keys 3-D
-// {128, L, n_cache} bf16, box {64, 128, 1}; queries 2-D {128, n_q*32}, box
-// {64, 32*G}; both 128-byte swizzled.
-cudaError_t launch_idx_score_tc(int G, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
+// {128, L, n_cache}, queries 2-D {128, n_q*32}, both 128-byte swizzled with
+// 128-byte boxes: bf16 boxes {64, 128, 1} / {64, 32*G}, FP8 (uint8) boxes
+// {128, 128, 1} / {128, 32*G}.
+cudaError_t launch_idx_score_tc(int G, bool fp8, const CUtensorMap &tmap_k, const CUtensorMap &tmap_q,
                                 const IdxTcArgs &a, int num_sms, cudaStream_t st);
 
 struct IdxGenericArgs {

@@ -15,6 +15,11 @@ indices can be compared bit for bit):
 With |q.k| <= 128 * 16 and at most 32 heads, each score is a multiple of 2^-3
 below 2^17, which float32 holds exactly whatever the summation order.
 
+FP8 indexer variant (fp8_indexer_inputs): the same integer queries and keys
+stored as E4M3 bytes (integers up to 16 are exact in E4M3), with per-(query,
+head) scales 2^e, e in [-1, 1], and per-key scales 2^e, e in [-2, 0]: every
+score is then a multiple of 2^-6 below 2^19 -- still exact in float32.
+
 Random numbers come from torch.Generator objects seeded per tensor (seed, tensor
 id), on the device the tensors are created on.
 """
@@ -27,7 +32,7 @@ from dataclasses import dataclass, field
 import torch
 
 # tensor ids used to derive independent streams from one workload seed
-_T_QIDX, _T_W, _T_KIDX, _T_QMLA, _T_KV = 1, 2, 3, 4, 5
+_T_QIDX, _T_W, _T_KIDX, _T_QMLA, _T_KV, _T_QSCALE, _T_KSCALE = 1, 2, 3, 4, 5, 6, 7
 
 
 @dataclass(frozen=True)
@@ -180,3 +185,20 @@ def random_scores(n_q, L, seed, device="cpu", mode="ties"):
         s[:, 3::11] = 0.0
         s[:, 5::13] = -0.0
     return s
+
+
+def fp8_indexer_inputs(w: Workload, x: dict, device="cpu") -> dict:
+    """FP8 (E4M3) versions of a workload's indexer inputs: the same integer
+    values as x["q_idx"] / x["k_idx"] stored as float8_e4m3fn, plus seeded
+    power-of-two scales q_scale [n_q][heads] and k_scale [n_cache][L]."""
+    n_cache = x["k_idx"].shape[0]
+    gq = _gen(w.seed, _T_QSCALE, device)
+    gk = _gen(w.seed, _T_KSCALE, device)
+    eq = torch.randint(-1, 2, (w.n_q, w.idx_heads), generator=gq, device=device, dtype=torch.int32)
+    ek = torch.randint(-2, 1, (n_cache, w.L), generator=gk, device=device, dtype=torch.int32)
+    return {
+        "q8": x["q_idx"].to(device).float().to(torch.float8_e4m3fn),
+        "k8": x["k_idx"].to(device).float().to(torch.float8_e4m3fn),
+        "q_scale": torch.pow(2.0, eq.to(torch.float32)),
+        "k_scale": torch.pow(2.0, ek.to(torch.float32)),
+    }

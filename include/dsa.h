@@ -72,7 +72,9 @@ typedef enum {
     DSA_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (device) */
 } dsa_status;
 
-typedef enum { DSA_BF16 = 0, DSA_F32 = 1 } dsa_dtype;
+/* DSA_FP8_E4M3: OCP 8-bit float E4M3 (no infinities), indexer q and k only,
+ * with per-row scales (dsa_indexer.q_scale / k_scale). */
+typedef enum { DSA_BF16 = 0, DSA_F32 = 1, DSA_FP8_E4M3 = 2 } dsa_dtype;
 
 /* Flags of dsa_indexer.flags and of dsa_topk. */
 enum {
@@ -130,13 +132,23 @@ typedef struct {
 /*
  * Lightning indexer of one full layer [TM, Indexer-selected sparse attention].
  *   heads, dim    32 and 128 for GLM-5.2 (any positive values on the generic path)
- *   dtype         DSA_BF16 or DSA_F32, for q and k
+ *   dtype         DSA_BF16 or DSA_F32, for q and k; or DSA_FP8_E4M3 (32 x 128
+ *                 only, tensor cores), where the operands are
+ *                   q[i,h,d] = e4m3(q[i,h,d]) * q_scale[i*heads + h]
+ *                   k[s,d]   = e4m3(k[s,d]) * k_scale[b*ks_seq_stride + s]
+ *                 (the FP8 variant: half the key bytes of bf16)
  *   q             [n_q][heads][dim], contiguous, post-RoPE
  *   w             float32 [n_q][heads], contiguous
  *   k             row s of sequence b at k + b*k_seq_stride + s*k_row_stride
  *                 (strides in elements; k_seq_stride 0 = all sequences share one
  *                 cache).  Tensor-core path: row and sequence strides multiple of
- *                 8 elements, k and q 16-byte aligned.
+ *                 8 elements (16 for FP8), k and q 16-byte aligned.
+ *   q_scale       FP8 only: float32 [n_q][heads], or NULL (all 1); positive
+ *   k_scale       FP8 only: float32, sequence b's row s at
+ *                 k_scale[b*ks_seq_stride + s] (ks_seq_stride 0 = shared), or
+ *                 NULL (all 1); positive.  A positive scale factors out of the
+ *                 ReLU, which the kernel uses (non-positive scales are not
+ *                 supported and give unspecified scores).
  */
 typedef struct {
     int32_t heads;
@@ -148,6 +160,9 @@ typedef struct {
     const void *k;
     int64_t k_seq_stride;
     int64_t k_row_stride;
+    const float *q_scale;  /* FP8 only */
+    const float *k_scale;  /* FP8 only */
+    int64_t ks_seq_stride; /* FP8 only, elements */
 } dsa_indexer;
 
 /*

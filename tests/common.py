@@ -55,6 +55,27 @@ def oracle_selection(w: wl.Workload, xh: dict, rows=None):
     return sc, idx, cnt
 
 
+def fp8_indexer(w: wl.Workload, f8: dict, x: dict, flags: int = 0) -> B.Indexer:
+    """Indexer descriptor of the FP8 (E4M3) variant from wl.fp8_indexer_inputs."""
+    k8 = f8["k8"][0] if w.shared_cache else f8["k8"]
+    ks = f8["k_scale"][0] if w.shared_cache else f8["k_scale"]
+    return B.Indexer(f8["q8"], x["w"], k8, flags=flags, q_scale=f8["q_scale"], k_scale=ks)
+
+
+def oracle_selection_fp8(w: wl.Workload, f8h: dict, xh: dict, rows=None):
+    """Oracle scores (on the exact dequantised E4M3 operands) + top-k."""
+    rows = np.arange(w.n_q) if rows is None else np.asarray(rows)
+    q_seq = xh["q_seq"].numpy()[rows]
+    q_pos = xh["q_pos"].numpy()[rows]
+    q_seq_o = np.zeros_like(q_seq) if w.shared_cache else q_seq
+    q8 = f8h["q8"].view(torch.uint8).numpy()[rows]
+    k8 = f8h["k8"].view(torch.uint8).numpy()
+    sc = oracle.index_scores_e4m3(q8, f8h["q_scale"].numpy()[rows], host_f32(xh["w"])[rows], k8,
+                                  f8h["k_scale"].numpy(), q_seq_o, q_pos)
+    idx, cnt = oracle.topk(sc, q_pos, w.topk)
+    return sc, idx, cnt
+
+
 def oracle_mla(w: wl.Workload, xh: dict, layer: int, idx, cnt, rows=None):
     rows = np.arange(w.n_q) if rows is None else np.asarray(rows)
     q_seq = xh["q_seq"].numpy()[rows]

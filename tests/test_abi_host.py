@@ -103,6 +103,25 @@ def test_index_scores_rejects(case):
     assert st == B.DSA_ERR_INVALID
 
 
+@pytest.mark.parametrize("case,expect", [
+    ("heads16", "unsupported"), ("row_stride_136", "unsupported"), ("seq_stride_not16", "unsupported"),
+    ("ks_stride_short", "invalid"), ("ks_stride_negative", "invalid"),
+])
+def test_index_scores_fp8_validation(case, expect):
+    """FP8 (E4M3) indexers run on the tensor-core path only (32 x 128, 16-element
+    TMA strides); a per-key scale array must cover max_ctx rows per sequence."""
+    lib = B.lib()
+    q = _q()
+    ix = _idx(dtype=B.DSA_FP8_E4M3)
+    if case == "heads16": ix.heads = 16
+    if case == "row_stride_136": ix.k_row_stride = 136
+    if case == "seq_stride_not16": ix.k_seq_stride = 1000 * 128 + 8
+    if case == "ks_stride_short": ix.k_scale, ix.ks_seq_stride = 0xA000, 500
+    if case == "ks_stride_negative": ix.ks_seq_stride = -1
+    st = lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(ix), 0x9000, 1000, _FakeWs.ptr, _FakeWs.size, None)
+    assert st == (B.DSA_ERR_UNSUPPORTED if expect == "unsupported" else B.DSA_ERR_INVALID)
+
+
 def test_workspace_checks():
     lib = B.lib()
     q, ix = _q(), _idx()

@@ -60,3 +60,33 @@ def test_named_workload_full_size(cuda_ok, name):
                                          np.arange(len(sel), dtype=np.int32)[None], rcnt, w.d_lat, w.scale)
             C.assert_attention_close(m.out[i:i + 1], out, w.dtype, f"query {i} layer {layer}")
             C.assert_lse_close(m.lse[i:i + 1], lse, w.dtype)
+
+
+@pytest.mark.parametrize("name", ["decode_32k", "decode_1m"])
+def test_fp8_indexer_full_size(cuda_ok, name):
+    """FP8 (E4M3) indexer variant at full size with the fused histogram and the
+    top-k, as the benchmark's --indexer-fp8 option runs it: scores bit-exact over
+    every visible key and indices bit-exact for a sampled query."""
+    w = wl.NAMED[name]
+    dev = torch.device("cuda")
+    x = wl.make_inputs(w, device=dev, layers=[])
+    f8 = wl.fp8_indexer_inputs(w, x, device=dev)
+    q, _, _ = C.descriptors(w, x, seq_run=1)
+    ix = C.fp8_indexer(w, f8, x, flags=B.DSA_INDEXER_TOPK_HIST)
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, 1, dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    idx = torch.empty((w.n_q, w.topk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.n_q,), dtype=torch.int32, device=dev)
+    B.dsa_index_scores(q, ix, scores, ws)
+    B.dsa_topk(q, scores, w.topk, idx, cnt, ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    i = w.n_q - 1
+    b, t = w.q_seq[i], w.q_pos[i]
+    sc = oracle.index_scores_e4m3(f8["q8"][i:i + 1].view(torch.uint8).cpu().numpy(),
+                                  f8["q_scale"][i:i + 1].cpu().numpy(), C.host_f32(x["w"][i:i + 1]),
+                                  f8["k8"][b:b + 1].view(torch.uint8).cpu().numpy(),
+                                  f8["k_scale"][b:b + 1].cpu().numpy(), [0], [t])
+    np.testing.assert_array_equal(scores[i, : t + 1].cpu().double().numpy(), sc[0, : t + 1])
+    ridx, rcnt = oracle.topk(sc, [t], w.topk)
+    np.testing.assert_array_equal(idx[i].cpu().numpy(), ridx[0])
+    assert int(cnt[i]) == int(rcnt[0])

@@ -91,6 +91,70 @@ def test_repeated_steps_one_workspace(dev, name, L_long):
         np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
 
 
+FP8_CASES = ["decode_edges", "decode_ragged", "prefill_small", "shared_cache", "ties"]
+
+
+@pytest.mark.parametrize("name", FP8_CASES)
+def test_fp8_index_scores_bit_exact(dev, name):
+    """FP8 (E4M3) indexer with per-(query, head) and per-key scales: every visible
+    score equals the oracle's (exact on the recipe's values)."""
+    w = SMALL[name]
+    xh = wl.make_inputs(w, layers=[])
+    f8h = wl.fp8_indexer_inputs(w, xh)
+    x, f8 = C.to_device(xh), C.to_device(f8h)
+    q, _, _ = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ix = C.fp8_indexer(w, f8, x)
+    ws = B.workspace(B.DSA_OP_INDEX_SCORES, q, device=dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    scores.fill_(float("nan"))
+    B.dsa_index_scores(q, ix, scores, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    ref, _, _ = C.oracle_selection_fp8(w, f8h, xh)
+    got = scores[:, : w.L].cpu().double().numpy()
+    for i, t in enumerate(w.q_pos):
+        np.testing.assert_array_equal(got[i, : t + 1], ref[i, : t + 1], err_msg=f"query {i}")
+
+
+@pytest.mark.parametrize("name", ["decode_edges", "decode_ragged", "ties"])
+@pytest.mark.parametrize("L_long", [False, True])
+def test_fp8_fused_topk_matches_oracle(dev, name, L_long):
+    """FP8 indexer with the fused first-digit histogram, then the top-k (row and
+    split schedules), twice on one workspace: indices bit-exact both times."""
+    w = SMALL[name]
+    if L_long:
+        w = wl.scaled(w, L=20000, q_pos=tuple(min(19999, p + 15000) for p in w.q_pos))
+    xh = wl.make_inputs(w, layers=[])
+    f8h = wl.fp8_indexer_inputs(w, xh)
+    x, f8 = C.to_device(xh), C.to_device(f8h)
+    q, _, _ = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ix = C.fp8_indexer(w, f8, x, flags=B.DSA_INDEXER_TOPK_HIST)
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, 1, dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    _, ridx, rcnt = C.oracle_selection_fp8(w, f8h, xh)
+    for step in range(2):
+        idx = torch.full((w.n_q, w.topk), -7, dtype=torch.int32, device=dev)
+        cnt = torch.full((w.n_q,), -7, dtype=torch.int32, device=dev)
+        B.dsa_index_scores(q, ix, scores, ws)
+        B.dsa_topk(q, scores, w.topk, idx, cnt, ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+        assert B.dsa_check_status(ws) == B.DSA_OK
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt, err_msg=f"step {step}")
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
+
+
+def test_fp8_unsupported_shape_is_rejected(dev):
+    """The tiny workload's 4 x 32 indexer has no FP8 path: rejected before launch."""
+    w = SMALL["tiny"]
+    xh = wl.make_inputs(w, layers=[])
+    x = C.to_device(xh)
+    q, _, _ = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ix = B.Indexer(x["q_idx"].to(torch.float8_e4m3fn), x["w"], x["k_idx"].to(torch.float8_e4m3fn))
+    ws = B.workspace(B.DSA_OP_INDEX_SCORES, q, device=dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    with pytest.raises(B.DsaError) as e:
+        B.dsa_index_scores(q, ix, scores, ws)
+    assert e.value.status == B.DSA_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 def test_index_scores_bit_exact(dev, name):
     w = SMALL[name]
