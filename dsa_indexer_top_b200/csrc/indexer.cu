@@ -37,13 +37,14 @@ struct IdxCfg {
     static constexpr int kTileBytes = kTileKeys * kIdxDim * kElem;  // 32 KB bf16, 16 KB FP8
     static constexpr int kBoxes = kElem;                          // 128-byte-wide boxes per row
     static constexpr int kKSteps = F8 ? kIdxDim / 32 : kIdxDim / 16;  // MMA K = 32 (8-bit) or 16
-    // One query per tile: two CTAs per SM, 64 KB of key stages each.  Two
-    // independent load -> MMA -> epilogue pipelines per SM keep the key stream
-    // at the rate of a plain TMA read stream, where one CTA with deeper
-    // buffering loses about 6% to the MMA turnaround of each stage; more than
-    // about 128 KB in flight per SM lowers the stream rate again.
-    static constexpr int kCtasPerSm = G == 1 ? 2 : 1;
-    static constexpr int kStages = G == 1 ? (F8 ? 4 : 2) : 4;
+    // One query per tile: several independent load -> MMA -> epilogue pipelines
+    // per SM keep the key stream at the rate of a plain TMA read stream, where one
+    // CTA with deeper buffering loses about 6% to the MMA turnaround of each
+    // stage, and more than about 128 KB in flight per SM lowers the stream rate
+    // again.  bf16: two CTAs x two 32 KB stages; FP8 (half the bytes per key, the
+    // same epilogue work): three CTAs x three 16 KB stages (measured best).
+    static constexpr int kCtasPerSm = G == 1 ? (F8 ? 3 : 2) : 1;
+    static constexpr int kStages = G == 1 ? (F8 ? 3 : 2) : 4;
     static constexpr int kBBytes = N * kIdxDim * kElem;
     static constexpr int kTmemCols = (2 * N < 32) ? 32 : 2 * N;
     static constexpr int kSmem = kStages * kTileBytes + kBBytes + 1024;
@@ -309,13 +310,14 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
             if (seq < 0 || j * kTileKeys > max_pos) continue;
             const int acc = static_cast<int>(k_tiles & 1);
             const int acc_use = static_cast<int>(k_tiles >> 1);
-            if (!mbar_wait(&tmem_full[acc], acc_use & 1, a.status, &abort_flag)) break;
-            tc_fence_after();
             const int s = j * kTileKeys + quad * 32 + lane;
-            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * N;
-            // FP8: the key's positive scale factors out of every head's ReLU
+            // FP8: the key's positive scale factors out of every head's ReLU (loaded
+            // before the wait for the accumulator, so its latency is hidden)
             const float ks = (F8 && a.k_scale && s < a.L) ? __ldg(a.k_scale + static_cast<int64_t>(seq) * a.ks_seq_stride + s)
                                                          : 1.f;
+            if (!mbar_wait(&tmem_full[acc], acc_use & 1, a.status, &abort_flag)) break;
+            tc_fence_after();
+            const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + acc * N;
 #pragma unroll
             for (int ii = 0; ii < kQPerWarp; ++ii) {
                 const int i = qlo + ii;
