@@ -41,6 +41,9 @@ L2_FLUSH_BYTES = 256 << 20
 # full size (67.61 MB); one sequence of 1M keys (275.13 MB), whose 4-sequence
 # launch streams 4 such caches (traffic x 4).  Absent workloads report null.
 NCU_INDEXER_TRAFFIC = {"decode_32k": 67.61e6, "decode_1m": 4 * 275.13e6}
+# the same for the FP8 variant (profiles/idx_score_tc_fp8_decode.md): 8 x 32K at
+# full size 34.68 MB; one 1M sequence 142.76 MB (x 4 for the 4-sequence launch)
+NCU_INDEXER_TRAFFIC_FP8 = {"decode_32k": 34.68e6, "decode_1m": 4 * 142.76e6}
 
 
 def measured_peaks():
@@ -514,7 +517,8 @@ def main():
                    "l2": "flushed before every timed step (256 MB write)", "graph": "CUDA graph per step"},
         "roofline": {"bound": "hbm", "kernel": "idx_score_tc (dsa_index_scores)", "achieved": idx_gbs,
                      "peak": hbm_peak, "unit": "GB/s", "frac": idx_gbs / hbm_peak,
-                     "traffic": None if fp8 else NCU_INDEXER_TRAFFIC.get(w.name), "peak_kind": f"{peak_kind} hbm_gbs",
+                     "traffic": (NCU_INDEXER_TRAFFIC_FP8 if fp8 else NCU_INDEXER_TRAFFIC).get(w.name),
+                     "peak_kind": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes": by["indexer"], "avg_launch_us": idx_ms * 1e3},
         "path_roofline": {"bytes": by["path"], "t_roof_us": t_roof_us,
                           "frac": t_roof_us / (ms_per_step * 1e3), "peak_kind": f"{peak_kind} hbm_gbs"},
