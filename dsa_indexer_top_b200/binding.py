@@ -73,6 +73,8 @@ def lib():
         h.dsa_workspace_bytes.restype = SZ
         h.dsa_workspace_init.argtypes = [P, SZ, P]
         h.dsa_check_status.argtypes = [P, P]
+        h.dsa_debug_bounded_wait.argtypes = [P, SZ, ctypes.c_uint64, P]
+        h.dsa_debug_bounded_wait.restype = st
         h.dsa_status_str.argtypes = [st]
         h.dsa_status_str.restype = ctypes.c_char_p
         for name in ("dsa_index_scores", "dsa_topk", "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill",
@@ -178,6 +180,11 @@ def dsa_workspace_init(ws: torch.Tensor, stream=None):
 def dsa_check_status(ws: torch.Tensor, stream=None) -> int:
     """Synchronise, read and clear the workspace status word (returns the code)."""
     return int(lib().dsa_check_status(_ptr(ws), _stream(stream)))
+
+
+def dsa_debug_bounded_wait(ws: torch.Tensor, limit_ns: int, stream=None):
+    _check(lib().dsa_debug_bounded_wait(_ptr(ws), ws.numel() * ws.element_size(), int(limit_ns), _stream(stream)),
+           "dsa_debug_bounded_wait")
 
 
 def dsa_index_scores(queries: Queries, indexer: Indexer, scores: torch.Tensor, ws: torch.Tensor, stream=None):

@@ -351,6 +351,14 @@ dsa_status dsa_workspace_init(void *ws, size_t ws_bytes, void *stream) {
                                                                                                : DSA_ERR_CUDA;
 }
 
+dsa_status dsa_debug_bounded_wait(void *ws, size_t ws_bytes, uint64_t limit_ns, void *stream) {
+    if (!ws_ok(ws, ws_bytes, kStatusBytes)) return DSA_ERR_INVALID;
+    if (limit_ns > kDeviceWaitLimitNs) return DSA_ERR_INVALID;
+    return launch_bounded_wait_probe(status_word(ws), limit_ns, static_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? DSA_OK
+               : DSA_ERR_CUDA;
+}
+
 dsa_status dsa_check_status(void *ws, void *stream) {
     if (!ws) return DSA_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);

@@ -114,6 +114,14 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st);
 // First-digit histograms only (into a.ghist, which must be zeroed), every query.
 cudaError_t launch_topk_hist(const TopkArgs &a, int num_sms, cudaStream_t st);
 
+// ------------------------------------------------------------------ diagnostics
+// The limit of every device-side wait (the same value as kWaitLimitNs of the
+// PTX wrappers): 2 s.
+constexpr uint64_t kDeviceWaitLimitNs = 2000000000ull;
+// One thread waits (bounded, limit_ns) on a barrier nothing completes and
+// reports DSA_ERR_TIMEOUT into *status.
+cudaError_t launch_bounded_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t st);
+
 // ------------------------------------------------------------------ sparse MLA
 struct MlaLayerPtrs {
     const void *q;

@@ -90,14 +90,14 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
 // kWaitLimitNs, records DSA_ERR_TIMEOUT, raises the CTA abort flag and returns
 // false.  Returns false at once when the abort flag is already raised.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t *status,
-                                          volatile int *abort_flag) {
+                                          volatile int *abort_flag, uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     uint64_t t0 = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 63u) == 0) {
             if (abort_flag && *abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 report_status(status, DSA_ERR_TIMEOUT);
                 if (abort_flag) *abort_flag = 1;
                 return false;

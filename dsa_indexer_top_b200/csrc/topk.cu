@@ -831,6 +831,23 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
     return launch_pdl(topk_split_kernel, dim3(P, a.n_q), dim3(kT), sizeof(SplitSmem), st, a, chunk, P);
 }
 
+static_assert(kWaitLimitNs == kDeviceWaitLimitNs, "one device wait limit");
+
+namespace {
+// The bounded-wait probe: the barrier expects one arrival that never comes.
+__global__ void bounded_wait_probe_kernel(uint32_t *status, uint64_t limit_ns) {
+    __shared__ uint64_t bar;
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait(&bar, 0, status, nullptr, limit_ns);
+}
+}  // namespace
+
+cudaError_t launch_bounded_wait_probe(uint32_t *status, uint64_t limit_ns, cudaStream_t st) {
+    bounded_wait_probe_kernel<<<1, 1, 0, st>>>(status, limit_ns);
+    return cudaGetLastError();
+}
+
 size_t topk_zeroed_bytes(int n_q) { return sizeof(uint32_t) * (static_cast<size_t>(kBins) + 1) * n_q; }
 
 // Scratch: [n_q][4096] first-digit histograms, then [n_q] tickets.  Both are

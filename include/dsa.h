@@ -313,6 +313,20 @@ dsa_status dsa_check_status(void *ws, void *stream);
 /* Human-readable name of a status code (static string). */
 const char *dsa_status_str(dsa_status status);
 
+/*
+ * Diagnostic (no counterpart on the pages): exercises the device-side bounded
+ * wait every kernel of this library uses.  Launches one thread that waits on a
+ * shared-memory barrier nothing completes, with the library's wait routine and
+ * a limit of `limit_ns` nanoseconds (at most 2 s, the limit the kernels use);
+ * when the limit runs out the wait gives up, the thread writes
+ * DSA_ERR_TIMEOUT into the workspace status word and exits, and the context
+ * stays usable.  Read the result with dsa_check_status().  Nothing else is
+ * launched or touched; no copy or tensor-core work is in flight during the
+ * wait.  DSA_ERR_INVALID for a null or too-small workspace or a limit above
+ * 2 s.
+ */
+dsa_status dsa_debug_bounded_wait(void *ws, size_t ws_bytes, uint64_t limit_ns, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

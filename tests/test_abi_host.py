@@ -122,6 +122,13 @@ def test_index_scores_fp8_validation(case, expect):
     assert st == (B.DSA_ERR_UNSUPPORTED if expect == "unsupported" else B.DSA_ERR_INVALID)
 
 
+def test_debug_bounded_wait_validation():
+    lib = B.lib()
+    lib.dsa_debug_bounded_wait.argtypes = [ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64, ctypes.c_void_p]
+    assert lib.dsa_debug_bounded_wait(None, 0, 1000, None) == B.DSA_ERR_INVALID
+    assert lib.dsa_debug_bounded_wait(_FakeWs.ptr, _FakeWs.size, 3_000_000_000, None) == B.DSA_ERR_INVALID
+
+
 def test_workspace_checks():
     lib = B.lib()
     q, ix = _q(), _idx()

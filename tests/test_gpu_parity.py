@@ -91,6 +91,24 @@ def test_repeated_steps_one_workspace(dev, name, L_long):
         np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
 
 
+def test_bounded_wait_times_out_and_context_stays_usable(dev):
+    """A device wait on a barrier that nothing completes gives up after its limit,
+    reports DSA_ERR_TIMEOUT through the workspace status word (no hang, no
+    fault), and the next calls on the same context are correct."""
+    w = SMALL["decode_edges"]
+    xh = wl.make_inputs(w)
+    x = C.to_device(xh)
+    q, _, _ = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, w.n_layers, dev)
+    B.dsa_debug_bounded_wait(ws, 20_000_000)  # 20 ms
+    assert B.dsa_check_status(ws) == B.DSA_ERR_TIMEOUT
+    assert B.dsa_check_status(ws) == B.DSA_OK  # read-and-clear
+    _, idx, cnt, mlas = _run_steps(w, x)
+    _, ridx, rcnt = C.oracle_selection(w, xh)
+    np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+    np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+
+
 FP8_CASES = ["decode_edges", "decode_ragged", "prefill_small", "shared_cache", "ties"]
 
 
