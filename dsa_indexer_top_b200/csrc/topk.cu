@@ -646,15 +646,17 @@ struct SplitSmem {
     int last;
 };
 
-struct StagedSegs {  // warp w: candidates [wbeg[w], wbeg[w] + wcnt[w]) of one array
+// The staged candidates are one array in position order, so warp w may take
+// an equal share of it regardless of chunk boundaries: [w*M/16, (w+1)*M/16).
+struct StagedSegs {
     const uint2 *cand;
-    const uint32_t *coff;  // chunk offsets
-    const int n_chunks;
+    const uint32_t total;  // M
     __device__ int pieces(int) const { return 1; }
-    __device__ const uint2 *ptr(int w, int) const { return cand + coff[w * n_chunks / kWarps]; }
-    __device__ uint32_t count(int w, int) const {
-        return coff[(w + 1) * n_chunks / kWarps] - coff[w * n_chunks / kWarps];
+    __device__ uint32_t begin(int w) const {
+        return static_cast<uint32_t>((static_cast<uint64_t>(total) * w) / kWarps);
     }
+    __device__ const uint2 *ptr(int w, int) const { return cand + begin(w); }
+    __device__ uint32_t count(int w, int) const { return begin(w + 1) - begin(w); }
 };
 
 // Finish query i from the chunks' candidates (written by other CTAs of this
@@ -698,7 +700,7 @@ __device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
-        const StagedSegs sg{sm.cand, sm.coff, n_chunks};
+        const StagedSegs sg{sm.cand, sm.coff[n_chunks]};
         if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out)) {
             uint32_t T, need_eq;
             seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
