@@ -35,6 +35,7 @@ UNIT = "qtok/s/layer"
 ROOT = os.path.dirname(os.path.abspath(__file__))
 DECODE_MAX_QUERIES = 256    # the MLA decode (split-K) schedule up to this many queries
 L2_FLUSH_BYTES = 256 << 20
+REFERENCE_BUDGET_S = 120.0  # timed oracle work of one --impl reference run
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch, from the ncu
 # captures summarised in profiles/idx_score_tc_decode.md: 8 x 32K keys captured at
@@ -412,13 +413,18 @@ def run_reference(args, w: wl.Workload, world: int, rank: int):
     x = wl.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
     order = list(range(w.n_q))
     h = host_copies(w, x, order)
-    for s in range(args.warmup):
+    for s in range(min(args.warmup, 3)):
         oracle_sample_time(w, h, [order[s % w.n_q]])
-    t = 0.0
+    # bounded: stop after REFERENCE_BUDGET_S of timed oracle work (long contexts
+    # take seconds per query) and report the steps actually timed
+    t, done = 0.0, 0
     for s in range(args.steps):
         t += oracle_sample_time(w, h, [order[s % w.n_q]])
-    value = args.steps * w.n_layers / t
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        done += 1
+        if t > REFERENCE_BUDGET_S:
+            break
+    value = done * w.n_layers / t
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": done,
             "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
             "config": {**w.describe(), "sample_per_step": "1 query, all layers"},
