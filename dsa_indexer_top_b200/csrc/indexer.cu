@@ -16,8 +16,14 @@
 //               ReLU, multiply by w and sum the 32 heads inside the thread, causal
 //               mask, coalesced fp32 store of one score per key per query.
 // Work items are (query group, key tile) pairs split into contiguous ranges over
-// a grid of at most two CTAs per SM (one query per tile) or one (several);
-// tiles past the group's last visible key are skipped.
+// a grid of at most two CTAs per SM (one query per tile; three for FP8) or one
+// (several); tiles past the group's last visible key are skipped.
+//
+// FP8 variant (E4M3 queries and keys, each row scaled by a positive float): the
+// same kernel with 16 KB tiles (one 128-byte box of E4M3 bytes per tile), four
+// K = 32 tcgen05.mma.kind::f8f6f4 steps per tile, the query scale folded into w
+// and the key scale applied to the finished score -- both factor out of the
+// ReLU because they are positive.
 #include <algorithm>
 #include <cuda_bf16.h>
 
