@@ -448,11 +448,15 @@ def main():
                          "not the bf16 headline)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="decode workloads: override the batch (a smaller case for profiling; not a bench line)")
+    ap.add_argument("--n-q", type=int, default=0,
+                    help="prefill: keep the last N queries of the chunk (a smaller case for profiling; not a bench line)")
     args = ap.parse_args()
     w = wl.NAMED[args.workload]
     if args.n_seq and len(set(w.q_seq)) == w.n_q:
         w = wl.scaled(w, n_seq=args.n_seq, q_pos=w.q_pos[:1] * args.n_seq, q_seq=tuple(range(args.n_seq)),
                       name=f"{w.name}_b{args.n_seq}")
+    if args.n_q and len(set(w.q_seq)) == 1 and args.n_q < w.n_q:
+        w = wl.scaled(w, q_pos=w.q_pos[-args.n_q:], q_seq=w.q_seq[-args.n_q:], name=f"{w.name}_q{args.n_q}")
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
