@@ -12,9 +12,11 @@
 //   warp 1      tcgen05.mma issuer: D[128 keys][32G] = K_tile (M=128, K-major)
 //               x Q^T (N = 32G, K-major), K = 128 in eight K=16 steps, fp32
 //               accumulators in TMEM, double-buffered.
-//   warps 2-5   epilogue: tcgen05.ld of its 32 TMEM lanes (one key per lane),
-//               ReLU, multiply by w and sum the 32 heads inside the thread, causal
-//               mask, coalesced fp32 store of one score per key per query.
+//   warps 2..   epilogue (4, 8 or 16 warps for 1, 2-4 or 8 queries per tile;
+//               warp w reads TMEM lane quadrant w % 4 and its share of the
+//               queries): tcgen05.ld of its 32 lanes (one key per lane), ReLU,
+//               multiply by w and sum the 32 heads inside the thread, causal mask,
+//               coalesced fp32 store of one score per key per query.
 // Work items are (query group, key tile) pairs split into contiguous ranges over
 // a grid of at most two CTAs per SM (one query per tile; three for FP8) or one
 // (several); tiles past the group's last visible key are skipped.
@@ -55,9 +57,11 @@ struct IdxCfg {
     static constexpr int kTmemCols = (2 * N < 32) ? 32 : 2 * N;
     static constexpr int kSmem = kStages * kTileBytes + kBBytes + 1024;
     static constexpr uint32_t kIdesc = F8 ? idesc_e4m3(128, N) : idesc_bf16(128, N, false, false);
-    // epilogue warps: two per TMEM lane quadrant when a tile holds several
-    // queries (each takes half of them), one otherwise
-    static constexpr int kEpiWarps = G >= 2 ? 8 : 4;
+    // epilogue warps: one per TMEM lane quadrant for one query per tile, two
+    // (each half of the queries) for 2 or 4, four (each a quarter) for 8 -- with
+    // 8 queries per tile the ReLU-weighted head sums outweigh the MMA, so the
+    // epilogue gets four warps per scheduler
+    static constexpr int kEpiWarps = G >= 8 ? 16 : (G >= 2 ? 8 : 4);
     static constexpr int kThreads = (2 + kEpiWarps) * 32;
 };
 
@@ -249,8 +253,8 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
         // ------------------------------------------------------------ epilogue
         const int quad = warp & 3;  // TMEM lane quadrant this warp may access
         // queries of the tile this warp handles
-        constexpr int kQPerWarp = E == 8 ? G / 2 : G;
-        const int qlo = E == 8 ? ((warp - 2) >> 2) * kQPerWarp : 0;
+        constexpr int kQPerWarp = G / (E / 4);
+        const int qlo = ((warp - 2) >> 2) * kQPerWarp;
         float *w_mine = w_sh[warp - 2];
         const int etid = threadIdx.x - 64;
         int cur_g = -1, seq = -1, max_pos = -1;
