@@ -4,6 +4,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "dsa.h"
 #include "kernels.cuh"
 
@@ -313,6 +315,15 @@ dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, co
 
 }  // namespace
 
+namespace {
+// An NVTX range around each compute entry point (header-only NVTX v3: without a
+// profiler attached a push/pop is a few nanoseconds of host time).
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+};
+}  // namespace
+
 extern "C" {
 
 const char *dsa_status_str(dsa_status s) {
@@ -371,6 +382,7 @@ dsa_status dsa_check_status(void *ws, void *stream) {
 
 dsa_status dsa_index_scores(const dsa_queries *queries, const dsa_indexer *indexer, float *scores,
                             int64_t ld_scores, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange range("dsa_index_scores");
     if (!valid_queries(queries)) return DSA_ERR_INVALID;
     if (!ws_ok(ws, ws_bytes, ws_index_scores())) return DSA_ERR_WORKSPACE;
     dsa_status s = check_indexer(queries, indexer);
@@ -387,6 +399,7 @@ dsa_status dsa_index_scores(const dsa_queries *queries, const dsa_indexer *index
 
 dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_scores, int32_t topk, int32_t flags,
                     int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange range("dsa_topk");
     if (!valid_queries(queries)) return DSA_ERR_INVALID;
     if (!ws_ok(ws, ws_bytes, ws_topk(queries->n_q, queries->max_ctx))) return DSA_ERR_WORKSPACE;
     if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
@@ -412,17 +425,20 @@ static dsa_status mla_entry(const dsa_queries *queries, const dsa_mla *mla, cons
 
 dsa_status dsa_sparse_mla_decode(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,
                                  const int32_t *cnt, int32_t topk, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange range("dsa_sparse_mla_decode");
     return mla_entry(queries, mla, idx, cnt, topk, ws, ws_bytes, stream, true);
 }
 
 dsa_status dsa_sparse_mla_prefill(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,
                                   const int32_t *cnt, int32_t topk, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange range("dsa_sparse_mla_prefill");
     return mla_entry(queries, mla, idx, cnt, topk, ws, ws_bytes, stream, false);
 }
 
 dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *indexer, const dsa_mla *layers,
                                 int32_t n_layers, int32_t topk, int32_t *idx, int32_t *cnt, void *ws,
                                 size_t ws_bytes, void *stream) {
+    NvtxRange range("dsa_indexshare_group");
     if (!valid_queries(queries)) return DSA_ERR_INVALID;
     if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
     dsa_status s = check_indexer(queries, indexer);
