@@ -159,6 +159,34 @@ def test_fp8_fused_topk_matches_oracle(dev, name, L_long):
         np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
 
 
+@pytest.mark.parametrize("which", ["no_q_scale", "no_k_scale", "no_scales"])
+def test_fp8_null_scales_mean_one(dev, which):
+    """FP8 scale arrays may be NULL (all 1): scores equal the oracle's with unit
+    scales for the missing side."""
+    w = SMALL["decode_ragged"]
+    xh = wl.make_inputs(w, layers=[])
+    f8h = wl.fp8_indexer_inputs(w, xh)
+    if which in ("no_q_scale", "no_scales"):
+        f8h["q_scale"] = torch.ones_like(f8h["q_scale"])
+    if which in ("no_k_scale", "no_scales"):
+        f8h["k_scale"] = torch.ones_like(f8h["k_scale"])
+    x, f8 = C.to_device(xh), C.to_device(f8h)
+    q, _, _ = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ix = C.fp8_indexer(w, f8, x)
+    if which in ("no_q_scale", "no_scales"):
+        ix.q_scale = None
+    if which in ("no_k_scale", "no_scales"):
+        ix.k_scale = None
+    ws = B.workspace(B.DSA_OP_INDEX_SCORES, q, device=dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    B.dsa_index_scores(q, ix, scores, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    ref, _, _ = C.oracle_selection_fp8(w, f8h, xh)
+    got = scores[:, : w.L].cpu().double().numpy()
+    for i, t in enumerate(w.q_pos):
+        np.testing.assert_array_equal(got[i, : t + 1], ref[i, : t + 1], err_msg=f"query {i}")
+
+
 def test_fp8_unsupported_shape_is_rejected(dev):
     """The tiny workload's 4 x 32 indexer has no FP8 path: rejected before launch."""
     w = SMALL["tiny"]
