@@ -35,7 +35,7 @@ constexpr int kMlaHeads = 64;   // num_attention_heads of GLM-5.2
 constexpr int kLatent = 512;    // kv_lora_rank
 constexpr int kRope = 64;       // qk_rope_head_dim
 constexpr int kRow = kLatent + kRope;
-constexpr int kRowsPerChunk = 128;  // rows per split of the workspace bound (ceil(topk / 128) splits)
+constexpr int kRowsPerChunk = 128;  // splits <= ceil(topk / 128): every CTA walks >= 2 chunks of 64 rows
 constexpr int kMlaChunk = 64;       // selected rows per tensor-core pipeline chunk
 constexpr int kMaxTopk = 4096;
 constexpr int kMaxLayers = 4;
@@ -145,7 +145,7 @@ struct MlaArgs {
     uint32_t *status;
     // split-K schedule (tensor-core path)
     int n_splits;        // CTAs per query
-    int chunks_per_cta;  // 128-row chunks walked by one CTA
+    int chunks_per_cta;  // 64-row chunks walked by one CTA
     float *part_o;       // [layers][n_q][n_splits][64][512] unnormalised
     float *part_ml;      // [layers][n_q][n_splits][64][2] (max, sum) in log2 units
 };
