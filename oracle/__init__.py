@@ -14,6 +14,10 @@ Functions and the passages they follow (page title, section):
   topk             -- same row: min(index_topk, n) largest scores, int32 indices.
   sparse_mla       -- same page, rows Multi-head latent attention / Learnable
                       attention sink / Partial RoPE (absorbed form, plain softmax).
+  sparse_mla_fp8   -- sparse_mla over a cache with 8-bit (E4M3) latents and one
+                      float32 scale per row ("GLM-5.2 -- Model techniques map",
+                      inference quantization: FP8 inference; row format read
+                      here, the pages give none).
   dense_mla        -- textbook causal attention (the topk >= n special case).
   indexshare_group -- "GLM 5.2 -- Hermosa AI", "MLA + DSA with IndexShare".
 Every function is pinned by tests in tests/test_oracle_pins.py.
@@ -66,6 +70,8 @@ def _load():
                                       _i32p, _i32p, _i32p, ci, _f64p, ctypes.c_void_p]
     lib.oracle_dense_mla.argtypes = [ci, ci, ci, ci, ctypes.c_double, _f32p, _f32p, i64, i64,
                                      _i32p, _i32p, _f64p, ctypes.c_void_p]
+    lib.oracle_sparse_mla_fp8.argtypes = [ci, ci, ci, ci, ctypes.c_double, _f32p, _u8p, i64, i64,
+                                          _i32p, _i32p, _i32p, ci, _f64p, ctypes.c_void_p]
     _lib = lib
     return lib
 
@@ -152,6 +158,28 @@ def sparse_mla(q, kv, q_seq, idx, cnt, d_lat, scale):
     lse = np.empty((n_q, heads), dtype=np.float64)
     _load().oracle_sparse_mla(n_q, heads, d_lat, dk - d_lat, float(scale), q, kv, L * dk, dk,
                               q_seq, idx, cnt, topk_, out, lse.ctypes.data)
+    return out, lse
+
+
+def sparse_mla_fp8(q, kv8, q_seq, idx, cnt, d_lat, d_rope, scale):
+    """FP8 latent cache: q [n_q,H,d_lat+d_rope] float, kv8 [n_seq,L,row_bytes] uint8
+    rows [E4M3 latent codes (d_lat) | bf16 RoPE key (2*d_rope bytes) | float32 scale |
+    padding], idx [n_q,topk], cnt [n_q] -> (out [n_q,H,d_lat], lse [n_q,H]) float64,
+    attending over c = scale_row * e4m3(code)."""
+    q = _f32(q)
+    kv8 = np.ascontiguousarray(np.asarray(kv8, dtype=np.uint8))
+    q_seq, idx, cnt = _i32(q_seq), _i32(idx), _i32(cnt)
+    n_q, heads, dk = q.shape
+    n_seq, L, row_bytes = kv8.shape
+    assert dk == d_lat + d_rope and row_bytes >= d_lat + 2 * d_rope + 4 and d_lat % 4 == 0
+    topk_ = idx.shape[1]
+    for i in range(n_q):
+        sel = idx[i, : cnt[i]]
+        assert np.all((sel >= 0) & (sel < L)), "selected index out of range"
+    out = np.empty((n_q, heads, d_lat), dtype=np.float64)
+    lse = np.empty((n_q, heads), dtype=np.float64)
+    _load().oracle_sparse_mla_fp8(n_q, heads, d_lat, d_rope, float(scale), q, kv8, L * row_bytes, row_bytes,
+                                  q_seq, idx, cnt, topk_, out, lse.ctypes.data)
     return out, lse
 
 

@@ -287,3 +287,87 @@ void oracle_dense_mla(int n_q, int heads, int d_lat, int d_rope, double scale, c
         free(buf);
     }
 }
+
+/* Value of a bf16 bit pattern: the upper half of an IEEE binary32. */
+static double bf16_bits_to_double(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/*
+ * attend_one_head on rows already widened to double: rows is [n_rows][d_lat +
+ * d_rope], row j = [c_j | r_j].  The same steps in the same order.
+ */
+static void attend_one_head_f64(const float *qh, const double *rows, int n_rows, int d_lat, int d_rope,
+                                double scale, double *logit_buf, double *out, double *lse) {
+    int dk = d_lat + d_rope;
+    double m = -INFINITY;
+    for (int j = 0; j < n_rows; j++) {
+        double dot = 0.0;
+        for (int d = 0; d < dk; d++) dot += (double)qh[d] * rows[(int64_t)j * dk + d];
+        logit_buf[j] = scale * dot;
+        if (logit_buf[j] > m) m = logit_buf[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < n_rows; j++) {
+        logit_buf[j] = exp(logit_buf[j] - m);
+        l += logit_buf[j];
+    }
+    for (int d = 0; d < d_lat; d++) out[d] = 0.0;
+    for (int j = 0; j < n_rows; j++) {
+        double p = logit_buf[j] / l;
+        for (int d = 0; d < d_lat; d++) out[d] += p * rows[(int64_t)j * dk + d];
+    }
+    *lse = m + log(l);
+}
+
+/*
+ * Sparse absorbed MLA over a cache that keeps the latent in 8 bits (the FP8
+ * variant: "GLM-5.2 -- Model techniques map" lists FP8 inference under
+ * inference quantization, and the key-facts table of "GLM-5.2 -- LLM atlas"
+ * gives fp8 as the precision; the cache format below is this oracle's reading,
+ * the pages give none).  Row s of sequence b is the byte string at
+ * kv8 + b*kv_seq_stride + s*kv_row_stride (strides in bytes):
+ *   bytes [0, d_lat)                    E4M3 codes c8[d] of the latent
+ *   bytes [d_lat, d_lat + 2*d_rope)     the RoPE key r as bf16, little-endian
+ *   bytes [d_lat + 2*d_rope, + 4)       float32 scale sigma, little-endian
+ * and the latent the attention sees is c[d] = sigma * e4m3(c8[d]).  Every
+ * selected row is widened to double exactly (one product per latent value) and
+ * attended as in oracle_sparse_mla.
+ */
+void oracle_sparse_mla_fp8(int n_q, int heads, int d_lat, int d_rope, double scale, const float *q,
+                           const uint8_t *kv8, int64_t kv_seq_stride, int64_t kv_row_stride,
+                           const int32_t *q_seq, const int32_t *idx, const int32_t *cnt, int topk,
+                           double *out, double *lse) {
+    int dk = d_lat + d_rope;
+    double lut[256];
+    for (int c = 0; c < 256; c++) lut[c] = oracle_e4m3_to_double((uint8_t)c);
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t e = 0; e < (int64_t)n_q * heads; e++) {
+        int i = (int)(e / heads);
+        int n_rows = cnt[i];
+        size_t nr = (size_t)(n_rows > 0 ? n_rows : 1);
+        double *rows = (double *)malloc(sizeof(double) * nr * (size_t)dk);
+        double *buf = (double *)malloc(sizeof(double) * nr);
+        const uint8_t *base = kv8 + (int64_t)q_seq[i] * kv_seq_stride;
+        for (int j = 0; j < n_rows; j++) {
+            const uint8_t *row = base + (int64_t)idx[(int64_t)i * topk + j] * kv_row_stride;
+            float sigma;
+            memcpy(&sigma, row + d_lat + 2 * d_rope, sizeof sigma);
+            double *dst = rows + (int64_t)j * dk;
+            for (int d = 0; d < d_lat; d++) dst[d] = (double)sigma * lut[row[d]];
+            for (int d = 0; d < d_rope; d++) {
+                uint16_t bits;
+                memcpy(&bits, row + d_lat + 2 * d, sizeof bits);
+                dst[d_lat + d] = bf16_bits_to_double(bits);
+            }
+        }
+        double l;
+        attend_one_head_f64(q + e * dk, rows, n_rows, d_lat, d_rope, scale, buf, out + e * d_lat, &l);
+        if (lse) lse[e] = l;
+        free(rows);
+        free(buf);
+    }
+}

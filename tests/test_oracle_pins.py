@@ -14,7 +14,10 @@ transposed operand -- breaks at least one):
   * closed forms: constant rows, a single row, q = 0 (uniform weights);
   * the E4M3 8-bit float format's defining values and torch's float8_e4m3fn
     decoding, for the FP8 indexer variant, and the positive homogeneity of ReLU
-    (a per-row scale of the keys or of a head's query factors out).
+    (a per-row scale of the keys or of a head's query factors out);
+  * for the FP8 latent cache: torch's float8 / bf16 decoding of the packed bytes,
+    SDPA on the exact values, and sparse_mla itself where power-of-two scales keep
+    every value exact in float32.
 """
 import json
 import math
@@ -420,3 +423,127 @@ def test_fp8_scales_factor_out_of_relu():
         dots = np.einsum("hd,sd->hs", qv[i].astype(np.float64), kv[q_seq[i], : t + 1].astype(np.float64))
         ref_q = ((w[i].astype(np.float64) * q_scale[i].astype(np.float64))[:, None] * np.maximum(dots, 0)).sum(0)
         np.testing.assert_allclose(with_q[i, : t + 1], ref_q, rtol=1e-12)
+
+
+# --------------------------------------------------------------------------- FP8 latent cache
+def _pack_fp8_rows(codes_u8, rope_bf16, sigma_f32, row_bytes):
+    """Byte rows [codes | RoPE bf16 | float32 scale | zero padding] from torch tensors
+    ([..., d_lat] uint8, [..., d_rope] bf16, [...] float32)."""
+    d_lat, d_rope = codes_u8.shape[-1], rope_bf16.shape[-1]
+    rows = torch.zeros(codes_u8.shape[:-1] + (row_bytes,), dtype=torch.uint8)
+    rows[..., :d_lat] = codes_u8
+    rows[..., d_lat: d_lat + 2 * d_rope] = rope_bf16.contiguous().view(torch.uint8)
+    rows[..., d_lat + 2 * d_rope: d_lat + 2 * d_rope + 4] = sigma_f32.contiguous().unsqueeze(-1).view(torch.uint8)
+    return rows
+
+
+def _fp8_cache(seed, n_seq, L, d_lat, d_rope, pow2_scales=False):
+    """A random packed cache plus its exact values: (rows uint8, c float64, r float64)."""
+    g = torch.Generator().manual_seed(seed)
+    code = (torch.randn((n_seq, L, d_lat), generator=g) * 64).clamp(-448, 448).to(torch.float8_e4m3fn)
+    rope = torch.randn((n_seq, L, d_rope), generator=g).to(torch.bfloat16)
+    if pow2_scales:
+        sigma = torch.pow(2.0, torch.randint(-7, -4, (n_seq, L), generator=g).float())
+    else:
+        sigma = torch.rand((n_seq, L), generator=g) * 0.05 + 0.003
+    rows = _pack_fp8_rows(code.view(torch.uint8), rope, sigma, wl.fp8_row_bytes(d_lat, d_rope))
+    # exact values through torch's own float8 / bf16 decoding
+    c = code.to(torch.float64) * sigma.to(torch.float64)[..., None]
+    r = rope.to(torch.float64)
+    return rows.numpy(), c.numpy(), r.numpy()
+
+
+def test_fp8_latent_single_row_is_the_scaled_row():
+    """One selected row: the softmax weight is 1, so the output is that row's latent
+    sigma * e4m3(code) exactly, and lse is the row's scaled logit (which also reads
+    the RoPE bytes)."""
+    d_lat, d_rope, H = 512, 64, 4
+    rows, c, r = _fp8_cache(11, 1, 40, d_lat, d_rope)
+    rng = np.random.default_rng(12)
+    q = rng.standard_normal((1, H, d_lat + d_rope)).astype(np.float32)
+    out, lse = oracle.sparse_mla_fp8(q, rows, [0], np.array([[29]], np.int32), [1], d_lat, d_rope, 0.0625)
+    np.testing.assert_array_equal(out[0], np.broadcast_to(c[0, 29], (H, d_lat)))
+    row = np.concatenate([c[0, 29], r[0, 29]])
+    np.testing.assert_allclose(lse[0], 0.0625 * (q[0].astype(np.float64) @ row), rtol=1e-13, atol=1e-13)
+
+
+def test_fp8_latent_equals_sdpa_on_the_exact_cache():
+    """Random selections on small dims against torch SDPA (float64) over the exact
+    values; with topk covering every visible row, against dense causal SDPA."""
+    d_lat, d_rope, H, L, n_seq, n_q = 12, 4, 3, 23, 2, 4
+    rows, c, r = _fp8_cache(13, n_seq, L, d_lat, d_rope)
+    kv = np.concatenate([c, r], axis=-1)
+    rng = np.random.default_rng(14)
+    q = rng.standard_normal((n_q, H, d_lat + d_rope)).astype(np.float32)
+    q_seq = np.array([0, 1, 1, 0], np.int32)
+    q_pos = np.array([4, 22, 9, 17], np.int32)
+    topk = 8
+    idx = np.full((n_q, topk), -1, np.int32)
+    cnt = np.zeros(n_q, np.int32)
+    for i in range(n_q):
+        sel = np.sort(rng.choice(q_pos[i] + 1, size=min(topk, q_pos[i] + 1), replace=False))
+        idx[i, : len(sel)] = sel
+        cnt[i] = len(sel)
+    scale = 1 / math.sqrt(11.0)
+    out, _ = oracle.sparse_mla_fp8(q, rows, q_seq, idx, cnt, d_lat, d_rope, scale)
+    full = np.full((n_q, L), -1, np.int32)
+    for i in range(n_q):
+        full[i, : q_pos[i] + 1] = np.arange(q_pos[i] + 1)
+    out_all, _ = oracle.sparse_mla_fp8(q, rows, q_seq, full, q_pos + 1, d_lat, d_rope, scale)
+    for i in range(n_q):
+        for sel, o in ((idx[i, : cnt[i]], out[i]), (np.arange(q_pos[i] + 1), out_all[i])):
+            mask = np.zeros(L, dtype=bool)
+            mask[sel] = True
+            ref = _sdpa(q[i][None], kv[q_seq[i]][None, None], c[q_seq[i]][None, None],
+                        np.broadcast_to(mask, (1, 1, H, L)).copy(), scale)
+            np.testing.assert_allclose(o, ref.reshape(H, d_lat), atol=1e-12)
+
+
+def test_fp8_latent_with_power_of_two_scales_equals_the_float_oracle():
+    """With power-of-two scales every latent value is exact in float32, so the FP8
+    form must agree with sparse_mla on the float cache (same arithmetic order:
+    bit for bit), at the GLM-5.2 sizes."""
+    d_lat, d_rope, H, L = 512, 64, 8, 300
+    rows, c, r = _fp8_cache(15, 2, L, d_lat, d_rope, pow2_scales=True)
+    kv = np.concatenate([c, r], axis=-1).astype(np.float32)
+    assert np.array_equal(kv.astype(np.float64), np.concatenate([c, r], axis=-1))
+    rng = np.random.default_rng(16)
+    q = rng.standard_normal((3, H, d_lat + d_rope)).astype(np.float32)
+    q_seq = np.array([1, 0, 1], np.int32)
+    idx = np.full((3, 64), -1, np.int32)
+    cnt = np.array([64, 17, 1], np.int32)
+    for i in range(3):
+        idx[i, : cnt[i]] = np.sort(rng.choice(L, size=cnt[i], replace=False))
+    a, la = oracle.sparse_mla_fp8(q, rows, q_seq, idx, cnt, d_lat, d_rope, 0.0625)
+    b, lb = oracle.sparse_mla(q, kv, q_seq, idx, cnt, d_lat, 0.0625)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(la, lb)
+
+
+def test_fp8_latent_padding_bytes_are_ignored():
+    d_lat, d_rope = 512, 64
+    rows, _, _ = _fp8_cache(17, 1, 50, d_lat, d_rope)
+    noisy = rows.copy()
+    noisy[..., d_lat + 2 * d_rope + 4:] = np.random.default_rng(18).integers(0, 256, size=noisy[..., 644:].shape)
+    rng = np.random.default_rng(19)
+    q = rng.standard_normal((2, 4, d_lat + d_rope)).astype(np.float32)
+    idx = np.array([[0, 7, 33, 49], [2, 3, -1, -1]], np.int32)
+    a, la = oracle.sparse_mla_fp8(q, rows, [0, 0], idx, [4, 2], d_lat, d_rope, 0.0625)
+    b, lb = oracle.sparse_mla_fp8(q, noisy, [0, 0], idx, [4, 2], d_lat, d_rope, 0.0625)
+    np.testing.assert_array_equal(a, b)
+    np.testing.assert_array_equal(la, lb)
+
+
+def test_fp8_latent_generator_layout():
+    """fp8_latent_inputs packs the layer's bf16 RoPE key, finite codes and scales in
+    the ranges stated, and zero padding."""
+    w = wl.scaled(wl.NAMED["decode_32k"], n_seq=2, L=64, q_pos=(63, 10), q_seq=(0, 1))
+    x = wl.make_inputs(w)
+    rows = wl.fp8_latent_inputs(w, x)[0]
+    assert rows.shape == (2, 64, 656) and rows.dtype == torch.uint8
+    assert torch.equal(rows[..., 512:640].contiguous().view(torch.bfloat16), x["kv"][0][..., 512:])
+    sigma = rows[..., 640:644].contiguous().view(torch.float32)
+    assert float(sigma.min()) >= 1 / 128 and float(sigma.max()) < 1 / 32
+    codes = rows[..., :512].contiguous().view(torch.float8_e4m3fn).float()
+    assert not torch.isnan(codes).any() and float(codes.abs().max()) <= 448
+    assert int(rows[..., 644:].sum()) == 0
