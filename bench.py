@@ -57,10 +57,11 @@ def measured_peaks():
 
 
 # ------------------------------------------------------------------ algorithmic bytes
-def path_bytes(w: wl.Workload, seq_run: int, indexer_fp8: bool = False):
+def path_bytes(w: wl.Workload, seq_run: int, indexer_fp8: bool = False, mla_fp8: bool = False):
     """Algorithmic HBM bytes of one step (each input byte once, outputs once).
     indexer_fp8: E4M3 indexer keys and queries (1 byte per value) plus a float32
-    scale per key and per (query, head)."""
+    scale per key and per (query, head).  mla_fp8: each selected cache row is one
+    packed 656-byte FP8 row (codes, bf16 RoPE key, scale, padding)."""
     vis = np.array(w.q_pos, dtype=np.int64) + 1
     seqs = {}
     for s, t in zip(w.q_seq, w.q_pos):
@@ -73,7 +74,8 @@ def path_bytes(w: wl.Workload, seq_run: int, indexer_fp8: bool = False):
     idx_in = key_rows * key_b + w.n_q * w.idx_heads * qry_b
     idx_out = int(vis.sum()) * 4
     cnt = np.minimum(vis, w.topk)
-    rows = int(cnt.sum()) * (w.d_lat + w.d_rope) * eb
+    row_b = wl.fp8_row_bytes(w.d_lat, w.d_rope) if mla_fp8 else (w.d_lat + w.d_rope) * eb
+    rows = int(cnt.sum()) * row_b
     q_out = w.n_q * w.mla_heads * ((w.d_lat + w.d_rope) * eb + w.d_lat * eb + 4)
     return {
         "indexer": idx_in + idx_out,
@@ -150,7 +152,8 @@ class ClockSampler:
 class Step:
     """Device buffers, descriptors and the captured CUDA graph of one step."""
 
-    def __init__(self, w: wl.Workload, dev, seed_offset: int = 0, indexer_fp8: bool = False):
+    def __init__(self, w: wl.Workload, dev, seed_offset: int = 0, indexer_fp8: bool = False,
+                 mla_fp8: bool = False):
         self.w = w
         self.dev = dev
         w = wl.scaled(w, seed=w.seed + seed_offset) if seed_offset else w
@@ -170,11 +173,16 @@ class Step:
         else:
             self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"],
                                 flags=B.DSA_INDEXER_TOPK_HIST)
+        self.kv8 = None
+        if mla_fp8:  # the FP8 variant of the latent cache: packed E4M3 rows with a per-row scale
+            self.kv8 = wl.fp8_latent_inputs(w, x, device=dev)
+            x["kv"] = None  # the bf16 caches are not read
         self.mlas = []
         for layer in range(w.n_layers):
             out = torch.empty((w.n_q, w.mla_heads, w.d_lat), dtype=w.torch_dtype, device=dev)
             lse = torch.empty((w.n_q, w.mla_heads), dtype=torch.float32, device=dev)
-            kv = x["kv"][layer][0] if w.shared_cache else x["kv"][layer]
+            caches = self.kv8 if mla_fp8 else x["kv"]
+            kv = caches[layer][0] if w.shared_cache else caches[layer]
             self.mlas.append(B.Mla(x["q_mla"][layer], kv, out, w.d_lat, w.scale, lse))
         self.ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, self.q, w.topk, w.n_layers, dev)
         self.scores = B.scores_buffer(w.n_q, w.L, dev)
@@ -446,6 +454,9 @@ def main():
     ap.add_argument("--indexer-fp8", action="store_true",
                     help="the FP8 variant: E4M3 indexer queries/keys with per-row scales (a separate line, "
                          "not the bf16 headline)")
+    ap.add_argument("--mla-fp8", action="store_true",
+                    help="the FP8 latent cache: packed E4M3 rows with a per-row scale, bf16 RoPE key "
+                         "(a separate line, not the bf16 headline)")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="decode workloads: override the batch (a smaller case for profiling; not a bench line)")
     ap.add_argument("--n-q", type=int, default=0,
@@ -468,7 +479,7 @@ def main():
     torch.cuda.set_device(dev)
     B.lib()
 
-    step = Step(w, dev, seed_offset=rank, indexer_fp8=args.indexer_fp8)
+    step = Step(w, dev, seed_offset=rank, indexer_fp8=args.indexer_fp8, mla_fp8=args.mla_fp8)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     step.capture()
     for _ in range(args.warmup):
@@ -512,8 +523,17 @@ def main():
     ms_per_step = tot_max / args.steps
     value = weak_scaling_value(world, w.n_q, w.n_layers, args.steps, tot_max)
     hbm_peak, tc_peak, peak_kind = measured_peaks()
-    fp8 = args.indexer_fp8
-    by = path_bytes(w, step.seq_run, indexer_fp8=fp8)
+    fp8, mla_fp8 = args.indexer_fp8, args.mla_fp8
+    by = path_bytes(w, step.seq_run, indexer_fp8=fp8, mla_fp8=mla_fp8)
+    dtype = w.dtype
+    if fp8 or mla_fp8:
+        dtype = ", ".join(p for p in ("e4m3 indexer" if fp8 else "",
+                                      "e4m3 latent cache" if mla_fp8 else "", w.dtype + " MLA") if p)
+    variant = {}
+    if fp8:
+        variant["indexer_dtype"] = "e4m3 + per-row fp32 scales (FP8 variant)"
+    if mla_fp8:
+        variant["latent_cache"] = "e4m3 + per-row fp32 scale, bf16 RoPE key, 656-byte rows (FP8 variant)"
     idx_ms = idx_t / n_bd
     idx_gbs = by["indexer"] / (idx_ms * 1e-3) / 1e9
     t_roof_us = by["path"] / (hbm_peak * 1e9) * 1e6
@@ -521,8 +541,8 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": ("e4m3 indexer, " + w.dtype + " MLA") if fp8 else w.dtype, "data": "synthetic",
-        "config": {**w.describe(), **({"indexer_dtype": "e4m3 + per-row fp32 scales (FP8 variant)"} if fp8 else {}),
+        "vs_baseline": None, "dtype": dtype, "data": "synthetic",
+        "config": {**w.describe(), **variant,
                    "parallelism": f"dp{world} (independent batches per GPU)",
                    "l2": "flushed before every timed step (256 MB write)", "graph": "CUDA graph per step"},
         "roofline": {"bound": "hbm", "kernel": "idx_score_tc (dsa_index_scores)", "achieved": idx_gbs,
@@ -557,7 +577,7 @@ def main():
                        "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "steps": n_e2e}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = None if fp8 else cpu_baseline(w, step.x)
+        line["cpu_baseline"] = None if (fp8 or mla_fp8) else cpu_baseline(w, step.x)
 
     if rank == 0:
         print(json.dumps(line), flush=True)

@@ -23,6 +23,7 @@ DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, D
 DSA_BF16, DSA_F32, DSA_FP8_E4M3 = 0, 1, 2
 DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_MLA_DECODE, DSA_OP_MLA_PREFILL, DSA_OP_INDEXSHARE_GROUP = range(5)
 DSA_INDEXER_TOPK_HIST = 1
+DSA_MLA_FP8_ROW_BYTES = 656
 DSA_TOPK_HIST_FROM_INDEXER = 1
 
 
@@ -46,7 +47,7 @@ class _Indexer(ctypes.Structure):
 
 class _Mla(ctypes.Structure):
     _fields_ = [("heads", ctypes.c_int32), ("d_latent", ctypes.c_int32), ("d_rope", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("scale", ctypes.c_float), ("reserved", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("scale", ctypes.c_float), ("kv_dtype", ctypes.c_int32),
                 ("q", ctypes.c_void_p), ("kv", ctypes.c_void_p), ("kv_seq_stride", ctypes.c_int64),
                 ("kv_row_stride", ctypes.c_int64), ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p)]
 
@@ -151,7 +152,8 @@ class Indexer:
 @dataclass
 class Mla:
     q: torch.Tensor              # [n_q, heads, d_latent + d_rope]
-    kv: torch.Tensor             # [n_seq, L, d_latent + d_rope] or [L, ...] (shared)
+    kv: torch.Tensor             # [n_seq, L, d_latent + d_rope] or [L, ...] (shared), q's dtype;
+                                 # or uint8 [n_seq, L, >= DSA_MLA_FP8_ROW_BYTES]: packed FP8 rows
     out: torch.Tensor            # [n_q, heads, d_latent]
     d_latent: int
     scale: float
@@ -161,7 +163,8 @@ class Mla:
         shared = self.kv.dim() == 2
         seq_stride = 0 if shared else self.kv.stride(0)
         heads, dk = self.q.shape[1], self.q.shape[2]
-        return _Mla(heads, self.d_latent, dk - self.d_latent, _dtype_code(self.q), float(self.scale), 0,
+        kv_dtype = DSA_FP8_E4M3 if self.kv.dtype == torch.uint8 else 0
+        return _Mla(heads, self.d_latent, dk - self.d_latent, _dtype_code(self.q), float(self.scale), kv_dtype,
                     self.q.data_ptr(), self.kv.data_ptr(), seq_stride, self.kv.stride(-2),
                     self.out.data_ptr(), self.lse.data_ptr() if self.lse is not None else None)
 

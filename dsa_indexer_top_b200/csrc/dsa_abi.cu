@@ -72,18 +72,30 @@ bool indexer_tc_ok(const dsa_indexer *ix) {
            ix->k_row_stride >= kIdxDim;
 }
 
+bool mla_kv_fp8(const dsa_mla *m) { return m->kv_dtype == DSA_FP8_E4M3; }
+
 bool mla_tc_ok(const dsa_mla *m) {
-    return m->dtype == DSA_BF16 && m->heads == kMlaHeads && m->d_latent == kLatent && m->d_rope == kRope &&
-           aligned16(m->q) && aligned16(m->kv) && aligned16(m->out) && m->kv_row_stride % 8 == 0 &&
-           m->kv_seq_stride % 8 == 0 && m->kv_row_stride >= kRow;
+    const bool shape = m->dtype == DSA_BF16 && m->heads == kMlaHeads && m->d_latent == kLatent &&
+                       m->d_rope == kRope && aligned16(m->q) && aligned16(m->kv) && aligned16(m->out);
+    if (mla_kv_fp8(m))  // packed rows, strides in bytes
+        return shape && m->kv_row_stride % 16 == 0 && m->kv_seq_stride % 16 == 0 && m->kv_row_stride >= kFp8Row;
+    return shape && m->kv_row_stride % 8 == 0 && m->kv_seq_stride % 8 == 0 && m->kv_row_stride >= kRow;
 }
 
 size_t ws_index_scores() { return kStatusBytes; }
 size_t ws_topk(int n_q, int max_ctx) { return kStatusBytes + align256(topk_scratch_bytes(n_q, max_ctx)); }
 int decode_splits(int topk) { return mla_max_splits(topk); }
-size_t ws_mla_decode(int n_q, int topk, int n_layers) {
+// The histograms and tickets that dsa_index_scores / dsa_topk keep zero between
+// calls head the scratch; the decode attention's partials start after them, so
+// the separate calls of a step can share one workspace.
+size_t ws_zeroed_head(int n_q) { return align256(topk_zeroed_bytes(n_q)); }
+size_t ws_mla_partials(int n_q, int topk, int n_layers) {
     const int ns = decode_splits(topk);
-    return kStatusBytes + (ns > 1 ? align256(mla_partial_bytes(n_layers, n_q, ns)) : 0);
+    return ns > 1 ? align256(mla_partial_bytes(n_layers, n_q, ns)) : 0;
+}
+size_t ws_mla_decode(int n_q, int topk, int n_layers) {
+    const size_t part = ws_mla_partials(n_q, topk, n_layers);
+    return kStatusBytes + (part ? ws_zeroed_head(n_q) + part : 0);
 }
 size_t ws_scores(int n_q, int max_ctx) {
     return align256(static_cast<size_t>(n_q) * round4(max_ctx) * sizeof(float));
@@ -91,7 +103,7 @@ size_t ws_scores(int n_q, int max_ctx) {
 bool group_uses_decode(int n_q) { return n_q <= kDecodeMaxQueries; }
 size_t ws_group(int n_q, int max_ctx, int topk, int n_layers) {
     size_t b = kStatusBytes + ws_scores(n_q, max_ctx) + align256(topk_scratch_bytes(n_q, max_ctx));
-    if (group_uses_decode(n_q)) b += ws_mla_decode(n_q, topk, n_layers) - kStatusBytes;
+    if (group_uses_decode(n_q)) b += ws_mla_partials(n_q, topk, n_layers);  // after the whole top-k scratch
     return b;
 }
 
@@ -256,9 +268,14 @@ dsa_status check_mla_layers(const dsa_mla *layers, int n_layers) {
         if (!m.q || !m.kv || !m.out) return DSA_ERR_INVALID;
         if (m.heads < 1 || m.d_latent < 1 || m.d_rope < 0 || (m.dtype != DSA_BF16 && m.dtype != DSA_F32))
             return DSA_ERR_INVALID;
-        if (m.kv_row_stride < m.d_latent + m.d_rope || m.kv_seq_stride < 0) return DSA_ERR_INVALID;
+        if (m.kv_dtype != 0 && m.kv_dtype != m.dtype && m.kv_dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID;
+        // a packed FP8 row holds d_latent codes, d_rope bf16 values and a float32 scale
+        const int64_t min_row = mla_kv_fp8(&m) ? int64_t(m.d_latent) + 2 * int64_t(m.d_rope) + 4
+                                               : int64_t(m.d_latent) + m.d_rope;
+        if (m.kv_row_stride < min_row || m.kv_seq_stride < 0) return DSA_ERR_INVALID;
         if (m.heads != m0.heads || m.d_latent != m0.d_latent || m.d_rope != m0.d_rope || m.dtype != m0.dtype ||
-            m.scale != m0.scale || m.kv_row_stride != m0.kv_row_stride || m.kv_seq_stride != m0.kv_seq_stride)
+            m.scale != m0.scale || m.kv_row_stride != m0.kv_row_stride || m.kv_seq_stride != m0.kv_seq_stride ||
+            mla_kv_fp8(&m) != mla_kv_fp8(&m0))
             return DSA_ERR_INVALID;
     }
     return DSA_OK;
@@ -291,9 +308,11 @@ dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, co
     a.d_rope = m.d_rope;
     a.scale = m.scale;
     a.is_bf16 = m.dtype == DSA_BF16;
+    a.kv_fp8 = mla_kv_fp8(&m) ? 1 : 0;
     a.status = status;
     bool tc = true;
     for (int l = 0; l < n_layers; ++l) tc = tc && mla_tc_ok(&layers[l]);
+    if (a.kv_fp8 && !tc) return DSA_ERR_UNSUPPORTED;  // packed FP8 caches: tensor-core path only
     if (tc) {
         int n_splits, cpc;
         mla_plan(qs->n_q, n_layers, topk, decode, num_sms_current(), kMlaMaxSplits, n_splits, cpc);
@@ -419,8 +438,10 @@ static dsa_status mla_entry(const dsa_queries *queries, const dsa_mla *mla, cons
     const size_t need = decode ? ws_mla_decode(queries->n_q, topk, 1) : kStatusBytes;
     if (!ws_ok(ws, ws_bytes, need)) return DSA_ERR_WORKSPACE;
     if (queries->n_q == 0) return DSA_OK;
-    return do_mla(queries, mla, 1, idx, cnt, topk, decode, static_cast<uint8_t *>(ws) + kStatusBytes,
-                  status_word(ws), static_cast<cudaStream_t>(stream));
+    // partials after the region the indexer / top-k keep zero (see ws_zeroed_head)
+    uint8_t *scratch = static_cast<uint8_t *>(ws) + kStatusBytes + ws_zeroed_head(queries->n_q);
+    return do_mla(queries, mla, 1, idx, cnt, topk, decode, scratch, status_word(ws),
+                  static_cast<cudaStream_t>(stream));
 }
 
 dsa_status dsa_sparse_mla_decode(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,

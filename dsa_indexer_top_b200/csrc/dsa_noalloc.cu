@@ -57,12 +57,15 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
     if (queries->n_q > 0 && (!queries->q_seq || !queries->q_pos)) return DSA_ERR_INVALID;
     if (topk < 1 || topk > kMaxTopk || !idx || !cnt || !mla) return DSA_ERR_INVALID;
     const dsa_mla &m = *mla;
-    if (!m.q || !m.kv || !m.out || m.kv_seq_stride < 0 || m.kv_row_stride < m.d_latent + m.d_rope)
-        return DSA_ERR_INVALID;
-    // Only the tensor-core shape uses scratch: bf16, 64 heads, 512 + 64.
+    if (m.kv_dtype != 0 && m.kv_dtype != m.dtype && m.kv_dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID;
+    const bool fp8 = m.kv_dtype == DSA_FP8_E4M3;  // packed rows, strides in bytes
+    const int64_t min_row = fp8 ? int64_t(m.d_latent) + 2 * int64_t(m.d_rope) + 4 : int64_t(m.d_latent) + m.d_rope;
+    if (!m.q || !m.kv || !m.out || m.kv_seq_stride < 0 || m.kv_row_stride < min_row) return DSA_ERR_INVALID;
+    // Only the tensor-core shape uses scratch: bf16 queries, 64 heads, 512 + 64.
+    const int64_t al = fp8 ? 16 : 8;
     if (m.dtype != DSA_BF16 || m.heads != kMlaHeads || m.d_latent != kLatent || m.d_rope != kRope ||
-        !aligned16(m.q) || !aligned16(m.kv) || !aligned16(m.out) || m.kv_row_stride % 8 != 0 ||
-        m.kv_seq_stride % 8 != 0)
+        !aligned16(m.q) || !aligned16(m.kv) || !aligned16(m.out) || m.kv_row_stride % al != 0 ||
+        m.kv_seq_stride % al != 0 || (fp8 && m.kv_row_stride < kFp8Row))
         return DSA_ERR_UNSUPPORTED;
     const int n_splits = (topk + kRowsPerChunk - 1) / kRowsPerChunk;
     const size_t need = kStatusBytes + (n_splits > 1 ? mla_partial_bytes(1, queries->n_q, n_splits) : 0);
@@ -95,6 +98,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
     a.d_rope = m.d_rope;
     a.scale = m.scale;
     a.is_bf16 = 1;
+    a.kv_fp8 = fp8 ? 1 : 0;
     a.status = reinterpret_cast<uint32_t *>(scratch);
     int dev = 0, sms = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||

@@ -35,6 +35,11 @@ constexpr int kMlaHeads = 64;   // num_attention_heads of GLM-5.2
 constexpr int kLatent = 512;    // kv_lora_rank
 constexpr int kRope = 64;       // qk_rope_head_dim
 constexpr int kRow = kLatent + kRope;
+// Packed FP8 latent-cache row (bytes): 512 E4M3 codes, the 64 bf16 RoPE values,
+// the float32 row scale, 12 bytes of padding -- 41 aligned 16-byte pieces.
+constexpr int kFp8RopeOff = kLatent;
+constexpr int kFp8ScaleOff = kLatent + 2 * kRope;
+constexpr int kFp8Row = kFp8ScaleOff + 16;
 constexpr int kRowsPerChunk = 128;  // splits <= ceil(topk / 128): every CTA walks >= 2 chunks of 64 rows
 constexpr int kMlaChunk = 64;       // selected rows per tensor-core pipeline chunk
 constexpr int kMaxTopk = 4096;
@@ -142,6 +147,7 @@ struct MlaArgs {
     int heads, d_lat, d_rope;
     float scale;
     int is_bf16;
+    int kv_fp8;          // caches are packed FP8 rows (kFp8Row bytes; strides in bytes)
     uint32_t *status;
     // split-K schedule (tensor-core path)
     int n_splits;        // CTAs per query
@@ -150,8 +156,9 @@ struct MlaArgs {
     float *part_ml;      // [layers][n_q][n_splits][64][2] (max, sum) in log2 units
 };
 
-// Tensor-core sparse MLA (bf16, 64 heads, 512 + 64).  n_splits == 1 writes the
-// final output; otherwise partials followed by launch_mla_combine.
+// Tensor-core sparse MLA (bf16 queries and outputs, 64 heads, 512 + 64; bf16 or
+// packed FP8 caches).  n_splits == 1 writes the final output; otherwise partials
+// followed by launch_mla_combine.
 cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st);
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st);
 cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st);

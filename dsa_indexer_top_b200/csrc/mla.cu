@@ -30,6 +30,8 @@
 //            per query) or fp32 partials + (max, sum) per head for a split-K
 //            merge (decode with few queries).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -55,6 +57,21 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Two E4M3 codes (low byte first) times a row scale, as two bf16 (low half
+// first): the codes widen exactly to half and float, the product is rounded
+// once to float, then to bf16.
+__device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t two, float sigma) {
+    const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
+    const float2 f = __half22float2(__half2(hr));
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sigma, f.y * sigma);
+    return *reinterpret_cast<const uint32_t *>(&b);
+}
+
+// kFp8: the caches are packed FP8 rows [512 E4M3 codes | 64 bf16 RoPE | float32
+// scale | padding]; the producers widen each latent to bf16 (scale applied) into
+// the same shared-memory tiles the bf16 cache fills, so the MMAs and the softmax
+// are the same for both.
+template <bool kFp8>
 __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -109,6 +126,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     const int c_begin = split * a.chunks_per_cta;
     const int nloc = max(0, min(c_begin + a.chunks_per_cta, nch) - c_begin);
     const __nv_bfloat16 *kv = static_cast<const __nv_bfloat16 *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
+    const uint8_t *kv8 = static_cast<const uint8_t *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(lp.q) + static_cast<int64_t>(i) * kMlaHeads * kRow;
     const uint32_t q_addr = smem_u32(q_sm);
 
@@ -141,19 +159,57 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                 }
             }
             const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
-            for (int rr = 0; rr < 16; ++rr) {
-                const int row = 16 * pw + rr;
-                const int src = __shfl_sync(0xffffffffu, r, rr);
+            if constexpr (!kFp8) {
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int row = 16 * pw + rr;
+                    const int src = __shfl_sync(0xffffffffu, r, rr);
 #pragma unroll
-                for (int tt = 0; tt < 3; ++tt) {
-                    const int ch = lane + 32 * tt;
-                    if (ch < kRow / 8) {
-                        const uint32_t dst = sb + (ch >> 3) * kBlockBytes + sw128_offset(row, ch & 7);
-                        if (src >= 0)
-                            cp_async_16(dst, kv + static_cast<int64_t>(src) * a.kv_row_stride + ch * 8);
-                        else
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+                    for (int tt = 0; tt < 3; ++tt) {
+                        const int ch = lane + 32 * tt;
+                        if (ch < kRow / 8) {
+                            const uint32_t dst = sb + (ch >> 3) * kBlockBytes + sw128_offset(row, ch & 7);
+                            if (src >= 0)
+                                cp_async_16(dst, kv + static_cast<int64_t>(src) * a.kv_row_stride + ch * 8);
+                            else
+                                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
+                        }
                     }
+                }
+            } else {
+                // Lane l takes latent dims 16l..16l+15 of each of the warp's 16 rows:
+                // all 16 code loads (and scales) are issued before any is widened;
+                // lanes 0-7 copy the row's RoPE key (bf16) straight into block 8.
+                uint4 code[16];
+                float sig[16];
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int src = __shfl_sync(0xffffffffu, r, rr);
+                    code[rr] = make_uint4(0u, 0u, 0u, 0u);
+                    sig[rr] = 0.f;
+                    const uint32_t rope_dst = sb + 8 * kBlockBytes + sw128_offset(16 * pw + rr, lane & 7);
+                    if (src >= 0) {
+                        const uint8_t *row = kv8 + static_cast<int64_t>(src) * a.kv_row_stride;
+                        code[rr] = __ldg(reinterpret_cast<const uint4 *>(row) + lane);
+                        sig[rr] = __ldg(reinterpret_cast<const float *>(row + kFp8ScaleOff));
+                        if (lane < 8) cp_async_16(rope_dst, row + kFp8RopeOff + 16 * lane);
+                    } else if (lane < 8) {
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(rope_dst), "r"(0u) : "memory");
+                    }
+                }
+                const uint32_t blk = sb + (lane >> 2) * kBlockBytes;  // dims 16l.. lie in block l / 4
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int row = 16 * pw + rr;
+                    const float sg = sig[rr];
+                    const uint32_t w0 = code[rr].x, w1 = code[rr].y, w2 = code[rr].z, w3 = code[rr].w;
+                    const uint32_t lo0 = e4m3x2_scaled_bf16x2(w0 & 0xffffu, sg), lo1 = e4m3x2_scaled_bf16x2(w0 >> 16, sg);
+                    const uint32_t lo2 = e4m3x2_scaled_bf16x2(w1 & 0xffffu, sg), lo3 = e4m3x2_scaled_bf16x2(w1 >> 16, sg);
+                    const uint32_t hi0 = e4m3x2_scaled_bf16x2(w2 & 0xffffu, sg), hi1 = e4m3x2_scaled_bf16x2(w2 >> 16, sg);
+                    const uint32_t hi2 = e4m3x2_scaled_bf16x2(w3 & 0xffffu, sg), hi3 = e4m3x2_scaled_bf16x2(w3 >> 16, sg);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane) & 7)),
+                                 "r"(lo0), "r"(lo1), "r"(lo2), "r"(lo3) : "memory");
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane + 1) & 7)),
+                                 "r"(hi0), "r"(hi1), "r"(hi2), "r"(hi3) : "memory");
                 }
             }
             cp_async_commit();
@@ -536,13 +592,18 @@ __global__ void __launch_bounds__(128) mla_generic_kernel(const MlaArgs a) {
     if (threadIdx.x == 0 && lp.lse) lp.lse[static_cast<int64_t>(i) * a.heads + h] = cnt > 0 ? m + logf(s) : -INFINITY;
 }
 
+template <bool kFp8>
+cudaError_t launch_mla_tc_t(const MlaArgs &a, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(a.n_splits, a.n_q, a.n_layers);
+    return launch_pdl(mla_tc_kernel<kFp8>, grid, dim3(kMlaThreads), kMlaSmem, st, a);
+}
+
 }  // namespace
 
 cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
-    if (e != cudaSuccess) return e;
-    dim3 grid(a.n_splits, a.n_q, a.n_layers);
-    return launch_pdl(mla_tc_kernel, grid, dim3(kMlaThreads), kMlaSmem, st, a);
+    return a.kv_fp8 ? launch_mla_tc_t<true>(a, st) : launch_mla_tc_t<false>(a, st);
 }
 
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st) {

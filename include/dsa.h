@@ -42,6 +42,10 @@
  *    kernels set on device-detected errors (out-of-range positions or indices,
  *    a bounded wait that ran out).  Zero the workspace once with
  *    dsa_workspace_init(); read (and clear) the status with dsa_check_status().
+ *    One workspace of dsa_workspace_bytes(DSA_OP_INDEXSHARE_GROUP, ...) bytes
+ *    serves the separate calls of a step (dsa_index_scores, dsa_topk,
+ *    dsa_sparse_mla_*) on the same queries: every call's scratch leaves alone
+ *    the histograms and tickets that the indexer and top-k keep zero.
  *  - Errors: invalid arguments are rejected synchronously, before any launch,
  *    with DSA_ERR_INVALID (null pointer, bad size, misaligned row, workspace too
  *    small -> DSA_ERR_WORKSPACE); a launch failure returns DSA_ERR_CUDA.  A call
@@ -72,8 +76,9 @@ typedef enum {
     DSA_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (device) */
 } dsa_status;
 
-/* DSA_FP8_E4M3: OCP 8-bit float E4M3 (no infinities), indexer q and k only,
- * with per-row scales (dsa_indexer.q_scale / k_scale). */
+/* DSA_FP8_E4M3: OCP 8-bit float E4M3 (no infinities) with per-row scales: the
+ * indexer's q and k (dsa_indexer.q_scale / k_scale) and the MLA latent cache
+ * (dsa_mla.kv_dtype, packed rows with their scale). */
 typedef enum { DSA_BF16 = 0, DSA_F32 = 1, DSA_FP8_E4M3 = 2 } dsa_dtype;
 
 /* Flags of dsa_indexer.flags and of dsa_topk. */
@@ -169,24 +174,42 @@ typedef struct {
  * Absorbed MLA of one layer [TM, Multi-head latent attention; Partial RoPE].
  *   heads              64 for GLM-5.2
  *   d_latent, d_rope   512 and 64 for GLM-5.2
- *   dtype              DSA_BF16 or DSA_F32 for q, kv and out
+ *   dtype              DSA_BF16 or DSA_F32 for q and out (and kv, see kv_dtype)
  *   scale              softmax scale (1/sqrt(192 + 64) for GLM-5.2)
+ *   kv_dtype           0 or `dtype`: the cache holds `dtype` values (below);
+ *                      DSA_FP8_E4M3: the cache holds packed 8-bit rows, see
+ *                      DSA_MLA_FP8_ROW_BYTES (dtype DSA_BF16, 64 x (512 + 64) only,
+ *                      else DSA_ERR_UNSUPPORTED).  Every layer of a call agrees.
  *   q                  [n_q][heads][d_latent + d_rope], contiguous
  *   kv                 cache row s of sequence b at kv + b*kv_seq_stride +
  *                      s*kv_row_stride, laid out [c (d_latent) | r (d_rope)];
  *                      tensor-core path: strides multiple of 8 elements, 16-byte
- *                      aligned base
+ *                      aligned base.  Packed FP8 rows: strides in bytes, multiples
+ *                      of 16, row stride >= DSA_MLA_FP8_ROW_BYTES
  *   out                [n_q][heads][d_latent], dtype `dtype`
  *   lse                float32 [n_q][heads] (natural log of the softmax
  *                      normaliser of the scaled logits), or NULL
  */
+/*
+ * Packed FP8 latent-cache row (kv_dtype = DSA_FP8_E4M3) [TM, inference
+ * quantization: FP8 inference; LA, key facts: precision fp8 -- the pages give no
+ * format, this one is the library's]:
+ *   bytes [0, 512)     E4M3 codes c8[d] of the latent
+ *   bytes [512, 640)   the RoPE key r, 64 bf16 values
+ *   bytes [640, 644)   float32 row scale sigma (positive, finite)
+ *   bytes [644, 656)   unused
+ * The latent attended over is c[d] = sigma * e4m3(c8[d]); the kernel rounds each
+ * such product to bf16 once before its tensor-core products.
+ */
+#define DSA_MLA_FP8_ROW_BYTES 656
+
 typedef struct {
     int32_t heads;
     int32_t d_latent;
     int32_t d_rope;
     int32_t dtype;
     float scale;
-    int32_t reserved;
+    int32_t kv_dtype; /* 0 = dtype, or DSA_FP8_E4M3 */
     const void *q;
     const void *kv;
     int64_t kv_seq_stride;
@@ -252,8 +275,8 @@ dsa_status dsa_sparse_mla_prefill(const dsa_queries *queries, const dsa_mla *mla
  * they run attention (a runtime or plugin that hands over only its input and
  * output tensors, or memory that was planned and fixed up front), so they have
  * no workspace to pass.  Same arguments and result as dsa_sparse_mla_decode
- * (tensor-core shape only: bf16, 64 heads, 512 + 64; other shapes return
- * DSA_ERR_UNSUPPORTED), minus `ws`.
+ * (tensor-core shape only: bf16 queries and outputs, 64 heads, 512 + 64, a bf16
+ * or packed FP8 cache; other shapes return DSA_ERR_UNSUPPORTED), minus `ws`.
  *  - Scratch: a fixed 32 MiB device array inside the library (status word +
  *    split-K partials), held by every GPU that loads the library until the
  *    process exits.  Calls that need more -- 256 + ceil(topk/128) * n_q *

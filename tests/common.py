@@ -85,6 +85,28 @@ def oracle_mla(w: wl.Workload, xh: dict, layer: int, idx, cnt, rows=None):
                              w.d_lat, w.scale)
 
 
+def with_fp8_caches(w: wl.Workload, mlas, kv8_layers):
+    """The same Mla descriptors reading packed FP8 latent caches (uint8 rows from
+    wl.fp8_latent_inputs) instead of the bf16 ones; outputs reset to NaN."""
+    out = []
+    for m, kv8 in zip(mlas, kv8_layers):
+        m.out.fill_(float("nan"))
+        if m.lse is not None:
+            m.lse.fill_(float("nan"))
+        out.append(B.Mla(m.q, kv8[0] if w.shared_cache else kv8, m.out, m.d_latent, m.scale, m.lse))
+    return out
+
+
+def oracle_mla_fp8(w: wl.Workload, xh: dict, kv8h, layer: int, idx, cnt, rows=None):
+    """Oracle attention of one layer over its packed FP8 cache (host uint8 rows)."""
+    rows = np.arange(w.n_q) if rows is None else np.asarray(rows)
+    q_seq = xh["q_seq"].numpy()[rows]
+    if w.shared_cache:
+        q_seq = np.zeros_like(q_seq)
+    return oracle.sparse_mla_fp8(host_f32(xh["q_mla"][layer])[rows], kv8h[layer].cpu().numpy(), q_seq, idx, cnt,
+                                 w.d_lat, w.d_rope, w.scale)
+
+
 def assert_attention_close(got: torch.Tensor, ref: np.ndarray, dtype: str, what: str = "out"):
     g = got.detach().float().cpu().numpy().astype(np.float64)
     max_abs, mean_abs, _ = TOL[dtype]

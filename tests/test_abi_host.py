@@ -54,8 +54,10 @@ def test_workspace_bytes():
     q2 = _q(n_q=8, L=8192)
     assert lib.dsa_workspace_bytes(B.DSA_OP_TOPK, ctypes.byref(q2), 2048, 64, 512, 1) == 256 + hist
     dec = lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 2048, 64, 512, 1)
-    # up to 32 splits (64-row chunks) x 8 queries x 64 heads x (512 + 2) floats, 256-aligned, + status
-    assert dec == 256 + ((8 * 32 * 64 * 514 * 4 + 255) // 256) * 256
+    # status + the region the indexer / top-k keep zero (left alone, so the calls of
+    # a step can share one workspace) + up to 32 splits (64-row chunks) x 8 queries
+    # x 64 heads x (512 + 2) floats, 256-aligned
+    assert dec == 256 + hist + ((8 * 32 * 64 * 514 * 4 + 255) // 256) * 256
     assert lib.dsa_workspace_bytes(B.DSA_OP_MLA_DECODE, ctypes.byref(q), 64, 64, 512, 1) == 256
     grp = lib.dsa_workspace_bytes(B.DSA_OP_INDEXSHARE_GROUP, ctypes.byref(q), 2048, 64, 512, 4)
     scores = 8 * 32768 * 4
@@ -193,3 +195,55 @@ def test_zero_queries_is_a_noop():
     q = _q(n_q=0)
     assert lib.dsa_index_scores(ctypes.byref(q), ctypes.byref(_idx()), 0x9000, 1000, _FakeWs.ptr, _FakeWs.size,
                                 None) == B.DSA_OK
+
+
+@pytest.mark.parametrize("case,expect", [
+    ("kv_dtype_unknown", "invalid"), ("row_too_short", "invalid"), ("row_not16", "unsupported"),
+    ("row_below_packed", "unsupported"), ("seq_not16", "unsupported"), ("f32_queries", "unsupported"),
+    ("heads32", "unsupported"), ("kv_unaligned", "unsupported"),
+])
+def test_mla_fp8_cache_validation(case, expect):
+    """Packed FP8 latent caches (kv_dtype = DSA_FP8_E4M3): byte strides, multiples
+    of 16, rows of at least 656 bytes, tensor-core shape only; a row shorter than
+    codes + RoPE + scale is invalid for any shape."""
+    lib = B.lib()
+    q = _q()
+    m = _mla(kss=1000 * 656, krs=656)
+    m.kv_dtype = B.DSA_FP8_E4M3
+    if case == "kv_dtype_unknown": m.kv_dtype = 7
+    if case == "row_too_short": m.kv_row_stride = 640
+    if case == "row_not16": m.kv_row_stride = 664
+    if case == "row_below_packed": m.kv_row_stride = 648
+    if case == "seq_not16": m.kv_seq_stride = 1000 * 656 + 8
+    if case == "f32_queries": m.dtype = B.DSA_F32
+    if case == "heads32": m.heads = 32
+    if case == "kv_unaligned": m.kv = 0x7008
+    want = B.DSA_ERR_INVALID if expect == "invalid" else B.DSA_ERR_UNSUPPORTED
+    for fn in (lib.dsa_sparse_mla_prefill, lib.dsa_sparse_mla_decode):
+        assert fn(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, _FakeWs.ptr, _FakeWs.size, None) == want
+    assert lib.dsa_sparse_mla_decode_noalloc(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, None) == want
+
+
+def test_group_rejects_mixed_cache_types():
+    lib = B.lib()
+    q, ix = _q(), _idx()
+    m8 = _mla(kss=1000 * 656, krs=656)
+    m8.kv_dtype = B.DSA_FP8_E4M3
+    m16 = _mla(kss=1000 * 656, krs=656)
+    arr = (B._Mla * 2)(m8, m16)
+    assert lib.dsa_indexshare_group(ctypes.byref(q), ctypes.byref(ix), arr, 2, 2048, 0xA000, 0xB000, _FakeWs.ptr,
+                                    _FakeWs.size, None) == B.DSA_ERR_INVALID
+
+
+def test_mla_kv_dtype_same_as_dtype_is_accepted_by_validation():
+    """kv_dtype equal to dtype means the plain cache: validation passes through to
+    the workspace check (a too-small workspace is then the first error)."""
+    lib = B.lib()
+    q = _q()
+    m = _mla()
+    m.kv_dtype = B.DSA_BF16
+    assert lib.dsa_sparse_mla_prefill(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, _FakeWs.ptr, 128,
+                                      None) == B.DSA_ERR_WORKSPACE
+    m.dtype = m.kv_dtype = B.DSA_F32
+    assert lib.dsa_sparse_mla_prefill(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, _FakeWs.ptr, 128,
+                                      None) == B.DSA_ERR_WORKSPACE

@@ -91,6 +91,37 @@ def test_repeated_steps_one_workspace(dev, name, L_long):
         np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
 
 
+@pytest.mark.parametrize("L_long", [False, True])
+def test_repeated_full_steps_one_workspace(dev, L_long):
+    """The benchmark's step -- fused indexer, top-k, decode attention as three
+    calls on one workspace -- three times in a row: the attention's split-K
+    partials must not land on the histograms and tickets the next step's indexer
+    and top-k expect zero, so every step matches the oracle."""
+    w = SMALL["decode_edges"]
+    if L_long:
+        w = wl.scaled(w, L=20000, q_pos=tuple(min(19999, p + 15000) for p in w.q_pos))
+    xh = wl.make_inputs(w)
+    x = C.to_device(xh)
+    _, ridx, rcnt = C.oracle_selection(w, xh)
+    ref, ref_lse = C.oracle_mla(w, xh, 0, ridx, rcnt)
+    q, ix, mlas = C.descriptors(w, x, seq_run=seq_run_of(w))
+    ix.flags = B.DSA_INDEXER_TOPK_HIST
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, 1, dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    for step in range(3):
+        idx = torch.full((w.n_q, w.topk), -7, dtype=torch.int32, device=dev)
+        cnt = torch.full((w.n_q,), -7, dtype=torch.int32, device=dev)
+        mlas[0].out.fill_(float("nan"))
+        B.dsa_index_scores(q, ix, scores, ws)
+        B.dsa_topk(q, scores, w.topk, idx, cnt, ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+        B.dsa_sparse_mla_decode(q, mlas[0], idx, cnt, w.topk, ws)
+        assert B.dsa_check_status(ws) == B.DSA_OK, f"step {step}"
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt, err_msg=f"step {step}")
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
+        C.assert_attention_close(mlas[0].out, ref, w.dtype, f"step {step}")
+        C.assert_lse_close(mlas[0].lse, ref_lse, w.dtype)
+
+
 def test_bounded_wait_times_out_and_context_stays_usable(dev):
     """A device wait on a barrier that nothing completes gives up after its limit,
     reports DSA_ERR_TIMEOUT through the workspace status word (no hang, no
