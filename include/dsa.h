@@ -45,7 +45,10 @@
  *    One workspace of dsa_workspace_bytes(DSA_OP_INDEXSHARE_GROUP, ...) bytes
  *    serves the separate calls of a step (dsa_index_scores, dsa_topk,
  *    dsa_sparse_mla_*) on the same queries: every call's scratch leaves alone
- *    the histograms and tickets that the indexer and top-k keep zero.
+ *    the histograms and tickets that the indexer and top-k keep zero.  The
+ *    group call lays its scratch out differently (scores first): a workspace
+ *    moved between dsa_indexshare_group and the separate calls must be
+ *    re-initialised with dsa_workspace_init() in between.
  *  - Errors: invalid arguments are rejected synchronously, before any launch,
  *    with DSA_ERR_INVALID (null pointer, bad size, misaligned row, workspace too
  *    small -> DSA_ERR_WORKSPACE); a launch failure returns DSA_ERR_CUDA.  A call
