@@ -1,8 +1,9 @@
 """Property tests on random small shapes (Hypothesis, derandomized so every run
 draws the same cases).
 
-CPU: the oracle's top-k against numpy's stable argsort and its indexer against
-the ReLU identity (a plain matmul), on random shapes and values.
+CPU: the oracle's top-k against numpy's stable argsort, its indexer against
+the ReLU identity (a plain matmul), and its FP8-latent attention against plain
+softmax attention on the exact latents, on random shapes and values.
 GPU: the whole chain (indexer -> top-k -> sparse MLA, decode and prefill
 schedules, with and without the fused histogram) on random contexts, positions,
 batch sizes and top-k sizes; indices bit-exact and outputs within tolerance of
@@ -55,6 +56,42 @@ def test_oracle_indexer_is_relu_of_a_matmul(heads, dim, L, seed):
         ref = (w[i][:, None] * (dots + np.abs(dots)) / 2).sum(0)
         t = q_pos[i]
         np.testing.assert_array_equal(got[i, : t + 1], ref[: t + 1])
+
+
+@CPU_SETTINGS
+@given(heads=st.integers(1, 4), d_lat=st.sampled_from([4, 8, 16, 32]), d_rope=st.integers(0, 8),
+       L=st.integers(1, 30), k=st.integers(1, 12), seed=st.integers(0, 2**31 - 1))
+def test_oracle_fp8_latent_attention_is_softmax_attention(heads, d_lat, d_rope, L, k, seed):
+    """The FP8-cache oracle on random packed rows (any codes but NaN, any positive
+    scale) equals a plain float64 softmax attention over the exact latents, which
+    torch's own float8 / bf16 decoding gives."""
+    g = torch.Generator().manual_seed(seed)
+    codes = torch.randint(0, 256, (1, L, d_lat), generator=g, dtype=torch.int32).to(torch.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0x38                      # no NaN codes (0x38 is 1.0)
+    sigma = torch.exp2(torch.rand((1, L), generator=g) * 12 - 10)
+    rope = torch.randn((1, L, d_rope), generator=g).to(torch.bfloat16)
+    rb = wl.fp8_row_bytes(d_lat, d_rope)
+    rows = torch.zeros((1, L, rb), dtype=torch.uint8)
+    rows[..., :d_lat] = codes
+    rows[..., d_lat: d_lat + 2 * d_rope] = rope.view(torch.uint8)
+    rows[..., d_lat + 2 * d_rope: d_lat + 2 * d_rope + 4] = sigma.contiguous().unsqueeze(-1).view(torch.uint8)
+    c = codes.view(torch.float8_e4m3fn).double() * sigma.double()[..., None]
+    kv = torch.cat([c, rope.double()], -1)[0].numpy()
+    q = torch.randn((1, heads, d_lat + d_rope), generator=g).numpy().astype(np.float32) * 0.05
+    n = L
+    kk = min(k, n)
+    sel = np.sort(np.random.default_rng(seed).choice(n, size=kk, replace=False)).astype(np.int32)
+    idx = np.full((1, k), -1, np.int32)
+    idx[0, :kk] = sel
+    scale = 0.3
+    out, lse = oracle.sparse_mla_fp8(q, rows.numpy(), [0], idx, [kk], d_lat, d_rope, scale)
+    logits = scale * (q[0].astype(np.float64) @ kv[sel].T)               # [heads, kk]
+    m = logits.max(1, keepdims=True)
+    p = np.exp(logits - m)
+    ref = (p / p.sum(1, keepdims=True)) @ kv[sel, :d_lat]
+    scale_out = max(1.0, float(np.abs(kv[sel, :d_lat]).max()))
+    np.testing.assert_allclose(out[0], ref, rtol=0, atol=1e-12 * scale_out)
+    np.testing.assert_allclose(lse[0], m[:, 0] + np.log(p.sum(1)), rtol=0, atol=1e-11 * max(1.0, float(np.abs(m).max())))
 
 
 @pytest.mark.gpu
