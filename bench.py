@@ -2,9 +2,13 @@
 
 One step = one pass of the whole path over one batch of synthetic inputs already
 resident in HBM: dsa_index_scores -> dsa_topk -> sparse MLA for every layer of
-the workload (through the C ABI).  The step is captured once in a CUDA graph with
-CUDA events between the calls, so per-kernel device times come from the same
-timed replays; L2 is flushed (256 MB write) before every timed step.
+the workload (through the C ABI, on one workspace).  The step is captured once in
+a CUDA graph with CUDA events at its two ends only (events between the calls
+would keep each kernel from launching while its predecessor finishes); a second
+graph with events between the calls gives the per-stage breakdown.  L2 is flushed
+(256 MB write) before every timed step.  After timing, the results the graph
+left are compared bitwise with one eager step on a freshly initialised workspace
+(`self_check` in the JSON line).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_32k]
     python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
@@ -332,6 +336,33 @@ class E2EStep:
         torch.cuda.synchronize()
 
 
+def self_check(step: Step) -> str:
+    """The results the timed graph left (indices, counts, every layer's output)
+    against one eager step on a freshly initialised workspace: the path is
+    deterministic (exact histogram counts, a fixed merge order), so they must be
+    bitwise equal.  A step whose calls corrupt each other's scratch across
+    replays fails this.  Reports; never raises."""
+    try:
+        w = step.w
+        idx0, cnt0 = step.idx.clone(), step.cnt.clone()
+        outs0 = [m.out.clone() for m in step.mlas]
+        saved = step.ws
+        step.ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, step.q, w.topk, w.n_layers, step.dev)
+        try:
+            step.run(events=False)
+            torch.cuda.synchronize()
+            st = B.dsa_check_status(step.ws)
+        finally:
+            step.ws = saved
+        if st != B.DSA_OK:
+            return f"fresh step status {B.status_str(st)}"
+        same = torch.equal(idx0, step.idx) and torch.equal(cnt0, step.cnt)
+        same = same and all(torch.equal(o0, m.out) for o0, m in zip(outs0, step.mlas))
+        return "bitwise equal to a fresh-workspace step" if same else "MISMATCH with a fresh-workspace step"
+    except Exception as e:  # the check reports; the measurement stands on its own
+        return f"error: {type(e).__name__}: {e}"
+
+
 # ------------------------------------------------------------------ CPU oracle timing
 def host_copies(w: wl.Workload, dev_x: dict, queries) -> dict:
     """Host copies of what the sampled queries read (their sequences only)."""
@@ -575,6 +606,8 @@ def main():
         te = max_over_ranks(te, world, dev)
         line["e2e"] = {"value": world * w.n_q * w.n_layers * n_e2e / (te * 1e-3), "unit": UNIT,
                        "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "steps": n_e2e}
+
+    line["self_check"] = self_check(step)
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = None if (fp8 or mla_fp8) else cpu_baseline(w, step.x)
