@@ -24,7 +24,6 @@ import json
 import os
 import statistics
 import subprocess
-import sys
 import threading
 import time
 

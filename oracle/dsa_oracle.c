@@ -249,7 +249,6 @@ void oracle_sparse_mla(int n_q, int heads, int d_lat, int d_rope, double scale, 
 #pragma omp parallel for schedule(dynamic, 1)
     for (int64_t e = 0; e < (int64_t)n_q * heads; e++) {
         int i = (int)(e / heads);
-        int h = (int)(e % heads);
         int n_rows = cnt[i];
         const float **rows = (const float **)malloc(sizeof(float *) * (size_t)(n_rows > 0 ? n_rows : 1));
         double *buf = (double *)malloc(sizeof(double) * (size_t)(n_rows > 0 ? n_rows : 1));

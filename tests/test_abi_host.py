@@ -6,7 +6,6 @@ import os
 import re
 
 import pytest
-import torch
 
 from dsa_indexer_top_b200 import binding as B
 
