@@ -90,3 +90,41 @@ def test_fp8_indexer_full_size(cuda_ok, name):
     ridx, rcnt = oracle.topk(sc, [t], w.topk)
     np.testing.assert_array_equal(idx[i].cpu().numpy(), ridx[0])
     assert int(cnt[i]) == int(rcnt[0])
+
+
+@pytest.mark.parametrize("name", ["indexshare_128k", "decode_1m"])
+def test_fp8_latent_cache_full_size(cuda_ok, name):
+    """FP8 latent caches at full size, as the benchmark's --mla-fp8 option runs them
+    (bf16 indexer with the fused histogram, top-k, decode attention on every layer's
+    packed FP8 cache): indices bit-exact and every layer's attention within tolerance
+    of the oracle for sampled queries."""
+    w = wl.NAMED[name]
+    dev = torch.device("cuda")
+    x = wl.make_inputs(w, device=dev)
+    kv8 = wl.fp8_latent_inputs(w, x, device=dev)
+    q, ix, mlas = C.descriptors(w, x, seq_run=1)
+    mlas = C.with_fp8_caches(w, mlas, kv8)
+    ix.flags = B.DSA_INDEXER_TOPK_HIST
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, w.n_layers, dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    idx = torch.empty((w.n_q, w.topk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.n_q,), dtype=torch.int32, device=dev)
+    B.dsa_index_scores(q, ix, scores, ws)
+    B.dsa_topk(q, scores, w.topk, idx, cnt, ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+    for m in mlas:
+        B.dsa_sparse_mla_decode(q, m, idx, cnt, w.topk, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    for i in SAMPLES[name]:
+        b, t = w.q_seq[i], w.q_pos[i]
+        k_h = x["k_idx"][b].cpu().float().numpy()[None]
+        sc = oracle.index_scores(C.host_f32(x["q_idx"][i:i + 1]), C.host_f32(x["w"][i:i + 1]), k_h, [0], [t])
+        ridx, rcnt = oracle.topk(sc, [t], w.topk)
+        np.testing.assert_array_equal(idx[i].cpu().numpy(), ridx[0], err_msg=f"indices of query {i}")
+        sel = torch.from_numpy(ridx[0, : rcnt[0]].astype(np.int64))
+        for layer, m in enumerate(mlas):
+            rows = kv8[layer][b].cpu()[sel].numpy()[None]            # the selected packed rows only
+            out, lse = oracle.sparse_mla_fp8(C.host_f32(x["q_mla"][layer][i:i + 1]), rows, [0],
+                                             np.arange(len(sel), dtype=np.int32)[None], rcnt, w.d_lat, w.d_rope,
+                                             w.scale)
+            C.assert_attention_close(m.out[i:i + 1], out, "bf16", f"query {i} layer {layer}")
+            C.assert_lse_close(m.lse[i:i + 1], lse, "bf16")
