@@ -19,6 +19,10 @@
  *  [AE] "GLM-5.2 -- LLM architectures explained", section "Modelled costs" --
  *       93 KiB of BF16 cache per token pins the per-layer row of 576 bf16 and the
  *       128-bf16 indexer key on full layers.
+ *  [TM] section "inference & serving", inference quantization -- FP8 inference;
+ *  [LA] "GLM-5.2 -- LLM atlas", key facts -- precision fp8.  Neither gives a
+ *       format: the FP8 variants below (E4M3 with per-row scales) are this
+ *       library's reading.
  *
  * Details the pages leave open, fixed here:
  *  - score(t,s) = sum_h w[t,h] * max(0, q_idx[t,h] . k_idx[s]) (post-RoPE
@@ -53,10 +57,12 @@
  *    with DSA_ERR_INVALID (null pointer, bad size, misaligned row, workspace too
  *    small -> DSA_ERR_WORKSPACE); a launch failure returns DSA_ERR_CUDA.  A call
  *    with n_q == 0 does nothing and returns DSA_OK.
- *  - Fast paths: bf16 indexers with 32 heads x 128 dims run on tcgen05 tensor
- *    cores fed by TMA; bf16 MLA with 64 heads x (512 + 64) runs on tcgen05 with
- *    TMEM accumulators.  Other shapes and float32 inputs run generic CUDA-core
- *    kernels.  There is no CPU path.
+ *  - Fast paths: bf16 or FP8 (E4M3) indexers with 32 heads x 128 dims run on
+ *    tcgen05 tensor cores fed by TMA; MLA with bf16 queries, 64 heads x (512 +
+ *    64) and a bf16 or packed FP8 latent cache runs on tcgen05 with TMEM
+ *    accumulators.  Other shapes and float32 inputs run generic CUDA-core
+ *    kernels; the FP8 forms have no generic path (DSA_ERR_UNSUPPORTED).  There
+ *    is no CPU path.
  *  - Thread safety: calls are re-entrant; the only global state is one-time
  *    per-device kernel attribute setup.
  */
