@@ -20,6 +20,9 @@ Functions and the passages they follow (page title, section):
                       here, the pages give none).
   dense_mla        -- textbook causal attention (the topk >= n special case).
   indexshare_group -- "GLM 5.2 -- Hermosa AI", "MLA + DSA with IndexShare".
+  sparse_mla_mtp   -- "GLM-5.2 -- LLM atlas", raw config.json fields
+                      (index_share_for_mtp_iteration): the queries of one MTP
+                      iteration share one selection.
 Every function is pinned by tests in tests/test_oracle_pins.py.
 """
 from __future__ import annotations
@@ -211,3 +214,15 @@ def indexshare_group(q_idx, w, k_idx, q_seq, q_pos, topk_, q_mla_layers, kv_laye
         outs.append(o)
         lses.append(l)
     return idx, cnt, outs, lses
+
+
+def sparse_mla_mtp(q, kv, q_seq, idx_g, cnt_g, draft_tokens, d_lat, scale):
+    """Queries in groups of `draft_tokens` consecutive queries; every query of
+    group g attends over selection row g (idx_g [n_q / D, topk], cnt_g [n_q / D]).
+    Composed from sparse_mla with the group's selection repeated per query
+    ("GLM-5.2 -- LLM atlas", raw config.json fields: index_share_for_mtp_iteration
+    -- the tokens of an MTP iteration share the index selection)."""
+    idx_g, cnt_g = _i32(idx_g), _i32(cnt_g)
+    assert np.asarray(q).shape[0] == idx_g.shape[0] * draft_tokens
+    return sparse_mla(q, kv, q_seq, np.repeat(idx_g, draft_tokens, axis=0), np.repeat(cnt_g, draft_tokens),
+                      d_lat, scale)

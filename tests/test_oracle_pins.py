@@ -552,3 +552,34 @@ def test_fp8_latent_generator_layout():
     err = (codes * sigma - c).abs()
     assert torch.all(err <= torch.maximum(c.abs() * 2.0 ** -4, sigma * 2.0 ** -10) * (1 + 1e-6))
     assert int(rows[..., 644:].sum()) == 0
+
+
+def test_mtp_shared_selection_equals_masked_sdpa_per_query():
+    """sparse_mla_mtp: every query of a group attends over its group's one
+    selection -- checked per query against float64 SDPA with that selection as
+    the mask (no oracle call on the reference side), and with one draft token
+    per group it is sparse_mla itself."""
+    rng = np.random.default_rng(61)
+    D, n_g, H, d_lat, d_rope, L = 3, 2, 3, 10, 4, 23
+    q = rng.standard_normal((n_g * D, H, d_lat + d_rope)).astype(np.float32)
+    kv = rng.standard_normal((n_g, L, d_lat + d_rope)).astype(np.float32)
+    q_seq = np.repeat(np.arange(n_g, dtype=np.int32), D)
+    topk = 6
+    idx_g = np.full((n_g, topk), -1, dtype=np.int32)
+    cnt_g = np.array([6, 4], dtype=np.int32)
+    for g in range(n_g):
+        idx_g[g, : cnt_g[g]] = np.sort(rng.choice(15, size=cnt_g[g], replace=False))
+    out, lse = oracle.sparse_mla_mtp(q, kv, q_seq, idx_g, cnt_g, D, d_lat, 0.3)
+    for i in range(n_g * D):
+        g = i // D
+        mask = np.zeros(L, dtype=bool)
+        mask[idx_g[g, : cnt_g[g]]] = True
+        ref = _sdpa(q[i][None], kv[q_seq[i]][None, None], kv[q_seq[i], :, :d_lat][None, None],
+                    np.broadcast_to(mask, (1, 1, H, L)).copy(), 0.3)
+        np.testing.assert_allclose(out[i], ref.reshape(H, d_lat), atol=1e-12)
+    # queries of one group differ (their own q), so their outputs differ
+    assert not np.allclose(out[0], out[1])
+    o1, l1 = oracle.sparse_mla_mtp(q[:n_g], kv, np.arange(n_g, dtype=np.int32), idx_g, cnt_g, 1, d_lat, 0.3)
+    o2, l2 = oracle.sparse_mla(q[:n_g], kv, np.arange(n_g, dtype=np.int32), idx_g, cnt_g, d_lat, 0.3)
+    np.testing.assert_array_equal(o1, o2)
+    np.testing.assert_array_equal(l1, l2)
