@@ -1,25 +1,38 @@
 """Benchmark of the DSA hot path: query-tokens/s per layer and % of HBM roofline.
 
 One step = one pass of the whole path over one batch of synthetic inputs already
-resident in HBM: dsa_index_scores -> dsa_topk -> sparse MLA for every layer of
-the workload (through the C ABI, on one workspace).  The step is captured once in
-a CUDA graph with CUDA events at its two ends only (events between the calls
-would keep each kernel from launching while its predecessor finishes); a second
-graph with events between the calls gives the per-stage breakdown.  L2 is flushed
-(256 MB write) before every timed step.  After timing, the results the graph
-left are compared bitwise with one eager step on a freshly initialised workspace
-(`self_check` in the JSON line).
+resident in HBM, made by ONE call of the public C ABI: dsa_indexshare_group
+(indexer -> top-k -> sparse MLA of every layer of the workload; with one layer it
+is the plain full-layer step).  The step is captured once in a CUDA graph with
+CUDA events at its two ends; L2 is flushed (256 MB write) before every timed
+step.  A second graph made of the separate calls (dsa_index_scores, dsa_topk,
+dsa_sparse_mla_*) with events between them gives the per-stage breakdown and the
+per-kernel rooflines.  After timing, the results of the timed graph are compared
+bitwise with one eager step on a freshly initialised workspace and with the
+separate calls' results (`self_check`).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_32k]
+The headline line is the 4 x 1,048,576 decode (the configuration the HBM
+roofline target is set on).  The same JSON line carries, under `per_config`,
+the other named workloads (tiny, decode 8 x 32K, prefill 4096 x 64K, IndexShare
+4 x 32 x 128K) and the FP8 variants of the two long-context decodes, each with
+its own value, step time, breakdown, rooflines and self-check.
+
+`e2e` times the same step end to end through the public API with host buffers,
+eagerly, every step: the step's query inputs are copied from pinned host memory,
+dsa_indexshare_group is called (argument checks, tensor-map encoding, launches),
+and the outputs and indices are copied back to pinned host memory.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode_1m]
     python bench.py --impl reference ...   # the fp64 CPU oracle on host cores
 
-With N > 1 (torchrun, one process per GPU) every rank runs its own batch of the
+With N > 1 (torchrun, one process per GPU) every rank runs its own batch of each
 workload (independent sequences, no collective on the data path: weak scaling);
-the time is the max over ranks and `value` counts every rank's queries.
+times are the max over ranks and `value` counts every rank's queries.
 """
 from __future__ import annotations
 
 import argparse
+import gc
 import json
 import os
 import statistics
@@ -36,18 +49,20 @@ from dsa_indexer_top_b200 import workloads as wl
 METRIC = "query-tokens/s per layer (indexer+top-k+sparse MLA); % of HBM roofline"
 UNIT = "qtok/s/layer"
 ROOT = os.path.dirname(os.path.abspath(__file__))
-DECODE_MAX_QUERIES = 256    # the MLA decode (split-K) schedule up to this many queries
+DECODE_MAX_QUERIES = 256    # the group call's MLA uses the decode (split-K) schedule up to this many queries
 L2_FLUSH_BYTES = 256 << 20
 REFERENCE_BUDGET_S = 120.0  # timed oracle work of one --impl reference run
+HEADLINE = "decode_1m"
+# the other workloads reported inside the headline line, with the FP8 variants
+# (indexer keys and latent cache both in E4M3) of the two long-context decodes
+PER_CONFIG = [("decode_32k", False), ("prefill_64k", False), ("indexshare_128k", False), ("tiny", False),
+              ("decode_1m", True), ("indexshare_128k", True)]
+PER_CONFIG_MAX_STEPS = 50
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one indexer launch, from the ncu
-# captures summarised in profiles/idx_score_tc_decode.md: 8 x 32K keys captured at
-# full size (67.61 MB); one sequence of 1M keys (275.13 MB), whose 4-sequence
-# launch streams 4 such caches (traffic x 4).  Absent workloads report null.
-NCU_INDEXER_TRAFFIC = {"decode_32k": 67.61e6, "decode_1m": 4 * 275.13e6}
-# the same for the FP8 variant (profiles/idx_score_tc_fp8_decode.md): 8 x 32K at
-# full size 34.68 MB; one 1M sequence 142.76 MB (x 4 for the 4-sequence launch)
-NCU_INDEXER_TRAFFIC_FP8 = {"decode_32k": 34.68e6, "decode_1m": 4 * 142.76e6}
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of a stage's kernel,
+# from an ncu capture of the current kernels (workload, stage, fp8) -> bytes.
+# Entries are removed when the kernel changes; missing entries report null.
+NCU_TRAFFIC: dict = {}
 
 
 def measured_peaks():
@@ -59,8 +74,8 @@ def measured_peaks():
     return 6650.0, 1590.0, "fallback"
 
 
-# ------------------------------------------------------------------ algorithmic bytes
-def path_bytes(w: wl.Workload, seq_run: int, indexer_fp8: bool = False, mla_fp8: bool = False):
+# ------------------------------------------------------------------ algorithmic bytes / flops
+def path_bytes(w: wl.Workload, indexer_fp8: bool = False, mla_fp8: bool = False):
     """Algorithmic HBM bytes of one step (each input byte once, outputs once).
     indexer_fp8: E4M3 indexer keys and queries (1 byte per value) plus a float32
     scale per key and per (query, head).  mla_fp8: each selected cache row is one
@@ -83,10 +98,20 @@ def path_bytes(w: wl.Workload, seq_run: int, indexer_fp8: bool = False, mla_fp8:
     return {
         "indexer": idx_in + idx_out,
         "topk": idx_out + w.n_q * (w.topk + 1) * 4,
-        "mla_per_layer": rows + q_out,
+        "mla": w.n_layers * (rows + q_out),
         # the path's roofline bytes: indexer keys + gathered rows + q/out
         "path": key_rows * key_b + w.n_layers * (rows + q_out) + w.n_q * w.idx_heads * qry_b,
     }
+
+
+def path_flops(w: wl.Workload):
+    """Tensor-core FLOPs of a step: the indexer's q.k products over every visible
+    key, and the MLA's S (576-deep) and O (512-deep) products over the selection."""
+    vis = np.array(w.q_pos, dtype=np.int64) + 1
+    cnt = np.minimum(vis, w.topk)
+    idx = 2 * w.idx_heads * w.idx_dim * int(vis.sum())
+    mla = 2 * w.mla_heads * (2 * w.d_lat + w.d_rope) * int(cnt.sum()) * w.n_layers
+    return {"indexer": idx, "mla": mla}
 
 
 # ------------------------------------------------------------------ clocks
@@ -98,6 +123,7 @@ class ClockSampler:
     def __init__(self, device_index: int):
         self.samples = []
         self.proc = None
+        self.windows = []
         sel = str(device_index)
         try:
             uuid = str(torch.cuda.get_device_properties(device_index).uuid)
@@ -106,7 +132,6 @@ class ClockSampler:
             pass
         self.cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
                     "-i", sel]
-        self.active = False
 
     def start(self):
         try:
@@ -123,12 +148,8 @@ class ClockSampler:
             if len(parts) == 7:
                 self.samples.append((time.time(), parts))
 
-    def mark(self, on: bool):
-        self.active = on
-        if on:
-            self.t_on = time.time()
-        else:
-            self.t_off = time.time()
+    def window(self, t0, t1):
+        self.windows.append((t0, t1))
 
     def stop(self):
         if self.proc:
@@ -138,11 +159,12 @@ class ClockSampler:
             except Exception:
                 self.proc.kill()
 
-    def summary(self):
+    def summary(self, t0=None, t1=None):
         if not self.samples:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        t0, t1 = getattr(self, "t_on", 0), getattr(self, "t_off", time.time())
-        inside = [p for t, p in self.samples if t0 - 0.06 <= t <= t1 + 0.06] or [p for _, p in self.samples]
+        wins = [(t0, t1)] if t0 is not None else self.windows
+        inside = [p for t, p in self.samples if any(a - 0.06 <= t <= b + 0.06 for a, b in wins)]
+        inside = inside or [p for _, p in self.samples]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[j] for p in inside for j in range(4) if p[3 + j].lower() == "active"})
         sm = [float(p[0]) for p in inside if p[0].replace(".", "").isdigit()]
@@ -151,138 +173,154 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside)}
 
 
+def count_kernel_nodes(fn) -> int | None:
+    """Kernels one call of fn() launches: fn is captured into a throw-away CUDA
+    graph whose kernel nodes are counted (events and memsets are not kernels)."""
+    try:
+        from cuda.bindings import runtime as rt
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+        with torch.cuda.graph(g, capture_error_mode="thread_local"):
+            fn()
+        err, _, n = rt.cudaGraphGetNodes(g.raw_cuda_graph(), 0)
+        err, nodes, n = rt.cudaGraphGetNodes(g.raw_cuda_graph(), n)
+        kinds = [rt.cudaGraphNodeGetType(nd)[1] for nd in nodes]
+        cnt = sum(1 for k in kinds if k == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+        del g
+        return cnt
+    except Exception:
+        return None
+
+
 # ------------------------------------------------------------------ the step
 class Step:
-    """Device buffers, descriptors and the captured CUDA graph of one step."""
+    """Device buffers and descriptors of one workload; the timed step is one
+    dsa_indexshare_group call, the breakdown step the separate calls."""
 
-    def __init__(self, w: wl.Workload, dev, seed_offset: int = 0, indexer_fp8: bool = False,
-                 mla_fp8: bool = False):
+    def __init__(self, w: wl.Workload, dev, seed_offset: int = 0, fp8: bool = False):
         self.w = w
         self.dev = dev
+        self.fp8 = fp8
         w = wl.scaled(w, seed=w.seed + seed_offset) if seed_offset else w
         self.x = wl.make_inputs(w, device=dev)
         self.seq_run = w.n_q if len(set(w.q_seq)) == 1 else 1
         x = self.x
         self.q = B.Queries(x["q_seq"], x["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=self.seq_run)
-        # the indexer leaves the top-k's first-digit histograms in the workspace
         self.f8 = None
-        if indexer_fp8:  # the FP8 variant: E4M3 indexer queries and keys with per-row scales
+        if fp8:  # E4M3 indexer queries and keys with per-row scales
             self.f8 = wl.fp8_indexer_inputs(w, x, device=dev)
             f8 = self.f8
             self.ix = B.Indexer(f8["q8"], x["w"], f8["k8"][0] if w.shared_cache else f8["k8"],
-                                flags=B.DSA_INDEXER_TOPK_HIST, q_scale=f8["q_scale"],
-                                k_scale=f8["k_scale"][0] if w.shared_cache else f8["k_scale"])
+                                q_scale=f8["q_scale"], k_scale=f8["k_scale"][0] if w.shared_cache else f8["k_scale"])
             x["k_idx"] = None  # the bf16 keys are not read
         else:
-            self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"],
-                                flags=B.DSA_INDEXER_TOPK_HIST)
-        self.kv8 = None
-        if mla_fp8:  # the FP8 variant of the latent cache: packed E4M3 rows with a per-row scale
-            self.kv8 = wl.fp8_latent_inputs(w, x, device=dev)
+            self.ix = B.Indexer(x["q_idx"], x["w"], x["k_idx"][0] if w.shared_cache else x["k_idx"])
+        # the separate calls: the indexer leaves the top-k's first-digit histograms
+        self.ix_sep = B.Indexer(self.ix.q, self.ix.w, self.ix.k, flags=B.DSA_INDEXER_TOPK_HIST,
+                                q_scale=self.ix.q_scale, k_scale=self.ix.k_scale)
+        if fp8:  # packed E4M3 latent rows with a per-row scale
+            caches = wl.fp8_latent_inputs(w, x, device=dev)
             x["kv"] = None  # the bf16 caches are not read
-        self.mlas = []
+        else:
+            caches = x["kv"]
+        self.mlas, self.mlas_sep = [], []
         for layer in range(w.n_layers):
-            out = torch.empty((w.n_q, w.mla_heads, w.d_lat), dtype=w.torch_dtype, device=dev)
-            lse = torch.empty((w.n_q, w.mla_heads), dtype=torch.float32, device=dev)
-            caches = self.kv8 if mla_fp8 else x["kv"]
             kv = caches[layer][0] if w.shared_cache else caches[layer]
-            self.mlas.append(B.Mla(x["q_mla"][layer], kv, out, w.d_lat, w.scale, lse))
+            for lst in (self.mlas, self.mlas_sep):
+                out = torch.empty((w.n_q, w.mla_heads, w.d_lat), dtype=w.torch_dtype, device=dev)
+                lse = torch.empty((w.n_q, w.mla_heads), dtype=torch.float32, device=dev)
+                lst.append(B.Mla(x["q_mla"][layer], kv, out, w.d_lat, w.scale, lse))
         self.ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, self.q, w.topk, w.n_layers, dev)
+        self.ws_sep = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, self.q, w.topk, w.n_layers, dev)
         self.scores = B.scores_buffer(w.n_q, w.L, dev)
         self.idx = torch.empty((w.n_q, w.topk), dtype=torch.int32, device=dev)
         self.cnt = torch.empty((w.n_q,), dtype=torch.int32, device=dev)
+        self.idx_sep = torch.empty_like(self.idx)
+        self.cnt_sep = torch.empty_like(self.cnt)
         self.decode = w.n_q <= DECODE_MAX_QUERIES
         self.mla_fn = B.dsa_sparse_mla_decode if self.decode else B.dsa_sparse_mla_prefill
-        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
         self.graph = None      # the timed step: events at its two ends only
-        self.graph_bd = None   # the same step with events between the stages (breakdown)
+        self.graph_bd = None   # the separate calls with events between the stages (breakdown)
 
-    def launches_per_step(self) -> int:
-        w = self.w
-        n_chunks = (w.topk + 127) // 128
-        mla = 2 if (self.decode and n_chunks > 1) else 1
-        return 2 + w.n_layers * mla
-
-    def run(self, events: bool, breakdown: bool = False):
-        # Events between the stages would sit between the kernels in the graph
-        # and stop each kernel from being launched while its predecessor
-        # finishes (programmatic dependent launch), so the timed graph has
-        # events at its two ends only; the breakdown graph adds the inner two.
+    def run(self, events: bool = False):
         if events:
             self.ev[0].record()
-        B.dsa_index_scores(self.q, self.ix, self.scores, self.ws)
-        if breakdown:
+        B.dsa_indexshare_group(self.q, self.ix, self.mlas, self.w.topk, self.idx, self.cnt, self.ws)
+        if events:
             self.ev[1].record()
-        B.dsa_topk(self.q, self.scores, self.w.topk, self.idx, self.cnt, self.ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
-        if breakdown:
+
+    def run_separate(self, events: bool = False):
+        if events:
             self.ev[2].record()
-        for m in self.mlas:
-            self.mla_fn(self.q, m, self.idx, self.cnt, self.w.topk, self.ws)
+        B.dsa_index_scores(self.q, self.ix_sep, self.scores, self.ws_sep)
         if events:
             self.ev[3].record()
+        B.dsa_topk(self.q, self.scores, self.w.topk, self.idx_sep, self.cnt_sep, self.ws_sep,
+                   flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+        if events:
+            self.ev[4].record()
+        for m in self.mlas_sep:
+            self.mla_fn(self.q, m, self.idx_sep, self.cnt_sep, self.w.topk, self.ws_sep)
+        if events:
+            self.ev[5].record()
 
     def capture(self):
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            self.run(events=False)      # one eager pass: one-time kernel attribute setup
+            self.run()              # one eager pass each: one-time kernel attribute setup
+            self.run_separate()
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
+        self.launches = count_kernel_nodes(self.run)
         self.graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
             self.run(events=True)
         torch.cuda.synchronize()
         self.graph_bd = torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.graph_bd, capture_error_mode="thread_local"):
-            self.run(events=True, breakdown=True)
+            self.run_separate(events=True)
         torch.cuda.synchronize()
 
     def step_ms(self):
-        return self.ev[0].elapsed_time(self.ev[3])
+        return self.ev[0].elapsed_time(self.ev[1])
 
     def breakdown_ms(self):
         e = self.ev
-        return (e[0].elapsed_time(e[1]), e[1].elapsed_time(e[2]), e[2].elapsed_time(e[3]))
+        return (e[2].elapsed_time(e[3]), e[3].elapsed_time(e[4]), e[4].elapsed_time(e[5]))
+
+    def release(self):
+        self.graph = None
+        self.graph_bd = None
 
 
 class E2EStep:
-    """The same step through the public API with host buffers: the step's query
-    inputs are copied from pinned host memory, the library calls run, and the
-    outputs (attention output of every layer, the selected indices) are copied
-    back.  Inputs and outputs are packed into 256-byte aligned views of a few
-    device buffers, as a caller batching its per-step host traffic would, and
-    the copies overlap the work that does not need them: the MLA queries (most
-    of the input bytes) travel on a side stream while the indexer runs, and the
-    indices go back while the MLA runs."""
+    """The step end to end through the public API with host buffers, eager: the
+    step's query inputs (indexer queries and weights, positions, every layer's
+    MLA queries) are copied from pinned host memory into one device buffer,
+    dsa_indexshare_group runs on them, and every layer's output plus the
+    selected indices and counts are copied back into pinned host memory.  The
+    caches stay resident (model state)."""
 
     def __init__(self, step: Step):
         self.s = step
         w, x = step.w, step.x
         dev = step.dev
-        ix_in = [("q_idx", step.ix.q), ("w", x["w"]), ("q_seq", x["q_seq"]), ("q_pos", x["q_pos"])]
-        if step.f8 is not None:
-            ix_in.append(("q_scale", step.ix.q_scale))
-        self.d_in_ix, self.h_in_ix, vix = self._pack(ix_in, dev, fill=True)
-        self.d_in_mla, self.h_in_mla, vmla = self._pack(
-            [(f"q_mla{l}", t) for l, t in enumerate(x["q_mla"])], dev, fill=True)
-        self.d_out, self.h_out, vout = self._pack([(f"out{l}", m.out) for l, m in enumerate(step.mlas)], dev,
-                                                  fill=False)
-        self.d_idx, self.h_idx, vidx = self._pack([("idx", step.idx)], dev, fill=False)
-        self.h2d = self.h_in_ix.numel() + self.h_in_mla.numel()
-        self.d2h = self.h_out.numel() + self.h_idx.numel()
-        # descriptors over the packed views (caches, scores, counts and workspace are the step's)
-        self.q = B.Queries(vix["q_seq"], vix["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=step.seq_run)
-        self.ix = B.Indexer(vix["q_idx"], vix["w"], step.ix.k, flags=B.DSA_INDEXER_TOPK_HIST,
-                            q_scale=vix.get("q_scale"), k_scale=step.ix.k_scale)
-        self.mlas = [B.Mla(vmla[f"q_mla{l}"], m.kv, vout[f"out{l}"], m.d_latent, m.scale, m.lse)
+        ins = [("q_idx", step.ix.q), ("w", x["w"]), ("q_seq", x["q_seq"]), ("q_pos", x["q_pos"])]
+        if step.ix.q_scale is not None:
+            ins.append(("q_scale", step.ix.q_scale))
+        ins += [(f"q_mla{l}", t) for l, t in enumerate(x["q_mla"])]
+        self.d_in, self.h_in, vin = self._pack(ins, dev, fill=True)
+        outs = [(f"out{l}", m.out) for l, m in enumerate(step.mlas)] + [("idx", step.idx), ("cnt", step.cnt)]
+        self.d_out, self.h_out, vout = self._pack(outs, dev, fill=False)
+        self.h2d = self.h_in.numel()
+        self.d2h = self.h_out.numel()
+        self.q = B.Queries(vin["q_seq"], vin["q_pos"], n_seq=w.n_seq, max_ctx=w.L, seq_run=step.seq_run)
+        self.ix = B.Indexer(vin["q_idx"], vin["w"], step.ix.k, q_scale=vin.get("q_scale"), k_scale=step.ix.k_scale)
+        self.mlas = [B.Mla(vin[f"q_mla{l}"], m.kv, vout[f"out{l}"], m.d_latent, m.scale, m.lse)
                      for l, m in enumerate(step.mlas)]
-        self.idx = vidx["idx"]
-        self.side = torch.cuda.Stream(device=dev)
-        self.ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)]
-        self.ev_mla_in = torch.cuda.Event()
-        self.ev_topk = torch.cuda.Event()
-        self.ev_idx_out = torch.cuda.Event()
-        self.graph = None
+        self.idx, self.cnt = vout["idx"], vout["cnt"]
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
 
     @staticmethod
     def _pack(items, dev, fill):
@@ -304,43 +342,23 @@ class E2EStep:
 
     def run(self):
         s = self.s
-        main = torch.cuda.current_stream()
         self.ev[0].record()
-        self.side.wait_stream(main)
-        with torch.cuda.stream(self.side):
-            self.d_in_mla.copy_(self.h_in_mla, non_blocking=True)
-            self.ev_mla_in.record()
-        self.d_in_ix.copy_(self.h_in_ix, non_blocking=True)
-        B.dsa_index_scores(self.q, self.ix, s.scores, s.ws)
-        main.wait_event(self.ev_mla_in)
-        B.dsa_topk(self.q, s.scores, s.w.topk, self.idx, s.cnt, s.ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
-        self.ev_topk.record()
-        for m in self.mlas:
-            s.mla_fn(self.q, m, self.idx, s.cnt, s.w.topk, s.ws)
-        with torch.cuda.stream(self.side):
-            self.side.wait_event(self.ev_topk)
-            self.h_idx.copy_(self.d_idx, non_blocking=True)
-            self.ev_idx_out.record()
+        self.d_in.copy_(self.h_in, non_blocking=True)
+        B.dsa_indexshare_group(self.q, self.ix, self.mlas, s.w.topk, self.idx, self.cnt, s.ws)
         self.h_out.copy_(self.d_out, non_blocking=True)
-        main.wait_event(self.ev_idx_out)
         self.ev[1].record()
 
-    def capture(self):
-        torch.cuda.synchronize()
-        self.run()  # one eager pass
-        torch.cuda.synchronize()
-        self.graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(self.graph, capture_error_mode="thread_local"):
-            self.run()
-        torch.cuda.synchronize()
+    def ms(self):
+        return self.ev[0].elapsed_time(self.ev[1])
 
 
 def self_check(step: Step) -> str:
     """The results the timed graph left (indices, counts, every layer's output)
-    against one eager step on a freshly initialised workspace: the path is
-    deterministic (exact histogram counts, a fixed merge order), so they must be
-    bitwise equal.  A step whose calls corrupt each other's scratch across
-    replays fails this.  Reports; never raises."""
+    against one eager group call on a freshly initialised workspace, and against
+    the separate calls' results: the path is deterministic (exact histogram
+    counts, a fixed merge order), so all three must be bitwise equal.  A step
+    whose calls corrupt each other's scratch across replays fails this.
+    Reports; never raises."""
     try:
         w = step.w
         idx0, cnt0 = step.idx.clone(), step.cnt.clone()
@@ -348,7 +366,7 @@ def self_check(step: Step) -> str:
         saved = step.ws
         step.ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, step.q, w.topk, w.n_layers, step.dev)
         try:
-            step.run(events=False)
+            step.run()
             torch.cuda.synchronize()
             st = B.dsa_check_status(step.ws)
         finally:
@@ -357,7 +375,20 @@ def self_check(step: Step) -> str:
             return f"fresh step status {B.status_str(st)}"
         same = torch.equal(idx0, step.idx) and torch.equal(cnt0, step.cnt)
         same = same and all(torch.equal(o0, m.out) for o0, m in zip(outs0, step.mlas))
-        return "bitwise equal to a fresh-workspace step" if same else "MISMATCH with a fresh-workspace step"
+        if not same:
+            return "MISMATCH with a fresh-workspace step"
+        if not (torch.equal(idx0, step.idx_sep) and torch.equal(cnt0, step.cnt_sep)):
+            return "MISMATCH between the group call's and the separate calls' indices"
+        # the group call plans its attention over all layers at once, the separate
+        # calls per layer: with different split counts the partial sums are added
+        # in another order, so outputs agree to rounding, not bit for bit
+        diff = max(float((o0.float() - m.out.float()).abs().max()) for o0, m in zip(outs0, step.mlas_sep))
+        if diff == 0.0:
+            return "bitwise equal to a fresh-workspace step and to the separate calls"
+        if diff <= 2e-2:
+            return (f"bitwise equal to a fresh-workspace step; indices equal to the separate calls', "
+                    f"outputs within {diff:.1e} (different split plans)")
+        return f"MISMATCH between the group call and the separate calls: max-abs {diff:.3e}"
     except Exception as e:  # the check reports; the measurement stands on its own
         return f"error: {type(e).__name__}: {e}"
 
@@ -442,6 +473,132 @@ def barrier(world):
         dist.barrier()
 
 
+def config_of(w: wl.Workload, world: int, fp8: bool = False) -> dict:
+    c = {**w.describe(), "parallelism": f"dp{world} (independent batches per GPU)",
+         "l2": "flushed before every timed step (256 MB write)", "graph": "CUDA graph per step",
+         "entry_point": "dsa_indexshare_group"}
+    if fp8:
+        c["indexer_dtype"] = "e4m3 + per-row fp32 scales (FP8 variant)"
+        c["latent_cache"] = "e4m3 + per-row fp32 scale, bf16 RoPE key, 656-byte rows (FP8 variant)"
+    return c
+
+
+def stage_rooflines(w: wl.Workload, fp8: bool, t_us: dict, hbm_peak: float, tc_peak: float, peak_kind: str):
+    """Per-stage achieved rates against their bound, and the dominant stage."""
+    by = path_bytes(w, indexer_fp8=fp8, mla_fp8=fp8)
+    fl = path_flops(w)
+    prefill = w.n_q > DECODE_MAX_QUERIES
+    st = {}
+    for name, key in (("index_scores", "indexer"), ("topk", "topk"), ("sparse_mla", "mla")):
+        us = t_us[name]
+        gbs = by[key] / (us * 1e-6) / 1e9
+        e = {"kernel": {"index_scores": "idx_score_tc", "topk": "topk", "sparse_mla": "mla_tc (+ mla_combine)"}[name],
+             "us": us, "algorithmic_bytes": by[key], "achieved_gbs": gbs, "hbm_frac": gbs / hbm_peak}
+        if key in fl:
+            tf = fl[key] / (us * 1e-6) / 1e12
+            e["flops"] = fl[key]
+            e["achieved_tflops"] = tf
+            e["tensor_frac"] = tf / tc_peak
+        st[name] = e
+    dom = max(st, key=lambda k: st[k]["us"])
+    d = st[dom]
+    tensor_bound = prefill and dom in ("index_scores", "sparse_mla")
+    if tensor_bound:
+        roof = {"bound": "tensor", "kernel": d["kernel"], "achieved": d["achieved_tflops"], "peak": tc_peak,
+                "unit": "TFLOP/s", "frac": d["tensor_frac"], "peak_kind": f"{peak_kind} bf16_tflops (burst)",
+                "algorithmic_flops": d["flops"]}
+    else:
+        roof = {"bound": "hbm", "kernel": d["kernel"], "achieved": d["achieved_gbs"], "peak": hbm_peak, "unit": "GB/s",
+                "frac": d["hbm_frac"], "peak_kind": f"{peak_kind} hbm_gbs", "algorithmic_bytes": d["algorithmic_bytes"]}
+    roof["avg_launch_us"] = d["us"]
+    roof["stage"] = dom
+    roof["traffic"] = NCU_TRAFFIC.get((w.name, dom, fp8))
+    return roof, st
+
+
+def measure(w: wl.Workload, fp8: bool, args, world: int, rank: int, dev, flush, clocks, steps: int,
+            headline: bool):
+    """Time one workload; returns its result dict (and the step, for e2e / baseline)."""
+    step = Step(w, dev, seed_offset=rank, fp8=fp8)
+    step.capture()
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step.graph.replay()
+    torch.cuda.synchronize()
+    st = B.dsa_check_status(step.ws)
+    if st != B.DSA_OK:
+        raise SystemExit(f"{w.name}: device status {B.status_str(st)}")
+    barrier(world)
+    torch.cuda.synchronize()
+    t_on = time.time()
+    tot = 0.0
+    for _ in range(steps):
+        flush.fill_(1)
+        step.graph.replay()
+        torch.cuda.synchronize()
+        tot += step.step_ms()
+    t_off = time.time()
+    clocks.window(t_on, t_off)
+    barrier(world)
+    tot_max = max_over_ranks(tot, world, dev)
+    # per-stage times (separate calls, events between the stages)
+    idx_t = topk_t = mla_t = 0.0
+    n_bd = max(5, min(steps, 50))
+    for _ in range(n_bd):
+        flush.fill_(1)
+        step.graph_bd.replay()
+        torch.cuda.synchronize()
+        b, c, d = step.breakdown_ms()
+        idx_t += b
+        topk_t += c
+        mla_t += d
+    t_us = {"index_scores": idx_t / n_bd * 1e3, "topk": topk_t / n_bd * 1e3, "sparse_mla": mla_t / n_bd * 1e3}
+    ms_per_step = tot_max / steps
+    hbm_peak, tc_peak, peak_kind = measured_peaks()
+    by = path_bytes(w, indexer_fp8=fp8, mla_fp8=fp8)
+    roof, stages = stage_rooflines(w, fp8, t_us, hbm_peak, tc_peak, peak_kind)
+    t_roof_us = by["path"] / (hbm_peak * 1e9) * 1e6
+    res = {
+        "value": weak_scaling_value(world, w.n_q, w.n_layers, steps, tot_max), "unit": UNIT,
+        "ms_per_step": ms_per_step, "steps": steps,
+        "dtype": ("e4m3 indexer, e4m3 latent cache, " + w.dtype + " MLA") if fp8 else w.dtype,
+        "config": config_of(w, world, fp8),
+        "roofline": roof,
+        "path_roofline": {"bytes": by["path"], "t_roof_us": t_roof_us, "frac": t_roof_us / (ms_per_step * 1e3),
+                          "peak_kind": f"{peak_kind} hbm_gbs"},
+        "breakdown_us": {**t_us, "note": "separate calls in a graph with events between the stages"},
+        "stages": stages,
+        "gpu_launches": None if step.launches is None else step.launches * steps,
+        "launches_per_step": step.launches,
+        "clocks": clocks.summary(t_on, t_off),
+    }
+    res["self_check"] = self_check(step)
+    return res, step
+
+
+def e2e_measure(step: Step, world: int, dev, flush, steps: int):
+    e2e = E2EStep(step)
+    for _ in range(3):
+        e2e.run()
+    torch.cuda.synchronize()
+    barrier(world)
+    te, wall = 0.0, 0.0
+    for _ in range(steps):
+        flush.fill_(1)
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        e2e.run()
+        torch.cuda.synchronize()
+        wall += time.perf_counter() - t0
+        te += e2e.ms()
+    te = max_over_ranks(te, world, dev)
+    w = step.w
+    return {"value": world * w.n_q * w.n_layers * steps / (te * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "steps": steps,
+            "host_wall_ms_per_step": 1e3 * wall / steps,
+            "how": "eager each step: pinned H2D of the query inputs, dsa_indexshare_group, D2H of outputs + indices"}
+
+
 def run_reference(args, w: wl.Workload, world: int, rank: int):
     """The oracle as it stands on host cores: each step one query's full path."""
     if rank != 0:
@@ -463,9 +620,9 @@ def run_reference(args, w: wl.Workload, world: int, rank: int):
             break
     value = done * w.n_layers / t
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": done,
-            "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": 1e3 * t / done, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {**w.describe(), "sample_per_step": "1 query, all layers"},
+            "config": config_of(w, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.max_threads(), "kind": "oracle",
                              "sample": "each step: one query of the workload, full path, all layers"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -475,29 +632,29 @@ def run_reference(args, w: wl.Workload, world: int, rank: int):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="decode_32k", choices=list(wl.NAMED))
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=HEADLINE, choices=list(wl.NAMED))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--fp8", action="store_true",
+                    help="the headline workload with the FP8 variants (E4M3 indexer keys/queries and latent cache)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--indexer-fp8", action="store_true",
-                    help="the FP8 variant: E4M3 indexer queries/keys with per-row scales (a separate line, "
-                         "not the bf16 headline)")
-    ap.add_argument("--mla-fp8", action="store_true",
-                    help="the FP8 latent cache: packed E4M3 rows with a per-row scale, bf16 RoPE key "
-                         "(a separate line, not the bf16 headline)")
+    ap.add_argument("--no-per-config", action="store_true", help="only the headline workload")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="decode workloads: override the batch (a smaller case for profiling; not a bench line)")
     ap.add_argument("--n-q", type=int, default=0,
                     help="prefill: keep the last N queries of the chunk (a smaller case for profiling; not a bench line)")
     args = ap.parse_args()
     w = wl.NAMED[args.workload]
+    small = False
     if args.n_seq and len(set(w.q_seq)) == w.n_q:
         w = wl.scaled(w, n_seq=args.n_seq, q_pos=w.q_pos[:1] * args.n_seq, q_seq=tuple(range(args.n_seq)),
                       name=f"{w.name}_b{args.n_seq}")
+        small = True
     if args.n_q and len(set(w.q_seq)) == 1 and args.n_q < w.n_q:
         w = wl.scaled(w, q_pos=w.q_pos[-args.n_q:], q_seq=w.q_seq[-args.n_q:], name=f"{w.name}_q{args.n_q}")
+        small = True
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
@@ -508,115 +665,49 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     B.lib()
-
-    step = Step(w, dev, seed_offset=rank, indexer_fp8=args.indexer_fp8, mla_fp8=args.mla_fp8)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    step.capture()
-    for _ in range(args.warmup):
-        flush.fill_(1)
-        step.graph.replay()
-    torch.cuda.synchronize()
-    st = B.dsa_check_status(step.ws)
-    if st != B.DSA_OK:
-        raise SystemExit(f"device status {B.status_str(st)}")
-
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    barrier(world)
-    torch.cuda.synchronize()
-    clocks.mark(True)
-    tot = 0.0
-    for _ in range(args.steps):
-        flush.fill_(1)
-        step.graph.replay()
-        torch.cuda.synchronize()
-        tot += step.step_ms()
-    torch.cuda.synchronize()
-    barrier(world)
-    clocks.mark(False)
-    time.sleep(0.1)
-    clocks.stop()
-    tot_max = max_over_ranks(tot, world, dev)
-    # per-stage times (events between the stages: not the timed graph)
-    idx_t = topk_t = mla_t = 0.0
-    n_bd = max(10, min(args.steps, 200))
-    for _ in range(n_bd):
-        flush.fill_(1)
-        step.graph_bd.replay()
-        torch.cuda.synchronize()
-        b, c, d = step.breakdown_ms()
-        idx_t += b
-        topk_t += c
-        mla_t += d
 
-    ms_per_step = tot_max / args.steps
-    value = weak_scaling_value(world, w.n_q, w.n_layers, args.steps, tot_max)
-    hbm_peak, tc_peak, peak_kind = measured_peaks()
-    fp8, mla_fp8 = args.indexer_fp8, args.mla_fp8
-    by = path_bytes(w, step.seq_run, indexer_fp8=fp8, mla_fp8=mla_fp8)
-    dtype = w.dtype
-    if fp8 or mla_fp8:
-        dtype = ", ".join(p for p in ("e4m3 indexer" if fp8 else "",
-                                      "e4m3 latent cache" if mla_fp8 else "", w.dtype + " MLA") if p)
-    variant = {}
-    if fp8:
-        variant["indexer_dtype"] = "e4m3 + per-row fp32 scales (FP8 variant)"
-    if mla_fp8:
-        variant["latent_cache"] = "e4m3 + per-row fp32 scale, bf16 RoPE key, 656-byte rows (FP8 variant)"
-    idx_ms = idx_t / n_bd
-    idx_gbs = by["indexer"] / (idx_ms * 1e-3) / 1e9
-    t_roof_us = by["path"] / (hbm_peak * 1e9) * 1e6
-
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": dtype, "data": "synthetic",
-        "config": {**w.describe(), **variant,
-                   "parallelism": f"dp{world} (independent batches per GPU)",
-                   "l2": "flushed before every timed step (256 MB write)", "graph": "CUDA graph per step"},
-        "roofline": {"bound": "hbm", "kernel": "idx_score_tc (dsa_index_scores)", "achieved": idx_gbs,
-                     "peak": hbm_peak, "unit": "GB/s", "frac": idx_gbs / hbm_peak,
-                     "traffic": (NCU_INDEXER_TRAFFIC_FP8 if fp8 else NCU_INDEXER_TRAFFIC).get(w.name),
-                     "peak_kind": f"{peak_kind} hbm_gbs",
-                     "algorithmic_bytes": by["indexer"], "avg_launch_us": idx_ms * 1e3},
-        "path_roofline": {"bytes": by["path"], "t_roof_us": t_roof_us,
-                          "frac": t_roof_us / (ms_per_step * 1e3), "peak_kind": f"{peak_kind} hbm_gbs"},
-        "breakdown_us": {"index_scores": idx_ms * 1e3, "topk": topk_t / n_bd * 1e3,
-                         "sparse_mla": mla_t / n_bd * 1e3, "note": "separate graph with events between stages"},
-        "gpu_launches": step.launches_per_step() * args.steps,
-        "clocks": clocks.summary(),
-    }
-
+    res, step = measure(w, args.fp8, args, world, rank, dev, flush, clocks, args.steps, True)
+    line = {"metric": METRIC, "value": res["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": res["dtype"], "data": "synthetic",
+            "config": res["config"]}
+    for k in ("roofline", "path_roofline", "breakdown_us", "stages", "gpu_launches", "launches_per_step",
+              "clocks", "self_check"):
+        line[k] = res[k]
     if not args.no_e2e:
-        e2e = E2EStep(step)
-        e2e.capture()
-        for _ in range(3):
-            e2e.graph.replay()
-        torch.cuda.synchronize()
-        barrier(world)
-        te = 0.0
-        n_e2e = max(10, min(args.steps, 500))
-        for _ in range(n_e2e):
-            flush.fill_(1)
-            e2e.graph.replay()
-            torch.cuda.synchronize()
-            te += e2e.ev[0].elapsed_time(e2e.ev[1])
-        te = max_over_ranks(te, world, dev)
-        line["e2e"] = {"value": world * w.n_q * w.n_layers * n_e2e / (te * 1e-3), "unit": UNIT,
-                       "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "steps": n_e2e}
+        line["e2e"] = e2e_measure(step, world, dev, flush, max(10, min(args.steps, 200)))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fp8:
+        line["cpu_baseline"] = cpu_baseline(w, step.x)
+    step.release()
+    del step
+    gc.collect()
+    torch.cuda.empty_cache()
 
-    line["self_check"] = self_check(step)
-
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = None if (fp8 or mla_fp8) else cpu_baseline(w, step.x)
-
+    if not args.no_per_config and not small:
+        per = {}
+        n = min(args.steps, PER_CONFIG_MAX_STEPS)
+        for name, fp8 in PER_CONFIG:
+            if name == args.workload and fp8 == args.fp8:
+                continue
+            r, s = measure(wl.NAMED[name], fp8, args, world, rank, dev, flush, clocks, n, False)
+            s.release()
+            del s
+            gc.collect()
+            torch.cuda.empty_cache()
+            per[name + ("+fp8" if fp8 else "")] = r
+        line["per_config"] = per
+        line["gpu_launches"] = (line["gpu_launches"] or 0) + sum((r["gpu_launches"] or 0) for r in per.values())
+    clocks.stop()
+    time.sleep(0.05)
+    line["clocks"] = clocks.summary()
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        step.graph = None
-        step.graph_bd = None
         dist.destroy_process_group()
 
 

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libdsa.so")
 
 DSA_OK, DSA_ERR_INVALID, DSA_ERR_UNSUPPORTED, DSA_ERR_WORKSPACE, DSA_ERR_CUDA, DSA_ERR_TIMEOUT = range(6)
 DSA_BF16, DSA_F32, DSA_FP8_E4M3 = 0, 1, 2
-DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_MLA_DECODE, DSA_OP_MLA_PREFILL, DSA_OP_INDEXSHARE_GROUP = range(5)
+DSA_OP_INDEX_SCORES, DSA_OP_TOPK, DSA_OP_MLA_DECODE, DSA_OP_MLA_PREFILL, DSA_OP_INDEXSHARE_GROUP, DSA_OP_SHARD_MERGE = range(6)
 DSA_INDEXER_TOPK_HIST = 1
 DSA_MLA_FP8_ROW_BYTES = 656
 DSA_TOPK_HIST_FROM_INDEXER = 1
@@ -43,6 +43,16 @@ class _Indexer(ctypes.Structure):
                 ("flags", ctypes.c_int32), ("q", ctypes.c_void_p), ("w", ctypes.c_void_p),
                 ("k", ctypes.c_void_p), ("k_seq_stride", ctypes.c_int64), ("k_row_stride", ctypes.c_int64),
                 ("q_scale", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("ks_seq_stride", ctypes.c_int64)]
+
+
+class _CacheWriter(ctypes.Structure):
+    _fields_ = [("n_tok", ctypes.c_int32), ("hidden", ctypes.c_int32), ("h", ctypes.c_void_p),
+                ("h_row_stride", ctypes.c_int64), ("w", ctypes.c_void_p), ("rms_weight", ctypes.c_void_p),
+                ("ln_weight", ctypes.c_void_p), ("ln_bias", ctypes.c_void_p), ("tok_seq", ctypes.c_void_p),
+                ("tok_pos", ctypes.c_void_p), ("n_seq", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
+                ("kv", ctypes.c_void_p), ("kv_seq_stride", ctypes.c_int64), ("kv_row_stride", ctypes.c_int64),
+                ("k_idx", ctypes.c_void_p), ("k_seq_stride", ctypes.c_int64), ("k_row_stride", ctypes.c_int64),
+                ("eps", ctypes.c_float), ("rope_theta", ctypes.c_float)]
 
 
 class _Mla(ctypes.Structure):
@@ -68,8 +78,19 @@ def lib():
         h.dsa_topk.argtypes = [ctypes.POINTER(_Queries), P, I64, I32, I32, P, P, P, SZ, P]
         for name in ("dsa_sparse_mla_decode", "dsa_sparse_mla_prefill"):
             getattr(h, name).argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Mla), P, P, I32, P, SZ, P]
+        h.dsa_sparse_mla_mtp.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Mla), P, P, I32, I32, P, SZ, P]
+        h.dsa_sparse_mla_decode_noalloc.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Mla), P, P, I32, P]
+        h.dsa_noalloc_check_status.argtypes = [P]
         h.dsa_indexshare_group.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Indexer),
                                            ctypes.POINTER(_Mla), I32, I32, P, P, P, SZ, P]
+        h.dsa_shard_candidates.argtypes = [ctypes.POINTER(_Queries), P, I64, P, P, I32, I32, P, P, P, SZ, P]
+        h.dsa_shard_merge.argtypes = [ctypes.POINTER(_Queries), I32, P, P, I32, I32, I32, P, P, P, P, P, SZ, P]
+        h.dsa_shard_combine.argtypes = [ctypes.POINTER(_Queries), I32, I32, I32, P, P, P, P, P, P]
+        h.dsa_write_cache_rows.argtypes = [ctypes.POINTER(_CacheWriter), P, SZ, P]
+        h.dsa_cache_writer_workspace_bytes.argtypes = [I32, I32]
+        h.dsa_cache_writer_workspace_bytes.restype = SZ
+        h.dsa_absorb_queries.argtypes = [I32, I32, P, P, P, P, ctypes.c_float, P, P, SZ, P]
+        h.dsa_up_project.argtypes = [I32, I32, P, P, P, P, SZ, P]
         h.dsa_workspace_bytes.argtypes = [I32, ctypes.POINTER(_Queries), I32, I32, I32, I32]
         h.dsa_workspace_bytes.restype = SZ
         h.dsa_workspace_init.argtypes = [P, SZ, P]
@@ -79,7 +100,10 @@ def lib():
         h.dsa_status_str.argtypes = [st]
         h.dsa_status_str.restype = ctypes.c_char_p
         for name in ("dsa_index_scores", "dsa_topk", "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill",
-                     "dsa_indexshare_group", "dsa_workspace_init", "dsa_check_status"):
+                     "dsa_sparse_mla_mtp", "dsa_sparse_mla_decode_noalloc", "dsa_noalloc_check_status",
+                     "dsa_indexshare_group", "dsa_workspace_init", "dsa_check_status",
+                     "dsa_shard_candidates", "dsa_shard_merge", "dsa_shard_combine",
+                     "dsa_write_cache_rows", "dsa_absorb_queries", "dsa_up_project"):
             getattr(h, name).restype = st
         _lib_handle = h
     return _lib_handle
@@ -169,6 +193,32 @@ class Mla:
                     self.out.data_ptr(), self.lse.data_ptr() if self.lse is not None else None)
 
 
+@dataclass
+class CacheWriter:
+    h: torch.Tensor              # bf16 [n_tok, hidden]
+    w: torch.Tensor              # bf16 [704, hidden]: latent 512 | RoPE key 64 | indexer key 128
+    rms_weight: torch.Tensor     # float32 [512]
+    ln_weight: torch.Tensor      # float32 [128]
+    ln_bias: torch.Tensor        # float32 [128]
+    tok_seq: torch.Tensor        # int32 [n_tok]
+    tok_pos: torch.Tensor        # int32 [n_tok]
+    kv: Optional[torch.Tensor]   # bf16 [n_seq, L, 576] latent cache, or None
+    k_idx: Optional[torch.Tensor]  # bf16 [n_seq, L, 128] indexer keys, or None
+    eps: float = 1e-5
+    rope_theta: float = 8.0e6
+
+    def c(self) -> _CacheWriter:
+        ref = self.kv if self.kv is not None else self.k_idx
+        return _CacheWriter(self.h.shape[0], self.h.shape[1], self.h.data_ptr(), self.h.stride(0), self.w.data_ptr(),
+                            self.rms_weight.data_ptr(), self.ln_weight.data_ptr(), self.ln_bias.data_ptr(),
+                            self.tok_seq.data_ptr(), self.tok_pos.data_ptr(), ref.shape[0], ref.shape[1],
+                            None if self.kv is None else self.kv.data_ptr(),
+                            0 if self.kv is None else self.kv.stride(0), 0 if self.kv is None else self.kv.stride(1),
+                            None if self.k_idx is None else self.k_idx.data_ptr(),
+                            0 if self.k_idx is None else self.k_idx.stride(0),
+                            0 if self.k_idx is None else self.k_idx.stride(1), self.eps, self.rope_theta)
+
+
 # ------------------------------------------------------------------ entry points
 def dsa_workspace_bytes(op: int, queries: Queries, topk: int = 1, mla_heads: int = 64, d_latent: int = 512,
                         n_layers: int = 1) -> int:
@@ -217,6 +267,25 @@ def dsa_sparse_mla_prefill(queries: Queries, mla: Mla, idx: torch.Tensor, cnt: t
                                         ws.numel() * ws.element_size(), _stream(stream)), "dsa_sparse_mla_prefill")
 
 
+def dsa_sparse_mla_mtp(queries: Queries, mla: Mla, idx: torch.Tensor, cnt: torch.Tensor, topk: int,
+                       draft_tokens: int, ws: torch.Tensor, stream=None):
+    qc, mc = queries.c(), mla.c()
+    _check(lib().dsa_sparse_mla_mtp(ctypes.byref(qc), ctypes.byref(mc), _ptr(idx), _ptr(cnt), topk, draft_tokens,
+                                    _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)), "dsa_sparse_mla_mtp")
+
+
+def dsa_sparse_mla_decode_noalloc(queries: Queries, mla: Mla, idx: torch.Tensor, cnt: torch.Tensor, topk: int,
+                                  stream=None):
+    qc, mc = queries.c(), mla.c()
+    _check(lib().dsa_sparse_mla_decode_noalloc(ctypes.byref(qc), ctypes.byref(mc), _ptr(idx), _ptr(cnt), topk,
+                                               _stream(stream)), "dsa_sparse_mla_decode_noalloc")
+
+
+def dsa_noalloc_check_status(stream=None) -> int:
+    """Synchronise, read and clear the no-workspace calls' status word (returns the code)."""
+    return int(lib().dsa_noalloc_check_status(_stream(stream)))
+
+
 def dsa_indexshare_group(queries: Queries, indexer: Indexer, layers: Sequence[Mla], topk: int, idx: torch.Tensor,
                          cnt: torch.Tensor, ws: torch.Tensor, stream=None):
     qc, ic = queries.c(), indexer.c()
@@ -224,6 +293,59 @@ def dsa_indexshare_group(queries: Queries, indexer: Indexer, layers: Sequence[Ml
     _check(lib().dsa_indexshare_group(ctypes.byref(qc), ctypes.byref(ic), arr, len(layers), topk, _ptr(idx),
                                       _ptr(cnt), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "dsa_indexshare_group")
+
+
+def dsa_shard_candidates(queries: Queries, scores: torch.Tensor, idx: torch.Tensor, cnt: torch.Tensor, topk: int,
+                         row_offset: int, cand_score: torch.Tensor, cand_pos: torch.Tensor, ws: torch.Tensor,
+                         stream=None):
+    qc = queries.c()
+    _check(lib().dsa_shard_candidates(ctypes.byref(qc), _ptr(scores), scores.stride(0), _ptr(idx), _ptr(cnt), topk,
+                                      row_offset, _ptr(cand_score), _ptr(cand_pos), _ptr(ws),
+                                      ws.numel() * ws.element_size(), _stream(stream)), "dsa_shard_candidates")
+
+
+def dsa_shard_merge(queries: Queries, n_shards: int, cand_score: torch.Tensor, cand_pos: torch.Tensor, topk: int,
+                    row_begin: int, row_end: int, idx: torch.Tensor, cnt: torch.Tensor, local_idx: torch.Tensor,
+                    local_cnt: torch.Tensor, ws: torch.Tensor, stream=None):
+    qc = queries.c()
+    _check(lib().dsa_shard_merge(ctypes.byref(qc), n_shards, _ptr(cand_score), _ptr(cand_pos), topk, row_begin,
+                                 row_end, _ptr(idx), _ptr(cnt), _ptr(local_idx), _ptr(local_cnt), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)), "dsa_shard_merge")
+
+
+def dsa_shard_combine(queries: Queries, part_out: torch.Tensor, part_lse: torch.Tensor, part_cnt: torch.Tensor,
+                      out: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None):
+    """part_out [n_parts, n_q, heads, d_latent] bf16, part_lse [n_parts, n_q, heads], part_cnt [n_parts, n_q]."""
+    qc = queries.c()
+    n_parts, _, heads, d_lat = part_out.shape
+    _check(lib().dsa_shard_combine(ctypes.byref(qc), n_parts, heads, d_lat, _ptr(part_out), _ptr(part_lse),
+                                   _ptr(part_cnt), _ptr(out), _ptr(lse), _stream(stream)), "dsa_shard_combine")
+
+
+def dsa_cache_writer_workspace_bytes(n_tok: int, hidden: int) -> int:
+    return int(lib().dsa_cache_writer_workspace_bytes(n_tok, hidden))
+
+
+def dsa_write_cache_rows(writer: CacheWriter, ws: torch.Tensor, stream=None):
+    wc = writer.c()
+    _check(lib().dsa_write_cache_rows(ctypes.byref(wc), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_write_cache_rows")
+
+
+def dsa_absorb_queries(q_nope: torch.Tensor, q_rope: torch.Tensor, w_uk_t: torch.Tensor, pos: torch.Tensor,
+                       rope_theta: float, q_out: torch.Tensor, ws: torch.Tensor, stream=None):
+    """q_nope [n, H, 192], q_rope [n, H, 64], w_uk_t [H, 512, 192], pos int32 [n] -> q_out [n, H, 576]."""
+    n, heads = q_nope.shape[0], q_nope.shape[1]
+    _check(lib().dsa_absorb_queries(n, heads, _ptr(q_nope), _ptr(q_rope), _ptr(w_uk_t), _ptr(pos), rope_theta,
+                                    _ptr(q_out), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dsa_absorb_queries")
+
+
+def dsa_up_project(o_lat: torch.Tensor, w_uv: torch.Tensor, out: torch.Tensor, ws: torch.Tensor, stream=None):
+    """o_lat [n, H, 512], w_uv [H, 256, 512] -> out [n, H, 256]."""
+    n, heads = o_lat.shape[0], o_lat.shape[1]
+    _check(lib().dsa_up_project(n, heads, _ptr(o_lat), _ptr(w_uv), _ptr(out), _ptr(ws),
+                                ws.numel() * ws.element_size(), _stream(stream)), "dsa_up_project")
 
 
 # ------------------------------------------------------------------ conveniences

@@ -6,6 +6,8 @@
 
 #include <nvtx3/nvToolsExt.h>
 
+#include "abi_checks.cuh"
+#include "tma_encode.cuh"
 #include "dsa.h"
 #include "kernels.cuh"
 
@@ -17,8 +19,6 @@ constexpr size_t kStatusBytes = 256;
 constexpr int kDecodeMaxQueries = 256;  // IndexShare group: split-K MLA up to this many queries
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
-
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int64_t round4(int64_t x) { return (x + 3) & ~static_cast<int64_t>(3); }
 
@@ -34,29 +34,7 @@ int num_sms_current() {
     return cache[dev];
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
-                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    });
-    return fn;
-}
-
-bool valid_queries(const dsa_queries *qs) {
-    if (!qs) return false;
-    if (qs->n_q < 0 || qs->n_seq < 1 || qs->max_ctx < 1 || qs->seq_run < 1) return false;
-    if (qs->n_q > 0 && (!qs->q_seq || !qs->q_pos)) return false;
-    return true;
-}
+EncodeTiledFn encode_fn() { return tma_encode_fn(); }
 
 uint32_t *status_word(void *ws) { return static_cast<uint32_t *>(ws); }
 
@@ -70,16 +48,6 @@ bool indexer_tc_ok(const dsa_indexer *ix) {
     return (ix->dtype == DSA_BF16 || ix->dtype == DSA_FP8_E4M3) && ix->heads == kIdxHeads && ix->dim == kIdxDim &&
            aligned16(ix->q) && aligned16(ix->k) && ix->k_row_stride % al == 0 && ix->k_seq_stride % al == 0 &&
            ix->k_row_stride >= kIdxDim;
-}
-
-bool mla_kv_fp8(const dsa_mla *m) { return m->kv_dtype == DSA_FP8_E4M3; }
-
-bool mla_tc_ok(const dsa_mla *m) {
-    const bool shape = m->dtype == DSA_BF16 && m->heads == kMlaHeads && m->d_latent == kLatent &&
-                       m->d_rope == kRope && aligned16(m->q) && aligned16(m->kv) && aligned16(m->out);
-    if (mla_kv_fp8(m))  // packed rows, strides in bytes
-        return shape && m->kv_row_stride % 16 == 0 && m->kv_seq_stride % 16 == 0 && m->kv_row_stride >= kFp8Row;
-    return shape && m->kv_row_stride % 8 == 0 && m->kv_seq_stride % 8 == 0 && m->kv_row_stride >= kRow;
 }
 
 size_t ws_index_scores() { return kStatusBytes; }
@@ -101,6 +69,31 @@ size_t ws_scores(int n_q, int max_ctx) {
     return align256(static_cast<size_t>(n_q) * round4(max_ctx) * sizeof(float));
 }
 bool group_uses_decode(int n_q) { return n_q <= kDecodeMaxQueries; }
+// dsa_shard_merge: [status][merged scores][merged positions][merged counts - 1]
+// [top-k of the merged list: indices, counts][top-k scratch of the merged list]
+int64_t shard_merged_ld(int n_shards, int topk) { return round4(static_cast<int64_t>(n_shards) * topk); }
+struct ShardMergeLayout {
+    size_t score, pos, last, sel, sel_cnt, topk_scratch, total;
+};
+ShardMergeLayout shard_merge_layout(int n_q, int n_shards, int topk) {
+    const int64_t ld = shard_merged_ld(n_shards, topk);
+    ShardMergeLayout l;
+    size_t o = kStatusBytes;
+    l.score = o;
+    o += align256(static_cast<size_t>(n_q) * ld * sizeof(float));
+    l.pos = o;
+    o += align256(static_cast<size_t>(n_q) * ld * sizeof(int32_t));
+    l.last = o;
+    o += align256(static_cast<size_t>(n_q) * sizeof(int32_t));
+    l.sel = o;
+    o += align256(static_cast<size_t>(n_q) * topk * sizeof(int32_t));
+    l.sel_cnt = o;
+    o += align256(static_cast<size_t>(n_q) * sizeof(int32_t));
+    l.topk_scratch = o;
+    o += align256(topk_scratch_bytes(n_q, static_cast<int>(ld)));
+    l.total = o;
+    return l;
+}
 size_t ws_group(int n_q, int max_ctx, int topk, int n_layers) {
     size_t b = kStatusBytes + ws_scores(n_q, max_ctx) + align256(topk_scratch_bytes(n_q, max_ctx));
     if (group_uses_decode(n_q)) b += ws_mla_partials(n_q, topk, n_layers);  // after the whole top-k scratch
@@ -260,32 +253,12 @@ bool scores_ok(const float *scores, int64_t ld, int max_ctx) {
 }
 
 // ------------------------------------------------------------------ MLA
-dsa_status check_mla_layers(const dsa_mla *layers, int n_layers) {
-    if (!layers || n_layers < 1 || n_layers > kMaxLayers) return DSA_ERR_INVALID;
-    const dsa_mla &m0 = layers[0];
-    for (int l = 0; l < n_layers; ++l) {
-        const dsa_mla &m = layers[l];
-        if (!m.q || !m.kv || !m.out) return DSA_ERR_INVALID;
-        if (m.heads < 1 || m.d_latent < 1 || m.d_rope < 0 || (m.dtype != DSA_BF16 && m.dtype != DSA_F32))
-            return DSA_ERR_INVALID;
-        if (m.kv_dtype != 0 && m.kv_dtype != m.dtype && m.kv_dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID;
-        // a packed FP8 row holds d_latent codes, d_rope bf16 values and a float32 scale
-        const int64_t min_row = mla_kv_fp8(&m) ? int64_t(m.d_latent) + 2 * int64_t(m.d_rope) + 4
-                                               : int64_t(m.d_latent) + m.d_rope;
-        if (m.kv_row_stride < min_row || m.kv_seq_stride < 0) return DSA_ERR_INVALID;
-        if (m.heads != m0.heads || m.d_latent != m0.d_latent || m.d_rope != m0.d_rope || m.dtype != m0.dtype ||
-            m.scale != m0.scale || m.kv_row_stride != m0.kv_row_stride || m.kv_seq_stride != m0.kv_seq_stride ||
-            mla_kv_fp8(&m) != mla_kv_fp8(&m0))
-            return DSA_ERR_INVALID;
-    }
-    return DSA_OK;
-}
-
 dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, const int32_t *idx,
                   const int32_t *cnt, int topk, bool decode, uint8_t *scratch, uint32_t *status,
-                  cudaStream_t st) {
+                  cudaStream_t st, int sel_group = 1) {
     MlaArgs a;
     std::memset(&a, 0, sizeof(a));
+    a.sel_group = sel_group;
     for (int l = 0; l < n_layers; ++l) {
         a.layer[l].q = layers[l].q;
         a.layer[l].kv = layers[l].kv;
@@ -371,6 +344,8 @@ size_t dsa_workspace_bytes(int32_t op, const dsa_queries *qs, int32_t topk, int3
         case DSA_OP_INDEXSHARE_GROUP:
             return ws_group(n_q, qs->max_ctx > 0 ? qs->max_ctx : 1, topk > 0 ? topk : 1,
                             n_layers > 0 ? n_layers : 1);
+        case DSA_OP_SHARD_MERGE:  // the last argument is the number of shards
+            return shard_merge_layout(n_q, n_layers > 0 ? n_layers : 1, topk > 0 ? topk : 1).total;
     }
     return 0;
 }
@@ -430,7 +405,7 @@ dsa_status dsa_topk(const dsa_queries *queries, const float *scores, int64_t ld_
 }
 
 static dsa_status mla_entry(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx, const int32_t *cnt,
-                            int32_t topk, void *ws, size_t ws_bytes, void *stream, bool decode) {
+                            int32_t topk, void *ws, size_t ws_bytes, void *stream, bool decode, int sel_group = 1) {
     if (!valid_queries(queries)) return DSA_ERR_INVALID;
     if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
     dsa_status s = check_mla_layers(mla, 1);
@@ -441,7 +416,7 @@ static dsa_status mla_entry(const dsa_queries *queries, const dsa_mla *mla, cons
     // partials after the region the indexer / top-k keep zero (see ws_zeroed_head)
     uint8_t *scratch = static_cast<uint8_t *>(ws) + kStatusBytes + ws_zeroed_head(queries->n_q);
     return do_mla(queries, mla, 1, idx, cnt, topk, decode, scratch, status_word(ws),
-                  static_cast<cudaStream_t>(stream));
+                  static_cast<cudaStream_t>(stream), sel_group);
 }
 
 dsa_status dsa_sparse_mla_decode(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,
@@ -454,6 +429,16 @@ dsa_status dsa_sparse_mla_prefill(const dsa_queries *queries, const dsa_mla *mla
                                   const int32_t *cnt, int32_t topk, void *ws, size_t ws_bytes, void *stream) {
     NvtxRange range("dsa_sparse_mla_prefill");
     return mla_entry(queries, mla, idx, cnt, topk, ws, ws_bytes, stream, false);
+}
+
+dsa_status dsa_sparse_mla_mtp(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,
+                              const int32_t *cnt, int32_t topk, int32_t draft_tokens, void *ws, size_t ws_bytes,
+                              void *stream) {
+    NvtxRange range("dsa_sparse_mla_mtp");
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (draft_tokens < 1 || queries->n_q % draft_tokens != 0) return DSA_ERR_INVALID;
+    return mla_entry(queries, mla, idx, cnt, topk, ws, ws_bytes, stream, queries->n_q <= kDecodeMaxQueries,
+                     draft_tokens);
 }
 
 dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *indexer, const dsa_mla *layers,
@@ -481,6 +466,105 @@ dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *i
     if (s != DSA_OK) return s;
     return do_mla(queries, layers, n_layers, idx, cnt, topk, group_uses_decode(queries->n_q), scratch,
                   status_word(ws), st);
+}
+
+// ------------------------------------------------------------------ key-range shards
+dsa_status dsa_shard_candidates(const dsa_queries *queries, const float *scores, int64_t ld_scores,
+                                const int32_t *idx, const int32_t *cnt, int32_t topk, int32_t row_offset,
+                                float *cand_score, int32_t *cand_pos, void *ws, size_t ws_bytes, void *stream) {
+    NvtxRange range("dsa_shard_candidates");
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (!ws_ok(ws, ws_bytes, kStatusBytes)) return DSA_ERR_WORKSPACE;
+    if (topk < 1 || topk > kMaxTopk || !idx || !cnt || !cand_score || !cand_pos || row_offset < 0)
+        return DSA_ERR_INVALID;
+    if (!scores || ld_scores < queries->max_ctx) return DSA_ERR_INVALID;
+    if (queries->n_q == 0) return DSA_OK;
+    ShardArgs a = {};
+    a.n_q = queries->n_q;
+    a.topk = topk;
+    a.L = queries->max_ctx;
+    a.status = status_word(ws);
+    a.scores = scores;
+    a.ld = ld_scores;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.row_offset = row_offset;
+    a.cand_score = cand_score;
+    a.cand_pos = cand_pos;
+    return launch_shard_candidates(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status dsa_shard_merge(const dsa_queries *queries, int32_t n_shards, const float *cand_score,
+                           const int32_t *cand_pos, int32_t topk, int32_t row_begin, int32_t row_end, int32_t *idx,
+                           int32_t *cnt, int32_t *local_idx, int32_t *local_cnt, void *ws, size_t ws_bytes,
+                           void *stream) {
+    NvtxRange range("dsa_shard_merge");
+    if (!queries || queries->n_q < 0) return DSA_ERR_INVALID;
+    if (n_shards < 1 || n_shards > kMaxShards || topk < 1 || topk > kMaxTopk) return DSA_ERR_INVALID;
+    if (!cand_score || !cand_pos || !idx || !cnt || !local_idx || !local_cnt) return DSA_ERR_INVALID;
+    if (row_begin < 0 || row_end < row_begin) return DSA_ERR_INVALID;
+    const ShardMergeLayout lay = shard_merge_layout(queries->n_q, n_shards, topk);
+    if (!ws_ok(ws, ws_bytes, lay.total)) return DSA_ERR_WORKSPACE;
+    if (queries->n_q == 0) return DSA_OK;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    const int64_t ld = shard_merged_ld(n_shards, topk);
+    ShardArgs a = {};
+    a.n_q = queries->n_q;
+    a.topk = topk;
+    a.status = status_word(ws);
+    a.cand_score = const_cast<float *>(cand_score);
+    a.cand_pos = const_cast<int32_t *>(cand_pos);
+    a.n_shards = n_shards;
+    a.merged_ld = ld;
+    a.merged_score = reinterpret_cast<float *>(base + lay.score);
+    a.merged_pos = reinterpret_cast<int32_t *>(base + lay.pos);
+    a.merged_last = reinterpret_cast<int32_t *>(base + lay.last);
+    int32_t *sel = reinterpret_cast<int32_t *>(base + lay.sel);
+    int32_t *sel_cnt = reinterpret_cast<int32_t *>(base + lay.sel_cnt);
+    a.sel = sel;
+    a.sel_cnt = sel_cnt;
+    a.out_idx = idx;
+    a.out_cnt = cnt;
+    a.local_idx = local_idx;
+    a.local_cnt = local_cnt;
+    a.row_begin = row_begin;
+    a.row_end = row_end;
+    if (launch_shard_compact(a, st) != cudaSuccess) return DSA_ERR_CUDA;
+    // the top-k of each query's merged list (ascending in position), ties to the
+    // lower list index = the lower position
+    dsa_queries mq;
+    mq.n_q = queries->n_q;
+    mq.n_seq = 1;
+    mq.max_ctx = static_cast<int32_t>(ld);
+    mq.seq_run = 1;
+    mq.q_seq = a.merged_last;  // not read by the top-k
+    mq.q_pos = a.merged_last;
+    dsa_status s = do_topk(&mq, a.merged_score, ld, topk, sel, sel_cnt, a.status, base + lay.topk_scratch, false, st);
+    if (s != DSA_OK) return s;
+    return launch_shard_map(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+dsa_status dsa_shard_combine(const dsa_queries *queries, int32_t n_parts, int32_t heads, int32_t d_latent,
+                             const void *part_out, const float *part_lse, const int32_t *part_cnt, void *out,
+                             float *lse, void *stream) {
+    NvtxRange range("dsa_shard_combine");
+    if (!queries || queries->n_q < 0) return DSA_ERR_INVALID;
+    if (n_parts < 1 || n_parts > kMaxShards || !part_out || !part_lse || !part_cnt || !out) return DSA_ERR_INVALID;
+    if (heads < 2 || heads % 2 != 0 || d_latent < 4 || d_latent % 4 != 0 || d_latent > 512) return DSA_ERR_UNSUPPORTED;
+    if ((reinterpret_cast<uintptr_t>(part_out) & 7u) || (reinterpret_cast<uintptr_t>(out) & 7u)) return DSA_ERR_INVALID;
+    if (queries->n_q == 0) return DSA_OK;
+    ShardCombineArgs a;
+    a.n_parts = n_parts;
+    a.n_q = queries->n_q;
+    a.heads = heads;
+    a.d_lat = d_latent;
+    a.part_out = part_out;
+    a.part_lse = part_lse;
+    a.part_cnt = part_cnt;
+    a.out = out;
+    a.lse = lse;
+    return launch_shard_combine(a, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 }  // extern "C"

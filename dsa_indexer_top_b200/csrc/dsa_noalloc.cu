@@ -1,16 +1,18 @@
 // dsa_noalloc.cu -- dsa_sparse_mla_decode_noalloc: the split-K sparse MLA decode
 // with its scratch in a fixed, file-scope device array instead of a
-// caller-provided workspace.
+// caller-provided workspace, and dsa_noalloc_check_status, which reads that
+// array's status word.
 //
 // Some callers cannot allocate device memory at the point where they run the
 // attention step: code running inside a captured or pre-planned execution whose
 // memory was fixed up front, plugins and runtimes that hand a kernel only its
 // input/output tensors, or hosts where cudaMalloc is not allowed on the serving
-// path.  For them this entry point needs no workspace: its split-K partials
-// live in g_mla_decode_scratch below, which every GPU that loads the library
-// keeps until the process exits.
+// path.  For them this entry point needs no workspace: its status word and
+// split-K partials live in g_mla_decode_scratch below, which every GPU that
+// loads the library keeps until the process exits.
 #include <mutex>
 
+#include "abi_checks.cuh"
 #include "dsa.h"
 #include "kernels.cuh"
 
@@ -19,8 +21,9 @@ using namespace dsa;
 namespace {
 
 constexpr size_t kStatusBytes = 256;
-// Size of the static scratch: status word + split-K partials.  32 MiB holds
-// the partials of up to 15 queries at topk = 2048 (2,105,344 bytes per query).
+// Size of the static scratch: status word + split-K partials.  The decode plan
+// gives a query at most (SMs / queries) splits, so its partials stay below
+// SMs x 131,584 bytes (about 19.5 MB on a 148-SM B200) whatever the batch.
 constexpr size_t kNoallocScratchBytes = static_cast<size_t>(32) << 20;
 
 __device__ __align__(256) uint8_t g_mla_decode_scratch[kNoallocScratchBytes];
@@ -30,14 +33,18 @@ std::mutex g_setup_mutex;
 void *g_scratch_ptr[kMaxDevices] = {};
 
 // Device address of the scratch array for the current device.  The host-side
-// symbol is only a stand-in; the real address comes from cudaGetSymbolAddress,
-// looked up once per device (with that device current) and cached.
-dsa_status scratch_for_current_device(uint8_t **out) {
+// symbol is only a stand-in; the real address comes from cudaGetSymbolAddress
+// with the device current.  It is looked up again on every call made outside
+// stream capture (so a context re-created after a device reset gets its own
+// address) and cached per device for calls made while `st` is capturing.
+dsa_status scratch_for_current_device(cudaStream_t st, uint8_t **out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
     if (dev < 0 || dev >= kMaxDevices) return DSA_ERR_UNSUPPORTED;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(st, &cap) != cudaSuccess) return DSA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
+    if (cap == cudaStreamCaptureStatusNone || !g_scratch_ptr[dev]) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, g_mla_decode_scratch) != cudaSuccess || !p) return DSA_ERR_CUDA;
         g_scratch_ptr[dev] = p;
@@ -46,37 +53,39 @@ dsa_status scratch_for_current_device(uint8_t **out) {
     return DSA_OK;
 }
 
-bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int num_sms(int dev) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    return sms;
+}
 
 }  // namespace
 
 extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, const dsa_mla *mla,
                                                     const int32_t *idx, const int32_t *cnt, int32_t topk,
                                                     void *stream) {
-    if (!queries || queries->n_q < 0 || queries->n_seq < 1 || queries->max_ctx < 1) return DSA_ERR_INVALID;
-    if (queries->n_q > 0 && (!queries->q_seq || !queries->q_pos)) return DSA_ERR_INVALID;
-    if (topk < 1 || topk > kMaxTopk || !idx || !cnt || !mla) return DSA_ERR_INVALID;
-    const dsa_mla &m = *mla;
-    if (m.kv_dtype != 0 && m.kv_dtype != m.dtype && m.kv_dtype != DSA_FP8_E4M3) return DSA_ERR_INVALID;
-    const bool fp8 = m.kv_dtype == DSA_FP8_E4M3;  // packed rows, strides in bytes
-    const int64_t min_row = fp8 ? int64_t(m.d_latent) + 2 * int64_t(m.d_rope) + 4 : int64_t(m.d_latent) + m.d_rope;
-    if (!m.q || !m.kv || !m.out || m.kv_seq_stride < 0 || m.kv_row_stride < min_row) return DSA_ERR_INVALID;
+    // the same checks as dsa_sparse_mla_decode (shared validators)
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
+    const dsa_status chk = check_mla_layers(mla, 1);
+    if (chk != DSA_OK) return chk;
     // Only the tensor-core shape uses scratch: bf16 queries, 64 heads, 512 + 64.
-    const int64_t al = fp8 ? 16 : 8;
-    if (m.dtype != DSA_BF16 || m.heads != kMlaHeads || m.d_latent != kLatent || m.d_rope != kRope ||
-        !aligned16(m.q) || !aligned16(m.kv) || !aligned16(m.out) || m.kv_row_stride % al != 0 ||
-        m.kv_seq_stride % al != 0 || (fp8 && m.kv_row_stride < kFp8Row))
-        return DSA_ERR_UNSUPPORTED;
-    const int n_splits = (topk + kRowsPerChunk - 1) / kRowsPerChunk;
+    if (!mla_tc_ok(mla)) return DSA_ERR_UNSUPPORTED;
+    const dsa_mla &m = *mla;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DSA_ERR_CUDA;
+    // the split plan of this call (the one the launch uses) sizes the scratch
+    int n_splits, cpc;
+    mla_plan(queries->n_q, 1, topk, true, num_sms(dev), kMlaMaxSplits, n_splits, cpc);
     const size_t need = kStatusBytes + (n_splits > 1 ? mla_partial_bytes(1, queries->n_q, n_splits) : 0);
     if (need > kNoallocScratchBytes) return DSA_ERR_WORKSPACE;  // beyond the static scratch
     uint8_t *scratch = nullptr;
-    dsa_status s = scratch_for_current_device(&scratch);
+    dsa_status s = scratch_for_current_device(st, &scratch);
     if (s != DSA_OK) return s;
     if (queries->n_q == 0) return DSA_OK;
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // The status word must start at zero; the partials are fully rewritten.
-    if (cudaMemsetAsync(scratch, 0, kStatusBytes, st) != cudaSuccess) return DSA_ERR_CUDA;
+    // The status word starts at zero when the library loads and is cleared by
+    // dsa_noalloc_check_status; the partials are fully rewritten by each call.
 
     MlaArgs a = {};
     a.layer[0].q = m.q;
@@ -98,22 +107,29 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
     a.d_rope = m.d_rope;
     a.scale = m.scale;
     a.is_bf16 = 1;
-    a.kv_fp8 = fp8 ? 1 : 0;
+    a.kv_fp8 = mla_kv_fp8(&m) ? 1 : 0;
+    a.sel_group = 1;
     a.status = reinterpret_cast<uint32_t *>(scratch);
-    int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
-        sms = 148;
-    int plan_splits, cpc;
-    mla_plan(queries->n_q, 1, topk, true, sms, n_splits, plan_splits, cpc);  // at most the bound above
-    a.n_splits = plan_splits;
+    a.n_splits = n_splits;
     a.chunks_per_cta = cpc;
-    if (plan_splits > 1) {
+    if (n_splits > 1) {
         a.part_o = reinterpret_cast<float *>(scratch + kStatusBytes);
-        const size_t rows = static_cast<size_t>(queries->n_q) * plan_splits * kMlaHeads;
+        const size_t rows = static_cast<size_t>(queries->n_q) * n_splits * kMlaHeads;
         a.part_ml = reinterpret_cast<float *>(scratch + kStatusBytes + rows * kLatent * sizeof(float));
         if (launch_mla_tc(a, st) != cudaSuccess) return DSA_ERR_CUDA;
         return launch_mla_combine(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
     }
     return launch_mla_tc(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+}
+
+extern "C" dsa_status dsa_noalloc_check_status(void *stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *scratch = nullptr;
+    dsa_status s = scratch_for_current_device(st, &scratch);
+    if (s != DSA_OK) return s;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, scratch, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cudaStreamSynchronize(st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (v != 0 && cudaMemsetAsync(scratch, 0, sizeof(v), st) != cudaSuccess) return DSA_ERR_CUDA;
+    return static_cast<dsa_status>(v);
 }

@@ -1,0 +1,175 @@
+// gemm.cu -- the dense contractions upstream and downstream of the attention
+// path ("GLM-5.2 -- Model techniques map", "Checked in its code": Multi-head
+// latent attention -- kv_a_proj_with_mqa, the per-head kv_b_proj halves W_UK /
+// W_UV of the absorbed form; QK normalization -- the indexer key projection wk):
+//   C[b][m][n] = sum_k A[b][m][k] * B[b][n][k]      (bf16 operands, fp32 sums)
+// with both operands K-major, i.e. B in the [out][in] layout of a linear layer's
+// weight.  A tcgen05 kernel: one CTA per (128 x BN output tile, K split, batch);
+//   warp 0      TMA producer: 128 x 64 tiles of A and BN x 64 tiles of B
+//               (128-byte swizzle) into a ring of shared-memory stages;
+//   warp 1      MMA issuer: tcgen05.mma kind::f16, M = 128, N = BN, K = 16 steps,
+//               fp32 accumulator in TMEM;
+//   warps 2-5   epilogue: tcgen05.ld of one TMEM lane quadrant each (one output
+//               row per thread), fp32 or bf16 stores.
+// Split-K (grid y) writes fp32 partials that a consumer sums in a fixed order.
+#include <cuda_bf16.h>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace dsa {
+namespace {
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 64;
+constexpr int kGemmStages = 3;
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmCfg {
+    static constexpr int kATile = kGemmBM * kGemmBK * 2;  // 16 KB
+    static constexpr int kBTile = BN * kGemmBK * 2;
+    static constexpr int kStage = kATile + kBTile;
+    static constexpr int kSmem = kGemmStages * kStage + 1024;
+    static constexpr int kTmemCols = BN < 32 ? 32 : BN;
+    static constexpr uint32_t kIdesc = idesc_bf16(kGemmBM, BN, false, false);
+};
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads) gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                                                               const __grid_constant__ CUtensorMap tmap_b,
+                                                               const GemmArgs g) {
+    using Cfg = GemmCfg<BN>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t full_bar[kGemmStages], empty_bar[kGemmStages], acc_full;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ int abort_flag;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nt = blockIdx.x, mt = blockIdx.y % g.m_tiles, split = blockIdx.y / g.m_tiles, b = blockIdx.z;
+    const int kb_total = (g.K + kGemmBK - 1) / kGemmBK;
+    const int kb0 = split * g.kb_per_split;
+    const int nkb = max(0, min(kb0 + g.kb_per_split, kb_total) - kb0);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGemmStages; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        mbar_init(&acc_full, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+        tma_prefetch_desc(&tmap_a);
+        tma_prefetch_desc(&tmap_b);
+    }
+    if (warp == 1) {
+        tmem_alloc(&tmem_base_sh, Cfg::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base_sh;
+    griddep_wait();
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int last_use[kGemmStages];
+            for (int s = 0; s < kGemmStages; ++s) last_use[s] = -1;
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % kGemmStages, use = kb / kGemmStages;
+                if (!mbar_wait(&empty_bar[s], (use & 1) ^ 1, g.status, &abort_flag)) break;
+                uint8_t *dst = smem + s * Cfg::kStage;
+                mbar_arrive_expect_tx(&full_bar[s], Cfg::kStage);
+                const int kx = (kb0 + kb) * kGemmBK;
+                if (g.a_batch_inner)
+                    tma_load_3d(dst, &tmap_a, &full_bar[s], kx, b, mt * kGemmBM);
+                else
+                    tma_load_3d(dst, &tmap_a, &full_bar[s], kx, mt * kGemmBM, b);
+                if (g.b_batch_inner)
+                    tma_load_3d(dst + Cfg::kATile, &tmap_b, &full_bar[s], kx, b, nt * BN);
+                else
+                    tma_load_3d(dst + Cfg::kATile, &tmap_b, &full_bar[s], kx, nt * BN, b);
+                last_use[s] = use;
+            }
+            // every copy this thread issued has landed before the CTA moves on
+            for (int s = 0; s < kGemmStages; ++s)
+                if (last_use[s] >= 0) mbar_wait(&full_bar[s], last_use[s] & 1, g.status, nullptr);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            for (int kb = 0; kb < nkb; ++kb) {
+                const int s = kb % kGemmStages, use = kb / kGemmStages;
+                if (!mbar_wait(&full_bar[s], use & 1, g.status, &abort_flag)) break;
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + s * Cfg::kStage);
+                const uint64_t adesc = sdesc_sw128(a_addr, 16, 1024);
+                const uint64_t bdesc = sdesc_sw128(a_addr + Cfg::kATile, 16, 1024);
+#pragma unroll
+                for (int kk = 0; kk < kGemmBK / 16; ++kk)  // 32 bytes of each 128-byte row per step
+                    umma_bf16(tbase, adesc + static_cast<uint64_t>(kk * 2), bdesc + static_cast<uint64_t>(kk * 2),
+                              Cfg::kIdesc, (kb > 0 || kk > 0) ? 1u : 0u);
+                umma_commit(&empty_bar[s]);
+            }
+            umma_commit(&acc_full);  // also when no MMA ran (nkb == 0): the epilogue writes zeros
+        }
+    } else {
+        // epilogue: warp w reads TMEM lanes 32 * (w % 4) .. + 31, one output row each
+        const int quad = warp & 3;
+        const int m = mt * kGemmBM + quad * 32 + lane;
+        const bool have = nkb > 0;
+        if (mbar_wait(&acc_full, 0, g.status, &abort_flag)) {
+            tc_fence_after();
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + c0, r);
+                tmem_ld_wait();
+                const int n0 = nt * BN + c0;
+                if (m >= g.M) continue;
+                if (g.out_f32) {
+                    float *o = g.out_f32 + split * g.s_split + b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n0;
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        if (n0 + x < g.N) o[x] = have ? u2f(r[x]) : 0.f;
+                } else {
+                    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(g.out_bf16) + b * g.s_batch +
+                                       static_cast<int64_t>(m) * g.ldc + n0;
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        if (n0 + x < g.N) o[x] = __float2bfloat16_rn(have ? u2f(r[x]) : 0.f);
+                }
+            }
+        }
+    }
+    griddep_launch_dependents();
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tbase, Cfg::kTmemCols);
+    }
+}
+
+template <int BN>
+cudaError_t launch_gemm_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st) {
+    using Cfg = GemmCfg<BN>;
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    if (e != cudaSuccess) return e;
+    const int n_tiles = (g.N + BN - 1) / BN;
+    dim3 grid(n_tiles, g.m_tiles * g.k_splits, g.batch);
+    return launch_pdl(gemm_tc_kernel<BN>, grid, dim3(kGemmThreads), Cfg::kSmem, st, ta, tb, g);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_tc(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st) {
+    switch (bn) {
+        case 64: return launch_gemm_bn<64>(ta, tb, g, st);
+        case 128: return launch_gemm_bn<128>(ta, tb, g, st);
+        case 256: return launch_gemm_bn<256>(ta, tb, g, st);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace dsa

@@ -152,7 +152,9 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            const uint64_t stream_policy = l2_evict_first_policy();  // keys are read once
+            // one query per tile (decode): keys are read once, evict them first; several
+            // (prefill): every query group re-reads the chunk's keys, keep them in L2
+            const uint64_t stream_policy = G == 1 ? l2_evict_first_policy() : l2_evict_last_policy();
             int cur_g = -1, seq = -1, max_pos = -1;
             bool group_loaded = false;
             int b_uses = 0;

@@ -119,6 +119,94 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st);
 // First-digit histograms only (into a.ghist, which must be zeroed), every query.
 cudaError_t launch_topk_hist(const TopkArgs &a, int num_sms, cudaStream_t st);
 
+// ------------------------------------------------------------------ key-range shards
+constexpr int kMaxShards = 64;
+
+struct ShardArgs {
+    int n_q, topk, L;
+    uint32_t *status;
+    // candidates of this rank's local top-k
+    const float *scores;
+    int64_t ld;
+    const int32_t *idx;      // [n_q][topk] local selection (shard rows), ascending, -1 padded
+    const int32_t *cnt;      // [n_q]
+    int row_offset;          // the shard's first row in the sequence
+    float *cand_score;       // [n_q][topk] (one rank) or [n_shards][n_q][topk] (gathered)
+    int32_t *cand_pos;       // same layout: sequence positions, -1 padded
+    // merge of the gathered candidates
+    int n_shards;
+    int64_t merged_ld;       // row stride of the merged list (>= n_shards * topk, multiple of 4)
+    float *merged_score;     // [n_q][merged_ld]
+    int32_t *merged_pos;     // [n_q][merged_ld]
+    int32_t *merged_last;    // [n_q] number of merged candidates - 1
+    const int32_t *sel;      // [n_q][topk] top-k of the merged list (indices into it)
+    const int32_t *sel_cnt;  // [n_q]
+    int32_t *out_idx, *out_cnt;      // global selection (sequence positions)
+    int32_t *local_idx, *local_cnt;  // this rank's part of it (shard rows)
+    int row_begin, row_end;
+};
+cudaError_t launch_shard_candidates(const ShardArgs &a, cudaStream_t st);
+cudaError_t launch_shard_compact(const ShardArgs &a, cudaStream_t st);
+cudaError_t launch_shard_map(const ShardArgs &a, cudaStream_t st);
+
+struct ShardCombineArgs {
+    int n_parts, n_q, heads, d_lat;
+    const void *part_out;     // bf16 [n_parts][n_q][heads][d_lat]
+    const float *part_lse;    // [n_parts][n_q][heads]
+    const int32_t *part_cnt;  // [n_parts][n_q] rows each part attended over (0: ignored)
+    void *out;                // bf16 [n_q][heads][d_lat]
+    float *lse;               // [n_q][heads] or null
+};
+cudaError_t launch_shard_combine(const ShardCombineArgs &a, cudaStream_t st);
+
+// ------------------------------------------------------------------ dense GEMM (producers)
+// C[b][m][n] = sum_k A[b][m][k] * B[b][n][k], bf16 operands read by TMA from
+// 3-D tensor maps {K, rows, batch} (128-byte swizzle, boxes {64, 128, 1} for A
+// and {64, BN, 1} for B), fp32 accumulation in TMEM.  Grid (N tiles, M tiles x
+// K splits, batch); split s of batch b writes rows of out_f32 + s * s_split +
+// b * s_batch (row stride ldc), or bf16 rows of out_bf16 (one split only).
+struct GemmArgs {
+    int M, N, K, batch;
+    int m_tiles, k_splits, kb_per_split;  // kb: blocks of 64 along K
+    float *out_f32;
+    void *out_bf16;
+    int64_t ldc, s_batch, s_split;        // elements
+    int a_batch_inner, b_batch_inner;     // operand map ordered {K, batch, rows} (see encode_gemm_operand)
+    uint32_t *status;
+};
+cudaError_t launch_gemm_tc(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st);
+
+// Cache-row writer epilogue: one CTA per token sums the split-K partials of
+// y = h . W^T (704 features: latent 512 | RoPE key 64 | indexer key 128) and
+// writes RMSNorm(latent) * gamma | RoPE(key) into the latent cache and
+// RoPE_last64(LayerNorm(indexer key) * w + b) into the indexer-key cache.
+struct CacheWriteArgs {
+    const float *y;            // [k_splits][n_tok][704]
+    int k_splits, n_tok;
+    const float *rms_weight, *ln_weight, *ln_bias;
+    const int32_t *tok_seq, *tok_pos;
+    void *kv;
+    int64_t kv_seq_stride, kv_row_stride;
+    void *k_idx;
+    int64_t k_seq_stride, k_row_stride;
+    int n_seq, L;
+    float eps;
+    double log2_theta;
+    uint32_t *status;
+};
+constexpr int kProjFeatures = kLatent + kRope + kIdxDim;  // 704
+cudaError_t launch_cache_write_epilogue(const CacheWriteArgs &a, cudaStream_t st);
+
+// RoPE of the absorbed queries' RoPE part: q[i][h][512 + d] = RoPE(q_rope[i][h], pos[i]).
+struct QueryRopeArgs {
+    const void *q_rope;  // bf16 [n][H][64]
+    void *q;             // bf16 [n][H][576]
+    const int32_t *pos;
+    int n, heads;
+    double log2_theta;
+};
+cudaError_t launch_query_rope(const QueryRopeArgs &a, cudaStream_t st);
+
 // ------------------------------------------------------------------ diagnostics
 // The limit of every device-side wait (the same value as kWaitLimitNs of the
 // PTX wrappers): 2 s.
@@ -148,6 +236,7 @@ struct MlaArgs {
     float scale;
     int is_bf16;
     int kv_fp8;          // caches are packed FP8 rows (kFp8Row bytes; strides in bytes)
+    int sel_group;       // queries per selection row: query i reads idx/cnt row i / sel_group (>= 1)
     uint32_t *status;
     // split-K schedule (tensor-core path)
     int n_splits;        // CTAs per query

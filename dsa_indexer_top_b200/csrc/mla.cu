@@ -54,6 +54,9 @@ constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, false);
 // this many powers of two (probabilities stay below 2^8); only then is the
 // accumulated O rescaled.
 constexpr float kRescaleLog2 = 8.0f;
+// Chunks prefetched into L2 ahead of a slot's gathers, counted in turns of the
+// slot (a slot takes every other chunk of the CTA).
+constexpr int kPrefetchSlots = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -71,6 +74,9 @@ __device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t two, float sig
 // scale | padding]; the producers widen each latent to bf16 (scale applied) into
 // the same shared-memory tiles the bf16 cache fills, so the MMAs and the softmax
 // are the same for both.
+// One CTA per SM (217 KB of shared memory).  Nine warps spread over the SM's
+// four sub-partitions (three on one of them, whose 16K-register file they
+// share) allow at most 168 registers per thread.
 template <bool kFp8>
 __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a) {
     extern __shared__ uint8_t smem_raw[];
@@ -83,7 +89,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     __shared__ uint64_t q_full, slot_full[2], s_full[2], p_full[2], o_done[2], fin, sm_bar;
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
-    __shared__ int row_idx[2][kChunk];
+    __shared__ int row_idx[2][kChunk];  // [slot][chunk row]: cache row, or -1 (padding)
     __shared__ float alpha_sm[kMlaHeads], m_fin[kMlaHeads], l_fin[kMlaHeads], inv_l[kMlaHeads];
     __shared__ int rescale_w[4];
 
@@ -95,7 +101,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     if (tid == 0) {
         mbar_init(&q_full, 4);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&slot_full[s], 4);
+            mbar_init(&slot_full[s], 2);
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], 4);
             mbar_init(&o_done[s], 1);
@@ -113,10 +119,29 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     __syncthreads();
     tc_fence_after();
     const uint32_t tbase = tmem_base_sh;
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(lp.q) + static_cast<int64_t>(i) * kMlaHeads * kRow;
+    const uint32_t q_addr = smem_u32(q_sm);
+    if (warp >= 4 && warp < 8) {
+        // The query tile is an input of the step, not written by the kernel this
+        // launch depends on: its copy (heads 16*pw .. 16*pw+15 per producer warp)
+        // is issued before the dependency wait.
+        const int pw = warp - 4;
+        for (int hh = 0; hh < 16; ++hh) {
+            const int h = 16 * pw + hh;
+#pragma unroll
+            for (int tt = 0; tt < 3; ++tt) {
+                const int ch = lane + 32 * tt;
+                if (ch < kRow / 8)
+                    cp_async_16(q_addr + (ch >> 3) * kBlockBytes + sw128_offset(h, ch & 7), q + h * kRow + ch * 8);
+            }
+        }
+        cp_async_commit();
+    }
     griddep_wait();
 
+    const int si = i / a.sel_group;  // the selection row this query reads
     int seq = a.q_seq[i];
-    int cnt = a.cnt[i];
+    int cnt = a.cnt[si];
     if (!(seq >= 0 && seq < a.n_seq && cnt >= 0 && cnt <= a.topk)) {
         if (tid == 0) report_status(a.status, DSA_ERR_INVALID);
         cnt = 0;
@@ -127,41 +152,54 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     const int nloc = max(0, min(c_begin + a.chunks_per_cta, nch) - c_begin);
     const __nv_bfloat16 *kv = static_cast<const __nv_bfloat16 *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
     const uint8_t *kv8 = static_cast<const uint8_t *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(lp.q) + static_cast<int64_t>(i) * kMlaHeads * kRow;
-    const uint32_t q_addr = smem_u32(q_sm);
+    const int32_t *sel = a.idx + static_cast<int64_t>(si) * a.topk;
 
     if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ producers
-        const int pw = warp - 4;  // rows (and, once, heads) 16*pw .. 16*pw+15
-        for (int t = 0; t < nloc; ++t) {
-            const int c = c_begin + t, s = t & 1, u = t >> 1;
-            if (t >= 2 && !mbar_wait(&o_done[s], (u - 1) & 1, a.status, &abort_flag)) break;
-            const int rl = 16 * pw + (lane & 15);
+        // Warps 4-5 fill slot 0 (even chunks of this CTA), warps 6-7 slot 1 (odd
+        // chunks), so the two slots fill concurrently; each warp gathers 32 of a
+        // chunk's 64 rows (lane l owns row 32 * half + l).  While gathering a
+        // chunk, each lane prefetches into L2 its row of the chunks this slot
+        // takes kPrefetchSlots turns later, so the gathers after the first read
+        // from L2 instead of waiting on HBM.
+        const int pw = warp - 4;
+        const int p = pw >> 1, half = pw & 1;
+        const int rl = 32 * half + lane;
+        const uint32_t row_bytes = kFp8 ? static_cast<uint32_t>(kFp8Row) : static_cast<uint32_t>(kRow * 2);
+        auto prefetch_chunk = [&](int t2) {
+            if (t2 >= nloc) return;
+            const int j = (c_begin + t2) * kChunk + rl;
+            if (j >= cnt) return;
+            const int r = __ldg(sel + j);
+            if (r < 0 || r >= a.L) return;
+            if constexpr (kFp8)
+                bulk_prefetch_l2(kv8 + static_cast<int64_t>(r) * a.kv_row_stride, row_bytes);
+            else
+                bulk_prefetch_l2(kv + static_cast<int64_t>(r) * a.kv_row_stride, row_bytes);
+        };
+        bool q_arrived = false;
+        for (int t = p; t < nloc; t += 2) {
+            const int c = c_begin + t, u = t >> 1;
+            if (t == p) {
+                for (int k = 1; k <= kPrefetchSlots; ++k) prefetch_chunk(t + 2 * k);
+            } else {
+                prefetch_chunk(t + 2 * kPrefetchSlots);
+            }
+            if (t >= 2 && !mbar_wait(&o_done[p], (u - 1) & 1, a.status, &abort_flag)) break;
             const int j = c * kChunk + rl;
             int r = -1;
             if (j < cnt) {
-                r = a.idx[static_cast<int64_t>(i) * a.topk + j];
+                r = __ldg(sel + j);
                 if (r < 0 || r >= a.L) {
                     report_status(a.status, DSA_ERR_INVALID);
                     r = -1;
                 }
             }
-            if (lane < 16) row_idx[s][rl] = r;
-            if (t == 0) {
-                for (int hh = 0; hh < 16; ++hh) {
-                    const int h = 16 * pw + hh;
-#pragma unroll
-                    for (int tt = 0; tt < 3; ++tt) {
-                        const int ch = lane + 32 * tt;
-                        if (ch < kRow / 8)
-                            cp_async_16(q_addr + (ch >> 3) * kBlockBytes + sw128_offset(h, ch & 7), q + h * kRow + ch * 8);
-                    }
-                }
-            }
-            const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
+            row_idx[p][rl] = r;
+            const uint32_t sb = smem_u32(slot_sm + p * kSlotBytes);
             if constexpr (!kFp8) {
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int row = 16 * pw + rr;
+                for (int rr = 0; rr < 32; ++rr) {
+                    const int row = 32 * half + rr;
                     const int src = __shfl_sync(0xffffffffu, r, rr);
 #pragma unroll
                     for (int tt = 0; tt < 3; ++tt) {
@@ -176,50 +214,64 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                     }
                 }
             } else {
-                // Lane l takes latent dims 16l..16l+15 of each of the warp's 16 rows:
+                // Lane l takes latent dims 16l..16l+15 of each of 16 rows at a time:
                 // all 16 code loads (and scales) are issued before any is widened;
                 // lanes 0-7 copy the row's RoPE key (bf16) straight into block 8.
-                uint4 code[16];
-                float sig[16];
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int src = __shfl_sync(0xffffffffu, r, rr);
-                    code[rr] = make_uint4(0u, 0u, 0u, 0u);
-                    sig[rr] = 0.f;
-                    const uint32_t rope_dst = sb + 8 * kBlockBytes + sw128_offset(16 * pw + rr, lane & 7);
-                    if (src >= 0) {
-                        const uint8_t *row = kv8 + static_cast<int64_t>(src) * a.kv_row_stride;
-                        code[rr] = __ldg(reinterpret_cast<const uint4 *>(row) + lane);
-                        sig[rr] = __ldg(reinterpret_cast<const float *>(row + kFp8ScaleOff));
-                        if (lane < 8) cp_async_16(rope_dst, row + kFp8RopeOff + 16 * lane);
-                    } else if (lane < 8) {
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(rope_dst), "r"(0u) : "memory");
-                    }
-                }
                 const uint32_t blk = sb + (lane >> 2) * kBlockBytes;  // dims 16l.. lie in block l / 4
+#pragma unroll 1
+                for (int rb = 0; rb < 32; rb += 16) {
+                    uint4 code[16];
+                    float sig[16];
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int row = 16 * pw + rr;
-                    const float sg = sig[rr];
-                    const uint32_t w0 = code[rr].x, w1 = code[rr].y, w2 = code[rr].z, w3 = code[rr].w;
-                    const uint32_t lo0 = e4m3x2_scaled_bf16x2(w0 & 0xffffu, sg), lo1 = e4m3x2_scaled_bf16x2(w0 >> 16, sg);
-                    const uint32_t lo2 = e4m3x2_scaled_bf16x2(w1 & 0xffffu, sg), lo3 = e4m3x2_scaled_bf16x2(w1 >> 16, sg);
-                    const uint32_t hi0 = e4m3x2_scaled_bf16x2(w2 & 0xffffu, sg), hi1 = e4m3x2_scaled_bf16x2(w2 >> 16, sg);
-                    const uint32_t hi2 = e4m3x2_scaled_bf16x2(w3 & 0xffffu, sg), hi3 = e4m3x2_scaled_bf16x2(w3 >> 16, sg);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane) & 7)),
-                                 "r"(lo0), "r"(lo1), "r"(lo2), "r"(lo3) : "memory");
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane + 1) & 7)),
-                                 "r"(hi0), "r"(hi1), "r"(hi2), "r"(hi3) : "memory");
+                    for (int rr = 0; rr < 16; ++rr) {
+                        const int src = __shfl_sync(0xffffffffu, r, rb + rr);
+                        code[rr] = make_uint4(0u, 0u, 0u, 0u);
+                        sig[rr] = 0.f;
+                        const uint32_t rope_dst = sb + 8 * kBlockBytes + sw128_offset(32 * half + rb + rr, lane & 7);
+                        if (src >= 0) {
+                            const uint8_t *row = kv8 + static_cast<int64_t>(src) * a.kv_row_stride;
+                            code[rr] = __ldg(reinterpret_cast<const uint4 *>(row) + lane);
+                            sig[rr] = __ldg(reinterpret_cast<const float *>(row + kFp8ScaleOff));
+                            if (lane < 8) cp_async_16(rope_dst, row + kFp8RopeOff + 16 * lane);
+                        } else if (lane < 8) {
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(rope_dst), "r"(0u) : "memory");
+                        }
+                    }
+#pragma unroll
+                    for (int rr = 0; rr < 16; ++rr) {
+                        const int row = 32 * half + rb + rr;
+                        const float sg = sig[rr];
+                        const uint32_t w0 = code[rr].x, w1 = code[rr].y, w2 = code[rr].z, w3 = code[rr].w;
+                        const uint32_t lo0 = e4m3x2_scaled_bf16x2(w0 & 0xffffu, sg), lo1 = e4m3x2_scaled_bf16x2(w0 >> 16, sg);
+                        const uint32_t lo2 = e4m3x2_scaled_bf16x2(w1 & 0xffffu, sg), lo3 = e4m3x2_scaled_bf16x2(w1 >> 16, sg);
+                        const uint32_t hi0 = e4m3x2_scaled_bf16x2(w2 & 0xffffu, sg), hi1 = e4m3x2_scaled_bf16x2(w2 >> 16, sg);
+                        const uint32_t hi2 = e4m3x2_scaled_bf16x2(w3 & 0xffffu, sg), hi3 = e4m3x2_scaled_bf16x2(w3 >> 16, sg);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane) & 7)),
+                                     "r"(lo0), "r"(lo1), "r"(lo2), "r"(lo3) : "memory");
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane + 1) & 7)),
+                                     "r"(hi0), "r"(hi1), "r"(hi2), "r"(hi3) : "memory");
+                    }
                 }
             }
             cp_async_commit();
+            if (!q_arrived) {
+                // the query tile (the older group) has landed: S may start on it
+                cp_async_wait_group<1>();
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&q_full);
+                q_arrived = true;
+            }
             cp_async_wait_all();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                if (t == 0) mbar_arrive(&q_full);
-                mbar_arrive(&slot_full[s]);
-            }
+            if (lane == 0) mbar_arrive(&slot_full[p]);
+        }
+        if (!q_arrived) {  // no chunk for this slot (or an abort): the query tile still counts
+            cp_async_wait_all();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_full);
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
@@ -448,7 +500,7 @@ __global__ void __launch_bounds__(256) mla_combine_kernel(const MlaArgs a) {
     const MlaLayerPtrs lp = a.layer[layer];
     __shared__ float wgt[kCombineHeads][32];
     griddep_wait();  // splits per query: at most 32 by the planner
-    int cnt = a.cnt[i];
+    int cnt = a.cnt[i / a.sel_group];
     if (cnt < 0 || cnt > a.topk) cnt = 0;
     const int nch = (cnt + kChunk - 1) / kChunk;
     const int ns = min(32, (nch + a.chunks_per_cta - 1) / a.chunks_per_cta);
@@ -547,7 +599,7 @@ __global__ void __launch_bounds__(128) mla_generic_kernel(const MlaArgs a) {
     for (int d = threadIdx.x; d < dk; d += blockDim.x) qs[d] = ld_f<T>(q + d);
     if (threadIdx.x == 0) bad = 0;
     int seq = a.q_seq[i];
-    int cnt = a.cnt[i];
+    int cnt = a.cnt[i / a.sel_group];
     if (seq < 0 || seq >= a.n_seq || cnt < 0 || cnt > a.topk) {
         if (threadIdx.x == 0 && h == 0) report_status(a.status, DSA_ERR_INVALID);
         seq = 0;
@@ -555,7 +607,7 @@ __global__ void __launch_bounds__(128) mla_generic_kernel(const MlaArgs a) {
     }
     __syncthreads();
     const T *kv = static_cast<const T *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
-    const int32_t *sel = a.idx + static_cast<int64_t>(i) * a.topk;
+    const int32_t *sel = a.idx + static_cast<int64_t>(i / a.sel_group) * a.topk;
     float m = -INFINITY;
     for (int j = threadIdx.x; j < cnt; j += blockDim.x) {
         const int r = sel[j];

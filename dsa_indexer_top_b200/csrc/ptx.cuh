@@ -136,6 +136,14 @@ __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     return pol;
 }
 
+// L2 policy for data every CTA re-reads (keys shared by all query groups of a
+// prefill chunk): evict last.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
 __device__ __forceinline__ void tma_load_3d_hint(void *dst, const void *map, uint64_t *bar, int x, int y, int z,
                                                  uint64_t policy) {
     asm volatile(
@@ -145,12 +153,21 @@ __device__ __forceinline__ void tma_load_3d_hint(void *dst, const void *map, uin
         : "memory");
 }
 
+// Bring `bytes` (a multiple of 16, 16-byte aligned source) into L2 ahead of
+// use; no completion to wait for.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // ----------------------------------------------------------------- cp.async (16 B)
 __device__ __forceinline__ void cp_async_16(uint32_t dst_smem, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst_smem), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still pending.
+template <int N>
+__device__ __forceinline__ void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 // Make this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tensor cores, TMA) -- needed before an MMA reads data written by

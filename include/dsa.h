@@ -117,7 +117,8 @@ typedef enum {
     DSA_OP_TOPK = 1,
     DSA_OP_MLA_DECODE = 2,
     DSA_OP_MLA_PREFILL = 3,
-    DSA_OP_INDEXSHARE_GROUP = 4
+    DSA_OP_INDEXSHARE_GROUP = 4,
+    DSA_OP_SHARD_MERGE = 5 /* dsa_shard_merge; dsa_workspace_bytes' last argument = shards */
 } dsa_op;
 
 /*
@@ -279,30 +280,67 @@ dsa_status dsa_sparse_mla_prefill(const dsa_queries *queries, const dsa_mla *mla
                                   size_t ws_bytes, void *stream);
 
 /*
+ * Sparse absorbed MLA for a multi-token-prediction (speculative) iteration
+ * [LA, raw config.json fields: index_share_for_mtp_iteration = true -- the
+ * tokens of an MTP iteration share the index selection instead of scoring
+ * again; HA, "78 layers, IndexShare pattern": one Multi-Token Prediction layer
+ * next to the 78].  The pages give only the flag; the reading here: the n_q
+ * queries come in groups of `draft_tokens` consecutive queries of one
+ * sequence, and every query of group g attends over the one selection
+ * idx[g*topk + 0..cnt[g]-1] -- exactly dsa_sparse_mla_decode with the selection
+ * row repeated for each query of the group.  The selection was made for a
+ * position no later than any query of the group, so it is causal for all of
+ * them.
+ *   idx        int32 [n_q / draft_tokens][topk];  cnt  int32 [n_q / draft_tokens]
+ *   draft_tokens  >= 1 and dividing n_q (else DSA_ERR_INVALID)
+ *   ws         dsa_workspace_bytes(DSA_OP_MLA_DECODE, queries, topk, ...) bytes
+ * The decode (split-K) schedule runs up to 256 queries, the prefill schedule
+ * above.  The queries of a group gather the same rows, so their CTAs read them
+ * from L2 after the first.
+ */
+dsa_status dsa_sparse_mla_mtp(const dsa_queries *queries, const dsa_mla *mla, const int32_t *idx,
+                              const int32_t *cnt, int32_t topk, int32_t draft_tokens, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/*
  * dsa_sparse_mla_decode without a workspace.  The pages have no counterpart to
  * this call: it exists for callers that cannot allocate device memory where
  * they run attention (a runtime or plugin that hands over only its input and
  * output tensors, or memory that was planned and fixed up front), so they have
- * no workspace to pass.  Same arguments and result as dsa_sparse_mla_decode
- * (tensor-core shape only: bf16 queries and outputs, 64 heads, 512 + 64, a bf16
- * or packed FP8 cache; other shapes return DSA_ERR_UNSUPPORTED), minus `ws`.
+ * no workspace to pass.  Same arguments, checks and result as
+ * dsa_sparse_mla_decode (tensor-core shape only: bf16 queries and outputs, 64
+ * heads, 512 + 64, a bf16 or packed FP8 cache; other shapes return
+ * DSA_ERR_UNSUPPORTED), minus `ws`.
  *  - Scratch: a fixed 32 MiB device array inside the library (status word +
  *    split-K partials), held by every GPU that loads the library until the
- *    process exits.  Calls that need more -- 256 + ceil(topk/128) * n_q *
- *    131,584 bytes, e.g. more than 15 queries at topk = 2048 -- are rejected
- *    with DSA_ERR_WORKSPACE before any launch.
- *  - Set-up: the first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before any stream capture.
+ *    process exits.  A call needs 256 + n_q * splits * 131,584 bytes, where
+ *    splits is the decode plan's split count (at most SMs / n_q, 1 for 75 or
+ *    more queries on 148 SMs, and no partials at all with one split): at most
+ *    about 19.5 MB on a B200.  A call whose plan needs more than the array (a
+ *    GPU with more than 255 SMs) is rejected with DSA_ERR_WORKSPACE before any
+ *    launch.
+ *  - Set-up: each call made outside stream capture looks up the array's device
+ *    address (cudaGetSymbolAddress) with the current device; calls made while
+ *    the stream is capturing reuse the address looked up last on that device,
+ *    so make one call on each device before capturing it.
  *  - Every call on a device shares the one array, so calls that overlap on the
  *    GPU (other streams, other host threads) race; serialise them.
- *  - Device-side checks (indices out of range) are applied -- such rows are
- *    skipped -- but not reported: there is no workspace status word to read.
+ *  - Device-detected errors (an index or count out of range, a bounded wait
+ *    that ran out) go to the array's status word, which keeps the first error
+ *    until dsa_noalloc_check_status reads and clears it.
  *  - Allocates nothing: no cudaMalloc/cudaFree, no allocating library call.
  */
 dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, const dsa_mla *mla,
                                          const int32_t *idx, const int32_t *cnt, int32_t topk,
                                          void *stream);
+
+/*
+ * Status of the dsa_sparse_mla_decode_noalloc calls made on the current device
+ * (no counterpart on the pages): synchronises `stream`, reads the status word of
+ * the library's fixed scratch array, clears it, and returns it (DSA_OK when no
+ * kernel reported an error since the last read).  Allocates nothing.
+ */
+dsa_status dsa_noalloc_check_status(void *stream);
 
 /*
  * IndexShare group [HA, MLA + DSA with IndexShare]: layer 0 (the full layer)
@@ -319,6 +357,150 @@ dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *i
                                 const dsa_mla *layers, int32_t n_layers, int32_t topk,
                                 int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
                                 void *stream);
+
+/*
+ * Key-range sharding of one long sequence over several GPUs.  The pages name
+ * attention data parallelism only ["GLM-5.2 -- Model techniques map",
+ * inference & serving]; splitting one sequence's cache by contiguous key
+ * ranges is this library's reading of how a 1M-token context
+ * ["GLM 5.2 -- Hermosa AI", "MLA + DSA with IndexShare": 1,048,576 tokens]
+ * spreads over GPUs, and it computes exactly the single-GPU result:
+ *   rank g holds rows [row_begin_g, row_end_g) of the sequence (contiguous,
+ *   in rank order) and, per query:
+ *   1. dsa_index_scores + dsa_topk on its shard (positions shard-relative);
+ *   2. dsa_shard_candidates: its <= topk (score, position) candidates;
+ *   3. an all-gather of every rank's candidates (the caller's collective);
+ *   4. dsa_shard_merge: the global selection (the top-k of all candidates,
+ *      ties to the lower position) and this rank's part of it;
+ *   5. dsa_sparse_mla_decode on its shard with that part;
+ *   6. an all-gather of the ranks' outputs, lse and part counts;
+ *   7. dsa_shard_combine: the log-sum-exp merge of the ranks' attentions.
+ * A row of the global top-k that lies in shard g is among shard g's top-k (its
+ * rank inside the shard is no worse than its global rank), so step 4 sees
+ * every row it needs.  Every query must see at least one row of every shard
+ * (decode at the end of the sequence).
+ */
+
+/*
+ * Step 2: candidates of this rank's local selection.
+ *   scores, ld_scores  the local scores (queries->max_ctx = shard rows)
+ *   idx, cnt           the local top-k (shard-relative, ascending, -1 padded)
+ *   row_offset         the shard's first row in the sequence
+ *   cand_score         float32 [n_q][topk]: the selected rows' scores, 0 after cnt
+ *   cand_pos           int32 [n_q][topk]: their sequence positions, -1 after cnt
+ *   ws                 at least 256 bytes (status word)
+ */
+dsa_status dsa_shard_candidates(const dsa_queries *queries, const float *scores, int64_t ld_scores,
+                                const int32_t *idx, const int32_t *cnt, int32_t topk, int32_t row_offset,
+                                float *cand_score, int32_t *cand_pos, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Step 4: merge of the gathered candidates (n_shards ranks, rank order).
+ *   cand_score, cand_pos  [n_shards][n_q][topk] as gathered from step 2
+ *   idx, cnt              the global selection: sequence positions, ascending,
+ *                         -1 padded; cnt = min(topk, candidates)
+ *   row_begin, row_end    this rank's rows
+ *   local_idx, local_cnt  [n_q][topk], [n_q]: the selected rows in
+ *                         [row_begin, row_end), shard-relative, ascending,
+ *                         -1 padded (the selection step 5 attends over)
+ *   ws                    dsa_workspace_bytes(DSA_OP_SHARD_MERGE, queries, topk,
+ *                         0, 0, n_shards) bytes, initialised once
+ */
+dsa_status dsa_shard_merge(const dsa_queries *queries, int32_t n_shards, const float *cand_score,
+                           const int32_t *cand_pos, int32_t topk, int32_t row_begin, int32_t row_end, int32_t *idx,
+                           int32_t *cnt, int32_t *local_idx, int32_t *local_cnt, void *ws, size_t ws_bytes,
+                           void *stream);
+
+/*
+ * Step 7: o = sum_g exp(lse_g - lse) o_g, lse = log sum_g exp(lse_g), over the
+ * parts g with part_cnt[g][i] > 0 (the others are ignored, whatever their
+ * out/lse hold).
+ *   part_out   bf16 [n_parts][n_q][heads][d_latent] (8-byte aligned)
+ *   part_lse   float32 [n_parts][n_q][heads];  part_cnt  int32 [n_parts][n_q]
+ *   out        bf16 [n_q][heads][d_latent];  lse  float32 [n_q][heads] or NULL
+ *   heads even, d_latent a multiple of 4 up to 512 (else DSA_ERR_UNSUPPORTED)
+ */
+dsa_status dsa_shard_combine(const dsa_queries *queries, int32_t n_parts, int32_t heads, int32_t d_latent,
+                             const void *part_out, const float *part_lse, const int32_t *part_cnt, void *out,
+                             float *lse, void *stream);
+
+/*
+ * Producers around the path (GLM-5.2 shapes only: latent 512, RoPE key 64,
+ * indexer key 128, no-RoPE query part 192, value 256) ["GLM-5.2 -- Model
+ * techniques map", "Checked in its code": Multi-head latent attention --
+ * kv_a_proj_with_mqa maps the hidden state to the 512-dim latent plus the
+ * 64-dim RoPE key, kv_a_layernorm (RMSNorm) normalises the latent, kv_b_proj
+ * holds per head a 192-dim no-RoPE key part (W_UK) and a 256-dim value (W_UV);
+ * QK normalization -- the indexer key is k_norm(wk(h)), k_norm a LayerNorm;
+ * Partial RoPE; "GLM 5.2 -- Hermosa AI", "MLA + DSA with IndexShare": RoPE
+ * theta 8e6; "GLM-5.2 -- LLM atlas", raw config.json fields: rope_interleave
+ * and indexer_rope_interleave true, rms_norm_eps].  Readings where the pages
+ * are silent: RoPE turns adjacent pairs (x[2i], x[2i+1]) of a 64-wide RoPE part
+ * by pos * theta^(-2i/64); the indexer key's RoPE part is its last 64 dims;
+ * LayerNorm has a weight and a bias, RMSNorm a weight.  Dense contractions run
+ * on tcgen05 tensor cores (bf16 operands, fp32 sums), bf16 results.
+ */
+
+/* One batch of tokens whose cache rows are written. */
+typedef struct {
+    int32_t n_tok;            /* tokens (>= 0) */
+    int32_t hidden;           /* hidden size (6144 for GLM-5.2), a multiple of 8, >= 64 */
+    const void *h;            /* bf16 [n_tok][hidden] hidden states, row stride h_row_stride
+                                 (elements, multiple of 8), 16-byte aligned */
+    int64_t h_row_stride;
+    const void *w;            /* bf16 [704][hidden] weights in the [out][in] layout: rows 0..511
+                                 the latent and 512..575 the RoPE key (kv_a_proj_with_mqa), rows
+                                 576..703 the indexer key (wk); 16-byte aligned */
+    const float *rms_weight;  /* [512] kv_a_layernorm weight */
+    const float *ln_weight;   /* [128] k_norm weight */
+    const float *ln_bias;     /* [128] k_norm bias */
+    const int32_t *tok_seq;   /* device [n_tok]: sequence of each token, in [0, n_seq) */
+    const int32_t *tok_pos;   /* device [n_tok]: its position = its cache row and RoPE position */
+    int32_t n_seq, max_ctx;
+    void *kv;                 /* bf16 latent cache [c | r] (the layout dsa_mla reads), or NULL */
+    int64_t kv_seq_stride, kv_row_stride;     /* elements */
+    void *k_idx;              /* bf16 indexer-key cache [128] rows, or NULL (not both NULL) */
+    int64_t k_seq_stride, k_row_stride;       /* elements */
+    float eps;                /* 1e-5 for GLM-5.2 (rms_norm_eps; also the LayerNorm's) */
+    float rope_theta;         /* 8e6 for GLM-5.2 */
+} dsa_cache_writer;
+
+/*
+ * Cache rows of a batch of tokens: y = h . W^T (704 outputs per token), then
+ *   kv[seq][pos]    = [ RMSNorm(y[0:512]) * rms_weight | RoPE(y[512:576], pos) ]
+ *   k_idx[seq][pos] = LayerNorm(y[576:704]) * ln_weight + ln_bias, its last 64
+ *                     dims turned by RoPE(pos)
+ *   ws   dsa_cache_writer_workspace_bytes(n_tok, hidden) bytes, 256-byte aligned
+ *        (status word + split-K partials of y)
+ * Out-of-range tok_seq / tok_pos skip the token and set DSA_ERR_INVALID in the
+ * workspace status word.
+ */
+dsa_status dsa_write_cache_rows(const dsa_cache_writer *writer, void *ws, size_t ws_bytes, void *stream);
+size_t dsa_cache_writer_workspace_bytes(int32_t n_tok, int32_t hidden);
+
+/*
+ * Absorbed MLA queries: per query i and head h
+ *   q_out[i][h][0:512]   = W_UK[h]^T q_nope[i][h]      (the no-RoPE key up-projection
+ *                                                      folded into the query)
+ *   q_out[i][h][512:576] = RoPE(q_rope[i][h], pos[i])
+ *   q_nope  bf16 [n_q][heads][192];  q_rope  bf16 [n_q][heads][64] (before RoPE)
+ *   w_uk_t  bf16 [heads][512][192]: W_UK[h] transposed (row j holds the weights
+ *           of latent dim j), the K-major layout the tensor cores read
+ *   pos     device int32 [n_q];  q_out  bf16 [n_q][heads][576] (the dsa_mla query)
+ *   ws      at least 256 bytes (status word)
+ */
+dsa_status dsa_absorb_queries(int32_t n_q, int32_t heads, const void *q_nope, const void *q_rope, const void *w_uk_t,
+                              const int32_t *pos, float rope_theta, void *q_out, void *ws, size_t ws_bytes,
+                              void *stream);
+
+/*
+ * Value up-projection of the absorbed attention output: per query i and head h
+ *   out[i][h][0:256] = W_UV[h] o_lat[i][h]
+ *   o_lat  bf16 [n_q][heads][512] (dsa_mla's out);  w_uv  bf16 [heads][256][512]
+ *   out    bf16 [n_q][heads][256];  ws  at least 256 bytes (status word)
+ */
+dsa_status dsa_up_project(int32_t n_q, int32_t heads, const void *o_lat, const void *w_uv, void *out, void *ws,
+                          size_t ws_bytes, void *stream);
 
 /*
  * Upper bound of the workspace bytes an operation needs (host only).

@@ -246,3 +246,58 @@ def test_mla_kv_dtype_same_as_dtype_is_accepted_by_validation():
     m.dtype = m.kv_dtype = B.DSA_F32
     assert lib.dsa_sparse_mla_prefill(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, _FakeWs.ptr, 128,
                                       None) == B.DSA_ERR_WORKSPACE
+
+
+def test_mtp_rejects_bad_group_size():
+    lib = B.lib()
+    q = _q(n_q=6)
+    m = _mla()
+    for d in (0, -1, 4):  # 4 does not divide 6
+        assert lib.dsa_sparse_mla_mtp(ctypes.byref(q), ctypes.byref(m), 0xA000, 0xB000, 2048, d, _FakeWs.ptr,
+                                      _FakeWs.size, None) == B.DSA_ERR_INVALID
+
+
+def test_shard_calls_validate():
+    lib = B.lib()
+    q = _q(n_q=2, L=5000)
+    P = 0xC000
+    # merge: shard count, ranges, workspace
+    assert lib.dsa_shard_merge(ctypes.byref(q), 0, P, P, 2048, 0, 10, P, P, P, P, _FakeWs.ptr, _FakeWs.size,
+                               None) == B.DSA_ERR_INVALID
+    assert lib.dsa_shard_merge(ctypes.byref(q), 65, P, P, 2048, 0, 10, P, P, P, P, _FakeWs.ptr, _FakeWs.size,
+                               None) == B.DSA_ERR_INVALID
+    assert lib.dsa_shard_merge(ctypes.byref(q), 2, P, P, 2048, 10, 5, P, P, P, P, _FakeWs.ptr, _FakeWs.size,
+                               None) == B.DSA_ERR_INVALID
+    need = lib.dsa_workspace_bytes(B.DSA_OP_SHARD_MERGE, ctypes.byref(q), 2048, 0, 0, 4)
+    # status + merged scores and positions (4 shards x 2048 per query) + counts + the
+    # merged top-k (indices, counts) + the top-k scratch of 8192-wide rows
+    assert need > 256 + 2 * (2 * 4 * 2048 * 4) + 2 * 2048 * 4
+    assert lib.dsa_shard_merge(ctypes.byref(q), 4, P, P, 2048, 0, 10, P, P, P, P, _FakeWs.ptr, need - 1,
+                               None) == B.DSA_ERR_WORKSPACE
+    # candidates: null outputs; combine: shapes the kernel does not cover
+    assert lib.dsa_shard_candidates(ctypes.byref(q), P, 5000, P, P, 2048, 0, None, P, _FakeWs.ptr, _FakeWs.size,
+                                    None) == B.DSA_ERR_INVALID
+    assert lib.dsa_shard_combine(ctypes.byref(q), 2, 63, 512, P, P, P, P, None, None) == B.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_shard_combine(ctypes.byref(q), 2, 64, 1024, P, P, P, P, None, None) == B.DSA_ERR_UNSUPPORTED
+    assert lib.dsa_shard_combine(ctypes.byref(q), 0, 64, 512, P, P, P, P, None, None) == B.DSA_ERR_INVALID
+
+
+def test_producer_calls_validate():
+    lib = B.lib()
+    P = 0xD000
+    w = B._CacheWriter(4, 6144, P, 6144, P, P, P, P, P, P, 2, 1000, P, 1000 * 576, 576, P, 1000 * 128, 128,
+                       1e-5, 8e6)
+    need = lib.dsa_cache_writer_workspace_bytes(4, 6144)
+    # 4 tokens: one M tile x 6 N tiles, split 24 ways along K (4 blocks of 64 each)
+    assert need == 256 + ((24 * 4 * 704 * 4 + 255) // 256) * 256
+    assert lib.dsa_write_cache_rows(ctypes.byref(w), _FakeWs.ptr, need - 1, None) == B.DSA_ERR_WORKSPACE
+    bad = B._CacheWriter(4, 6144, P, 6144, None, P, P, P, P, P, 2, 1000, P, 1000 * 576, 576, P, 1000 * 128, 128,
+                         1e-5, 8e6)
+    assert lib.dsa_write_cache_rows(ctypes.byref(bad), _FakeWs.ptr, need, None) == B.DSA_ERR_INVALID
+    odd = B._CacheWriter(4, 6100, P, 6100, P, P, P, P, P, P, 2, 1000, P, 1000 * 576, 576, P, 1000 * 128, 128,
+                         1e-5, 8e6)
+    assert lib.dsa_write_cache_rows(ctypes.byref(odd), _FakeWs.ptr, need, None) == B.DSA_ERR_INVALID
+    assert lib.dsa_absorb_queries(4, 64, P, P, None, P, 8e6, P, _FakeWs.ptr, 256, None) == B.DSA_ERR_INVALID
+    assert lib.dsa_absorb_queries(4, 64, P, P, P, P, 8e6, P, _FakeWs.ptr, 128, None) == B.DSA_ERR_WORKSPACE
+    assert lib.dsa_up_project(4, 64, P, P, None, _FakeWs.ptr, 256, None) == B.DSA_ERR_INVALID
+    assert lib.dsa_up_project(0, 64, P, P, P, _FakeWs.ptr, 256, None) == B.DSA_OK

@@ -1,8 +1,10 @@
 """Parity at the five named workloads' full sizes, in the call sequence the
 benchmark times (dsa_index_scores -> dsa_topk -> sparse MLA per layer, decode
 schedule up to 256 queries, prefill schedule above).  The GPU runs the whole
-batch; the oracle recomputes sampled queries one by one (scores bit-exact over
-every visible key, indices bit-exact, attention within tolerance)."""
+batch; the oracle recomputes every query of the decode workloads and, for the
+prefill chunk, every 16th query plus the first and the last 64 (scores
+bit-exact over every visible key, indices bit-exact, attention within
+tolerance)."""
 import numpy as np
 import pytest
 import torch
@@ -14,13 +16,69 @@ from tests import common as C
 
 pytestmark = pytest.mark.gpu
 
+def _prefill_sample(n_q):
+    """Every 16th query plus the first and the last 64."""
+    return sorted(set(range(0, n_q, 16)) | set(range(64)) | set(range(n_q - 64, n_q)))
+
+
 SAMPLES = {
     "tiny": None,                       # every query
     "decode_32k": None,
-    "prefill_64k": [0, 1, 2047, 4095],
-    "indexshare_128k": [0, 31],
-    "decode_1m": [2],
+    "prefill_64k": _prefill_sample(4096),
+    "indexshare_128k": None,            # all 32 queries, every layer
+    "decode_1m": None,                  # all 4 queries
 }
+
+
+def check_rows(w, x, rows, scores, idx, cnt, mlas, kv8=None):
+    """Oracle checks of the queries in `rows`, batched per sequence (the oracle
+    spreads (query, key) pairs and (query, head) pairs over the host's cores):
+    scores bit-exact over every visible key, indices and counts bit-exact, and
+    every layer's attention (over the oracle's own selection) within tolerance."""
+    rows = np.asarray(rows)
+    q_seq = np.asarray(w.q_seq)[rows]
+    q_pos = np.asarray(w.q_pos)[rows]
+    seqs = [0] if w.shared_cache else sorted(set(q_seq.tolist()))
+    got_idx = idx.cpu().numpy()
+    got_cnt = cnt.cpu().numpy()
+    batches = []
+    for b in seqs:
+        in_seq = rows if w.shared_cache else rows[q_seq == b]
+        batches += [(b, in_seq[j: j + 64]) for j in range(0, len(in_seq), 64)]  # bounded host memory
+    for b, sel_rows in batches:
+        pos = np.asarray(w.q_pos)[sel_rows]
+        k_h = x["k_idx"][b].cpu().float().numpy()[None]
+        sc = oracle.index_scores(C.host_f32(x["q_idx"][sel_rows]), C.host_f32(x["w"][sel_rows]), k_h,
+                                 np.zeros(len(sel_rows), np.int32), pos)
+        del k_h
+        if scores is not None:
+            got_sc = scores[torch.from_numpy(sel_rows)].cpu().double().numpy()
+            for j, i in enumerate(sel_rows):
+                t = pos[j]
+                np.testing.assert_array_equal(got_sc[j, : t + 1], sc[j, : t + 1], err_msg=f"scores of query {i}")
+        ridx, rcnt = oracle.topk(sc, pos, w.topk)
+        del sc
+        np.testing.assert_array_equal(got_idx[sel_rows], ridx, err_msg=f"indices of sequence {b}")
+        np.testing.assert_array_equal(got_cnt[sel_rows], rcnt)
+        # attention over the selected rows only: [n, topk, row] gathered per query
+        gidx = torch.from_numpy(np.where(ridx >= 0, ridx, 0).astype(np.int64))
+        local = np.where(np.arange(w.topk)[None, :] < rcnt[:, None], np.arange(w.topk)[None, :], -1).astype(np.int32)
+        for layer, m in enumerate(mlas):
+            qm = C.host_f32(x["q_mla"][layer][sel_rows])
+            if kv8 is None:
+                cache = x["kv"][layer][b]
+                rows_h = cache[gidx.to(cache.device)].cpu().float().numpy()
+                out, lse = oracle.sparse_mla(qm, rows_h, np.arange(len(sel_rows), dtype=np.int32), local, rcnt,
+                                             w.d_lat, w.scale)
+            else:
+                cache = kv8[layer][b]
+                rows_h = cache[gidx.to(cache.device)].cpu().numpy()
+                out, lse = oracle.sparse_mla_fp8(qm, rows_h, np.arange(len(sel_rows), dtype=np.int32), local, rcnt,
+                                                 w.d_lat, w.d_rope, w.scale)
+            sr = torch.from_numpy(sel_rows)
+            C.assert_attention_close(m.out[sr], out, "bf16" if kv8 is not None else w.dtype,
+                                     f"sequence {b} layer {layer}")
+            C.assert_lse_close(m.lse[sr], lse, "bf16" if kv8 is not None else w.dtype)
 
 
 @pytest.mark.parametrize("name", wl.NAMED_ORDER)
@@ -41,25 +99,27 @@ def test_named_workload_full_size(cuda_ok, name):
     for m in mlas:
         mla(q, m, idx, cnt, w.topk, ws)
     assert B.dsa_check_status(ws) == B.DSA_OK
-
     rows = list(range(w.n_q)) if SAMPLES[name] is None else SAMPLES[name]
-    for i in rows:
-        b = 0 if w.shared_cache else w.q_seq[i]
-        t = w.q_pos[i]
-        k_h = x["k_idx"][b].cpu().float().numpy()[None]
-        sc = oracle.index_scores(C.host_f32(x["q_idx"][i:i + 1]), C.host_f32(x["w"][i:i + 1]), k_h, [0], [t])
-        got_sc = scores[i, : t + 1].cpu().double().numpy()
-        np.testing.assert_array_equal(got_sc, sc[0, : t + 1], err_msg=f"scores of query {i}")
-        ridx, rcnt = oracle.topk(sc, [t], w.topk)
-        np.testing.assert_array_equal(idx[i].cpu().numpy(), ridx[0], err_msg=f"indices of query {i}")
-        assert int(cnt[i]) == int(rcnt[0])
-        sel = ridx[0, : rcnt[0]]
-        for layer, m in enumerate(mlas):
-            kv_rows = x["kv"][layer][b].cpu()[torch.from_numpy(sel.astype(np.int64))].float().numpy()[None]
-            out, lse = oracle.sparse_mla(C.host_f32(x["q_mla"][layer][i:i + 1]), kv_rows, [0],
-                                         np.arange(len(sel), dtype=np.int32)[None], rcnt, w.d_lat, w.scale)
-            C.assert_attention_close(m.out[i:i + 1], out, w.dtype, f"query {i} layer {layer}")
-            C.assert_lse_close(m.lse[i:i + 1], lse, w.dtype)
+    check_rows(w, x, rows, scores, idx, cnt, mlas)
+
+
+@pytest.mark.parametrize("name", wl.NAMED_ORDER)
+def test_named_workload_group_call_full_size(cuda_ok, name):
+    """The same workloads through the one-call entry point the benchmark times
+    (dsa_indexshare_group: scores in the workspace, decode schedule up to 256
+    queries, prefill above): indices and attention against the oracle."""
+    w = wl.NAMED[name]
+    dev = torch.device("cuda")
+    x = wl.make_inputs(w, device=dev)
+    seq_run = w.n_q if len(set(w.q_seq)) == 1 else 1
+    q, ix, mlas = C.descriptors(w, x, seq_run=seq_run)
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, w.n_layers, dev)
+    idx = torch.empty((w.n_q, w.topk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.n_q,), dtype=torch.int32, device=dev)
+    B.dsa_indexshare_group(q, ix, mlas, w.topk, idx, cnt, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    rows = list(range(w.n_q)) if SAMPLES[name] is None else SAMPLES[name][::4]
+    check_rows(w, x, rows, None, idx, cnt, mlas)
 
 
 @pytest.mark.parametrize("name", ["decode_32k", "decode_1m"])
@@ -114,17 +174,4 @@ def test_fp8_latent_cache_full_size(cuda_ok, name):
     for m in mlas:
         B.dsa_sparse_mla_decode(q, m, idx, cnt, w.topk, ws)
     assert B.dsa_check_status(ws) == B.DSA_OK
-    for i in SAMPLES[name]:
-        b, t = w.q_seq[i], w.q_pos[i]
-        k_h = x["k_idx"][b].cpu().float().numpy()[None]
-        sc = oracle.index_scores(C.host_f32(x["q_idx"][i:i + 1]), C.host_f32(x["w"][i:i + 1]), k_h, [0], [t])
-        ridx, rcnt = oracle.topk(sc, [t], w.topk)
-        np.testing.assert_array_equal(idx[i].cpu().numpy(), ridx[0], err_msg=f"indices of query {i}")
-        sel = torch.from_numpy(ridx[0, : rcnt[0]].astype(np.int64))
-        for layer, m in enumerate(mlas):
-            rows = kv8[layer][b].cpu()[sel].numpy()[None]            # the selected packed rows only
-            out, lse = oracle.sparse_mla_fp8(C.host_f32(x["q_mla"][layer][i:i + 1]), rows, [0],
-                                             np.arange(len(sel), dtype=np.int32)[None], rcnt, w.d_lat, w.d_rope,
-                                             w.scale)
-            C.assert_attention_close(m.out[i:i + 1], out, "bf16", f"query {i} layer {layer}")
-            C.assert_lse_close(m.lse[i:i + 1], lse, "bf16")
+    check_rows(w, x, list(range(w.n_q)), scores, idx, cnt, mlas, kv8=kv8)
