@@ -4,8 +4,9 @@ One step = one pass of the whole path over one batch of synthetic inputs already
 resident in HBM, made by ONE call of the public C ABI: dsa_indexshare_group
 (indexer -> top-k -> sparse MLA of every layer of the workload; with one layer it
 is the plain full-layer step).  The step is captured once in a CUDA graph with
-CUDA events at its two ends; L2 is flushed (256 MB write) before every timed
-step.  A second graph made of the separate calls (dsa_index_scores, dsa_topk,
+CUDA events at its two ends; L2 is flushed before every timed step (a 256 MB
+write, then a 256 MB read, so that no dirty line is written back inside the
+timed region).  A second graph made of the separate calls (dsa_index_scores, dsa_topk,
 dsa_sparse_mla_*) with events between them gives the per-stage breakdown and the
 per-kernel rooflines.  After timing, the results of the timed graph are compared
 bitwise with one eager step on a freshly initialised workspace and with the
@@ -51,6 +52,21 @@ UNIT = "qtok/s/layer"
 ROOT = os.path.dirname(os.path.abspath(__file__))
 DECODE_MAX_QUERIES = 256    # the group call's MLA uses the decode (split-K) schedule up to this many queries
 L2_FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Before every timed step: write a 256 MB buffer (evicts everything the
+    previous step left in the 126 MB L2), then read a second 256 MB buffer, so the
+    dirty lines of the write are written back here, outside the timed region, and
+    the step starts with an L2 of clean lines that hold none of its data."""
+
+    def __init__(self, dev):
+        self.w = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.zeros(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+
+    def fill_(self, v):
+        self.w.fill_(v)
+        self.r.amax()
 REFERENCE_BUDGET_S = 120.0  # timed oracle work of one --impl reference run
 HEADLINE = "decode_1m"
 # the other workloads reported inside the headline line, with the FP8 variants
@@ -475,7 +491,7 @@ def barrier(world):
 
 def config_of(w: wl.Workload, world: int, fp8: bool = False) -> dict:
     c = {**w.describe(), "parallelism": f"dp{world} (independent batches per GPU)",
-         "l2": "flushed before every timed step (256 MB write)", "graph": "CUDA graph per step",
+         "l2": "flushed before every timed step (256 MB write, then a 256 MB read so the step starts with clean lines)", "graph": "CUDA graph per step",
          "entry_point": "dsa_indexshare_group"}
     if fp8:
         c["indexer_dtype"] = "e4m3 + per-row fp32 scales (FP8 variant)"
@@ -599,6 +615,73 @@ def e2e_measure(step: Step, world: int, dev, flush, steps: int):
             "how": "eager each step: pinned H2D of the query inputs, dsa_indexshare_group, D2H of outputs + indices"}
 
 
+def producers_measure(dev, flush, steps: int, hbm_peak: float, tc_peak: float, peak_kind: str) -> dict:
+    """The producers around the path at GLM-5.2 shapes (hidden 6144, 64 heads), decode-sized (4 tokens)
+    and prefill-sized (4096 tokens) batches: cache-row writer, query absorption, value up-projection.
+    Each timed with CUDA events (L2 flushed before every launch) against its bound: the weights' HBM
+    bytes for decode sizes, the GEMM FLOPs at the bf16 tensor peak for prefill sizes."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    H, hidden = 64, 6144
+    out = {}
+
+    def timed(fn):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        fn()
+        torch.cuda.synchronize()
+        tot = 0.0
+        for _ in range(steps):
+            flush.fill_(1)
+            ev[0].record()
+            fn()
+            ev[1].record()
+            torch.cuda.synchronize()
+            tot += ev[0].elapsed_time(ev[1])
+        return tot / steps * 1e3  # us
+
+    def entry(us, weight_bytes, io_bytes, flops, prefill):
+        gbs = (weight_bytes + io_bytes) / (us * 1e-6) / 1e9
+        tf = flops / (us * 1e-6) / 1e12
+        e = {"us": us, "bytes": weight_bytes + io_bytes, "flops": flops, "achieved_gbs": gbs,
+             "achieved_tflops": tf}
+        if prefill:
+            e.update({"bound": "tensor", "frac": tf / tc_peak, "peak_kind": f"{peak_kind} bf16_tflops (burst)"})
+        else:
+            e.update({"bound": "hbm", "frac": gbs / hbm_peak, "peak_kind": f"{peak_kind} hbm_gbs"})
+        return e
+
+    w_cache = (torch.randn((704, hidden), generator=g, device=dev) / hidden ** 0.5).to(torch.bfloat16)
+    rms = torch.ones(512, device=dev)
+    lnw, lnb = torch.ones(128, device=dev), torch.zeros(128, device=dev)
+    w_uk_t = (torch.randn((H, 512, 192), generator=g, device=dev) / 192 ** 0.5).to(torch.bfloat16)
+    w_uv = (torch.randn((H, 256, 512), generator=g, device=dev) / 512 ** 0.5).to(torch.bfloat16)
+    for n in (4, 4096):
+        pre = n > 256
+        h = torch.randn((n, hidden), generator=g, device=dev).to(torch.bfloat16)
+        seq = torch.zeros(n, dtype=torch.int32, device=dev)
+        pos = torch.arange(n, dtype=torch.int32, device=dev)
+        kv = torch.empty((1, n, 576), dtype=torch.bfloat16, device=dev)
+        kidx = torch.empty((1, n, 128), dtype=torch.bfloat16, device=dev)
+        cw = B.CacheWriter(h, w_cache, rms, lnw, lnb, seq, pos, kv, kidx)
+        ws = torch.zeros(max(256, B.dsa_cache_writer_workspace_bytes(n, hidden)), dtype=torch.uint8, device=dev)
+        us = timed(lambda: B.dsa_write_cache_rows(cw, ws))
+        out[f"write_cache_rows_{n}"] = entry(us, w_cache.numel() * 2, n * (hidden + 704) * 2,
+                                             2 * n * hidden * 704, pre)
+        q_nope = torch.randn((n, H, 192), generator=g, device=dev).to(torch.bfloat16)
+        q_rope = torch.randn((n, H, 64), generator=g, device=dev).to(torch.bfloat16)
+        q_out = torch.empty((n, H, 576), dtype=torch.bfloat16, device=dev)
+        ws2 = torch.zeros(256, dtype=torch.uint8, device=dev)
+        us = timed(lambda: B.dsa_absorb_queries(q_nope, q_rope, w_uk_t, pos, 8.0e6, q_out, ws2))
+        out[f"absorb_queries_{n}"] = entry(us, w_uk_t.numel() * 2, n * H * (192 + 64 + 576) * 2,
+                                           2 * n * H * 192 * 512, pre)
+        o_lat = torch.randn((n, H, 512), generator=g, device=dev).to(torch.bfloat16)
+        o_v = torch.empty((n, H, 256), dtype=torch.bfloat16, device=dev)
+        us = timed(lambda: B.dsa_up_project(o_lat, w_uv, o_v, ws2))
+        out[f"up_project_{n}"] = entry(us, w_uv.numel() * 2, n * H * (512 + 256) * 2, 2 * n * H * 512 * 256, pre)
+        assert B.dsa_check_status(ws) == B.DSA_OK and B.dsa_check_status(ws2) == B.DSA_OK
+    return out
+
+
 def run_reference(args, w: wl.Workload, world: int, rank: int):
     """The oracle as it stands on host cores: each step one query's full path."""
     if rank != 0:
@@ -641,6 +724,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-per-config", action="store_true", help="only the headline workload")
+    ap.add_argument("--no-producers", action="store_true", help="skip the producer measurements")
     ap.add_argument("--n-seq", type=int, default=0,
                     help="decode workloads: override the batch (a smaller case for profiling; not a bench line)")
     ap.add_argument("--n-q", type=int, default=0,
@@ -665,7 +749,7 @@ def main():
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     B.lib()
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
@@ -687,6 +771,10 @@ def main():
     gc.collect()
     torch.cuda.empty_cache()
 
+    if not args.no_producers and not small:
+        hbm_peak, tc_peak, peak_kind = measured_peaks()
+        line["producers"] = producers_measure(dev, flush, min(args.steps, PER_CONFIG_MAX_STEPS), hbm_peak, tc_peak,
+                                              peak_kind)
     if not args.no_per_config and not small:
         per = {}
         n = min(args.steps, PER_CONFIG_MAX_STEPS)

@@ -1,6 +1,7 @@
 // dsa_abi.cu -- the extern "C" entry points declared in include/dsa.h:
 // argument validation, workspace layout, TMA descriptor encoding and dispatch to
 // the kernels.  No allocation, no synchronisation (except dsa_check_status).
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 
@@ -229,7 +230,7 @@ dsa_status check_indexer(const dsa_queries *qs, const dsa_indexer *ix) {
 // ------------------------------------------------------------------ top-k
 dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int topk, int32_t *idx,
                    int32_t *cnt, uint32_t *status, void *scratch, bool hist_ready, cudaStream_t st) {
-    TopkArgs a;
+    TopkArgs a = {};
     a.scores = scores;
     a.ld = ld;
     a.q_pos = qs->q_pos;

@@ -10,7 +10,8 @@
 //   warp 1      MMA issuer: tcgen05.mma kind::f16, M = 128, N = BN, K = 16 steps,
 //               fp32 accumulator in TMEM;
 //   warps 2-5   epilogue: tcgen05.ld of one TMEM lane quadrant each (one output
-//               row per thread), fp32 or bf16 stores.
+//               row per thread), fp32 or bf16 rows stored as 16-byte pieces
+//               (output rows and batch strides are multiples of 16 bytes).
 // Split-K (grid y) writes fp32 partials that a consumer sums in a fixed order.
 #include <cuda_bf16.h>
 
@@ -126,18 +127,40 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_tc_kernel(const __grid_cons
                 tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + c0, r);
                 tmem_ld_wait();
                 const int n0 = nt * BN + c0;
-                if (m >= g.M) continue;
+                if (m >= g.M || n0 >= g.N) continue;
+                if (!have) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) r[x] = 0u;
+                }
+                const bool full = n0 + 32 <= g.N;  // the row's 32 columns as 16-byte stores
                 if (g.out_f32) {
                     float *o = g.out_f32 + split * g.s_split + b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n0;
+                    if (full) {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        if (n0 + x < g.N) o[x] = have ? u2f(r[x]) : 0.f;
+                        for (int x = 0; x < 32; x += 4)
+                            *reinterpret_cast<uint4 *>(o + x) = make_uint4(r[x], r[x + 1], r[x + 2], r[x + 3]);
+                    } else {
+                        for (int x = 0; x < 32; ++x)
+                            if (n0 + x < g.N) o[x] = u2f(r[x]);
+                    }
                 } else {
                     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(g.out_bf16) + b * g.s_batch +
                                        static_cast<int64_t>(m) * g.ldc + n0;
+                    if (full) {
 #pragma unroll
-                    for (int x = 0; x < 32; ++x)
-                        if (n0 + x < g.N) o[x] = __float2bfloat16_rn(have ? u2f(r[x]) : 0.f);
+                        for (int x = 0; x < 32; x += 8) {
+                            uint32_t pk[4];
+#pragma unroll
+                            for (int y = 0; y < 4; ++y) {
+                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(u2f(r[x + 2 * y]), u2f(r[x + 2 * y + 1]));
+                                pk[y] = *reinterpret_cast<const uint32_t *>(&h2);
+                            }
+                            *reinterpret_cast<uint4 *>(o + x) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        }
+                    } else {
+                        for (int x = 0; x < 32; ++x)
+                            if (n0 + x < g.N) o[x] = __float2bfloat16_rn(u2f(r[x]));
+                    }
                 }
             }
         }
@@ -151,6 +174,85 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_tc_kernel(const __grid_cons
     }
 }
 
+// ---------------------------------------------------------------- few rows of A
+// The same contraction when A has at most kSkinnyM rows (decode-sized batches):
+// B (the weights) is streamed once with 16-byte loads, A's rows sit in shared
+// memory.  One CTA per (64 rows of B, K split, batch); each warp walks 8 rows of
+// B, its lanes splitting K in 8-element pieces; a row's M partial sums are
+// reduced across the warp and written like the tensor-core kernel's output
+// (fp32 split-K partials or bf16).  HBM-bound on B.
+constexpr int kSkinnyM = 16;
+constexpr int kSkinnyRows = 64;     // rows of B per CTA
+constexpr int kSkinnyThreads = 256;
+constexpr int kSkinnyMaxK = 2048;   // K per split held in shared memory (bf16)
+
+__global__ void __launch_bounds__(kSkinnyThreads) gemm_skinny_kernel(const GemmSkinnyArgs g) {
+    extern __shared__ __align__(16) uint8_t sm_raw[];
+    __nv_bfloat16 *a_sm = reinterpret_cast<__nv_bfloat16 *>(sm_raw);  // [M][kc]
+    const int nb = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int k0 = split * g.k_per_split;
+    const int kc = min(g.k_per_split, g.K - k0);  // a multiple of 8
+    griddep_wait();
+    // A rows [M][k0, k0 + kc) into shared memory, 16 bytes at a time
+    const int pieces = kc / 8;
+    for (int e = threadIdx.x; e < g.M * pieces; e += kSkinnyThreads) {
+        const int m = e / pieces, pc = e % pieces;
+        const __nv_bfloat16 *src = static_cast<const __nv_bfloat16 *>(g.a) + b * g.a_batch + static_cast<int64_t>(m) * g.a_row +
+                                   k0 + pc * 8;
+        *reinterpret_cast<uint4 *>(a_sm + m * kc + pc * 8) = __ldg(reinterpret_cast<const uint4 *>(src));
+    }
+    __syncthreads();
+    for (int rr = 0; rr < kSkinnyRows / 8; ++rr) {
+        const int n = nb * kSkinnyRows + warp * (kSkinnyRows / 8) + rr;
+        if (n >= g.N) break;
+        const __nv_bfloat16 *brow = static_cast<const __nv_bfloat16 *>(g.b) + b * g.b_batch + static_cast<int64_t>(n) * g.b_row + k0;
+        float acc[kSkinnyM];
+#pragma unroll
+        for (int m = 0; m < kSkinnyM; ++m) acc[m] = 0.f;
+        for (int pc = lane; pc < pieces; pc += 32) {
+            const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(brow + pc * 8));
+            float wf[8];
+            {
+                const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[y]));
+                    wf[2 * y] = f.x;
+                    wf[2 * y + 1] = f.y;
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < kSkinnyM; ++m) {
+                if (m >= g.M) break;
+                const uint4 av = *reinterpret_cast<const uint4 *>(a_sm + m * kc + pc * 8);
+                const uint32_t a4[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&a4[y]));
+                    acc[m] = fmaf(wf[2 * y], f.x, acc[m]);
+                    acc[m] = fmaf(wf[2 * y + 1], f.y, acc[m]);
+                }
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < kSkinnyM; ++m) {
+            if (m >= g.M) break;
+            float v = acc[m];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) {
+                if (g.out_f32)
+                    g.out_f32[split * g.s_split + b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n] = v;
+                else
+                    static_cast<__nv_bfloat16 *>(g.out_bf16)[b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n] =
+                        __float2bfloat16_rn(v);
+            }
+        }
+    }
+    griddep_launch_dependents();
+}
+
 template <int BN>
 cudaError_t launch_gemm_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st) {
     using Cfg = GemmCfg<BN>;
@@ -162,6 +264,16 @@ cudaError_t launch_gemm_bn(const CUtensorMap &ta, const CUtensorMap &tb, const G
 }
 
 }  // namespace
+
+cudaError_t launch_gemm_skinny(const GemmSkinnyArgs &g, cudaStream_t st) {
+    const size_t smem = static_cast<size_t>(g.M) * g.k_per_split * 2;
+    cudaError_t e = cudaFuncSetAttribute(gemm_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    const int k_splits = (g.K + g.k_per_split - 1) / g.k_per_split;
+    dim3 grid((g.N + kSkinnyRows - 1) / kSkinnyRows, k_splits, g.batch);
+    return launch_pdl(gemm_skinny_kernel, grid, dim3(kSkinnyThreads), smem, st, g);
+}
 
 cudaError_t launch_gemm_tc(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st) {
     switch (bn) {

@@ -106,6 +106,8 @@ struct TopkArgs {
     // scratch (workspace)
     uint32_t *ghist;   // [n_q][4096] first-digit histogram
     uint32_t *gticket; // [n_q] chunks of the query done (split schedule), after ghist
+    uint32_t *ghist2;  // [n_q][4096] second-digit histogram of the threshold-bin candidates
+                       // (split schedule), after the tickets
     uint32_t *gcount;  // [n_q][kSplitMax] candidates per chunk
     uint2 *gcand;      // [n_q][kSplitMax][kSplitCap] (key, position)
 };
@@ -175,6 +177,24 @@ struct GemmArgs {
     uint32_t *status;
 };
 cudaError_t launch_gemm_tc(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st);
+
+// The same contraction for at most 16 rows of A (decode-sized batches), on CUDA
+// cores: B streamed once with 16-byte loads; K split in pieces of k_per_split
+// (a multiple of 8, at most 2048); element (m, k) of batch b at a + b * a_batch +
+// m * a_row + k, (n, k) at b + b * b_batch + n * b_row + k (elements, 16-byte
+// aligned rows); outputs addressed as in GemmArgs.
+struct GemmSkinnyArgs {
+    int M, N, K, batch, k_per_split;
+    const void *a;
+    int64_t a_row, a_batch;
+    const void *b;
+    int64_t b_row, b_batch;
+    float *out_f32;
+    void *out_bf16;
+    int64_t ldc, s_batch, s_split;
+};
+constexpr int kSkinnyMaxM = 16;
+cudaError_t launch_gemm_skinny(const GemmSkinnyArgs &g, cudaStream_t st);
 
 // Cache-row writer epilogue: one CTA per token sums the split-K partials of
 // y = h . W^T (704 features: latent 512 | RoPE key 64 | indexer key 128) and

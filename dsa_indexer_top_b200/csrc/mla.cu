@@ -50,30 +50,43 @@ constexpr int kTmemCols = 512;                      // S slots: 0..127, O^T: 128
 constexpr int kOCol = 128;
 constexpr uint32_t kIdescS = idesc_bf16(64, 64, false, false);
 constexpr uint32_t kIdescO = idesc_bf16(128, 64, true, false);
+// Packed FP8 caches run the MMAs in fp16 (E4M3 codes, the queries and the RoPE
+// keys are exact in fp16): S has a latent half (codes, the row scale applied in
+// the softmax) in columns 64*slot and a RoPE half in columns kSRopeCol + 64*slot.
+constexpr uint32_t kIdescS16 = idesc_f16(64, 64, false, false);
+constexpr uint32_t kIdescO16 = idesc_f16(128, 64, true, false);
+constexpr int kSRopeCol = 384;
 // A running maximum is kept until a head's chunk maximum exceeds it by more than
 // this many powers of two (probabilities stay below 2^8); only then is the
 // accumulated O rescaled.
 constexpr float kRescaleLog2 = 8.0f;
-// Chunks prefetched into L2 ahead of a slot's gathers, counted in turns of the
-// slot (a slot takes every other chunk of the CTA).
-constexpr int kPrefetchSlots = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Two E4M3 codes (low byte first) times a row scale, as two bf16 (low half
-// first): the codes widen exactly to half and float, the product is rounded
-// once to float, then to bf16.
-__device__ __forceinline__ uint32_t e4m3x2_scaled_bf16x2(uint32_t two, float sigma) {
+// Two E4M3 codes (low byte first) as two fp16 (low half first): exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two) {
     const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-    const float2 f = __half22float2(__half2(hr));
-    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x * sigma, f.y * sigma);
-    return *reinterpret_cast<const uint32_t *>(&b);
+    return static_cast<uint32_t>(hr.x) | (static_cast<uint32_t>(hr.y) << 16);
+}
+
+// Eight bf16 values (one 16-byte piece) as eight fp16, rounded to nearest (exact
+// for bf16 values of magnitude within fp16's normal range).
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[k]));
+        const __half2 h = __floats2half2_rn(f.x, f.y);
+        w[k] = *reinterpret_cast<const uint32_t *>(&h);
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // kFp8: the caches are packed FP8 rows [512 E4M3 codes | 64 bf16 RoPE | float32
-// scale | padding]; the producers widen each latent to bf16 (scale applied) into
-// the same shared-memory tiles the bf16 cache fills, so the MMAs and the softmax
-// are the same for both.
+// scale | padding].  The producers widen the codes (exactly) and the RoPE keys and
+// queries to fp16 into the same swizzled tiles; the MMAs run kind::f16 on fp16;
+// the softmax scales each row's latent logit by its sigma and folds sigma into
+// the fp16 P, so O = sum_j p_j sigma_j code_j.
 // One CTA per SM (217 KB of shared memory).  Nine warps spread over the SM's
 // four sub-partitions (three on one of them, whose 16K-register file they
 // share) allow at most 168 registers per thread.
@@ -90,6 +103,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     __shared__ int row_idx[2][kChunk];  // [slot][chunk row]: cache row, or -1 (padding)
+    __shared__ float row_sigma[kFp8 ? 2 : 1][kChunk];  // FP8 caches: [slot][chunk row] row scale
     __shared__ float alpha_sm[kMlaHeads], m_fin[kMlaHeads], l_fin[kMlaHeads], inv_l[kMlaHeads];
     __shared__ int rescale_w[4];
 
@@ -101,7 +115,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     if (tid == 0) {
         mbar_init(&q_full, 4);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&slot_full[s], 2);
+            mbar_init(&slot_full[s], 4);
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], 4);
             mbar_init(&o_done[s], 1);
@@ -136,6 +150,30 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             }
         }
         cp_async_commit();
+        if constexpr (kFp8) {
+            // fp16 queries for the fp16 MMAs: each thread converts the pieces it
+            // copied, in place, while the previous kernel may still be running
+            cp_async_wait_all();
+            for (int hh = 0; hh < 16; ++hh) {
+                const int h = 16 * pw + hh;
+#pragma unroll
+                for (int tt = 0; tt < 3; ++tt) {
+                    const int ch = lane + 32 * tt;
+                    if (ch < kRow / 8) {
+                        const uint32_t adr = q_addr + (ch >> 3) * kBlockBytes + sw128_offset(h, ch & 7);
+                        uint4 v;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                     : "r"(adr)
+                                     : "memory");
+                        v = bf16x8_to_f16x8(v);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(v.x), "r"(v.y), "r"(v.z),
+                                     "r"(v.w)
+                                     : "memory");
+                    }
+                }
+            }
+        }
     }
     griddep_wait();
 
@@ -156,36 +194,12 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
 
     if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ producers
-        // Warps 4-5 fill slot 0 (even chunks of this CTA), warps 6-7 slot 1 (odd
-        // chunks), so the two slots fill concurrently; each warp gathers 32 of a
-        // chunk's 64 rows (lane l owns row 32 * half + l).  While gathering a
-        // chunk, each lane prefetches into L2 its row of the chunks this slot
-        // takes kPrefetchSlots turns later, so the gathers after the first read
-        // from L2 instead of waiting on HBM.
-        const int pw = warp - 4;
-        const int p = pw >> 1, half = pw & 1;
-        const int rl = 32 * half + lane;
-        const uint32_t row_bytes = kFp8 ? static_cast<uint32_t>(kFp8Row) : static_cast<uint32_t>(kRow * 2);
-        auto prefetch_chunk = [&](int t2) {
-            if (t2 >= nloc) return;
-            const int j = (c_begin + t2) * kChunk + rl;
-            if (j >= cnt) return;
-            const int r = __ldg(sel + j);
-            if (r < 0 || r >= a.L) return;
-            if constexpr (kFp8)
-                bulk_prefetch_l2(kv8 + static_cast<int64_t>(r) * a.kv_row_stride, row_bytes);
-            else
-                bulk_prefetch_l2(kv + static_cast<int64_t>(r) * a.kv_row_stride, row_bytes);
-        };
+        const int pw = warp - 4;  // rows (and the query tile's heads) 16*pw .. 16*pw+15
         bool q_arrived = false;
-        for (int t = p; t < nloc; t += 2) {
-            const int c = c_begin + t, u = t >> 1;
-            if (t == p) {
-                for (int k = 1; k <= kPrefetchSlots; ++k) prefetch_chunk(t + 2 * k);
-            } else {
-                prefetch_chunk(t + 2 * kPrefetchSlots);
-            }
-            if (t >= 2 && !mbar_wait(&o_done[p], (u - 1) & 1, a.status, &abort_flag)) break;
+        for (int t = 0; t < nloc; ++t) {
+            const int c = c_begin + t, s = t & 1, u = t >> 1;
+            if (t >= 2 && !mbar_wait(&o_done[s], (u - 1) & 1, a.status, &abort_flag)) break;
+            const int rl = 16 * pw + (lane & 15);
             const int j = c * kChunk + rl;
             int r = -1;
             if (j < cnt) {
@@ -195,11 +209,11 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                     r = -1;
                 }
             }
-            row_idx[p][rl] = r;
-            const uint32_t sb = smem_u32(slot_sm + p * kSlotBytes);
+            if (lane < 16) row_idx[s][rl] = r;
+            const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
             if constexpr (!kFp8) {
-                for (int rr = 0; rr < 32; ++rr) {
-                    const int row = 32 * half + rr;
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int row = 16 * pw + rr;
                     const int src = __shfl_sync(0xffffffffu, r, rr);
 #pragma unroll
                     for (int tt = 0; tt < 3; ++tt) {
@@ -214,60 +228,72 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                     }
                 }
             } else {
-                // Lane l takes latent dims 16l..16l+15 of each of 16 rows at a time:
-                // all 16 code loads (and scales) are issued before any is widened;
-                // lanes 0-7 copy the row's RoPE key (bf16) straight into block 8.
-                const uint32_t blk = sb + (lane >> 2) * kBlockBytes;  // dims 16l.. lie in block l / 4
-#pragma unroll 1
-                for (int rb = 0; rb < 32; rb += 16) {
-                    uint4 code[16];
-                    float sig[16];
+                // Lane l takes latent dims 16l..16l+15 of each of the warp's 16 rows:
+                // all 16 code loads are issued before any is widened (exactly, to
+                // fp16); lanes 0-7 copy the row's RoPE key (bf16) into block 8, to be
+                // converted to fp16 in place once it lands; the row scale goes to
+                // row_sigma.
+                uint4 code[16];
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) {
-                        const int src = __shfl_sync(0xffffffffu, r, rb + rr);
-                        code[rr] = make_uint4(0u, 0u, 0u, 0u);
-                        sig[rr] = 0.f;
-                        const uint32_t rope_dst = sb + 8 * kBlockBytes + sw128_offset(32 * half + rb + rr, lane & 7);
-                        if (src >= 0) {
-                            const uint8_t *row = kv8 + static_cast<int64_t>(src) * a.kv_row_stride;
-                            code[rr] = __ldg(reinterpret_cast<const uint4 *>(row) + lane);
-                            sig[rr] = __ldg(reinterpret_cast<const float *>(row + kFp8ScaleOff));
-                            if (lane < 8) cp_async_16(rope_dst, row + kFp8RopeOff + 16 * lane);
-                        } else if (lane < 8) {
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int src = __shfl_sync(0xffffffffu, r, rr);
+                    code[rr] = make_uint4(0u, 0u, 0u, 0u);
+                    const uint32_t rope_dst = sb + 8 * kBlockBytes + sw128_offset(16 * pw + rr, lane & 7);
+                    if (src >= 0) {
+                        const uint8_t *row = kv8 + static_cast<int64_t>(src) * a.kv_row_stride;
+                        code[rr] = __ldg(reinterpret_cast<const uint4 *>(row) + lane);
+                        if (lane < 8) cp_async_16(rope_dst, row + kFp8RopeOff + 16 * lane);
+                        if (lane == 8) row_sigma[s][16 * pw + rr] = __ldg(reinterpret_cast<const float *>(row + kFp8ScaleOff));
+                    } else {
+                        if (lane < 8)
                             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(rope_dst), "r"(0u) : "memory");
-                        }
+                        if (lane == 8) row_sigma[s][16 * pw + rr] = 0.f;
                     }
+                }
+                const uint32_t blk = sb + (lane >> 2) * kBlockBytes;  // dims 16l.. lie in block l / 4
 #pragma unroll
-                    for (int rr = 0; rr < 16; ++rr) {
-                        const int row = 32 * half + rb + rr;
-                        const float sg = sig[rr];
-                        const uint32_t w0 = code[rr].x, w1 = code[rr].y, w2 = code[rr].z, w3 = code[rr].w;
-                        const uint32_t lo0 = e4m3x2_scaled_bf16x2(w0 & 0xffffu, sg), lo1 = e4m3x2_scaled_bf16x2(w0 >> 16, sg);
-                        const uint32_t lo2 = e4m3x2_scaled_bf16x2(w1 & 0xffffu, sg), lo3 = e4m3x2_scaled_bf16x2(w1 >> 16, sg);
-                        const uint32_t hi0 = e4m3x2_scaled_bf16x2(w2 & 0xffffu, sg), hi1 = e4m3x2_scaled_bf16x2(w2 >> 16, sg);
-                        const uint32_t hi2 = e4m3x2_scaled_bf16x2(w3 & 0xffffu, sg), hi3 = e4m3x2_scaled_bf16x2(w3 >> 16, sg);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane) & 7)),
-                                     "r"(lo0), "r"(lo1), "r"(lo2), "r"(lo3) : "memory");
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane + 1) & 7)),
-                                     "r"(hi0), "r"(hi1), "r"(hi2), "r"(hi3) : "memory");
-                    }
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int row = 16 * pw + rr;
+                    const uint32_t w0 = code[rr].x, w1 = code[rr].y, w2 = code[rr].z, w3 = code[rr].w;
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane) & 7)),
+                                 "r"(e4m3x2_to_f16x2(w0 & 0xffffu)), "r"(e4m3x2_to_f16x2(w0 >> 16)),
+                                 "r"(e4m3x2_to_f16x2(w1 & 0xffffu)), "r"(e4m3x2_to_f16x2(w1 >> 16))
+                                 : "memory");
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane + 1) & 7)),
+                                 "r"(e4m3x2_to_f16x2(w2 & 0xffffu)), "r"(e4m3x2_to_f16x2(w2 >> 16)),
+                                 "r"(e4m3x2_to_f16x2(w3 & 0xffffu)), "r"(e4m3x2_to_f16x2(w3 >> 16))
+                                 : "memory");
                 }
             }
             cp_async_commit();
-            if (!q_arrived) {
-                // the query tile (the older group) has landed: S may start on it
-                cp_async_wait_group<1>();
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&q_full);
-                q_arrived = true;
+            cp_async_wait_all();  // the query tile (first chunk) and this chunk's rows
+            if constexpr (kFp8) {
+                // this lane's RoPE pieces (bf16, copied above) to fp16, in place
+                if (lane < 8) {
+#pragma unroll 4
+                    for (int rr = 0; rr < 16; ++rr) {
+                        const uint32_t adr = sb + 8 * kBlockBytes + sw128_offset(16 * pw + rr, lane & 7);
+                        uint4 v;
+                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                     : "r"(adr)
+                                     : "memory");
+                        v = bf16x8_to_f16x8(v);
+                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(v.x), "r"(v.y), "r"(v.z),
+                                     "r"(v.w)
+                                     : "memory");
+                    }
+                }
             }
-            cp_async_wait_all();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&slot_full[p]);
+            if (lane == 0) {
+                if (!q_arrived) mbar_arrive(&q_full);
+                mbar_arrive(&slot_full[s]);
+            }
+            q_arrived = true;
         }
-        if (!q_arrived) {  // no chunk for this slot (or an abort): the query tile still counts
+        if (!q_arrived) {  // no chunk for this CTA (or an abort): the query tile still counts
             cp_async_wait_all();
             fence_proxy_async_smem();
             __syncwarp();
@@ -297,10 +323,21 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                     tc_fence_after();
                     const int s = ts & 1;
                     const uint64_t cdesc = s ? cdesc1 : cdesc0;
+                    if constexpr (!kFp8) {
 #pragma unroll
-                    for (int kk = 0; kk < kRow / 16; ++kk) {
-                        const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
-                        umma_bf16(tbase + 64 * s, qdesc + koff, cdesc + koff, kIdescS, kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < kRow / 16; ++kk) {
+                            const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                            umma_bf16(tbase + 64 * s, qdesc + koff, cdesc + koff, kIdescS, kk > 0 ? 1u : 0u);
+                        }
+                    } else {
+                        // latent half (codes) and RoPE half into separate accumulators
+#pragma unroll
+                        for (int kk = 0; kk < kRow / 16; ++kk) {
+                            const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * kBlockBytes + (kk & 3) * 32) >> 4);
+                            const bool rope = kk >= kLatent / 16;
+                            umma_bf16(tbase + (rope ? kSRopeCol : 0) + 64 * s, qdesc + koff, cdesc + koff, kIdescS16,
+                                      (kk > 0 && kk != kLatent / 16) ? 1u : 0u);
+                        }
                     }
                     umma_commit(&s_full[s]);
                     ++ts;
@@ -317,7 +354,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                         for (int kk = 0; kk < kChunk / 16; ++kk) {
                             umma_bf16(tbase + kOCol + 64 * mt,
                                       adesc + static_cast<uint64_t>((2 * mt * kBlockBytes + kk * 2048) >> 4),
-                                      bdesc + static_cast<uint64_t>((kk * 32) >> 4), kIdescO, (to > 0 || kk > 0) ? 1u : 0u);
+                                      bdesc + static_cast<uint64_t>((kk * 32) >> 4), kFp8 ? kIdescO16 : kIdescO,
+                                      (to > 0 || kk > 0) ? 1u : 0u);
                         }
                     }
                     umma_commit(&o_done[sp]);
@@ -359,7 +397,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             {
                 uint32_t r[32];
                 tmem_ld16x2_32<32>(lane_base + 64 * s, r);
-                tmem_ld_wait();
+                if constexpr (kFp8) {
+                    // logit = sigma_j * (q_lat . code_j) + q_rope . r_j
+                    uint32_t rr[32];
+                    tmem_ld16x2_32<32>(lane_base + kSRopeCol + 64 * s, rr);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(fmaf(row_sigma[s][rbase + x], u2f(r[x]), u2f(rr[x])));
+                } else {
+                    tmem_ld_wait();
+                }
 #pragma unroll
                 for (int x = 0; x < 32; ++x)
                     if (row_idx[s][rbase + x] >= 0) mc = fmaxf(mc, u2f(r[x]));
@@ -404,22 +451,44 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             }
             uint32_t r[32];  // the chunk's logits again (cheaper than keeping them live)
             tmem_ld16x2_32<32>(lane_base + 64 * s, r);
-            tmem_ld_wait();
+            if constexpr (kFp8) {
+                uint32_t rr[32];
+                tmem_ld16x2_32<32>(lane_base + kSRopeCol + 64 * s, rr);
+                tmem_ld_wait();
+#pragma unroll
+                for (int x = 0; x < 32; ++x) r[x] = __float_as_uint(fmaf(row_sigma[s][rbase + x], u2f(r[x]), u2f(rr[x])));
+            } else {
+                tmem_ld_wait();
+            }
             {
                 uint8_t *pl = slot_sm + s * kSlotBytes + 8 * kBlockBytes;  // head h's P line
                 float sum = 0.f;
 #pragma unroll
                 for (int jc = 0; jc < 4; ++jc) {
-                    __align__(16) __nv_bfloat16 pb[8];
+                    if constexpr (!kFp8) {
+                        __align__(16) __nv_bfloat16 pb[8];
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) {
-                        const int xr = 8 * jc + x;
-                        const float pf = (row_idx[s][rbase + xr] >= 0) ? exp2f((u2f(r[xr]) - m) * c2) : 0.f;
-                        pb[x] = __float2bfloat16_rn(pf);
-                        sum += __bfloat162float(pb[x]);  // the sum uses the value the MMA sees
+                        for (int x = 0; x < 8; ++x) {
+                            const int xr = 8 * jc + x;
+                            const float pf = (row_idx[s][rbase + xr] >= 0) ? exp2f((u2f(r[xr]) - m) * c2) : 0.f;
+                            pb[x] = __float2bfloat16_rn(pf);
+                            sum += __bfloat162float(pb[x]);  // the sum uses the value the MMA sees
+                        }
+                        *reinterpret_cast<uint4 *>(pl + sw128_offset(h, (rbase >> 3) + jc)) =
+                            *reinterpret_cast<const uint4 *>(pb);
+                    } else {
+                        // P' = p * sigma in fp16 (the MMA multiplies it by the exact codes)
+                        __align__(16) __half pb[8];
+#pragma unroll
+                        for (int x = 0; x < 8; ++x) {
+                            const int xr = 8 * jc + x;
+                            const float pf = (row_idx[s][rbase + xr] >= 0) ? exp2f((u2f(r[xr]) - m) * c2) : 0.f;
+                            pb[x] = __float2half_rn(pf * row_sigma[s][rbase + xr]);
+                            sum += pf;
+                        }
+                        *reinterpret_cast<uint4 *>(pl + sw128_offset(h, (rbase >> 3) + jc)) =
+                            *reinterpret_cast<const uint4 *>(pb);
                     }
-                    *reinterpret_cast<uint4 *>(pl + sw128_offset(h, (rbase >> 3) + jc)) =
-                        *reinterpret_cast<const uint4 *>(pb);
                 }
                 sum += __shfl_xor_sync(0xffffffffu, sum, 16);
                 l = l * al + sum;
@@ -449,22 +518,25 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             const bool final_out = (a.n_splits == 1);
             for (int mt = mt0; mt < mt0 + 2; ++mt) {
                 const int d = mt * 128 + quad * 32 + lane;
+                // both 32-head halves of this lane's latent dim in flight before one wait
+                uint32_t r0[32], r1[32];
+                const uint32_t ta = tbase + (static_cast<uint32_t>(quad * 32) << 16) + kOCol + mt * 64;
+                tmem_ld32(ta, r0);
+                tmem_ld32(ta + 32, r1);
+                tmem_ld_wait();
+                if (final_out) {
+                    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(lp.out) + static_cast<int64_t>(i) * kMlaHeads * kLatent;
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r[32];
-                    tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + kOCol + mt * 64 + half * 32, r);
-                    tmem_ld_wait();
-                    if (final_out) {
-                        __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(lp.out) + static_cast<int64_t>(i) * kMlaHeads * kLatent;
+                    for (int x = 0; x < 32; ++x) {
+                        o[x * kLatent + d] = __float2bfloat16_rn(u2f(r0[x]) * inv_l[x]);
+                        o[(32 + x) * kLatent + d] = __float2bfloat16_rn(u2f(r1[x]) * inv_l[32 + x]);
+                    }
+                } else {
+                    float *po = a.part_o + ((static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits + split) * kMlaHeads * kLatent;
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) {
-                            const int hh = half * 32 + x;
-                            o[hh * kLatent + d] = __float2bfloat16_rn(u2f(r[x]) * inv_l[hh]);
-                        }
-                    } else {
-                        float *po = a.part_o + ((static_cast<int64_t>(layer) * a.n_q + i) * a.n_splits + split) * kMlaHeads * kLatent;
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) po[(half * 32 + x) * kLatent + d] = u2f(r[x]);
+                    for (int x = 0; x < 32; ++x) {
+                        po[x * kLatent + d] = u2f(r0[x]);
+                        po[(32 + x) * kLatent + d] = u2f(r1[x]);
                     }
                 }
             }
@@ -681,3 +753,4 @@ cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st) {
 }
 
 }  // namespace dsa
+

@@ -9,6 +9,8 @@
 //   dsa_absorb_queries    q_lat[h] = W_UK[h]^T q_nope[h] per head (batched GEMM over
 //                         heads) and the query's RoPE part rotated
 //   dsa_up_project        o[h] = W_UV[h] o_lat[h] per head (batched GEMM)
+// Batches of up to 16 tokens run the contractions on CUDA cores (the weights
+// streamed once, HBM-bound); larger batches on the tcgen05 GEMM.
 // ("GLM-5.2 -- Model techniques map", "Checked in its code": Multi-head latent
 // attention, QK normalization, Partial RoPE; "GLM 5.2 -- Hermosa AI", "MLA + DSA
 // with IndexShare": RoPE theta 8e6; "GLM-5.2 -- LLM atlas", raw config.json
@@ -61,11 +63,41 @@ __global__ void __launch_bounds__(kEpiThreads) cache_write_epilogue_kernel(const
         if (threadIdx.x == 0) report_status(a.status, DSA_ERR_INVALID);
         return;
     }
-    for (int f = threadIdx.x; f < kProjFeatures; f += kEpiThreads) {
-        float v = 0.f;
-        for (int s = 0; s < a.k_splits; ++s)  // fixed order: deterministic
-            v += a.y[(static_cast<int64_t>(s) * a.n_tok + t) * kProjFeatures + f];
-        y[f] = v;
+    {
+        // three features per thread (704 = 2.75 x 256), the split partials summed in a
+        // fixed order (deterministic) with the loads of four splits in flight at once
+        constexpr int kF = (kProjFeatures + kEpiThreads - 1) / kEpiThreads;
+        float v[kF];
+#pragma unroll
+        for (int q = 0; q < kF; ++q) v[q] = 0.f;
+        const int64_t split_stride = static_cast<int64_t>(a.n_tok) * kProjFeatures;
+        const float *yt = a.y + static_cast<int64_t>(t) * kProjFeatures;
+        int s = 0;
+        for (; s + 4 <= a.k_splits; s += 4) {
+            float x[4][kF];
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int q = 0; q < kF; ++q) {
+                    const int f = threadIdx.x + q * kEpiThreads;
+                    x[u][q] = f < kProjFeatures ? yt[(s + u) * split_stride + f] : 0.f;
+                }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+#pragma unroll
+                for (int q = 0; q < kF; ++q) v[q] += x[u][q];
+        }
+        for (; s < a.k_splits; ++s)
+#pragma unroll
+            for (int q = 0; q < kF; ++q) {
+                const int f = threadIdx.x + q * kEpiThreads;
+                if (f < kProjFeatures) v[q] += yt[s * split_stride + f];
+            }
+#pragma unroll
+        for (int q = 0; q < kF; ++q) {
+            const int f = threadIdx.x + q * kEpiThreads;
+            if (f < kProjFeatures) y[f] = v[q];
+        }
     }
     __syncthreads();
     // latent: RMSNorm over 512 features, times gamma
@@ -214,12 +246,32 @@ dsa_status dsa_write_cache_rows(const dsa_cache_writer *cw, void *ws, size_t ws_
     g.s_batch = 0;
     g.s_split = static_cast<int64_t>(cw->n_tok) * kProjFeatures;
     g.status = static_cast<uint32_t *>(ws);
-    CUtensorMap ta, tb;
-    if (!encode_gemm_operand(&ta, cw->h, cw->hidden, cw->n_tok, 1, cw->h_row_stride, 0, 128, &g.a_batch_inner))
-        return DSA_ERR_INVALID;
-    if (!encode_gemm_operand(&tb, cw->w, cw->hidden, kProjFeatures, 1, cw->hidden, 0, 128, &g.b_batch_inner))
-        return DSA_ERR_INVALID;
-    if (launch_gemm_tc(128, ta, tb, g, st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (cw->n_tok <= kSkinnyMaxM) {
+        // decode-sized batch: stream the weights once on CUDA cores (same partials)
+        GemmSkinnyArgs k = {};
+        k.M = cw->n_tok;
+        k.N = kProjFeatures;
+        k.K = cw->hidden;
+        k.batch = 1;
+        k.k_per_split = (((cw->hidden + g.k_splits - 1) / g.k_splits) + 7) / 8 * 8;
+        if (k.k_per_split > 2048) return DSA_ERR_UNSUPPORTED;
+        g.k_splits = (cw->hidden + k.k_per_split - 1) / k.k_per_split;  // what the epilogue sums
+        k.a = cw->h;
+        k.a_row = cw->h_row_stride;
+        k.b = cw->w;
+        k.b_row = cw->hidden;
+        k.out_f32 = y;
+        k.ldc = kProjFeatures;
+        k.s_split = g.s_split;
+        if (launch_gemm_skinny(k, st) != cudaSuccess) return DSA_ERR_CUDA;
+    } else {
+        CUtensorMap ta, tb;
+        if (!encode_gemm_operand(&ta, cw->h, cw->hidden, cw->n_tok, 1, cw->h_row_stride, 0, 128, &g.a_batch_inner))
+            return DSA_ERR_INVALID;
+        if (!encode_gemm_operand(&tb, cw->w, cw->hidden, kProjFeatures, 1, cw->hidden, 0, 128, &g.b_batch_inner))
+            return DSA_ERR_INVALID;
+        if (launch_gemm_tc(128, ta, tb, g, st) != cudaSuccess) return DSA_ERR_CUDA;
+    }
     CacheWriteArgs e;
     e.y = y;
     e.k_splits = g.k_splits;
@@ -264,14 +316,33 @@ dsa_status dsa_absorb_queries(int32_t n_q, int32_t heads, const void *q_nope, co
     g.ldc = static_cast<int64_t>(heads) * kRow;
     g.s_batch = kRow;
     g.status = static_cast<uint32_t *>(ws);
-    CUtensorMap ta, tb;
-    if (!encode_gemm_operand(&ta, q_nope, kDNope, n_q, heads, static_cast<int64_t>(heads) * kDNope, kDNope, 128,
-                             &g.a_batch_inner))
-        return DSA_ERR_INVALID;
-    if (!encode_gemm_operand(&tb, w_uk_t, kDNope, kLatent, heads, kDNope, static_cast<int64_t>(kLatent) * kDNope, 128,
-                             &g.b_batch_inner))
-        return DSA_ERR_INVALID;
-    if (launch_gemm_tc(128, ta, tb, g, st) != cudaSuccess) return DSA_ERR_CUDA;
+    if (n_q <= kSkinnyMaxM) {
+        GemmSkinnyArgs k = {};
+        k.M = n_q;
+        k.N = kLatent;
+        k.K = kDNope;
+        k.batch = heads;
+        k.k_per_split = kDNope;
+        k.a = q_nope;
+        k.a_row = static_cast<int64_t>(heads) * kDNope;
+        k.a_batch = kDNope;
+        k.b = w_uk_t;
+        k.b_row = kDNope;
+        k.b_batch = static_cast<int64_t>(kLatent) * kDNope;
+        k.out_bf16 = q_out;
+        k.ldc = g.ldc;
+        k.s_batch = g.s_batch;
+        if (launch_gemm_skinny(k, st) != cudaSuccess) return DSA_ERR_CUDA;
+    } else {
+        CUtensorMap ta, tb;
+        if (!encode_gemm_operand(&ta, q_nope, kDNope, n_q, heads, static_cast<int64_t>(heads) * kDNope, kDNope, 128,
+                                 &g.a_batch_inner))
+            return DSA_ERR_INVALID;
+        if (!encode_gemm_operand(&tb, w_uk_t, kDNope, kLatent, heads, kDNope, static_cast<int64_t>(kLatent) * kDNope,
+                                 128, &g.b_batch_inner))
+            return DSA_ERR_INVALID;
+        if (launch_gemm_tc(128, ta, tb, g, st) != cudaSuccess) return DSA_ERR_CUDA;
+    }
     QueryRopeArgs r;
     r.q_rope = q_rope;
     r.q = q_out;
@@ -301,6 +372,24 @@ dsa_status dsa_up_project(int32_t n_q, int32_t heads, const void *o_lat, const v
     g.ldc = static_cast<int64_t>(heads) * kDV;
     g.s_batch = kDV;
     g.status = static_cast<uint32_t *>(ws);
+    if (n_q <= kSkinnyMaxM) {
+        GemmSkinnyArgs k = {};
+        k.M = n_q;
+        k.N = kDV;
+        k.K = kLatent;
+        k.batch = heads;
+        k.k_per_split = kLatent;
+        k.a = o_lat;
+        k.a_row = static_cast<int64_t>(heads) * kLatent;
+        k.a_batch = kLatent;
+        k.b = w_uv;
+        k.b_row = kLatent;
+        k.b_batch = static_cast<int64_t>(kDV) * kLatent;
+        k.out_bf16 = out;
+        k.ldc = g.ldc;
+        k.s_batch = g.s_batch;
+        return launch_gemm_skinny(k, static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    }
     CUtensorMap ta, tb;
     if (!encode_gemm_operand(&ta, o_lat, kLatent, n_q, heads, static_cast<int64_t>(heads) * kLatent, kLatent, 128,
                              &g.a_batch_inner))

@@ -337,23 +337,27 @@ __device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t n
 // bounds-checked against k (they stay below k whenever the histogram the
 // threshold digit came from describes these scores).
 constexpr int kOwn = 9;
+// hist2_ready: `hist` already holds the second-digit histogram of the
+// candidates in bin d1 (built by the chunk CTAs), so it is not rebuilt here.
 template <class Segs>
 __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t r2, uint32_t k, uint32_t *hist,
-                                           uint64_t *scan, uint32_t *sel, int32_t *out) {
+                                           uint64_t *scan, uint32_t *sel, int32_t *out, bool hist2_ready = false) {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint2 *p = sg.ptr(w, 0);
     const uint32_t c = sg.count(w, 0);
     const uint32_t m = ((c + 31) / 32) | 1u;  // odd run length: the lanes' loads fall in distinct banks
-    zero_hist(hist, kBins);
+    if (!hist2_ready) zero_hist(hist, kBins);
     if (__syncthreads_or(m > static_cast<uint32_t>(kOwn) || sg.pieces(w) != 1)) return false;
     const uint32_t b0 = min(c, lane * m), b1 = min(c, b0 + m);
     uint32_t key[kOwn];
 #pragma unroll
     for (int j = 0; j < kOwn; ++j) key[j] = b0 + j < b1 ? p[b0 + j].x : 0u;
+    if (!hist2_ready) {
 #pragma unroll
-    for (int j = 0; j < kOwn; ++j)
-        if (b0 + j < b1 && first_digit(key[j]) == d1) atomicAdd(&hist[(key[j] >> 8) & 0xFFFu], 1u);
-    __syncthreads();
+        for (int j = 0; j < kOwn; ++j)
+            if (b0 + j < b1 && first_digit(key[j]) == d1) atomicAdd(&hist[(key[j] >> 8) & 0xFFFu], 1u);
+        __syncthreads();
+    }
     find_digit(hist, kBins, r2, scan, sel);
     const uint32_t d2 = sel[0];
     const uint32_t r3 = r2 - sel[1];
@@ -682,9 +686,15 @@ __device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int
     }
     __syncthreads();
     const bool overflow = sm.sel[2] != 0;
+    uint32_t *g2 = a.ghist2 + static_cast<int64_t>(i) * kBins;
     if (overflow) {
+        for (int b = threadIdx.x; b < kBins; b += kT) g2[b] = 0u;  // zero for the next launch
         finish_stream(row, n, k, d1, above1, sm.hist, sm.scan, sm.sel, out);
     } else {
+        // the second-digit histogram the chunk CTAs built (16-byte pieces, L2)
+        for (int e = threadIdx.x; e < kBins / 4; e += kT)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&sm.hist[4 * e])), "l"(g2 + 4 * e)
+                         : "memory");
         // stage: warp w copies chunks w, w + 16, ... with asynchronous copies
         // (all in flight at once).  The L1-allocating form is safe here: this
         // CTA is the only reader of these lines in this launch, after every
@@ -700,8 +710,9 @@ __device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int
         cp_async_commit();
         cp_async_wait_all();
         __syncthreads();
+        for (int b = threadIdx.x; b < kBins; b += kT) g2[b] = 0u;  // read above; zero for the next launch
         const StagedSegs sg{sm.cand, sm.coff[n_chunks]};
-        if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out)) {
+        if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out, true)) {
             uint32_t T, need_eq;
             seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
             seg_write(sg, T, need_eq, k, out, sm.wg, sm.we);
@@ -750,6 +761,17 @@ __global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int
         compact_batch(v, base0, whi, d1, cs.wbuf[warp], kWarpCap, cnt);
     }
     if (lane == 0) cs.wcount[warp] = cnt;
+    {
+        // second digit of this warp's candidates in the threshold bin, into the
+        // query's histogram (the finishing CTA reads it instead of building it)
+        __syncwarp();
+        uint32_t *g2 = a.ghist2 + static_cast<int64_t>(i) * kBins;
+        const uint32_t c = min(cnt, static_cast<uint32_t>(kWarpCap));
+        for (uint32_t j = lane; j < c; j += 32) {
+            const uint32_t u = cs.wbuf[warp][j].x;
+            if (first_digit(u) == d1) atomicAdd(&g2[(u >> 8) & 0xFFFu], 1u);
+        }
+    }
     __syncthreads();
     if (threadIdx.x == 0) {
         uint32_t o = 0;
@@ -771,6 +793,9 @@ __global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int
         for (uint32_t j = lane; j < c; j += 32) dst[cs.woff[warp] + j] = cs.wbuf[warp][j];
     }
     if (threadIdx.x == 0) a.gcount[static_cast<int64_t>(i) * kSplitMax + p] = total;
+    // The next kernel (the attention) may start its prologue on the SMs the chunk
+    // CTAs leave; it still waits for this whole grid before reading the selection.
+    griddep_launch_dependents();
 
     // ---- publish; the last CTA of the query finishes it
     __threadfence();
@@ -850,10 +875,16 @@ cudaError_t launch_bounded_wait_probe(uint32_t *status, uint64_t limit_ns, cudaS
     return cudaGetLastError();
 }
 
-size_t topk_zeroed_bytes(int n_q) { return sizeof(uint32_t) * (static_cast<size_t>(kBins) + 1) * n_q; }
+// The tickets are padded to a multiple of 4 words so that the second-digit
+// histograms after them start on a 16-byte boundary (they are copied with
+// 16-byte cp.async).
+static size_t ticket_words(int n_q) { return (static_cast<size_t>(n_q) + 3) & ~static_cast<size_t>(3); }
+size_t topk_zeroed_bytes(int n_q) {
+    return sizeof(uint32_t) * (2 * static_cast<size_t>(kBins) * n_q + ticket_words(n_q));
+}
 
-// Scratch: [n_q][4096] first-digit histograms, then [n_q] tickets.  Both are
-// zero between calls: dsa_workspace_init zeroes them, a top-k launch zeroes
+// Scratch: [n_q][4096] first-digit histograms, [n_q] tickets, then [n_q][4096]
+// second-digit histograms (split schedule).  All are zero between calls: dsa_workspace_init zeroes them, a top-k launch zeroes
 // each query's histogram and ticket once it has used them, and the one launch
 // that builds histograms without an indexer (hist_ready == 0) zeroes them first.
 // The split schedule adds [n_q][kSplitMax] candidate counts and the candidates.
@@ -871,6 +902,7 @@ void topk_bind_scratch(TopkArgs &a, void *scratch) {
     uint8_t *p = static_cast<uint8_t *>(scratch);
     a.ghist = reinterpret_cast<uint32_t *>(p);
     a.gticket = a.ghist + static_cast<size_t>(kBins) * a.n_q;
+    a.ghist2 = a.gticket + ticket_words(a.n_q);
     if (!topk_uses_split(a.n_q, a.L)) return;
     p += al(topk_zeroed_bytes(a.n_q));
     a.gcount = reinterpret_cast<uint32_t *>(p);

@@ -45,9 +45,10 @@ def test_workspace_bytes():
     lib = B.lib()
     q = _q(n_q=8, L=32768)
     assert lib.dsa_workspace_bytes(B.DSA_OP_INDEX_SCORES, ctypes.byref(q), 2048, 64, 512, 1) == 256
-    # top-k: status + first-digit histograms and one ticket per query (256-aligned)
-    # + (split schedule: 8 queries, ctx > 8192) per-chunk counts and candidates
-    hist = ((8 * 4096 * 4 + 8 * 4 + 255) // 256) * 256
+    # top-k: status + first-digit histograms, one ticket per query and the
+    # second-digit histograms (256-aligned) + (split schedule: 8 queries,
+    # ctx > 8192) per-chunk counts and candidates
+    hist = ((8 * 4096 * 4 + 8 * 4 + 8 * 4096 * 4 + 255) // 256) * 256  # tickets padded to 4 words
     split = hist + 8 * 64 * 4 + 8 * 64 * 1024 * 8
     assert lib.dsa_workspace_bytes(B.DSA_OP_TOPK, ctypes.byref(q), 2048, 64, 512, 1) == 256 + split
     q2 = _q(n_q=8, L=8192)

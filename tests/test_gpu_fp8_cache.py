@@ -3,9 +3,10 @@ DSA_FP8_E4M3): 512 E4M3 codes, the bf16 RoPE key and a float32 scale per row.
 
 Outputs are compared with the oracle's attention over the exact values
 sigma * e4m3(code) (fp64) within the bf16 tolerances; selections come from the
-indexer and stay bit-exact.  A second check needs no oracle: with power-of-two
-scales every sigma * e4m3(code) is exact in bf16, so the FP8 path must give the
-bf16 path's outputs bit for bit on the equivalent bf16 cache."""
+indexer and stay bit-exact.  A second check compares the two cache formats: with
+power-of-two scales every sigma * e4m3(code) is exact in bf16, so the bf16 path
+reads the same values from an equivalent bf16 cache; the FP8 path (fp16 tiles,
+sigma folded into an fp16 P) must be at least as close to the oracle."""
 import ctypes
 
 import numpy as np
@@ -114,13 +115,16 @@ def test_fp8_indexer_and_fp8_cache_chain(dev):
 
 
 @pytest.mark.parametrize("decode", [True, False])
-def test_fp8_cache_equals_bf16_cache_when_exact(dev, decode):
-    """Power-of-two row scales: sigma * e4m3(code) is exact in bf16, so both cache
-    formats put the same bf16 tiles in shared memory -- outputs and lse identical."""
+def test_fp8_cache_at_least_as_precise_as_bf16_cache(dev, decode):
+    """Power-of-two row scales: sigma * e4m3(code) is exact in bf16, so the bf16
+    path attends over exactly the FP8 cache's values.  Against the oracle, the FP8
+    path (exact fp16 codes, sigma applied to the logits and folded into an fp16 P)
+    is no less precise than the bf16 path (bf16 P), and both are within tolerance."""
     w = wl.scaled(D32, n_seq=2, L=2500, q_pos=(2499, 1000), q_seq=(0, 1), topk=2048, seed=31)
     xh = wl.make_inputs(w, layers=[0])
     kv8 = wl.fp8_latent_inputs(w, xh)[0]
-    e = torch.randint(-7, -4, (w.n_seq, w.L, 1), generator=torch.Generator().manual_seed(32)).float()
+    # 2^-8 .. 2^-7: about the recipe's amax / 448, so the latents keep their N(0, 1) size
+    e = torch.randint(-8, -6, (w.n_seq, w.L, 1), generator=torch.Generator().manual_seed(32)).float()
     kv8[..., 640:644] = torch.pow(2.0, e).contiguous().view(torch.uint8)
     c = kv8[..., :512].contiguous().view(torch.float8_e4m3fn).float() * torch.pow(2.0, e)
     kv16 = torch.cat([c.to(torch.bfloat16), kv8[..., 512:640].contiguous().view(torch.bfloat16)], dim=-1)
@@ -138,8 +142,32 @@ def test_fp8_cache_equals_bf16_cache_when_exact(dev, decode):
     got = B.Mla(ref.q, kv8.to(dev), out, w.d_lat, w.scale, lse)
     call(q, got, idx, cnt, w.topk, ws)
     assert B.dsa_check_status(ws) == B.DSA_OK
-    assert torch.equal(out, ref.out)
-    assert torch.equal(lse, ref.lse)
+    o_ref, l_ref = C.oracle_mla_fp8(w, xh, [kv8], 0, idx.cpu().numpy(), cnt.cpu().numpy())
+    C.assert_attention_close(out, o_ref, "bf16", "fp8 cache")
+    C.assert_attention_close(ref.out, o_ref, "bf16", "bf16 cache")
+    e8 = np.abs(out.float().cpu().numpy() - o_ref)
+    e16 = np.abs(ref.out.float().cpu().numpy() - o_ref)
+    assert e8.max() <= e16.max() * 1.05 and e8.mean() <= e16.mean() * 1.05, (e8.max(), e16.max(), e8.mean(), e16.mean())
+    C.assert_lse_close(lse, l_ref, "bf16")
+
+
+def test_fp8_cache_precision_margin(dev):
+    """The FP8 cache's worst error on a decode batch at GLM-5.2 shapes, with the
+    workload recipe's scales (amax / 448, not powers of two): well inside the
+    bf16 tolerance (measured max-abs is stated in the design notes)."""
+    w = wl.scaled(D32, n_seq=4, L=8000, q_pos=(7999, 7000, 5000, 3000), q_seq=(0, 1, 2, 3), topk=2048, seed=34)
+    xh = wl.make_inputs(w, layers=[0])
+    kv8h = wl.fp8_latent_inputs(w, xh)
+    x = C.to_device(xh)
+    q, _, mlas = C.descriptors(w, x)
+    m = C.with_fp8_caches(w, mlas, [t.to(dev) for t in kv8h])[0]
+    idx, cnt = C.random_selection(w, seed=35, device=dev)
+    ws = B.workspace(B.DSA_OP_MLA_DECODE, q, w.topk, device=dev)
+    B.dsa_sparse_mla_decode(q, m, idx, cnt, w.topk, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    o_ref, _ = C.oracle_mla_fp8(w, xh, kv8h, 0, idx.cpu().numpy(), cnt.cpu().numpy())
+    err = np.abs(m.out.float().cpu().numpy() - o_ref)
+    assert err.max() <= 1e-2 and err.mean() <= 1e-3, (err.max(), err.mean())
 
 
 def test_fp8_cache_noalloc(dev):
