@@ -632,6 +632,9 @@ def producers_measure(dev, flush, steps: int, hbm_peak: float, tc_peak: float, p
         tot = 0.0
         for _ in range(steps):
             flush.fill_(1)
+            # ~100 us of device spin so the eager call's host-side marshalling is
+            # enqueued before the start event fires: the kernels' time, not the host's
+            torch.cuda._sleep(200_000)
             ev[0].record()
             fn()
             ev[1].record()

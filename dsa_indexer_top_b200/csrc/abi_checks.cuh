@@ -3,6 +3,7 @@
 // the same inputs.  Internal; not part of the public header.
 #pragma once
 
+#include <climits>
 #include <cstdint>
 
 #include "dsa.h"
@@ -30,6 +31,15 @@ inline bool mla_tc_ok(const dsa_mla *m) {
     if (mla_kv_fp8(m))
         return shape && m->kv_row_stride % 16 == 0 && m->kv_seq_stride % 16 == 0 && m->kv_row_stride >= kFp8Row;
     return shape && m->kv_row_stride % 8 == 0 && m->kv_seq_stride % 8 == 0 && m->kv_row_stride >= kRow;
+}
+
+// bf16 caches on the tensor-core path are read by TMA row gathers over one 2-D
+// tensor of every sequence's rows: the sequence stride a whole number of rows
+// (or 0) and at most INT32_MAX rows in all.  Packed FP8 caches: no condition.
+inline bool mla_tc_rows_ok(const dsa_mla *m, int n_seq, int max_ctx) {
+    if (mla_kv_fp8(m)) return true;
+    const int64_t rows = mla_gather_rows(m->kv_seq_stride, m->kv_row_stride, n_seq, max_ctx);
+    return rows >= 1 && rows <= INT32_MAX;
 }
 
 // Every layer described and consistent with layer 0 (one shape, dtype, scale,

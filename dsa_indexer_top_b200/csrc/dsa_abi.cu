@@ -164,6 +164,14 @@ dsa_status do_index_scores(const dsa_queries *qs, const dsa_indexer *ix, float *
         const long long groups = (qs->n_q + G - 1) / G;
         a.total_items = groups * a.tiles_per_group;
         a.ghist = (ghist && G == 1) ? ghist : nullptr;  // fused into the epilogue
+        // Claimed work only where a claim rarely crosses into another query: one
+        // bf16 query per tile and at least 4096 key tiles per query.  A query
+        // change costs the CTA a pipeline drain for the new query tile and a
+        // histogram flush, which outweighs the balance on shorter contexts and on
+        // the FP8 form's smaller tiles (measured); those keep contiguous ranges.
+        a.work = (!f8 && G == 1 && a.tiles_per_group >= kIdxDynamicMinTiles)
+                     ? reinterpret_cast<unsigned long long *>(reinterpret_cast<uint8_t *>(status) + kIdxWorkOffset)
+                     : nullptr;
         a.q_scale = f8 ? ix->q_scale : nullptr;
         a.k_scale = f8 ? ix->k_scale : nullptr;
         a.ks_seq_stride = f8 ? ix->ks_seq_stride : 0;
@@ -286,8 +294,12 @@ dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, co
     a.status = status;
     bool tc = true;
     for (int l = 0; l < n_layers; ++l) tc = tc && mla_tc_ok(&layers[l]);
+    tc = tc && mla_tc_rows_ok(&m, qs->n_seq, qs->max_ctx);
     if (a.kv_fp8 && !tc) return DSA_ERR_UNSUPPORTED;  // packed FP8 caches: tensor-core path only
     if (tc) {
+        MlaMaps maps;
+        std::memset(&maps, 0, sizeof(maps));
+        if (!a.kv_fp8 && !encode_mla_maps(a, maps)) return DSA_ERR_CUDA;
         int n_splits, cpc;
         mla_plan(qs->n_q, n_layers, topk, decode, num_sms_current(), kMlaMaxSplits, n_splits, cpc);
         a.n_splits = n_splits;
@@ -296,10 +308,10 @@ dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, co
             a.part_o = reinterpret_cast<float *>(scratch);
             const size_t rows = static_cast<size_t>(n_layers) * qs->n_q * n_splits * kMlaHeads;
             a.part_ml = reinterpret_cast<float *>(scratch + rows * kLatent * sizeof(float));
-            if (launch_mla_tc(a, st) != cudaSuccess) return DSA_ERR_CUDA;
+            if (launch_mla_tc(a, maps, st) != cudaSuccess) return DSA_ERR_CUDA;
             return launch_mla_combine(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
         }
-        return launch_mla_tc(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+        return launch_mla_tc(a, maps, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
     }
     const size_t smem = sizeof(float) * (static_cast<size_t>(m.d_latent + m.d_rope) + topk);
     if (smem > 200 * 1024) return DSA_ERR_UNSUPPORTED;

@@ -10,6 +10,7 @@
 // path.  For them this entry point needs no workspace: its status word and
 // split-K partials live in g_mla_decode_scratch below, which every GPU that
 // loads the library keeps until the process exits.
+#include <cstring>
 #include <mutex>
 
 #include "abi_checks.cuh"
@@ -70,7 +71,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
     const dsa_status chk = check_mla_layers(mla, 1);
     if (chk != DSA_OK) return chk;
     // Only the tensor-core shape uses scratch: bf16 queries, 64 heads, 512 + 64.
-    if (!mla_tc_ok(mla)) return DSA_ERR_UNSUPPORTED;
+    if (!mla_tc_ok(mla) || !mla_tc_rows_ok(mla, queries->n_seq, queries->max_ctx)) return DSA_ERR_UNSUPPORTED;
     const dsa_mla &m = *mla;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     int dev = 0;
@@ -112,14 +113,17 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
     a.status = reinterpret_cast<uint32_t *>(scratch);
     a.n_splits = n_splits;
     a.chunks_per_cta = cpc;
+    MlaMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    if (!a.kv_fp8 && !encode_mla_maps(a, maps)) return DSA_ERR_CUDA;
     if (n_splits > 1) {
         a.part_o = reinterpret_cast<float *>(scratch + kStatusBytes);
         const size_t rows = static_cast<size_t>(queries->n_q) * n_splits * kMlaHeads;
         a.part_ml = reinterpret_cast<float *>(scratch + kStatusBytes + rows * kLatent * sizeof(float));
-        if (launch_mla_tc(a, st) != cudaSuccess) return DSA_ERR_CUDA;
+        if (launch_mla_tc(a, maps, st) != cudaSuccess) return DSA_ERR_CUDA;
         return launch_mla_combine(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
     }
-    return launch_mla_tc(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+    return launch_mla_tc(a, maps, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }
 
 extern "C" dsa_status dsa_noalloc_check_status(void *stream) {

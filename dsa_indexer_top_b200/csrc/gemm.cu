@@ -177,16 +177,21 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_tc_kernel(const __grid_cons
 // ---------------------------------------------------------------- few rows of A
 // The same contraction when A has at most kSkinnyM rows (decode-sized batches):
 // B (the weights) is streamed once with 16-byte loads, A's rows sit in shared
-// memory.  One CTA per (64 rows of B, K split, batch); each warp walks 8 rows of
-// B, its lanes splitting K in 8-element pieces; a row's M partial sums are
+// memory.  Each warp takes WR rows of B and keeps two 16-byte loads of each in
+// flight, its lanes splitting K in 8-element pieces; a row's M partial sums are
 // reduced across the warp and written like the tensor-core kernel's output
-// (fp32 split-K partials or bf16).  HBM-bound on B.
+// (fp32 split-K partials or bf16).  One CTA per (8 * WR rows of B, K split,
+// batch).  HBM-bound on B.  Two shapes: up to 4 rows of A with 8 rows of B per
+// warp, up to 16 rows of A with 4 (the accumulators fit the registers either way).
 constexpr int kSkinnyM = 16;
-constexpr int kSkinnyRows = 64;     // rows of B per CTA
 constexpr int kSkinnyThreads = 256;
-constexpr int kSkinnyMaxK = 2048;   // K per split held in shared memory (bf16)
+template <int MM, int WR>
+struct SkinnyCfg {
+    static constexpr int kRows = WR * (kSkinnyThreads / 32);  // rows of B per CTA
+};
 
-__global__ void __launch_bounds__(kSkinnyThreads) gemm_skinny_kernel(const GemmSkinnyArgs g) {
+template <int MM, int WR>
+__global__ void __launch_bounds__(kSkinnyThreads, 1) gemm_skinny_kernel(const GemmSkinnyArgs g) {
     extern __shared__ __align__(16) uint8_t sm_raw[];
     __nv_bfloat16 *a_sm = reinterpret_cast<__nv_bfloat16 *>(sm_raw);  // [M][kc]
     const int nb = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
@@ -203,50 +208,55 @@ __global__ void __launch_bounds__(kSkinnyThreads) gemm_skinny_kernel(const GemmS
         *reinterpret_cast<uint4 *>(a_sm + m * kc + pc * 8) = __ldg(reinterpret_cast<const uint4 *>(src));
     }
     __syncthreads();
-    for (int rr = 0; rr < kSkinnyRows / 8; ++rr) {
-        const int n = nb * kSkinnyRows + warp * (kSkinnyRows / 8) + rr;
-        if (n >= g.N) break;
-        const __nv_bfloat16 *brow = static_cast<const __nv_bfloat16 *>(g.b) + b * g.b_batch + static_cast<int64_t>(n) * g.b_row + k0;
-        float acc[kSkinnyM];
+    const int n0 = nb * SkinnyCfg<MM, WR>::kRows + warp * WR;
+    if (n0 < g.N) {
+        const int nr = min(WR, g.N - n0);
+        const __nv_bfloat16 *bbase = static_cast<const __nv_bfloat16 *>(g.b) + b * g.b_batch + static_cast<int64_t>(n0) * g.b_row + k0;
+        float acc[WR][MM];
 #pragma unroll
-        for (int m = 0; m < kSkinnyM; ++m) acc[m] = 0.f;
+        for (int r = 0; r < WR; ++r)
+#pragma unroll
+            for (int m = 0; m < MM; ++m) acc[r][m] = 0.f;
+#pragma unroll 2
         for (int pc = lane; pc < pieces; pc += 32) {
-            const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(brow + pc * 8));
-            float wf[8];
-            {
-                const uint32_t w4[4] = {wv.x, wv.y, wv.z, wv.w};
+            uint4 wv[WR];
 #pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[y]));
-                    wf[2 * y] = f.x;
-                    wf[2 * y + 1] = f.y;
-                }
-            }
+            for (int r = 0; r < WR; ++r)
+                wv[r] = r < nr ? __ldg(reinterpret_cast<const uint4 *>(bbase + r * g.b_row + pc * 8)) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
-            for (int m = 0; m < kSkinnyM; ++m) {
+            for (int m = 0; m < MM; ++m) {
                 if (m >= g.M) break;
                 const uint4 av = *reinterpret_cast<const uint4 *>(a_sm + m * kc + pc * 8);
                 const uint32_t a4[4] = {av.x, av.y, av.z, av.w};
 #pragma unroll
                 for (int y = 0; y < 4; ++y) {
-                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&a4[y]));
-                    acc[m] = fmaf(wf[2 * y], f.x, acc[m]);
-                    acc[m] = fmaf(wf[2 * y + 1], f.y, acc[m]);
+                    const float2 af = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&a4[y]));
+#pragma unroll
+                    for (int r = 0; r < WR; ++r) {
+                        const uint32_t w4[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+                        const float2 wf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[y]));
+                        acc[r][m] = fmaf(wf.x, af.x, acc[r][m]);
+                        acc[r][m] = fmaf(wf.y, af.y, acc[r][m]);
+                    }
                 }
             }
         }
 #pragma unroll
-        for (int m = 0; m < kSkinnyM; ++m) {
-            if (m >= g.M) break;
-            float v = acc[m];
+        for (int r = 0; r < WR; ++r) {
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) {
-                if (g.out_f32)
-                    g.out_f32[split * g.s_split + b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n] = v;
-                else
-                    static_cast<__nv_bfloat16 *>(g.out_bf16)[b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n] =
-                        __float2bfloat16_rn(v);
+            for (int m = 0; m < MM; ++m) {
+                if (m >= g.M) break;
+                float v = acc[r][m];
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+                if (lane == 0 && r < nr) {
+                    const int n = n0 + r;
+                    if (g.out_f32)
+                        g.out_f32[split * g.s_split + b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n] = v;
+                    else
+                        static_cast<__nv_bfloat16 *>(g.out_bf16)[b * g.s_batch + static_cast<int64_t>(m) * g.ldc + n] =
+                            __float2bfloat16_rn(v);
+                }
             }
         }
     }
@@ -263,16 +273,24 @@ cudaError_t launch_gemm_bn(const CUtensorMap &ta, const CUtensorMap &tb, const G
     return launch_pdl(gemm_tc_kernel<BN>, grid, dim3(kGemmThreads), Cfg::kSmem, st, ta, tb, g);
 }
 
-}  // namespace
 
-cudaError_t launch_gemm_skinny(const GemmSkinnyArgs &g, cudaStream_t st) {
+template <int MM, int WR>
+cudaError_t launch_skinny_cfg(const GemmSkinnyArgs &g, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(g.M) * g.k_per_split * 2;
-    cudaError_t e = cudaFuncSetAttribute(gemm_skinny_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_skinny_kernel<MM, WR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int k_splits = (g.K + g.k_per_split - 1) / g.k_per_split;
-    dim3 grid((g.N + kSkinnyRows - 1) / kSkinnyRows, k_splits, g.batch);
-    return launch_pdl(gemm_skinny_kernel, grid, dim3(kSkinnyThreads), smem, st, g);
+    constexpr int rows = SkinnyCfg<MM, WR>::kRows;
+    dim3 grid((g.N + rows - 1) / rows, k_splits, g.batch);
+    return launch_pdl(gemm_skinny_kernel<MM, WR>, grid, dim3(kSkinnyThreads), smem, st, g);
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_skinny(const GemmSkinnyArgs &g, cudaStream_t st) {
+    if (g.M < 1 || g.M > kSkinnyM) return cudaErrorInvalidValue;
+    return g.M <= 4 ? launch_skinny_cfg<4, 8>(g, st) : launch_skinny_cfg<16, 4>(g, st);
 }
 
 cudaError_t launch_gemm_tc(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st) {

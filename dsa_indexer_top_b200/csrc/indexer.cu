@@ -17,9 +17,13 @@
 //               queries): tcgen05.ld of its 32 lanes (one key per lane), ReLU,
 //               multiply by w and sum the 32 heads inside the thread, causal mask,
 //               coalesced fp32 store of one score per key per query.
-// Work items are (query group, key tile) pairs split into contiguous ranges over
-// a grid of at most two CTAs per SM (one query per tile; three for FP8) or one
-// (several); tiles past the group's last visible key are skipped.
+// Work items are (query group, key tile) pairs over a grid of at most two CTAs
+// per SM (one query per tile; three for FP8) or one (several): contiguous
+// ranges per CTA, or, for long bf16 contexts, claimed two at a time from a
+// counter in the workspace so that the CTAs of faster SMs take more of them and
+// all finish together.  The producer hands each item to the MMA issuer and the
+// epilogue through a small ring in shared memory.  Tiles past the group's last
+// visible key are skipped.
 //
 // FP8 variant (E4M3 queries and keys, each row scaled by a positive float): the
 // same kernel with 16 KB tiles (one 128-byte box of E4M3 bytes per tile), four
@@ -36,6 +40,8 @@ namespace dsa {
 namespace {
 
 constexpr int kTileKeys = 128;
+constexpr int kClaim = 2;  // work items per claim
+constexpr int kRing = 8;   // items in flight between the producer and the epilogue (> stages + 2)
 
 // F8: queries and keys are E4M3 bytes (the FP8 variant) instead of bf16.
 template <int G, bool F8>
@@ -83,6 +89,71 @@ __device__ __forceinline__ void group_info(const IdxTcArgs &a, int g, int &seq, 
     }
 }
 
+// A run of consecutive work items, as (query group, key tile), stepped without
+// a division per item: `left` items from tile j of group g.
+struct ItemRun {
+    long long left = 0;
+    int g = 0, j = 0;
+    __device__ __forceinline__ void start(long long first, long long count, int tpg) {
+        left = count;
+        g = static_cast<int>(first / tpg);
+        j = static_cast<int>(first - static_cast<long long>(g) * tpg);
+    }
+    __device__ __forceinline__ void take(int tpg, int &og, int &oj) {
+        og = g;
+        oj = j;
+        --left;
+        if (++j == tpg) {
+            j = 0;
+            ++g;
+        }
+    }
+    // the rest of the group just taken is skipped too (its tiles lie further
+    // past the last visible key, or the group has no valid query)
+    __device__ __forceinline__ void skip_group(int tpg) {
+        if (j != 0) {
+            left -= min(left, static_cast<long long>(tpg - j));
+            j = 0;
+            ++g;
+        }
+    }
+};
+
+// The work items a consumer role (MMA issuer, epilogue warp) walks, in the
+// producer's order: with claimed work the ring the producer fills (group -1
+// ends it); otherwise the CTA's contiguous range, skipping what the producer
+// skips.
+template <int G>
+struct ItemWalk {
+    ItemRun run;
+    int sg = -1, seq = -1, max_pos = -1;
+    __device__ __forceinline__ ItemWalk(long long begin, long long end, int tpg) { run.start(begin, end - begin, tpg); }
+    __device__ __forceinline__ bool next(const IdxTcArgs &a, int tpg, long long k, const int2 *ring,
+                                         uint64_t *ring_bar, int *abort_flag, int &g, int &j) {
+        if (!a.work) {
+            while (run.left > 0) {
+                run.take(tpg, g, j);
+                if (g != sg) {
+                    group_info<G>(a, g, seq, max_pos);
+                    sg = g;
+                }
+                if (seq < 0 || j * kTileKeys > max_pos) {
+                    run.skip_group(tpg);
+                    continue;
+                }
+                return true;
+            }
+            return false;
+        }
+        const int r = static_cast<int>(k % kRing);
+        if (!mbar_wait(&ring_bar[r], static_cast<uint32_t>((k / kRing) & 1), a.status, abort_flag)) return false;
+        const volatile int *v = reinterpret_cast<const volatile int *>(&ring[r]);
+        g = v[0];
+        j = v[1];
+        return g >= 0;
+    }
+};
+
 template <int G, bool F8>
 __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasPerSm)
     idx_score_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -109,6 +180,9 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
     // tile only), flushed into a.ghist when the epilogue moves to another query.
     __shared__ uint32_t ehist[G == 1 ? kTopkBins : 1];
     __shared__ uint64_t epi_bar;
+    __shared__ int2 item_q[kRing];          // claimed (group, tile) in issue order; group -1 ends the work
+    __shared__ uint64_t item_bar[kRing];    // item_q[r] written (one arrival per use)
+    static_assert(kRing >= S + 3, "the ring outlasts the producer's lead over the epilogue");
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -126,6 +200,7 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
         mbar_init(&b_empty, 1);
         mbar_init(&mma_done, 1);
         mbar_init(&epi_bar, 4);
+        for (int r = 0; r < kRing; ++r) mbar_init(&item_bar[r], 1);
         abort_flag = 0;
         fence_barrier_init();
         tma_prefetch_desc(&tmap_k);
@@ -145,8 +220,6 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
     griddep_wait();
 
     const long long total = a.total_items;
-    const long long begin = total * blockIdx.x / gridDim.x;
-    const long long end = total * (blockIdx.x + 1) / gridDim.x;
     const int tpg = a.tiles_per_group;
 
     if (warp == 0) {
@@ -161,15 +234,42 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
             long long k_tiles = 0;
             int last_use[S];
             for (int s = 0; s < S; ++s) last_use[s] = -1;
-            for (long long it = begin; it < end; ++it) {
-                const int g = static_cast<int>(it / tpg);
-                const int j = static_cast<int>(it % tpg);
+            // Claimed work: the claim after the current one is requested as soon as
+            // the current one starts, so its latency hides behind the current items.
+            // Otherwise one contiguous range per CTA.
+            ItemRun run;
+            long long next = total;
+            if (a.work) {
+                next = static_cast<long long>(atomicAdd(a.work, static_cast<unsigned long long>(kClaim)));
+            } else {
+                const long long begin = total * blockIdx.x / gridDim.x;
+                run.start(begin, total * (blockIdx.x + 1) / gridDim.x - begin, tpg);
+            }
+            for (;;) {
+                if (run.left == 0) {
+                    if (next >= total) break;
+                    run.start(next, min(static_cast<long long>(kClaim), total - next), tpg);
+                    next = static_cast<long long>(atomicAdd(a.work, static_cast<unsigned long long>(kClaim)));
+                }
+                int g, j;
+                run.take(tpg, g, j);
                 if (g != cur_g) {
                     group_info<G>(a, g, seq, max_pos);
                     cur_g = g;
                     group_loaded = false;
+                    // a group without one valid query is skipped whole, so the epilogue
+                    // never checks it: report it here
+                    if (seq < 0 || max_pos < 0) report_status(a.status, DSA_ERR_INVALID);
                 }
-                if (seq < 0 || j * kTileKeys > max_pos) continue;
+                if (seq < 0 || j * kTileKeys > max_pos) {
+                    run.skip_group(tpg);
+                    continue;
+                }
+                if (a.work) {  // claimed work: the consumers learn the item from the ring
+                    const int r = static_cast<int>(k_tiles % kRing);
+                    item_q[r] = make_int2(g, j);
+                    mbar_arrive(&item_bar[r]);
+                }
                 if (!group_loaded) {
                     if (b_uses > 0 &&
                         !mbar_wait(&b_empty, (b_uses - 1) & 1, a.status, &abort_flag))
@@ -194,6 +294,10 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
                 last_use[stage] = use;
                 ++k_tiles;
             }
+            if (a.work) {
+                item_q[k_tiles % kRing] = make_int2(-1, 0);  // the end (also after an abort: the consumers stop)
+                mbar_arrive(&item_bar[k_tiles % kRing]);
+            }
             // Drain: every copy this thread issued has landed before the CTA exits.
             for (int s = 0; s < S; ++s)
                 if (last_use[s] >= 0) mbar_wait(&full_bar[s], last_use[s] & 1, a.status, nullptr);
@@ -202,19 +306,17 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
-            int cur_g = -1, seq = -1, max_pos = -1;
+            int cur_g = -1;
             bool group_ready = false;
             int b_uses = 0;
             long long k_tiles = 0;
-            for (long long it = begin; it < end; ++it) {
-                const int g = static_cast<int>(it / tpg);
-                const int j = static_cast<int>(it % tpg);
+            ItemWalk<G> walk(total * blockIdx.x / gridDim.x, total * (blockIdx.x + 1) / gridDim.x, tpg);
+            int g, j;
+            while (walk.next(a, tpg, k_tiles, item_q, item_bar, &abort_flag, g, j)) {
                 if (g != cur_g) {
-                    group_info<G>(a, g, seq, max_pos);
                     cur_g = g;
                     group_ready = false;
                 }
-                if (seq < 0 || j * kTileKeys > max_pos) continue;
                 if (!group_ready) {
                     if (b_uses > 0) umma_commit(&b_empty);  // previous group's MMAs release B
                     if (!mbar_wait(&b_full, b_uses & 1, a.status, &abort_flag)) break;
@@ -284,9 +386,9 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
             }
             epi_sync();
         };
-        for (long long it = begin; it < end; ++it) {
-            const int g = static_cast<int>(it / tpg);
-            const int j = static_cast<int>(it % tpg);
+        ItemWalk<G> walk(total * blockIdx.x / gridDim.x, total * (blockIdx.x + 1) / gridDim.x, tpg);
+        int g, j;
+        while (walk.next(a, tpg, k_tiles, item_q, item_bar, &abort_flag, g, j)) {
             if (g != cur_g) {
                 if (fuse_hist && hist_dirty) {
                     flush_hist(cur_g);
@@ -319,7 +421,6 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
                     }
                 }
             }
-            if (seq < 0 || j * kTileKeys > max_pos) continue;
             const int acc = static_cast<int>(k_tiles & 1);
             const int acc_use = static_cast<int>(k_tiles >> 1);
             const int s = j * kTileKeys + quad * 32 + lane;
@@ -363,6 +464,14 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
     griddep_launch_dependents();
     tc_fence_before();
     __syncthreads();
+    if (threadIdx.x == 0 && a.work) {
+        // every role of this CTA is done claiming; the last CTA to get here leaves
+        // the counter zero for the next launch
+        if (atomicAdd(a.work + 1, 1ull) == gridDim.x - 1) {
+            atomicExch(a.work, 0ull);
+            atomicExch(a.work + 1, 0ull);
+        }
+    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);

@@ -46,6 +46,11 @@ constexpr int kMaxTopk = 4096;
 constexpr int kMaxLayers = 4;
 
 // ------------------------------------------------------------------ indexer
+// Byte offset, inside the workspace's 256-byte status block, of the indexer's
+// two work counters (unsigned 64-bit; zeroed with the workspace).
+constexpr size_t kIdxWorkOffset = 128;
+constexpr int kIdxDynamicMinTiles = 4096;  // key tiles per query from which work is claimed
+
 struct IdxTcArgs {
     const float *w;
     const int32_t *q_seq;
@@ -59,6 +64,9 @@ struct IdxTcArgs {
     long long total_items;
     uint32_t *ghist;      // non-null (one query per tile only): accumulate the top-k
                           // first-digit histogram [n_q][4096] of the scores written
+    unsigned long long *work;  // claimed work: [0] next work item, [1] CTAs finished,
+                               // zero between launches (the last CTA re-zeroes them);
+                               // null: contiguous ranges of items per CTA
     // FP8 (E4M3) operands only: positive per-(query, head) and per-key scales, or null
     const float *q_scale;    // [n_q][32]
     const float *k_scale;    // sequence b's key s at k_scale[b * ks_seq_stride + s]
@@ -265,10 +273,25 @@ struct MlaArgs {
     float *part_ml;      // [layers][n_q][n_splits][64][2] (max, sum) in log2 units
 };
 
+// TMA descriptors of the tensor-core MLA with a bf16 cache (one per layer):
+// kv 2-D {576, rows of all sequences}, boxes {64, 1} (the row gathers' unit,
+// four rows per gather); q 2-D {576, n_q * 64}, boxes {64, 64}; both 128-byte
+// swizzled.
+struct MlaMaps {
+    CUtensorMap kv[kMaxLayers];
+    CUtensorMap q[kMaxLayers];
+};
+
 // Tensor-core sparse MLA (bf16 queries and outputs, 64 heads, 512 + 64; bf16 or
 // packed FP8 caches).  n_splits == 1 writes the final output; otherwise partials
-// followed by launch_mla_combine.
-cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st);
+// followed by launch_mla_combine.  `maps` (bf16 caches; ignored for FP8) come
+// from encode_mla_maps.
+cudaError_t launch_mla_tc(const MlaArgs &a, const MlaMaps &maps, cudaStream_t st);
+bool encode_mla_maps(const MlaArgs &a, MlaMaps &maps);
+// Rows of the 2-D tensor the bf16 row gathers read (every sequence's rows, at
+// kv_row_stride apart): -1 when the sequence stride is not a whole number of
+// rows.  The tensor-core path needs 1 .. INT32_MAX.
+int64_t mla_gather_rows(int64_t kv_seq_stride, int64_t kv_row_stride, int n_seq, int max_ctx);
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st);
 cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st);
 

@@ -29,12 +29,15 @@
 //   epilogue (warps 0-7)  reads O^T from TMEM: the final bf16 output (one CTA
 //            per query) or fp32 partials + (max, sum) per head for a split-K
 //            merge (decode with few queries).
+#include <climits>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
+#include "tma_encode.cuh"
 
 namespace dsa {
 namespace {
@@ -91,7 +94,7 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
 // four sub-partitions (three on one of them, whose 16K-register file they
 // share) allow at most 168 registers per thread.
 template <bool kFp8>
-__global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a) {
+__global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a, const __grid_constant__ MlaMaps maps) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                 ~uintptr_t(1023));
@@ -113,9 +116,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     const float c2 = a.scale * kLog2e;
 
     if (tid == 0) {
-        mbar_init(&q_full, 4);
+        mbar_init(&q_full, kFp8 ? 4 : 1);  // bf16: one arrival with the TMA byte count
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&slot_full[s], 4);
+            mbar_init(&slot_full[s], 4);    // one per producer warp (+ the TMA bytes for bf16)
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], 4);
             mbar_init(&o_done[s], 1);
@@ -135,7 +138,17 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
     const uint32_t tbase = tmem_base_sh;
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(lp.q) + static_cast<int64_t>(i) * kMlaHeads * kRow;
     const uint32_t q_addr = smem_u32(q_sm);
-    if (warp >= 4 && warp < 8) {
+    if (!kFp8 && tid == 4 * 32) {
+        // The query tile is an input of the step, not written by the kernel this
+        // launch depends on: nine 64-head x 64-dim TMA boxes, issued before the
+        // dependency wait.
+        tma_prefetch_desc(&maps.q[layer]);
+        tma_prefetch_desc(&maps.kv[layer]);
+        mbar_arrive_expect_tx(&q_full, kQBytes);
+#pragma unroll 1
+        for (int b = 0; b < kBlocks; ++b) tma_load_2d(q_sm + b * kBlockBytes, &maps.q[layer], &q_full, 64 * b, i * kMlaHeads);
+    }
+    if (kFp8 && warp >= 4 && warp < 8) {
         // The query tile is an input of the step, not written by the kernel this
         // launch depends on: its copy (heads 16*pw .. 16*pw+15 per producer warp)
         // is issued before the dependency wait.
@@ -175,10 +188,19 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             }
         }
     }
+    int seq = a.q_seq[i];  // an input of the step, like the query tile
     griddep_wait();
 
     const int si = i / a.sel_group;  // the selection row this query reads
-    int seq = a.q_seq[i];
+    const int32_t *sel = a.idx + static_cast<int64_t>(si) * a.topk;
+    const int c_begin = split * a.chunks_per_cta;
+    // producers: the first chunk's indices are requested with the count, not after it
+    int r_first = -1, f_first = -1;
+    if (warp >= 4 && warp < 8 && c_begin * kChunk < a.topk) {
+        const int j0 = c_begin * kChunk + 16 * (warp - 4) + (lane & 15);
+        if (j0 < a.topk) r_first = __ldg(sel + j0);
+        f_first = __ldg(sel + c_begin * kChunk);
+    }
     int cnt = a.cnt[si];
     if (!(seq >= 0 && seq < a.n_seq && cnt >= 0 && cnt <= a.topk)) {
         if (tid == 0) report_status(a.status, DSA_ERR_INVALID);
@@ -186,24 +208,33 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
         seq = 0;
     }
     const int nch = (cnt + kChunk - 1) / kChunk;
-    const int c_begin = split * a.chunks_per_cta;
     const int nloc = max(0, min(c_begin + a.chunks_per_cta, nch) - c_begin);
-    const __nv_bfloat16 *kv = static_cast<const __nv_bfloat16 *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
     const uint8_t *kv8 = static_cast<const uint8_t *>(lp.kv) + static_cast<int64_t>(seq) * a.kv_seq_stride;
-    const int32_t *sel = a.idx + static_cast<int64_t>(si) * a.topk;
 
     if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ producers
         const int pw = warp - 4;  // rows (and the query tile's heads) 16*pw .. 16*pw+15
-        bool q_arrived = false;
+        bool q_arrived = false;   // FP8: this warp's share of the query tile is in
+        int issued = 0;           // bf16: chunks whose row gathers this warp has issued
+        // bf16: the rows of all sequences form one 2-D tensor (rows of kv_row_stride)
+        const int seq_row0 = a.kv_row_stride > 0 ? static_cast<int>(static_cast<int64_t>(seq) * (a.kv_seq_stride / a.kv_row_stride)) : 0;
+        const int rl = 16 * pw + (lane & 15);
+        int r_cur = r_first, f_cur = f_first;  // chunk t's index (this lane's row) and first row
         for (int t = 0; t < nloc; ++t) {
             const int c = c_begin + t, s = t & 1, u = t >> 1;
+            // chunk t + 1's indices are requested now: they land while this chunk
+            // waits for its slot and is issued
+            int r_nx = -1, f_nx = -1;
+            if (t + 1 < nloc) {
+                const int j1 = (c + 1) * kChunk + rl;
+                if (j1 < cnt) r_nx = __ldg(sel + j1);
+                f_nx = __ldg(sel + (c + 1) * kChunk);
+            }
             if (t >= 2 && !mbar_wait(&o_done[s], (u - 1) & 1, a.status, &abort_flag)) break;
-            const int rl = 16 * pw + (lane & 15);
             const int j = c * kChunk + rl;
             int r = -1;
             if (j < cnt) {
-                r = __ldg(sel + j);
+                r = r_cur;
                 if (r < 0 || r >= a.L) {
                     report_status(a.status, DSA_ERR_INVALID);
                     r = -1;
@@ -212,21 +243,32 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             if (lane < 16) row_idx[s][rl] = r;
             const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
             if constexpr (!kFp8) {
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int row = 16 * pw + rr;
-                    const int src = __shfl_sync(0xffffffffu, r, rr);
+                // The warp's 16 rows as 4 row gathers per 64-dim block (36 TMA ops,
+                // lanes 0-31 then 0-3): padding rows and rejected indices fetch the
+                // chunk's first row instead (in range; masked in the softmax), so
+                // every op moves whole rows and the byte count is fixed.
+                int f = f_cur;
+                if (f < 0 || f >= a.L) f = 0;
+                const int gr = seq_row0 + (r >= 0 ? r : f);
+                const int g0 = lane / 9, b0 = lane - 9 * g0;
+                int y0[4], y1[4];
 #pragma unroll
-                    for (int tt = 0; tt < 3; ++tt) {
-                        const int ch = lane + 32 * tt;
-                        if (ch < kRow / 8) {
-                            const uint32_t dst = sb + (ch >> 3) * kBlockBytes + sw128_offset(row, ch & 7);
-                            if (src >= 0)
-                                cp_async_16(dst, kv + static_cast<int64_t>(src) * a.kv_row_stride + ch * 8);
-                            else
-                                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
-                        }
-                    }
+                for (int qq = 0; qq < 4; ++qq) {
+                    y0[qq] = __shfl_sync(0xffffffffu, gr, 4 * g0 + qq);
+                    y1[qq] = __shfl_sync(0xffffffffu, gr, 12 + qq);
                 }
+                __syncwarp();  // row_idx written before the arrival releases it
+                if (lane == 0) mbar_arrive_expect_tx(&slot_full[s], 16 * kRow * 2);
+                const uint32_t wb = sb + (16 * pw) * 128;
+                tma_gather4(wb + b0 * kBlockBytes + g0 * 512, &maps.kv[layer], &slot_full[s], 64 * b0, y0[0], y0[1],
+                            y0[2], y0[3]);
+                if (lane < 4)
+                    tma_gather4(wb + (5 + lane) * kBlockBytes + 3 * 512, &maps.kv[layer], &slot_full[s],
+                                64 * (5 + lane), y1[0], y1[1], y1[2], y1[3]);
+                issued = t + 1;
+                r_cur = r_nx;
+                f_cur = f_nx;
+                continue;
             } else {
                 // Lane l takes latent dims 16l..16l+15 of each of the warp's 16 rows:
                 // all 16 code loads are issued before any is widened (exactly, to
@@ -267,7 +309,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
             }
             cp_async_commit();
             cp_async_wait_all();  // the query tile (first chunk) and this chunk's rows
-            if constexpr (kFp8) {
+            {
                 // this lane's RoPE pieces (bf16, copied above) to fp16, in place
                 if (lane < 8) {
 #pragma unroll 4
@@ -292,12 +334,22 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a)
                 mbar_arrive(&slot_full[s]);
             }
             q_arrived = true;
+            r_cur = r_nx;
+            f_cur = f_nx;
         }
-        if (!q_arrived) {  // no chunk for this CTA (or an abort): the query tile still counts
+        if (kFp8 && !q_arrived) {  // no chunk for this CTA (or an abort): the query tile still counts
             cp_async_wait_all();
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&q_full);
+        }
+        if (!kFp8 && lane == 0) {
+            // every TMA copy this warp requested has landed before the CTA may exit
+            // (the consumers may have stopped early on an abort): the last phase of
+            // each slot it filled, and the query tile
+            for (int t = max(0, issued - 2); t < issued; ++t)
+                mbar_wait(&slot_full[t & 1], (t >> 1) & 1, a.status, nullptr);
+            if (pw == 0) mbar_wait(&q_full, 0, a.status, nullptr);
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
@@ -717,17 +769,49 @@ __global__ void __launch_bounds__(128) mla_generic_kernel(const MlaArgs a) {
 }
 
 template <bool kFp8>
-cudaError_t launch_mla_tc_t(const MlaArgs &a, cudaStream_t st) {
+cudaError_t launch_mla_tc_t(const MlaArgs &a, const MlaMaps &maps, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_splits, a.n_q, a.n_layers);
-    return launch_pdl(mla_tc_kernel<kFp8>, grid, dim3(kMlaThreads), kMlaSmem, st, a);
+    return launch_pdl(mla_tc_kernel<kFp8>, grid, dim3(kMlaThreads), kMlaSmem, st, a, maps);
 }
 
 }  // namespace
 
-cudaError_t launch_mla_tc(const MlaArgs &a, cudaStream_t st) {
-    return a.kv_fp8 ? launch_mla_tc_t<true>(a, st) : launch_mla_tc_t<false>(a, st);
+int64_t mla_gather_rows(int64_t kv_seq_stride, int64_t kv_row_stride, int n_seq, int max_ctx) {
+    if (kv_row_stride <= 0 || kv_seq_stride % kv_row_stride != 0) return -1;
+    return static_cast<int64_t>(n_seq - 1) * (kv_seq_stride / kv_row_stride) + max_ctx;
+}
+
+bool encode_mla_maps(const MlaArgs &a, MlaMaps &maps) {
+    EncodeTiledFn enc = tma_encode_fn();
+    if (!enc) return false;
+    const int64_t rows = mla_gather_rows(a.kv_seq_stride, a.kv_row_stride, a.n_seq, a.L);
+    if (rows < 1 || rows > INT32_MAX || static_cast<int64_t>(a.n_q) * kMlaHeads > INT32_MAX) return false;
+    const cuuint32_t es[2] = {1, 1};
+    for (int l = 0; l < a.n_layers; ++l) {
+        // cache rows: {576 dims, rows}, one-row boxes of 64 dims (the gathers' unit)
+        const cuuint64_t kd[2] = {static_cast<cuuint64_t>(kRow), static_cast<cuuint64_t>(rows)};
+        const cuuint64_t ks[1] = {static_cast<cuuint64_t>(a.kv_row_stride) * 2};
+        const cuuint32_t kb[2] = {64, 1};
+        if (enc(&maps.kv[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.layer[l].kv), kd, ks, kb, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+        // queries: {576 dims, n_q * 64 heads}, boxes of 64 dims x 64 heads
+        const cuuint64_t qd[2] = {static_cast<cuuint64_t>(kRow), static_cast<cuuint64_t>(a.n_q) * kMlaHeads};
+        const cuuint64_t qs[1] = {static_cast<cuuint64_t>(kRow) * 2};
+        const cuuint32_t qb[2] = {64, static_cast<cuuint32_t>(kMlaHeads)};
+        if (enc(&maps.q[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.layer[l].q), qd, qs, qb, es,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return false;
+    }
+    return true;
+}
+
+cudaError_t launch_mla_tc(const MlaArgs &a, const MlaMaps &maps, cudaStream_t st) {
+    return a.kv_fp8 ? launch_mla_tc_t<true>(a, maps, st) : launch_mla_tc_t<false>(a, maps, st);
 }
 
 cudaError_t launch_mla_combine(const MlaArgs &a, cudaStream_t st) {
@@ -753,4 +837,3 @@ cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st) {
 }
 
 }  // namespace dsa
-

@@ -129,6 +129,19 @@ __device__ __forceinline__ void tma_load_3d(void *dst, const void *map, uint64_t
         : "memory");
 }
 
+// Four rows of a 2-D tensor map (row coordinates y0..y3, columns from x, a box
+// one row high) into four consecutive box-sized pieces of shared memory: the
+// row gather of sm_100 TMA.  With 128-byte swizzling the pieces are swizzled by
+// their shared-memory address, so four rows can fill half of an 8-row atom.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const void *map, uint64_t *bar, int x, int y0, int y1,
+                                            int y2, int y3) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+        : "memory");
+}
+
 // L2 policy for data read once (streamed keys): evict first.
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
     uint64_t pol;

@@ -40,12 +40,21 @@
  *    pointers unless stated otherwise; the library never allocates, frees or
  *    synchronises inside a compute call.  `stream` is a cudaStream_t (NULL =
  *    legacy default stream); work is enqueued on it and results are valid in
- *    stream order.
+ *    stream order.  Kernels are launched with programmatic dependent launch:
+ *    one may start while the previous kernel on the stream finishes and read
+ *    the inputs that no kernel of the call writes (the attention's query tile
+ *    and query sequences) before it waits for that kernel.  A kernel of the
+ *    caller's that writes those inputs just before the call must therefore not
+ *    release its dependents early (a kernel that never executes
+ *    griddepcontrol.launch_dependents does not).
  *  - Workspace: `ws` is a device buffer of at least dsa_workspace_bytes(...)
  *    bytes, 256-byte aligned.  Its first 256 bytes hold a status word that
  *    kernels set on device-detected errors (out-of-range positions or indices,
- *    a bounded wait that ran out).  Zero the workspace once with
- *    dsa_workspace_init(); read (and clear) the status with dsa_check_status().
+ *    a bounded wait that ran out) and the counters from which the tensor-core
+ *    indexer's CTAs claim their work (zero between calls).  Zero the workspace
+ *    once with dsa_workspace_init(); read (and clear) the status with
+ *    dsa_check_status().  Calls that share a workspace must run one after
+ *    another (one stream, or streams ordered by events), never concurrently.
  *    One workspace of dsa_workspace_bytes(DSA_OP_INDEXSHARE_GROUP, ...) bytes
  *    serves the separate calls of a step (dsa_index_scores, dsa_topk,
  *    dsa_sparse_mla_*) on the same queries: every call's scratch leaves alone

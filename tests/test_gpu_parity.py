@@ -322,10 +322,38 @@ def test_sparse_mla_alone(dev, decode, topk, L):
     C.assert_lse_close(mlas[0].lse, lse, "bf16")
 
 
-def test_device_detects_bad_positions(dev):
-    w = wl.scaled(D32, n_seq=2, L=1000, q_pos=(999, 500), q_seq=(0, 1))
+# 4096 key tiles per query: the tensor-core indexer's CTAs claim their work from
+# a counter in the workspace instead of taking contiguous ranges
+L_CLAIMED = 4096 * 128
+
+
+def test_claimed_work_repeated_steps_one_workspace(dev):
+    """Long-context indexer steps whose CTAs claim work from the workspace
+    counter: the last CTA of each launch re-zeroes it, so three fused indexer ->
+    top-k steps on one workspace all match the oracle."""
+    w = wl.scaled(D32, n_seq=2, L=L_CLAIMED, q_pos=(L_CLAIMED - 1, 300001), q_seq=(0, 1))
+    xh = wl.make_inputs(w, layers=[])
+    x = C.to_device(xh)
+    q, ix, _ = C.descriptors(w, x)
+    ix.flags = B.DSA_INDEXER_TOPK_HIST
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, 1, dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    _, ridx, rcnt = C.oracle_selection(w, xh)
+    for step in range(3):
+        idx = torch.full((w.n_q, w.topk), -7, dtype=torch.int32, device=dev)
+        cnt = torch.full((w.n_q,), -7, dtype=torch.int32, device=dev)
+        B.dsa_index_scores(q, ix, scores, ws)
+        B.dsa_topk(q, scores, w.topk, idx, cnt, ws, flags=B.DSA_TOPK_HIST_FROM_INDEXER)
+        assert B.dsa_check_status(ws) == B.DSA_OK
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt, err_msg=f"step {step}")
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx, err_msg=f"step {step}")
+
+
+@pytest.mark.parametrize("L", [1000, L_CLAIMED])
+def test_device_detects_bad_positions(dev, L):
+    w = wl.scaled(D32, n_seq=2, L=L, q_pos=(L - 1, 500), q_seq=(0, 1))
     x = C.to_device(wl.make_inputs(w, layers=[]))
-    x["q_pos"][1] = 5000  # beyond the cache
+    x["q_pos"][1] = L + 4000  # beyond the cache
     q, ix, _ = C.descriptors(w, x)
     ws = B.workspace(B.DSA_OP_INDEX_SCORES, q, device=dev)
     scores = B.scores_buffer(w.n_q, w.L, dev)
