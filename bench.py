@@ -360,7 +360,9 @@ class E2EStep:
         s = self.s
         self.ev[0].record()
         self.d_in.copy_(self.h_in, non_blocking=True)
+        t0 = time.perf_counter()
         B.dsa_indexshare_group(self.q, self.ix, self.mlas, s.w.topk, self.idx, self.cnt, s.ws)
+        self.call_s = time.perf_counter() - t0
         self.h_out.copy_(self.d_out, non_blocking=True)
         self.ev[1].record()
 
@@ -598,7 +600,7 @@ def e2e_measure(step: Step, world: int, dev, flush, steps: int):
         e2e.run()
     torch.cuda.synchronize()
     barrier(world)
-    te, wall = 0.0, 0.0
+    te, wall, call = 0.0, 0.0, 0.0
     for _ in range(steps):
         flush.fill_(1)
         torch.cuda.synchronize()
@@ -606,12 +608,14 @@ def e2e_measure(step: Step, world: int, dev, flush, steps: int):
         e2e.run()
         torch.cuda.synchronize()
         wall += time.perf_counter() - t0
+        call += e2e.call_s
         te += e2e.ms()
     te = max_over_ranks(te, world, dev)
     w = step.w
     return {"value": world * w.n_q * w.n_layers * steps / (te * 1e-3), "unit": UNIT,
             "h2d_bytes_per_step": e2e.h2d, "d2h_bytes_per_step": e2e.d2h, "steps": steps,
             "host_wall_ms_per_step": 1e3 * wall / steps,
+            "host_call_us": 1e6 * call / steps,  # the group call's own host time (checks, maps, launches)
             "how": "eager each step: pinned H2D of the query inputs, dsa_indexshare_group, D2H of outputs + indices"}
 
 

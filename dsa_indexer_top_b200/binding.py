@@ -122,8 +122,13 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(stream):
     if stream is None:
+        if _raw_stream is not None:
+            return ctypes.c_void_p(_raw_stream(torch.cuda.current_device()))
         stream = torch.cuda.current_stream()
     return ctypes.c_void_p(stream.cuda_stream)
 
@@ -139,22 +144,40 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 # ------------------------------------------------------------------ descriptors
+class _CStruct:
+    """A descriptor whose C struct (pointers, strides, sizes) is built on first
+    use and kept until a field is assigned: repeated calls skip the marshalling.
+    The tensors are held, so their pointers stay valid; a tensor whose storage is
+    replaced in place (Tensor.set_) needs its field assigned again."""
+
+    def __setattr__(self, name, value):
+        object.__setattr__(self, name, value)
+        object.__setattr__(self, "_cs", None)
+
+    def c(self):
+        cs = self.__dict__.get("_cs")
+        if cs is None:
+            cs = self._make()
+            object.__setattr__(self, "_cs", cs)
+        return cs
+
+
 @dataclass
-class Queries:
+class Queries(_CStruct):
     q_seq: torch.Tensor          # int32 [n_q]
     q_pos: torch.Tensor          # int32 [n_q]
     n_seq: int
     max_ctx: int
     seq_run: int = 1
 
-    def c(self) -> _Queries:
+    def _make(self) -> _Queries:
         return _Queries(self.q_pos.numel(), self.n_seq, self.max_ctx, self.seq_run,
                         self.q_seq.data_ptr() if self.q_seq.numel() else None,
                         self.q_pos.data_ptr() if self.q_pos.numel() else None)
 
 
 @dataclass
-class Indexer:
+class Indexer(_CStruct):
     q: torch.Tensor              # [n_q, heads, dim] (bf16, fp32 or float8_e4m3fn)
     w: torch.Tensor              # float32 [n_q, heads]
     k: torch.Tensor              # [n_seq, L, dim] or [L, dim] (shared cache), q's dtype
@@ -162,7 +185,7 @@ class Indexer:
     q_scale: Optional[torch.Tensor] = None   # FP8 only: float32 [n_q, heads], positive
     k_scale: Optional[torch.Tensor] = None   # FP8 only: float32 [n_seq, L] or [L] (shared), positive
 
-    def c(self) -> _Indexer:
+    def _make(self) -> _Indexer:
         shared = self.k.dim() == 2
         seq_stride = 0 if shared else self.k.stride(0)
         ks = self.k_scale
@@ -174,7 +197,7 @@ class Indexer:
 
 
 @dataclass
-class Mla:
+class Mla(_CStruct):
     q: torch.Tensor              # [n_q, heads, d_latent + d_rope]
     kv: torch.Tensor             # [n_seq, L, d_latent + d_rope] or [L, ...] (shared), q's dtype;
                                  # or uint8 [n_seq, L, >= DSA_MLA_FP8_ROW_BYTES]: packed FP8 rows
@@ -183,7 +206,7 @@ class Mla:
     scale: float
     lse: Optional[torch.Tensor] = None   # float32 [n_q, heads]
 
-    def c(self) -> _Mla:
+    def _make(self) -> _Mla:
         shared = self.kv.dim() == 2
         seq_stride = 0 if shared else self.kv.stride(0)
         heads, dk = self.q.shape[1], self.q.shape[2]
@@ -194,7 +217,7 @@ class Mla:
 
 
 @dataclass
-class CacheWriter:
+class CacheWriter(_CStruct):
     h: torch.Tensor              # bf16 [n_tok, hidden]
     w: torch.Tensor              # bf16 [704, hidden]: latent 512 | RoPE key 64 | indexer key 128
     rms_weight: torch.Tensor     # float32 [512]
@@ -207,7 +230,7 @@ class CacheWriter:
     eps: float = 1e-5
     rope_theta: float = 8.0e6
 
-    def c(self) -> _CacheWriter:
+    def _make(self) -> _CacheWriter:
         ref = self.kv if self.kv is not None else self.k_idx
         return _CacheWriter(self.h.shape[0], self.h.shape[1], self.h.data_ptr(), self.h.stride(0), self.w.data_ptr(),
                             self.rms_weight.data_ptr(), self.ln_weight.data_ptr(), self.ln_bias.data_ptr(),

@@ -237,7 +237,8 @@ dsa_status check_indexer(const dsa_queries *qs, const dsa_indexer *ix) {
 
 // ------------------------------------------------------------------ top-k
 dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int topk, int32_t *idx,
-                   int32_t *cnt, uint32_t *status, void *scratch, bool hist_ready, cudaStream_t st) {
+                   int32_t *cnt, uint32_t *status, void *scratch, bool hist_ready, cudaStream_t st,
+                   bool pos_early = true) {
     TopkArgs a = {};
     a.scores = scores;
     a.ld = ld;
@@ -249,6 +250,7 @@ dsa_status do_topk(const dsa_queries *qs, const float *scores, int64_t ld, int t
     a.L = qs->max_ctx;
     a.topk = topk;
     a.hist_ready = (hist_ready && (qs->seq_run & 1)) ? 1 : 0;
+    a.pos_early = pos_early ? 1 : 0;
     a.ghist = nullptr;
     a.gticket = nullptr;
     a.gcount = nullptr;
@@ -553,7 +555,9 @@ dsa_status dsa_shard_merge(const dsa_queries *queries, int32_t n_shards, const f
     mq.seq_run = 1;
     mq.q_seq = a.merged_last;  // not read by the top-k
     mq.q_pos = a.merged_last;
-    dsa_status s = do_topk(&mq, a.merged_score, ld, topk, sel, sel_cnt, a.status, base + lay.topk_scratch, false, st);
+    // (the merged lists' lengths are written by shard_compact, the kernel just before)
+    dsa_status s = do_topk(&mq, a.merged_score, ld, topk, sel, sel_cnt, a.status, base + lay.topk_scratch, false, st,
+                           false);
     if (s != DSA_OK) return s;
     return launch_shard_map(a, st) == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
 }

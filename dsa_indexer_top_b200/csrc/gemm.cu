@@ -266,7 +266,7 @@ __global__ void __launch_bounds__(kSkinnyThreads, 1) gemm_skinny_kernel(const Ge
 template <int BN>
 cudaError_t launch_gemm_bn(const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st) {
     using Cfg = GemmCfg<BN>;
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    cudaError_t e = set_max_dynamic_smem(gemm_tc_kernel<BN>, Cfg::kSmem);
     if (e != cudaSuccess) return e;
     const int n_tiles = (g.N + BN - 1) / BN;
     dim3 grid(n_tiles, g.m_tiles * g.k_splits, g.batch);
@@ -277,8 +277,7 @@ cudaError_t launch_gemm_bn(const CUtensorMap &ta, const CUtensorMap &tb, const G
 template <int MM, int WR>
 cudaError_t launch_skinny_cfg(const GemmSkinnyArgs &g, cudaStream_t st) {
     const size_t smem = static_cast<size_t>(g.M) * g.k_per_split * 2;
-    cudaError_t e = cudaFuncSetAttribute(gemm_skinny_kernel<MM, WR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+    cudaError_t e = set_max_dynamic_smem(gemm_skinny_kernel<MM, WR>, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     const int k_splits = (g.K + g.k_per_split - 1) / g.k_per_split;
     constexpr int rows = SkinnyCfg<MM, WR>::kRows;

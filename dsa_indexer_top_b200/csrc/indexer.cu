@@ -297,6 +297,12 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
             if (a.work) {
                 item_q[k_tiles % kRing] = make_int2(-1, 0);  // the end (also after an abort: the consumers stop)
                 mbar_arrive(&item_bar[k_tiles % kRing]);
+                // this CTA claims nothing more; the last CTA to get here leaves the
+                // counters zero for the next launch (while its pipeline drains)
+                if (atomicAdd(a.work + 1, 1ull) == gridDim.x - 1) {
+                    atomicExch(a.work, 0ull);
+                    atomicExch(a.work + 1, 0ull);
+                }
             }
             // Drain: every copy this thread issued has landed before the CTA exits.
             for (int s = 0; s < S; ++s)
@@ -464,14 +470,6 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
     griddep_launch_dependents();
     tc_fence_before();
     __syncthreads();
-    if (threadIdx.x == 0 && a.work) {
-        // every role of this CTA is done claiming; the last CTA to get here leaves
-        // the counter zero for the next launch
-        if (atomicAdd(a.work + 1, 1ull) == gridDim.x - 1) {
-            atomicExch(a.work, 0ull);
-            atomicExch(a.work + 1, 0ull);
-        }
-    }
     if (warp == 1) {
         tc_fence_after();
         tmem_dealloc(tmem_base, Cfg::kTmemCols);
@@ -525,8 +523,7 @@ cudaError_t launch_tc(const CUtensorMap &tk, const CUtensorMap &tq, const IdxTcA
     using Cfg = IdxCfg<G, F8>;
     const long long slots = static_cast<long long>(num_sms) * Cfg::kCtasPerSm;
     const int grid = static_cast<int>(a.total_items < slots ? a.total_items : slots);
-    cudaError_t e = cudaFuncSetAttribute(idx_score_tc_kernel<G, F8>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmem);
+    cudaError_t e = set_max_dynamic_smem(idx_score_tc_kernel<G, F8>, Cfg::kSmem);
     if (e != cudaSuccess) return e;
     return launch_pdl(idx_score_tc_kernel<G, F8>, dim3(grid), dim3(Cfg::kThreads), Cfg::kSmem, st, tk, tq, a);
 }
@@ -556,15 +553,11 @@ cudaError_t launch_idx_score_generic(const IdxGenericArgs &a, cudaStream_t st) {
     const int bx = std::min((a.L + 255) / 256, 1024);
     dim3 grid(bx, a.n_q);
     if (a.is_bf16) {
-        cudaError_t e = cudaFuncSetAttribute(idx_score_generic_kernel<__nv_bfloat16>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        cudaError_t e = set_max_dynamic_smem(idx_score_generic_kernel<__nv_bfloat16>, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         idx_score_generic_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(a);
     } else {
-        cudaError_t e = cudaFuncSetAttribute(idx_score_generic_kernel<float>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        cudaError_t e = set_max_dynamic_smem(idx_score_generic_kernel<float>, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         idx_score_generic_kernel<float><<<grid, 256, smem, st>>>(a);
     }

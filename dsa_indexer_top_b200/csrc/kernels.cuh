@@ -4,6 +4,9 @@
 
 #include <cstddef>
 #include <cstdint>
+#include <map>
+#include <mutex>
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -27,6 +30,24 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args &&>(args)...);
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per (kernel, device) and
+// size: a launch then pays only a lookup.
+template <typename... KArgs>
+cudaError_t set_max_dynamic_smem(void (*kernel)(KArgs...), int bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, int> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const void *key = reinterpret_cast<const void *>(kernel);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find({key, dev});
+    if (it != done.end() && it->second >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done[{key, dev}] = bytes;
+    return e;
 }
 
 constexpr int kIdxHeads = 32;   // index_n_heads of GLM-5.2
@@ -111,6 +132,8 @@ struct TopkArgs {
     uint32_t *status;
     int n_q, L, topk;
     int hist_ready;    // ghist already holds the first-digit histograms (indexer epilogue)
+    int pos_early;     // q_pos is an input of the call (no kernel of it writes q_pos): the
+                       // split schedule reads it before waiting for the previous kernel
     // scratch (workspace)
     uint32_t *ghist;   // [n_q][4096] first-digit histogram
     uint32_t *gticket; // [n_q] chunks of the query done (split schedule), after ghist

@@ -11,10 +11,12 @@
 // Tensor-core path (bf16, 64 heads, 512 + 64): one CTA per (query, split,
 // layer) walks its share of the selected rows in chunks of 64, software-pipelined
 // across warp roles with mbarriers (every wait bounded):
-//   producers (warps 4-7)  gather chunk c+1 -- 64 rows x 1152 B by 16-byte
-//            cp.async into nine 64-column blocks of 128-byte-swizzled shared
-//            memory -- into one of two 72 KB slots while chunk c is computed;
-//            the 64 x 576 query tile once per CTA.
+//   producers (warps 4-7)  gather chunk c+1 -- 64 rows x 1152 B into nine
+//            64-column blocks of 128-byte-swizzled shared memory -- into one of
+//            two 72 KB slots while chunk c is computed: bf16 caches by TMA row
+//            gathers (four rows per op, issued by the lanes), packed FP8 caches
+//            by per-lane loads widened to fp16; the 64 x 576 query tile once per
+//            CTA (TMA boxes for bf16).
 //   MMA issuer (warp 8)   S = Q . C^T (M = 64 heads, N = 64 rows, K = 576, both
 //            operands K-major): 36 tcgen05.mma into TMEM columns 64*slot; then
 //            O^T += C_lat^T . P^T (the row tile read MN-major: M = 4 x 128 latent
@@ -770,7 +772,7 @@ __global__ void __launch_bounds__(128) mla_generic_kernel(const MlaArgs a) {
 
 template <bool kFp8>
 cudaError_t launch_mla_tc_t(const MlaArgs &a, const MlaMaps &maps, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel<kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kMlaSmem);
+    cudaError_t e = set_max_dynamic_smem(mla_tc_kernel<kFp8>, kMlaSmem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.n_splits, a.n_q, a.n_layers);
     return launch_pdl(mla_tc_kernel<kFp8>, grid, dim3(kMlaThreads), kMlaSmem, st, a, maps);
@@ -823,13 +825,11 @@ cudaError_t launch_mla_generic(const MlaArgs &a, cudaStream_t st) {
     const size_t smem = sizeof(float) * (static_cast<size_t>(a.d_lat + a.d_rope) + a.topk);
     dim3 grid(a.n_q, a.heads, a.n_layers);
     if (a.is_bf16) {
-        cudaError_t e = cudaFuncSetAttribute(mla_generic_kernel<__nv_bfloat16>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaError_t e = set_max_dynamic_smem(mla_generic_kernel<__nv_bfloat16>, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         mla_generic_kernel<__nv_bfloat16><<<grid, 128, smem, st>>>(a);
     } else {
-        cudaError_t e = cudaFuncSetAttribute(mla_generic_kernel<float>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        cudaError_t e = set_max_dynamic_smem(mla_generic_kernel<float>, static_cast<int>(smem));
         if (e != cudaSuccess) return e;
         mla_generic_kernel<float><<<grid, 128, smem, st>>>(a);
     }

@@ -727,15 +727,17 @@ __global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int
     CollectSmem &cs = ss.u.c;
     const int i = blockIdx.y, p = blockIdx.x;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // positions that are inputs of the call are read before the wait, so the
+    // chunk's score loads go out together with the histogram's
+    const int n_early = a.pos_early ? visible_rows(a, i) : 0;
     griddep_wait();
-    // the histogram does not depend on the position: its loads go out first
     uint32_t hv[kBins / kT];
     {
         const uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
 #pragma unroll
         for (int j = 0; j < kBins / kT; ++j) hv[j] = __ldg(g + threadIdx.x + j * kT);
     }
-    const int n = visible_rows(a, i);
+    const int n = a.pos_early ? n_early : visible_rows(a, i);
     if (n <= a.topk) {  // every chunk of the query sees the same n
         if (p == 0) {
             write_all(a, i, n);
@@ -841,8 +843,7 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
     cudaError_t e;
     if (!topk_uses_split(a.n_q, a.L)) {
         const size_t smem = sizeof(RowSmem);
-        if ((e = cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                      static_cast<int>(smem))) != cudaSuccess)
+        if ((e = set_max_dynamic_smem(topk_row_kernel, static_cast<int>(smem))) != cudaSuccess)
             return e;
         return launch_pdl(topk_row_kernel, dim3(a.n_q), dim3(kT), smem, st, a);
     }
@@ -852,8 +853,7 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
         if ((e = cudaMemsetAsync(a.ghist, 0, topk_zeroed_bytes(a.n_q), st)) != cudaSuccess) return e;
         if ((e = launch_pdl(topk_hist_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk)) != cudaSuccess) return e;
     }
-    if ((e = cudaFuncSetAttribute(topk_split_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(sizeof(SplitSmem)))) != cudaSuccess)
+    if ((e = set_max_dynamic_smem(topk_split_kernel, static_cast<int>(sizeof(SplitSmem)))) != cudaSuccess)
         return e;
     return launch_pdl(topk_split_kernel, dim3(P, a.n_q), dim3(kT), sizeof(SplitSmem), st, a, chunk, P);
 }

@@ -42,8 +42,8 @@
  *    legacy default stream); work is enqueued on it and results are valid in
  *    stream order.  Kernels are launched with programmatic dependent launch:
  *    one may start while the previous kernel on the stream finishes and read
- *    the inputs that no kernel of the call writes (the attention's query tile
- *    and query sequences) before it waits for that kernel.  A kernel of the
+ *    the inputs that no kernel of the call writes (the query positions and
+ *    sequences, the attention's query tile) before it waits for that kernel.  A kernel of the
  *    caller's that writes those inputs just before the call must therefore not
  *    release its dependents early (a kernel that never executes
  *    griddepcontrol.launch_dependents does not).
