@@ -275,8 +275,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
                 // Lane l takes latent dims 16l..16l+15 of each of the warp's 16 rows:
                 // all 16 code loads are issued before any is widened (exactly, to
                 // fp16); lanes 0-7 copy the row's RoPE key (bf16) into block 8, to be
-                // converted to fp16 in place once it lands; the row scale goes to
-                // row_sigma.
+                // converted to fp16 in place once it lands; lane l < 16 loads the
+                // scale of its own row for row_sigma, stored only after the loads
+                // (a store right behind each load would wait for it, row by row).
+                float sig = 0.f;
+                if (lane < 16 && r >= 0)
+                    sig = __ldg(reinterpret_cast<const float *>(kv8 + static_cast<int64_t>(r) * a.kv_row_stride +
+                                                                kFp8ScaleOff));
                 uint4 code[16];
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) {
@@ -287,11 +292,9 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
                         const uint8_t *row = kv8 + static_cast<int64_t>(src) * a.kv_row_stride;
                         code[rr] = __ldg(reinterpret_cast<const uint4 *>(row) + lane);
                         if (lane < 8) cp_async_16(rope_dst, row + kFp8RopeOff + 16 * lane);
-                        if (lane == 8) row_sigma[s][16 * pw + rr] = __ldg(reinterpret_cast<const float *>(row + kFp8ScaleOff));
                     } else {
                         if (lane < 8)
                             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(rope_dst), "r"(0u) : "memory");
-                        if (lane == 8) row_sigma[s][16 * pw + rr] = 0.f;
                     }
                 }
                 const uint32_t blk = sb + (lane >> 2) * kBlockBytes;  // dims 16l.. lie in block l / 4
@@ -308,6 +311,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
                                  "r"(e4m3x2_to_f16x2(w3 & 0xffffu)), "r"(e4m3x2_to_f16x2(w3 >> 16))
                                  : "memory");
                 }
+                if (lane < 16) row_sigma[s][rl] = sig;
             }
             cp_async_commit();
             cp_async_wait_all();  // the query tile (first chunk) and this chunk's rows

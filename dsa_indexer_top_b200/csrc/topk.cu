@@ -337,6 +337,7 @@ __device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t n
 // bounds-checked against k (they stay below k whenever the histogram the
 // threshold digit came from describes these scores).
 constexpr int kOwn = 9;
+static_assert(kMaxTopk <= kBins, "seg_finish stages the output in the histogram");
 // hist2_ready: `hist` already holds the second-digit histogram of the
 // candidates in bin d1 (built by the chunk CTAs), so it is not rebuilt here.
 template <class Segs>
@@ -381,18 +382,25 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     uint64_t tot;
     const uint64_t ex = block_scan((static_cast<uint64_t>(te) << 32) | tg, scan, tot);
     uint32_t g = static_cast<uint32_t>(ex & 0xFFFFFFFFu), q = static_cast<uint32_t>(ex >> 32);
+    // The kept rows land in shared memory first (each lane's run is scattered
+    // over the output, which as global stores costs one sector per row), then
+    // the k slots go out coalesced.  The histogram is free again here: every
+    // thread has read the digits it held (find_digit ends with a barrier).
+    int32_t *stage = reinterpret_cast<int32_t *>(hist);  // k <= kMaxTopk = kBins slots
 #pragma unroll
     for (int j = 0; j < kOwn; ++j) {
         if (b0 + j >= b1) continue;
         if (key[j] > T) {
             const uint32_t slot = g + min(q, need_eq);
-            if (slot < k) out[slot] = static_cast<int32_t>(p[b0 + j].y);
+            if (slot < k) stage[slot] = static_cast<int32_t>(p[b0 + j].y);
             ++g;
         } else if (key[j] == T) {
-            if (q < need_eq && g + q < k) out[g + q] = static_cast<int32_t>(p[b0 + j].y);
+            if (q < need_eq && g + q < k) stage[g + q] = static_cast<int32_t>(p[b0 + j].y);
             ++q;
         }
     }
+    __syncthreads();
+    for (uint32_t x = threadIdx.x; x < k; x += kT) out[x] = stage[x];
     return true;
 }
 
