@@ -75,10 +75,21 @@ PER_CONFIG = [("decode_32k", False), ("prefill_64k", False), ("indexshare_128k",
               ("decode_1m", True), ("indexshare_128k", True)]
 PER_CONFIG_MAX_STEPS = 50
 
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch of a stage's kernel,
-# from an ncu capture of the current kernels (workload, stage, fp8) -> bytes.
-# Entries are removed when the kernel changes; missing entries report null.
-NCU_TRAFFIC: dict = {}
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch of a stage's kernels
+# (workload, stage, fp8) -> bytes, from one-kernel ncu captures of the current
+# kernels on the one-query case of the workload (`--n-seq 1`), times its 4
+# queries: every term of a decode stage's traffic grows with the queries (keys and
+# scores per sequence, selected rows, split-K partials).  The captures are cold
+# (ncu flushes the caches), so the attention's entry includes re-reading its
+# split-K partials, which stay in L2 inside a step.  Entries are removed when a
+# kernel changes; missing entries report null.
+NCU_TRAFFIC: dict = {
+    ("decode_1m", "index_scores", False): 4 * (268_491_008 + 5_246_720),
+    ("decode_1m", "index_scores", True): 4 * (138_483_712 + 4_256_768),
+    ("decode_1m", "topk", False): 4 * 4_316_416,
+    ("decode_1m", "sparse_mla", False): 4 * (2_501_632 + 2_118_400),   # mla_tc + mla_combine
+    ("decode_1m", "sparse_mla", True): 4 * (1_730_304 + 2_118_400),
+}
 
 
 def measured_peaks():

@@ -181,8 +181,9 @@ __global__ void __launch_bounds__(kGemmThreads) gemm_tc_kernel(const __grid_cons
 // flight, its lanes splitting K in 8-element pieces; a row's M partial sums are
 // reduced across the warp and written like the tensor-core kernel's output
 // (fp32 split-K partials or bf16).  One CTA per (8 * WR rows of B, K split,
-// batch).  HBM-bound on B.  Two shapes: up to 4 rows of A with 8 rows of B per
-// warp, up to 16 rows of A with 4 (the accumulators fit the registers either way).
+// batch).  HBM-bound on B.  Two shapes, both 4 rows of B per warp: up to 4 rows
+// of A in at most 85 registers, so three CTAs share an SM and more loads are in
+// flight per SM; up to 16 rows of A at one CTA per SM.
 constexpr int kSkinnyM = 16;
 constexpr int kSkinnyThreads = 256;
 template <int MM, int WR>
@@ -191,7 +192,7 @@ struct SkinnyCfg {
 };
 
 template <int MM, int WR>
-__global__ void __launch_bounds__(kSkinnyThreads, 1) gemm_skinny_kernel(const GemmSkinnyArgs g) {
+__global__ void __launch_bounds__(kSkinnyThreads, MM <= 4 ? 3 : 1) gemm_skinny_kernel(const GemmSkinnyArgs g) {
     extern __shared__ __align__(16) uint8_t sm_raw[];
     __nv_bfloat16 *a_sm = reinterpret_cast<__nv_bfloat16 *>(sm_raw);  // [M][kc]
     const int nb = blockIdx.x, split = blockIdx.y, b = blockIdx.z;
@@ -289,8 +290,10 @@ cudaError_t launch_skinny_cfg(const GemmSkinnyArgs &g, cudaStream_t st) {
 
 cudaError_t launch_gemm_skinny(const GemmSkinnyArgs &g, cudaStream_t st) {
     if (g.M < 1 || g.M > kSkinnyM) return cudaErrorInvalidValue;
-    return g.M <= 4 ? launch_skinny_cfg<4, 8>(g, st) : launch_skinny_cfg<16, 4>(g, st);
+    return g.M <= 4 ? launch_skinny_cfg<4, 4>(g, st) : launch_skinny_cfg<16, 4>(g, st);
 }
+
+int skinny_rows_per_cta(int M) { return M <= 4 ? SkinnyCfg<4, 4>::kRows : SkinnyCfg<16, 4>::kRows; }
 
 cudaError_t launch_gemm_tc(int bn, const CUtensorMap &ta, const CUtensorMap &tb, const GemmArgs &g, cudaStream_t st) {
     switch (bn) {

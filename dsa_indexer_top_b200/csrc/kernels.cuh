@@ -225,6 +225,7 @@ struct GemmSkinnyArgs {
     int64_t ldc, s_batch, s_split;
 };
 constexpr int kSkinnyMaxM = 16;
+int skinny_rows_per_cta(int M);  // rows of B per CTA of launch_gemm_skinny
 cudaError_t launch_gemm_skinny(const GemmSkinnyArgs &g, cudaStream_t st);
 
 // Cache-row writer epilogue: one CTA per token sums the split-K partials of

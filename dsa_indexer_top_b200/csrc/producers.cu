@@ -211,6 +211,18 @@ size_t cache_ws_bytes(int n_tok, int hidden) {
 
 bool a16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+int sm_count() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -253,7 +265,12 @@ dsa_status dsa_write_cache_rows(const dsa_cache_writer *cw, void *ws, size_t ws_
         k.N = kProjFeatures;
         k.K = cw->hidden;
         k.batch = 1;
-        k.k_per_split = (((cw->hidden + g.k_splits - 1) / g.k_splits) + 7) / 8 * 8;
+        // about two CTAs per SM in one wave: K splits for the 704 weight rows,
+        // no more than the workspace holds partials for
+        const int n_tiles = (kProjFeatures + skinny_rows_per_cta(cw->n_tok) - 1) / skinny_rows_per_cta(cw->n_tok);
+        int ks = 2 * sm_count() / n_tiles;
+        ks = ks < 1 ? 1 : (ks > g.k_splits ? g.k_splits : ks);
+        k.k_per_split = (((cw->hidden + ks - 1) / ks) + 7) / 8 * 8;
         if (k.k_per_split > 2048) return DSA_ERR_UNSUPPORTED;
         g.k_splits = (cw->hidden + k.k_per_split - 1) / k.k_per_split;  // what the epilogue sums
         k.a = cw->h;
