@@ -33,11 +33,10 @@ inline bool mla_tc_ok(const dsa_mla *m) {
     return shape && m->kv_row_stride % 8 == 0 && m->kv_seq_stride % 8 == 0 && m->kv_row_stride >= kRow;
 }
 
-// bf16 caches on the tensor-core path are read by TMA row gathers over one 2-D
-// tensor of every sequence's rows: the sequence stride a whole number of rows
-// (or 0) and at most INT32_MAX rows in all.  Packed FP8 caches: no condition.
+// Caches on the tensor-core path are read by TMA row gathers over one 2-D tensor
+// of every sequence's rows: the sequence stride a whole number of rows (or 0)
+// and at most INT32_MAX rows in all.
 inline bool mla_tc_rows_ok(const dsa_mla *m, int n_seq, int max_ctx) {
-    if (mla_kv_fp8(m)) return true;
     const int64_t rows = mla_gather_rows(m->kv_seq_stride, m->kv_row_stride, n_seq, max_ctx);
     return rows >= 1 && rows <= INT32_MAX;
 }

@@ -301,7 +301,7 @@ dsa_status do_mla(const dsa_queries *qs, const dsa_mla *layers, int n_layers, co
     if (tc) {
         MlaMaps maps;
         std::memset(&maps, 0, sizeof(maps));
-        if (!a.kv_fp8 && !encode_mla_maps(a, maps)) return DSA_ERR_CUDA;
+        if (!encode_mla_maps(a, maps)) return DSA_ERR_CUDA;
         int n_splits, cpc;
         mla_plan(qs->n_q, n_layers, topk, decode, num_sms_current(), kMlaMaxSplits, n_splits, cpc);
         a.n_splits = n_splits;

@@ -115,7 +115,7 @@ extern "C" dsa_status dsa_sparse_mla_decode_noalloc(const dsa_queries *queries, 
     a.chunks_per_cta = cpc;
     MlaMaps maps;
     std::memset(&maps, 0, sizeof(maps));
-    if (!a.kv_fp8 && !encode_mla_maps(a, maps)) return DSA_ERR_CUDA;
+    if (!encode_mla_maps(a, maps)) return DSA_ERR_CUDA;
     if (n_splits > 1) {
         a.part_o = reinterpret_cast<float *>(scratch + kStatusBytes);
         const size_t rows = static_cast<size_t>(queries->n_q) * n_splits * kMlaHeads;

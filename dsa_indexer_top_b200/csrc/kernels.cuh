@@ -297,13 +297,16 @@ struct MlaArgs {
     float *part_ml;      // [layers][n_q][n_splits][64][2] (max, sum) in log2 units
 };
 
-// TMA descriptors of the tensor-core MLA with a bf16 cache (one per layer):
-// kv 2-D {576, rows of all sequences}, boxes {64, 1} (the row gathers' unit,
-// four rows per gather); q 2-D {576, n_q * 64}, boxes {64, 64}; both 128-byte
-// swizzled.
+// TMA descriptors of the tensor-core MLA (one set per layer), over one 2-D
+// tensor of every sequence's rows (the row gathers read four rows per op).
+// bf16 caches: kv {576, rows}, boxes {64, 1}; q {576, n_q * 64}, boxes {64, 64};
+// both 128-byte swizzled.  Packed FP8 caches: kv {656 bytes, rows}, boxes
+// {128 bytes, 1}, unswizzled (staging for the widening); kvr the same rows as
+// {328 bf16, rows}, boxes {64, 1}, 128-byte swizzled (the RoPE key).
 struct MlaMaps {
-    CUtensorMap kv[kMaxLayers];
-    CUtensorMap q[kMaxLayers];
+    CUtensorMap kv[kMaxLayers];   // bf16: the rows; packed FP8: the rows' bytes, boxes {128 B, 1}, unswizzled
+    CUtensorMap q[kMaxLayers];    // bf16 only
+    CUtensorMap kvr[kMaxLayers];  // packed FP8 only: the rows as bf16, boxes {64, 1} at the RoPE key, swizzled
 };
 
 // Tensor-core sparse MLA (bf16 queries and outputs, 64 heads, 512 + 64; bf16 or

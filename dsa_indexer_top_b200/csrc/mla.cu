@@ -105,6 +105,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
 
     // o_done[s]: the O-MMA of the chunk in slot s completed (the slot may be refilled)
     __shared__ uint64_t q_full, slot_full[2], s_full[2], p_full[2], o_done[2], fin, sm_bar;
+    __shared__ uint64_t raw_full[2];  // FP8: a chunk's gathered bytes (before widening) are in the slot
     __shared__ uint32_t tmem_base_sh;
     __shared__ int abort_flag;
     __shared__ int row_idx[2][kChunk];  // [slot][chunk row]: cache row, or -1 (padding)
@@ -124,6 +125,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], 4);
             mbar_init(&o_done[s], 1);
+            mbar_init(&raw_full[s], 4);  // one per producer warp, with its bytes
         }
         mbar_init(&fin, 1);
         mbar_init(&sm_bar, 4);
@@ -188,6 +190,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
                     }
                 }
             }
+            // this warp's share of the fp16 query tile is in (for the MMAs' async reads)
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&q_full);
         }
     }
     int seq = a.q_seq[i];  // an input of the step, like the query tile
@@ -196,12 +202,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
     const int si = i / a.sel_group;  // the selection row this query reads
     const int32_t *sel = a.idx + static_cast<int64_t>(si) * a.topk;
     const int c_begin = split * a.chunks_per_cta;
-    // producers: the first chunk's indices are requested with the count, not after it
-    int r_first = -1, f_first = -1;
-    if (warp >= 4 && warp < 8 && c_begin * kChunk < a.topk) {
+    // producers: the first two chunks' indices (this lane's row, and the chunk's
+    // first row) are requested with the count, not after it; later chunks' two
+    // chunks ahead of their turn
+    int r_first = -1, f_first = -1, r_second = -1, f_second = -1;
+    if (warp >= 4 && warp < 8) {
         const int j0 = c_begin * kChunk + 16 * (warp - 4) + (lane & 15);
         if (j0 < a.topk) r_first = __ldg(sel + j0);
-        f_first = __ldg(sel + c_begin * kChunk);
+        if (c_begin * kChunk < a.topk) f_first = __ldg(sel + c_begin * kChunk);
+        if (j0 + kChunk < a.topk) r_second = __ldg(sel + j0 + kChunk);
+        if ((c_begin + 1) * kChunk < a.topk) f_second = __ldg(sel + (c_begin + 1) * kChunk);
     }
     int cnt = a.cnt[si];
     if (!(seq >= 0 && seq < a.n_seq && cnt >= 0 && cnt <= a.topk)) {
@@ -216,35 +226,35 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
     if (warp >= 4 && warp < 8) {
         // ------------------------------------------------------------ producers
         const int pw = warp - 4;  // rows (and the query tile's heads) 16*pw .. 16*pw+15
-        bool q_arrived = false;   // FP8: this warp's share of the query tile is in
-        int issued = 0;           // bf16: chunks whose row gathers this warp has issued
-        // bf16: the rows of all sequences form one 2-D tensor (rows of kv_row_stride)
+        // the rows of all sequences form one 2-D tensor (rows of kv_row_stride)
         const int seq_row0 = a.kv_row_stride > 0 ? static_cast<int>(static_cast<int64_t>(seq) * (a.kv_seq_stride / a.kv_row_stride)) : 0;
         const int rl = 16 * pw + (lane & 15);
-        int r_cur = r_first, f_cur = f_first;  // chunk t's index (this lane's row) and first row
-        for (int t = 0; t < nloc; ++t) {
-            const int c = c_begin + t, s = t & 1, u = t >> 1;
-            // chunk t + 1's indices are requested now: they land while this chunk
-            // waits for its slot and is issued
-            int r_nx = -1, f_nx = -1;
-            if (t + 1 < nloc) {
-                const int j1 = (c + 1) * kChunk + rl;
-                if (j1 < cnt) r_nx = __ldg(sel + j1);
-                f_nx = __ldg(sel + (c + 1) * kChunk);
-            }
-            if (t >= 2 && !mbar_wait(&o_done[s], (u - 1) & 1, a.status, &abort_flag)) break;
-            const int j = c * kChunk + rl;
-            int r = -1;
-            if (j < cnt) {
-                r = r_cur;
-                if (r < 0 || r >= a.L) {
-                    report_status(a.status, DSA_ERR_INVALID);
-                    r = -1;
+        if constexpr (!kFp8) {
+            int issued = 0;                        // chunks whose row gathers this warp has issued
+            int r_cur = r_first, f_cur = f_first;    // chunk t's index (this lane's row) and first row
+            int r_nx = r_second, f_nx = f_second;    // chunk t + 1's
+            for (int t = 0; t < nloc; ++t) {
+                const int c = c_begin + t, s = t & 1, u = t >> 1;
+                // chunk t + 2's indices are requested now: they land while this chunk
+                // and the next wait for their slots and are issued
+                int r_n2 = -1, f_n2 = -1;
+                if (t + 2 < nloc) {
+                    const int j2 = (c + 2) * kChunk + rl;
+                    if (j2 < a.topk) r_n2 = __ldg(sel + j2);
+                    f_n2 = __ldg(sel + (c + 2) * kChunk);
                 }
-            }
-            if (lane < 16) row_idx[s][rl] = r;
-            const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
-            if constexpr (!kFp8) {
+                if (t >= 2 && !mbar_wait(&o_done[s], (u - 1) & 1, a.status, &abort_flag)) break;
+                const int j = c * kChunk + rl;
+                int r = -1;
+                if (j < cnt) {
+                    r = r_cur;
+                    if (r < 0 || r >= a.L) {
+                        report_status(a.status, DSA_ERR_INVALID);
+                        r = -1;
+                    }
+                }
+                if (lane < 16) row_idx[s][rl] = r;
+                const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
                 // The warp's 16 rows as 4 row gathers per 64-dim block (36 TMA ops,
                 // lanes 0-31 then 0-3): padding rows and rejected indices fetch the
                 // chunk's first row instead (in range; masked in the softmax), so
@@ -270,92 +280,185 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_tc_kernel(const MlaArgs a,
                 issued = t + 1;
                 r_cur = r_nx;
                 f_cur = f_nx;
-                continue;
-            } else {
-                // Lane l takes latent dims 16l..16l+15 of each of the warp's 16 rows:
-                // all 16 code loads are issued before any is widened (exactly, to
-                // fp16); lanes 0-7 copy the row's RoPE key (bf16) into block 8, to be
-                // converted to fp16 in place once it lands; lane l < 16 loads the
-                // scale of its own row for row_sigma, stored only after the loads
-                // (a store right behind each load would wait for it, row by row).
-                float sig = 0.f;
-                if (lane < 16 && r >= 0)
-                    sig = __ldg(reinterpret_cast<const float *>(kv8 + static_cast<int64_t>(r) * a.kv_row_stride +
-                                                                kFp8ScaleOff));
-                uint4 code[16];
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int src = __shfl_sync(0xffffffffu, r, rr);
-                    code[rr] = make_uint4(0u, 0u, 0u, 0u);
-                    const uint32_t rope_dst = sb + 8 * kBlockBytes + sw128_offset(16 * pw + rr, lane & 7);
-                    if (src >= 0) {
-                        const uint8_t *row = kv8 + static_cast<int64_t>(src) * a.kv_row_stride;
-                        code[rr] = __ldg(reinterpret_cast<const uint4 *>(row) + lane);
-                        if (lane < 8) cp_async_16(rope_dst, row + kFp8RopeOff + 16 * lane);
-                    } else {
-                        if (lane < 8)
-                            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(rope_dst), "r"(0u) : "memory");
-                    }
-                }
-                const uint32_t blk = sb + (lane >> 2) * kBlockBytes;  // dims 16l.. lie in block l / 4
-#pragma unroll
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int row = 16 * pw + rr;
-                    const uint32_t w0 = code[rr].x, w1 = code[rr].y, w2 = code[rr].z, w3 = code[rr].w;
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane) & 7)),
-                                 "r"(e4m3x2_to_f16x2(w0 & 0xffffu)), "r"(e4m3x2_to_f16x2(w0 >> 16)),
-                                 "r"(e4m3x2_to_f16x2(w1 & 0xffffu)), "r"(e4m3x2_to_f16x2(w1 >> 16))
-                                 : "memory");
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(blk + sw128_offset(row, (2 * lane + 1) & 7)),
-                                 "r"(e4m3x2_to_f16x2(w2 & 0xffffu)), "r"(e4m3x2_to_f16x2(w2 >> 16)),
-                                 "r"(e4m3x2_to_f16x2(w3 & 0xffffu)), "r"(e4m3x2_to_f16x2(w3 >> 16))
-                                 : "memory");
-                }
-                if (lane < 16) row_sigma[s][rl] = sig;
+                r_nx = r_n2;
+                f_nx = f_n2;
             }
-            cp_async_commit();
-            cp_async_wait_all();  // the query tile (first chunk) and this chunk's rows
-            {
-                // this lane's RoPE pieces (bf16, copied above) to fp16, in place
-                if (lane < 8) {
-#pragma unroll 4
-                    for (int rr = 0; rr < 16; ++rr) {
-                        const uint32_t adr = sb + 8 * kBlockBytes + sw128_offset(16 * pw + rr, lane & 7);
-                        uint4 v;
-                        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                                     : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                                     : "r"(adr)
-                                     : "memory");
-                        v = bf16x8_to_f16x8(v);
-                        asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(v.x), "r"(v.y), "r"(v.z),
-                                     "r"(v.w)
-                                     : "memory");
-                    }
-                }
-            }
-            fence_proxy_async_smem();
-            __syncwarp();
             if (lane == 0) {
-                if (!q_arrived) mbar_arrive(&q_full);
-                mbar_arrive(&slot_full[s]);
+                // every TMA copy this warp requested has landed before the CTA may exit
+                // (the consumers may have stopped early on an abort): the last phase of
+                // each slot it filled, and the query tile
+                for (int t = max(0, issued - 2); t < issued; ++t)
+                    mbar_wait(&slot_full[t & 1], (t >> 1) & 1, a.status, nullptr);
+                if (pw == 0) mbar_wait(&q_full, 0, a.status, nullptr);
             }
-            q_arrived = true;
-            r_cur = r_nx;
-            f_cur = f_nx;
-        }
-        if (kFp8 && !q_arrived) {  // no chunk for this CTA (or an abort): the query tile still counts
-            cp_async_wait_all();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&q_full);
-        }
-        if (!kFp8 && lane == 0) {
-            // every TMA copy this warp requested has landed before the CTA may exit
-            // (the consumers may have stopped early on an abort): the last phase of
-            // each slot it filled, and the query tile
-            for (int t = max(0, issued - 2); t < issued; ++t)
-                mbar_wait(&slot_full[t & 1], (t >> 1) & 1, a.status, nullptr);
-            if (pw == 0) mbar_wait(&q_full, 0, a.status, nullptr);
+        } else {
+            // Packed FP8 rows.  Each chunk's bytes for this warp's 16 rows arrive by TMA
+            // row gathers on raw_full[slot]: the codes (four 128-byte boxes per row,
+            // unswizzled) into the slot's blocks 4..7 as staging, the RoPE key (one
+            // 64 x bf16 box, swizzled) into block 8.  The warp then widens them in the
+            // slot: codes to the fp16 tiles (exact), the RoPE key to fp16 in place, and
+            // marks the slot full.  Issuing a chunk (when its slot is free) and widening
+            // one (when its bytes are in) are polled, not waited for in turn, so the next
+            // chunk's gathers are in flight while this one is widened and computed.
+            // Padding rows fetch the chunk's first row (masked in the softmax, scale 0).
+            int n_iss = 0, n_conv = 0;             // chunks issued / widened by this warp
+            int r_iss = r_first, f_iss = f_first;    // chunk n_iss's index (this lane's row) and first row
+            int r_iss2 = r_second, f_iss2 = f_second;  // chunk n_iss + 1's
+            float sig0 = 0.f, sig1 = 0.f;          // lanes < 16: the scale of this lane's row, per slot
+            uint64_t t_idle = 0;
+            while (n_conv < nloc) {
+                bool did = false;
+                if (n_iss < nloc && n_iss < n_conv + 2) {
+                    const int s = n_iss & 1;
+                    bool free = n_iss < 2;
+                    if (!free) {
+                        uint32_t ok = 0;
+                        if (lane == 0) ok = mbar_test_wait(&o_done[s], ((n_iss >> 1) - 1) & 1) ? 1u : 0u;
+                        free = __shfl_sync(0xffffffffu, ok, 0) != 0u;
+                    }
+                    if (free) {
+                        const int c = c_begin + n_iss;
+                        const int j = c * kChunk + rl;
+                        int r = -1;
+                        if (j < cnt) {
+                            r = r_iss;
+                            if (r < 0 || r >= a.L) {
+                                report_status(a.status, DSA_ERR_INVALID);
+                                r = -1;
+                            }
+                        }
+                        int f = f_iss;
+                        if (f < 0 || f >= a.L) f = 0;
+                        // the indices of the chunk after next are requested now
+                        r_iss = r_iss2;
+                        f_iss = f_iss2;
+                        r_iss2 = -1;
+                        f_iss2 = -1;
+                        if (n_iss + 2 < nloc) {
+                            const int j2 = (c + 2) * kChunk + rl;
+                            if (j2 < a.topk) r_iss2 = __ldg(sel + j2);
+                            f_iss2 = __ldg(sel + (c + 2) * kChunk);
+                        }
+                        if (lane < 16) row_idx[s][rl] = r;
+                        const int gr = seq_row0 + (r >= 0 ? r : f);
+                        // lanes 0..15: codes of row group lane / 4, box lane % 4;
+                        // lanes 16..19: RoPE keys of row group lane - 16
+                        const int g = lane < 16 ? (lane >> 2) : (lane - 16) & 3;
+                        int y[4];
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) y[qq] = __shfl_sync(0xffffffffu, gr, 4 * g + qq);
+                        if (lane == 0) mbar_arrive_expect_tx(&raw_full[s], 16 * (kLatent + 2 * kRope));
+                        __syncwarp();
+                        const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
+                        const uint32_t rows_off = (16 * pw + 4 * g) * 128;
+                        if (lane < 16)
+                            tma_gather4(sb + (4 + (lane & 3)) * kBlockBytes + rows_off, &maps.kv[layer], &raw_full[s],
+                                        128 * (lane & 3), y[0], y[1], y[2], y[3]);
+                        else if (lane < 20)
+                            tma_gather4(sb + 8 * kBlockBytes + rows_off, &maps.kvr[layer], &raw_full[s], kFp8RopeOff / 2,
+                                        y[0], y[1], y[2], y[3]);
+                        // the scale of the row this lane's row fetched (a padding row's P is 0),
+                        // loaded straight into the slot's register: it is read only when the
+                        // chunk is widened, so nothing here waits for it
+                        if (lane < 16) {
+                            const float *sp = reinterpret_cast<const float *>(
+                                kv8 + static_cast<int64_t>(r >= 0 ? r : f) * a.kv_row_stride + kFp8ScaleOff);
+                            if (s == 0)
+                                sig0 = __ldg(sp);
+                            else
+                                sig1 = __ldg(sp);
+                        }
+                        ++n_iss;
+                        did = true;
+                    }
+                }
+                if (n_conv < n_iss) {
+                    const int s = n_conv & 1;
+                    uint32_t ok = 0;
+                    if (lane == 0) ok = mbar_test_wait(&raw_full[s], (n_conv >> 1) & 1) ? 1u : 0u;
+                    if (__shfl_sync(0xffffffffu, ok, 0) != 0u) {
+                        const uint32_t sb = smem_u32(slot_sm + s * kSlotBytes);
+                        // codes: 4 lanes per row (a 128-code quarter each), 8 rows per pass;
+                        // every read of a pass before any write (blocks 4..7 hold both the
+                        // staged codes and the widened tiles; a row only touches its own lines)
+#pragma unroll
+                        for (int pass = 0; pass < 2; ++pass) {
+                            const int row = 16 * pw + 8 * pass + (lane >> 2);
+                            const int q = lane & 3;
+                            const uint32_t src = sb + (4 + q) * kBlockBytes + row * 128;
+                            uint4 raw[8];
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const int kk = (k + lane) & 7;
+                                asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                             : "=r"(raw[k].x), "=r"(raw[k].y), "=r"(raw[k].z), "=r"(raw[k].w)
+                                             : "r"(src + 16 * kk)
+                                             : "memory");
+                            }
+                            __syncwarp();
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                const int kk = (k + lane) & 7;  // codes 128q + 16kk .. +15: block 2q + kk/4
+                                const uint32_t dst = sb + (2 * q + (kk >> 2)) * kBlockBytes;
+                                const int c0 = 2 * (kk & 3);
+                                const uint32_t w0 = raw[k].x, w1 = raw[k].y, w2 = raw[k].z, w3 = raw[k].w;
+                                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sw128_offset(row, c0)),
+                                             "r"(e4m3x2_to_f16x2(w0 & 0xffffu)), "r"(e4m3x2_to_f16x2(w0 >> 16)),
+                                             "r"(e4m3x2_to_f16x2(w1 & 0xffffu)), "r"(e4m3x2_to_f16x2(w1 >> 16))
+                                             : "memory");
+                                asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + sw128_offset(row, c0 + 1)),
+                                             "r"(e4m3x2_to_f16x2(w2 & 0xffffu)), "r"(e4m3x2_to_f16x2(w2 >> 16)),
+                                             "r"(e4m3x2_to_f16x2(w3 & 0xffffu)), "r"(e4m3x2_to_f16x2(w3 >> 16))
+                                             : "memory");
+                            }
+                            __syncwarp();
+                        }
+                        // RoPE keys (bf16, swizzled by the TMA) to fp16 in place: 16 rows x 8 pieces
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int idx = lane + 32 * e;
+                            const uint32_t adr = sb + 8 * kBlockBytes + sw128_offset(16 * pw + (idx >> 3), idx & 7);
+                            uint4 v;
+                            asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                                         : "r"(adr)
+                                         : "memory");
+                            v = bf16x8_to_f16x8(v);
+                            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(adr), "r"(v.x), "r"(v.y),
+                                         "r"(v.z), "r"(v.w)
+                                         : "memory");
+                        }
+                        if (lane < 16) row_sigma[s][rl] = s == 0 ? sig0 : sig1;
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&slot_full[s]);
+                        ++n_conv;
+                        did = true;
+                    }
+                }
+                if (did) {
+                    t_idle = 0;
+                } else {
+                    // nothing ready: bounded, like every wait, and stopped by an abort
+                    const uint64_t now = global_timer_ns();
+                    if (t_idle == 0) t_idle = now;
+                    uint32_t stop = 0;
+                    if (lane == 0) {
+                        if (*reinterpret_cast<volatile int *>(&abort_flag)) stop = 1;
+                        else if (now - t_idle > kWaitLimitNs) {
+                            report_status(a.status, DSA_ERR_TIMEOUT);
+                            abort_flag = 1;
+                            stop = 1;
+                        }
+                    }
+                    if (__shfl_sync(0xffffffffu, stop, 0) != 0u) break;
+                    __nanosleep(64);  // leave the issue slots to the softmax warp on this SM sub-partition
+                }
+            }
+            if (lane == 0) {
+                // every gather this warp issued has landed before the CTA may exit
+                for (int n = n_conv; n < n_iss; ++n) mbar_wait(&raw_full[n & 1], (n >> 1) & 1, a.status, nullptr);
+            }
         }
     } else if (warp == 8) {
         // ------------------------------------------------------------ MMA issuer
@@ -795,6 +898,26 @@ bool encode_mla_maps(const MlaArgs &a, MlaMaps &maps) {
     const int64_t rows = mla_gather_rows(a.kv_seq_stride, a.kv_row_stride, a.n_seq, a.L);
     if (rows < 1 || rows > INT32_MAX || static_cast<int64_t>(a.n_q) * kMlaHeads > INT32_MAX) return false;
     const cuuint32_t es[2] = {1, 1};
+    if (a.kv_fp8) {
+        for (int l = 0; l < a.n_layers; ++l) {
+            // packed rows as bytes {656, rows}: one-row boxes of 128 codes, unswizzled
+            const cuuint64_t kd[2] = {static_cast<cuuint64_t>(kFp8Row), static_cast<cuuint64_t>(rows)};
+            const cuuint64_t ks[1] = {static_cast<cuuint64_t>(a.kv_row_stride)};
+            const cuuint32_t kb[2] = {128, 1};
+            if (enc(&maps.kv[l], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(a.layer[l].kv), kd, ks, kb, es,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return false;
+            // the same rows as bf16 {328, rows}: one-row boxes of the 64-value RoPE key
+            const cuuint64_t rd[2] = {static_cast<cuuint64_t>(kFp8Row / 2), static_cast<cuuint64_t>(rows)};
+            const cuuint32_t rb[2] = {64, 1};
+            if (enc(&maps.kvr[l], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(a.layer[l].kv), rd, ks, rb,
+                    es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+                return false;
+        }
+        return true;
+    }
     for (int l = 0; l < a.n_layers; ++l) {
         // cache rows: {576 dims, rows}, one-row boxes of 64 dims (the gathers' unit)
         const cuuint64_t kd[2] = {static_cast<cuuint64_t>(kRow), static_cast<cuuint64_t>(rows)};
