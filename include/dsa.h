@@ -203,8 +203,13 @@ typedef struct {
  *   kv                 cache row s of sequence b at kv + b*kv_seq_stride +
  *                      s*kv_row_stride, laid out [c (d_latent) | r (d_rope)];
  *                      tensor-core path: strides multiple of 8 elements, 16-byte
- *                      aligned base.  Packed FP8 rows: strides in bytes, multiples
- *                      of 16, row stride >= DSA_MLA_FP8_ROW_BYTES
+ *                      aligned base, and the sequence stride a whole number of
+ *                      rows (or 0) -- the rows are gathered by TMA from one 2-D
+ *                      tensor of every sequence's rows (bf16 caches that miss it
+ *                      take the generic path).  Packed FP8 rows: strides in bytes,
+ *                      multiples of 16, row stride >= DSA_MLA_FP8_ROW_BYTES, the
+ *                      sequence stride a whole number of rows (else
+ *                      DSA_ERR_UNSUPPORTED)
  *   out                [n_q][heads][d_latent], dtype `dtype`
  *   lse                float32 [n_q][heads] (natural log of the softmax
  *                      normaliser of the scaled logits), or NULL
@@ -217,8 +222,10 @@ typedef struct {
  *   bytes [512, 640)   the RoPE key r, 64 bf16 values
  *   bytes [640, 644)   float32 row scale sigma (positive, finite)
  *   bytes [644, 656)   unused
- * The latent attended over is c[d] = sigma * e4m3(c8[d]); the kernel rounds each
- * such product to bf16 once before its tensor-core products.
+ * The latent attended over is c[d] = sigma * e4m3(c8[d]).  The kernel multiplies
+ * the exact codes (E4M3 values are exact in fp16) on fp16 tensor cores and applies
+ * sigma in fp32: to the row's logit, and to its softmax weight, rounded to fp16
+ * once before the product with the codes.
  */
 #define DSA_MLA_FP8_ROW_BYTES 656
 
