@@ -729,7 +729,14 @@ __device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int
     if (threadIdx.x == 0) a.cnt[i] = a.topk;
 }
 
-__global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int chunk, int n_chunks) {
+// kPerSm CTAs per SM.  One, where the plan gives each query enough chunks with
+// one CTA per SM: the finishing CTA's digit search and output then run in
+// registers (at two CTAs per SM the 64-register cap spills them, which costs
+// the finish about a microsecond per phase).  Two for many queries, which need
+// more chunks per query than one CTA per SM allows (a chunk's candidates must
+// fit its buffers).
+template <int kPerSm>
+__global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a, int chunk, int n_chunks) {
     extern __shared__ __align__(16) uint8_t smem_raw[];
     SplitSmem &ss = *reinterpret_cast<SplitSmem *>(smem_raw);
     CollectSmem &cs = ss.u.c;
@@ -827,10 +834,13 @@ __global__ void __launch_bounds__(kT, 2) topk_split_kernel(const TopkArgs a, int
     merge_query(a, i, n, n_chunks, d1, above1, ss.u.m);
 }
 
-// P chunks per query so that about two CTAs per SM take part; chunks are
-// multiples of 2048 rows.
-void split_plan(const TopkArgs &a, int num_sms, int &P, int &chunk) {
-    P = (2 * num_sms + a.n_q - 1) / a.n_q;
+// P chunks per query, chunks multiples of 2048 rows: about one CTA per SM when
+// that still gives every query kSplitMinChunks chunks (per_sm = 1), else about
+// two (per_sm = 2).
+constexpr int kSplitMinChunks = 8;  // a query's ~2-4K candidates stay within a chunk's buffers
+void split_plan(const TopkArgs &a, int num_sms, int &P, int &chunk, int &per_sm) {
+    per_sm = num_sms / a.n_q >= kSplitMinChunks ? 1 : 2;
+    P = per_sm == 1 ? num_sms / a.n_q : (2 * num_sms + a.n_q - 1) / a.n_q;
     P = P < 1 ? 1 : (P > kSplitMax ? kSplitMax : P);
     chunk = (a.L + P - 1) / P;
     chunk = (chunk + 2047) / 2048 * 2048;
@@ -842,8 +852,8 @@ void split_plan(const TopkArgs &a, int num_sms, int &P, int &chunk) {
 bool topk_uses_split(int n_q, int max_ctx) { return max_ctx > kTopkSplitMinCtx && n_q <= kTopkSplitMaxQueries; }
 
 cudaError_t launch_topk_hist(const TopkArgs &a, int num_sms, cudaStream_t st) {
-    int P, chunk;
-    split_plan(a, num_sms, P, chunk);
+    int P, chunk, per_sm;
+    split_plan(a, num_sms, P, chunk, per_sm);
     return launch_pdl(topk_hist_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk);
 }
 
@@ -855,15 +865,19 @@ cudaError_t launch_topk(const TopkArgs &a, int num_sms, cudaStream_t st) {
             return e;
         return launch_pdl(topk_row_kernel, dim3(a.n_q), dim3(kT), smem, st, a);
     }
-    int P, chunk;
-    split_plan(a, num_sms, P, chunk);
+    int P, chunk, per_sm;
+    split_plan(a, num_sms, P, chunk, per_sm);
     if (!a.hist_ready) {
         if ((e = cudaMemsetAsync(a.ghist, 0, topk_zeroed_bytes(a.n_q), st)) != cudaSuccess) return e;
         if ((e = launch_pdl(topk_hist_kernel, dim3(P, a.n_q), dim3(kT), 0, st, a, chunk)) != cudaSuccess) return e;
     }
-    if ((e = set_max_dynamic_smem(topk_split_kernel, static_cast<int>(sizeof(SplitSmem)))) != cudaSuccess)
-        return e;
-    return launch_pdl(topk_split_kernel, dim3(P, a.n_q), dim3(kT), sizeof(SplitSmem), st, a, chunk, P);
+    if (per_sm == 1) {
+        if ((e = set_max_dynamic_smem(topk_split_kernel<1>, static_cast<int>(sizeof(SplitSmem)))) != cudaSuccess)
+            return e;
+        return launch_pdl(topk_split_kernel<1>, dim3(P, a.n_q), dim3(kT), sizeof(SplitSmem), st, a, chunk, P);
+    }
+    if ((e = set_max_dynamic_smem(topk_split_kernel<2>, static_cast<int>(sizeof(SplitSmem)))) != cudaSuccess) return e;
+    return launch_pdl(topk_split_kernel<2>, dim3(P, a.n_q), dim3(kT), sizeof(SplitSmem), st, a, chunk, P);
 }
 
 static_assert(kWaitLimitNs == kDeviceWaitLimitNs, "one device wait limit");
