@@ -328,22 +328,19 @@ __device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t n
 }
 
 // Refine and write in one go with the candidates in registers: lane l of warp
-// w owns a contiguous run of at most kOwnT (odd) candidates of the warp's segment, so
+// w owns a contiguous run of at most kOwn (odd) candidates of the warp's segment, so
 // (warp, lane, run index) is position order.  Digit 2 and digit 3 are counted
 // with per-lane shared atomics over the owned keys only; the kept rows' output
 // slots come from one block scan of (rows > T, rows == T) per thread.  Returns
-// false, having written nothing, when a segment holds more than 32 * kOwnT
-// candidates (the caller then uses seg_refine + seg_write).  kOwnT = kOwn where
-// registers are capped at 64 (two 512-thread CTAs per SM), kOwnWide in the
-// one-CTA-per-SM finish.  Output slots are
+// false, having written nothing, when a segment holds more than 32 * kOwn
+// candidates (the caller then uses seg_refine + seg_write).  Output slots are
 // bounds-checked against k (they stay below k whenever the histogram the
 // threshold digit came from describes these scores).
 constexpr int kOwn = 9;
-constexpr int kOwnWide = 15;
 static_assert(kMaxTopk <= kBins, "seg_finish stages the output in the histogram");
 // hist2_ready: `hist` already holds the second-digit histogram of the
 // candidates in bin d1 (built by the chunk CTAs), so it is not rebuilt here.
-template <int kOwnT = kOwn, class Segs>
+template <class Segs>
 __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t r2, uint32_t k, uint32_t *hist,
                                            uint64_t *scan, uint32_t *sel, int32_t *out, bool hist2_ready = false) {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -351,14 +348,14 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     const uint32_t c = sg.count(w, 0);
     const uint32_t m = ((c + 31) / 32) | 1u;  // odd run length: the lanes' loads fall in distinct banks
     if (!hist2_ready) zero_hist(hist, kBins);
-    if (__syncthreads_or(m > static_cast<uint32_t>(kOwnT) || sg.pieces(w) != 1)) return false;
+    if (__syncthreads_or(m > static_cast<uint32_t>(kOwn) || sg.pieces(w) != 1)) return false;
     const uint32_t b0 = min(c, lane * m), b1 = min(c, b0 + m);
-    uint32_t key[kOwnT];
+    uint32_t key[kOwn];
 #pragma unroll
-    for (int j = 0; j < kOwnT; ++j) key[j] = b0 + j < b1 ? p[b0 + j].x : 0u;
+    for (int j = 0; j < kOwn; ++j) key[j] = b0 + j < b1 ? p[b0 + j].x : 0u;
     if (!hist2_ready) {
 #pragma unroll
-        for (int j = 0; j < kOwnT; ++j)
+        for (int j = 0; j < kOwn; ++j)
             if (b0 + j < b1 && first_digit(key[j]) == d1) atomicAdd(&hist[(key[j] >> 8) & 0xFFFu], 1u);
         __syncthreads();
     }
@@ -370,7 +367,7 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     if (threadIdx.x < kBins3) hist[threadIdx.x] = 0u;
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kOwnT; ++j)
+    for (int j = 0; j < kOwn; ++j)
         if (b0 + j < b1 && (key[j] >> 8) == p24) atomicAdd(&hist[key[j] & 0xFFu], 1u);
     __syncthreads();
     find_digit(hist, kBins3, r3, scan, sel);
@@ -378,7 +375,7 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     const uint32_t need_eq = r3 - sel[1];
     uint32_t tg = 0, te = 0;
 #pragma unroll
-    for (int j = 0; j < kOwnT; ++j) {
+    for (int j = 0; j < kOwn; ++j) {
         tg += (b0 + j < b1 && key[j] > T) ? 1u : 0u;
         te += (b0 + j < b1 && key[j] == T) ? 1u : 0u;
     }
@@ -391,7 +388,7 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     // thread has read the digits it held (find_digit ends with a barrier).
     int32_t *stage = reinterpret_cast<int32_t *>(hist);  // k <= kMaxTopk = kBins slots
 #pragma unroll
-    for (int j = 0; j < kOwnT; ++j) {
+    for (int j = 0; j < kOwn; ++j) {
         if (b0 + j >= b1) continue;
         if (key[j] > T) {
             const uint32_t slot = g + min(q, need_eq);
@@ -676,7 +673,6 @@ struct StagedSegs {
 
 // Finish query i from the chunks' candidates (written by other CTAs of this
 // launch: read through L2).
-template <int kOwnT>
 __device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int n_chunks, uint32_t d1,
                                             uint32_t above1, MergeSmem &sm) {
     const uint32_t k = static_cast<uint32_t>(a.topk);
@@ -724,7 +720,7 @@ __device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int
         __syncthreads();
         for (int b = threadIdx.x; b < kBins; b += kT) g2[b] = 0u;  // read above; zero for the next launch
         const StagedSegs sg{sm.cand, sm.coff[n_chunks]};
-        if (!seg_finish<kOwnT>(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out, true)) {
+        if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out, true)) {
             uint32_t T, need_eq;
             seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
             seg_write(sg, T, need_eq, k, out, sm.wg, sm.we);
@@ -835,7 +831,7 @@ __global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a
         for (int b = threadIdx.x; b < kBins; b += kT) g[b] = 0u;
         if (threadIdx.x == 0) a.gticket[i] = 0;
     }
-    merge_query<kPerSm == 1 ? kOwnWide : kOwn>(a, i, n, n_chunks, d1, above1, ss.u.m);
+    merge_query(a, i, n, n_chunks, d1, above1, ss.u.m);
 }
 
 // P chunks per query, chunks multiples of 2048 rows: about one CTA per SM when
