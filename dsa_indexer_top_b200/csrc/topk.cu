@@ -814,16 +814,20 @@ __global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a
     // CTAs leave; it still waits for this whole grid before reading the selection.
     griddep_launch_dependents();
 
-    // ---- publish; the last CTA of the query finishes it
-    __threadfence();
+    // ---- publish; the last CTA of the query finishes it.  The barrier orders every
+    // thread's candidate, count and histogram writes before thread 0's fence, which
+    // is cumulative: one device-scope fence releases them all with the ticket, and
+    // one more, in the last CTA, acquires the other chunks' writes for all its
+    // threads (their reads follow the second barrier).
     __syncthreads();
     if (threadIdx.x == 0) {
+        __threadfence();
         const uint32_t prev = atomicAdd(a.gticket + i, 1u);
         ss.last = prev == static_cast<uint32_t>(n_chunks - 1) ? 1 : 0;
+        if (ss.last) __threadfence();
     }
     __syncthreads();
     if (!ss.last) return;
-    __threadfence();
     // every chunk has read the histogram and taken its ticket: leave both zero
     // for the next launch
     {
