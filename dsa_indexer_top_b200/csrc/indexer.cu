@@ -237,8 +237,12 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
             // Claimed work: the claim after the current one is requested as soon as
             // the current one starts, so its latency hides behind the current items.
             // Otherwise one contiguous range per CTA.
+            // The last two rounds of claims take one item each, so the CTAs finish
+            // within about one item of each other.
             ItemRun run;
             long long next = total;
+            int next_sz = kClaim;  // items in the claim at `next`
+            const long long tail = 2LL * kClaim * gridDim.x;
             if (a.work) {
                 next = static_cast<long long>(atomicAdd(a.work, static_cast<unsigned long long>(kClaim)));
             } else {
@@ -248,8 +252,9 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
             for (;;) {
                 if (run.left == 0) {
                     if (next >= total) break;
-                    run.start(next, min(static_cast<long long>(kClaim), total - next), tpg);
-                    next = static_cast<long long>(atomicAdd(a.work, static_cast<unsigned long long>(kClaim)));
+                    run.start(next, min(static_cast<long long>(next_sz), total - next), tpg);
+                    next_sz = next + tail < total ? kClaim : 1;
+                    next = static_cast<long long>(atomicAdd(a.work, static_cast<unsigned long long>(next_sz)));
                 }
                 int g, j;
                 run.take(tpg, g, j);

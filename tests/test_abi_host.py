@@ -302,3 +302,28 @@ def test_producer_calls_validate():
     assert lib.dsa_absorb_queries(4, 64, P, P, P, P, 8e6, P, _FakeWs.ptr, 128, None) == B.DSA_ERR_WORKSPACE
     assert lib.dsa_up_project(4, 64, P, P, None, _FakeWs.ptr, 256, None) == B.DSA_ERR_INVALID
     assert lib.dsa_up_project(0, 64, P, P, P, _FakeWs.ptr, 256, None) == B.DSA_OK
+
+
+def test_descriptor_struct_follows_field_assignments():
+    """The binding's descriptors build their C struct once and rebuild it when a
+    field is assigned (so repeated calls skip the marshalling but never pass a
+    stale pointer, flag or size)."""
+    import torch
+
+    q = torch.zeros(4, 32, 128, dtype=torch.bfloat16)
+    w = torch.zeros(4, 32)
+    k = torch.zeros(4, 64, 128, dtype=torch.bfloat16)
+    ix = B.Indexer(q, w, k)
+    c0 = ix.c()
+    assert ix.c() is c0 and c0.flags == 0
+    ix.flags = B.DSA_INDEXER_TOPK_HIST
+    c1 = ix.c()
+    assert c1 is not c0 and c1.flags == B.DSA_INDEXER_TOPK_HIST
+    k2 = torch.zeros(4, 64, 128, dtype=torch.bfloat16)
+    ix.k = k2
+    assert ix.c().k == k2.data_ptr()
+    qs = B.Queries(torch.zeros(3, dtype=torch.int32), torch.zeros(3, dtype=torch.int32), n_seq=2, max_ctx=10)
+    assert qs.c().n_q == 3
+    qs.q_pos = torch.zeros(5, dtype=torch.int32)
+    qs.q_seq = torch.zeros(5, dtype=torch.int32)
+    assert qs.c().n_q == 5
