@@ -328,19 +328,22 @@ __device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t n
 }
 
 // Refine and write in one go with the candidates in registers: lane l of warp
-// w owns a contiguous run of at most kOwn (odd) candidates of the warp's segment, so
+// w owns a contiguous run of at most kO (odd) candidates of the warp's segment, so
 // (warp, lane, run index) is position order.  Digit 2 and digit 3 are counted
 // with per-lane shared atomics over the owned keys only; the kept rows' output
 // slots come from one block scan of (rows > T, rows == T) per thread.  Returns
-// false, having written nothing, when a segment holds more than 32 * kOwn
+// false, having written nothing, when a segment holds more than 32 * kO
 // candidates (the caller then uses seg_refine + seg_write).  Output slots are
 // bounds-checked against k (they stay below k whenever the histogram the
 // threshold digit came from describes these scores).
-constexpr int kOwn = 9;
+constexpr int kOwn = 9;         // row schedule: within its 64-register budget
+constexpr int kOwnStaged = 11;  // the split schedule's finish: up to 5,632 candidates, without
+                                // spills at one CTA per SM (4 x 1M decode queries' candidate
+                                // sets pass the 4,608 that 9 per lane hold)
 static_assert(kMaxTopk <= kBins, "seg_finish stages the output in the histogram");
 // hist2_ready: `hist` already holds the second-digit histogram of the
 // candidates in bin d1 (built by the chunk CTAs), so it is not rebuilt here.
-template <class Segs>
+template <int kO, class Segs>
 __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t r2, uint32_t k, uint32_t *hist,
                                            uint64_t *scan, uint32_t *sel, int32_t *out, bool hist2_ready = false) {
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -348,14 +351,14 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     const uint32_t c = sg.count(w, 0);
     const uint32_t m = ((c + 31) / 32) | 1u;  // odd run length: the lanes' loads fall in distinct banks
     if (!hist2_ready) zero_hist(hist, kBins);
-    if (__syncthreads_or(m > static_cast<uint32_t>(kOwn) || sg.pieces(w) != 1)) return false;
+    if (__syncthreads_or(m > static_cast<uint32_t>(kO) || sg.pieces(w) != 1)) return false;
     const uint32_t b0 = min(c, lane * m), b1 = min(c, b0 + m);
-    uint32_t key[kOwn];
+    uint32_t key[kO];
 #pragma unroll
-    for (int j = 0; j < kOwn; ++j) key[j] = b0 + j < b1 ? p[b0 + j].x : 0u;
+    for (int j = 0; j < kO; ++j) key[j] = b0 + j < b1 ? p[b0 + j].x : 0u;
     if (!hist2_ready) {
 #pragma unroll
-        for (int j = 0; j < kOwn; ++j)
+        for (int j = 0; j < kO; ++j)
             if (b0 + j < b1 && first_digit(key[j]) == d1) atomicAdd(&hist[(key[j] >> 8) & 0xFFFu], 1u);
         __syncthreads();
     }
@@ -367,7 +370,7 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     if (threadIdx.x < kBins3) hist[threadIdx.x] = 0u;
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < kOwn; ++j)
+    for (int j = 0; j < kO; ++j)
         if (b0 + j < b1 && (key[j] >> 8) == p24) atomicAdd(&hist[key[j] & 0xFFu], 1u);
     __syncthreads();
     find_digit(hist, kBins3, r3, scan, sel);
@@ -375,7 +378,7 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     const uint32_t need_eq = r3 - sel[1];
     uint32_t tg = 0, te = 0;
 #pragma unroll
-    for (int j = 0; j < kOwn; ++j) {
+    for (int j = 0; j < kO; ++j) {
         tg += (b0 + j < b1 && key[j] > T) ? 1u : 0u;
         te += (b0 + j < b1 && key[j] == T) ? 1u : 0u;
     }
@@ -388,7 +391,7 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     // thread has read the digits it held (find_digit ends with a barrier).
     int32_t *stage = reinterpret_cast<int32_t *>(hist);  // k <= kMaxTopk = kBins slots
 #pragma unroll
-    for (int j = 0; j < kOwn; ++j) {
+    for (int j = 0; j < kO; ++j) {
         if (b0 + j >= b1) continue;
         if (key[j] > T) {
             const uint32_t slot = g + min(q, need_eq);
@@ -400,7 +403,8 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
         }
     }
     __syncthreads();
-    for (uint32_t x = threadIdx.x; x < k; x += kT) out[x] = stage[x];
+    if (out != nullptr)  // null: a run that only brings this code into the caches
+        for (uint32_t x = threadIdx.x; x < k; x += kT) out[x] = stage[x];
     return true;
 }
 
@@ -599,7 +603,7 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
         }
         finish_stream(row, n, k, d1, above1, sm.hist, sm.scan, sm.sel, out);
     } else {
-        if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out)) {
+        if (!seg_finish<kOwn>(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out)) {
             uint32_t T, need_eq;
             seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
             seg_write(sg, T, need_eq, k, out, sm.wg, sm.we);
@@ -655,8 +659,19 @@ struct SplitSmem {
         CollectSmem c;
         MergeSmem m;
     } u;
-    int last;
+    int last;  // 1: this CTA finishes the query; 2: the first to finish its chunk
 };
+
+// The finishing CTA's refine and write, as one function that is not inlined, so
+// that a run of it on an empty candidate set executes the very instructions the
+// finish executes later.  The first chunk CTA of each query to
+// take its ticket makes that run before it exits: the finish is the only code of
+// the path that no other CTA runs first, and with its instructions fetched from
+// DRAM (the step's streams evict them from L2) its last phases took about 2 us
+// longer than with the lines cached.
+struct StagedSegs;
+__device__ __noinline__ bool seg_finish_staged(const StagedSegs sg, uint32_t d1, uint32_t r2, uint32_t k,
+                                               uint32_t *hist, uint64_t *scan, uint32_t *sel, int32_t *out);
 
 // The staged candidates are one array in position order, so warp w may take
 // an equal share of it regardless of chunk boundaries: [w*M/16, (w+1)*M/16).
@@ -670,6 +685,11 @@ struct StagedSegs {
     __device__ const uint2 *ptr(int w, int) const { return cand + begin(w); }
     __device__ uint32_t count(int w, int) const { return begin(w + 1) - begin(w); }
 };
+
+__device__ __noinline__ bool seg_finish_staged(const StagedSegs sg, uint32_t d1, uint32_t r2, uint32_t k,
+                                               uint32_t *hist, uint64_t *scan, uint32_t *sel, int32_t *out) {
+    return seg_finish<kOwnStaged>(sg, d1, r2, k, hist, scan, sel, out, true);
+}
 
 // Finish query i from the chunks' candidates (written by other CTAs of this
 // launch: read through L2).
@@ -720,7 +740,7 @@ __device__ __forceinline__ void merge_query(const TopkArgs &a, int i, int n, int
         __syncthreads();
         for (int b = threadIdx.x; b < kBins; b += kT) g2[b] = 0u;  // read above; zero for the next launch
         const StagedSegs sg{sm.cand, sm.coff[n_chunks]};
-        if (!seg_finish(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out, true)) {
+        if (!seg_finish_staged(sg, d1, k - above1, k, sm.hist, sm.scan, sm.sel, out)) {
             uint32_t T, need_eq;
             seg_refine(sg, d1, k - above1, sm.hist, sm.scan, sm.sel, T, need_eq);
             seg_write(sg, T, need_eq, k, out, sm.wg, sm.we);
@@ -823,11 +843,19 @@ __global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a
     if (threadIdx.x == 0) {
         __threadfence();
         const uint32_t prev = atomicAdd(a.gticket + i, 1u);
-        ss.last = prev == static_cast<uint32_t>(n_chunks - 1) ? 1 : 0;
-        if (ss.last) __threadfence();
+        ss.last = prev == static_cast<uint32_t>(n_chunks - 1) ? 1 : (prev == 0 ? 2 : 0);
+        if (ss.last == 1) __threadfence();
     }
     __syncthreads();
-    if (!ss.last) return;
+    if (ss.last == 2) {
+        // the query's first chunk to finish: run the finish on no candidates (no
+        // global writes; the shared memory it reads and writes is this CTA's own)
+        MergeSmem &wm = ss.u.m;
+        const StagedSegs none{wm.cand, 0u};
+        seg_finish_staged(none, 0u, 1u, 1u, wm.hist, wm.scan, wm.sel, nullptr);
+        return;
+    }
+    if (ss.last != 1) return;
     // every chunk has read the histogram and taken its ticket: leave both zero
     // for the next launch
     {
@@ -838,13 +866,15 @@ __global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a
     merge_query(a, i, n, n_chunks, d1, above1, ss.u.m);
 }
 
-// P chunks per query, chunks multiples of 2048 rows: about one CTA per SM when
-// that still gives every query kSplitMinChunks chunks (per_sm = 1), else about
-// two (per_sm = 2).
+// P chunks per query, chunks multiples of 2048 rows: at most one CTA per SM when
+// that still gives every query kSplitMinChunks chunks (per_sm = 1), else at most
+// two (per_sm = 2).  The grid stays within one wave of resident CTAs: a CTA left
+// for a second wave would start only when a first-wave CTA exits, and every
+// query's finish waits for its last chunk.
 constexpr int kSplitMinChunks = 8;  // a query's ~2-4K candidates stay within a chunk's buffers
 void split_plan(const TopkArgs &a, int num_sms, int &P, int &chunk, int &per_sm) {
     per_sm = num_sms / a.n_q >= kSplitMinChunks ? 1 : 2;
-    P = per_sm == 1 ? num_sms / a.n_q : (2 * num_sms + a.n_q - 1) / a.n_q;
+    P = per_sm * num_sms / a.n_q;
     P = P < 1 ? 1 : (P > kSplitMax ? kSplitMax : P);
     chunk = (a.L + P - 1) / P;
     chunk = (chunk + 2047) / 2048 * 2048;
