@@ -337,9 +337,11 @@ __device__ __forceinline__ void seg_write(const Segs &sg, uint32_t T, uint32_t n
 // bounds-checked against k (they stay below k whenever the histogram the
 // threshold digit came from describes these scores).
 constexpr int kOwn = 9;         // row schedule: within its 64-register budget
-constexpr int kOwnStaged = 11;  // the split schedule's finish: up to 5,632 candidates, without
-                                // spills at one CTA per SM (4 x 1M decode queries' candidate
-                                // sets pass the 4,608 that 9 per lane hold)
+// The split schedule's finish: up to 7,680 candidates, without spills at one CTA
+// per SM (1M-context decode queries' candidate sets reach 5-7K when the k-th
+// score falls in a dense bin; past 32 * kO per warp the slower two-pass refine
+// and write take over).
+constexpr int kOwnStaged = 15;
 static_assert(kMaxTopk <= kBins, "seg_finish stages the output in the histogram");
 // hist2_ready: `hist` already holds the second-digit histogram of the
 // candidates in bin d1 (built by the chunk CTAs), so it is not rebuilt here.
@@ -408,10 +410,11 @@ __device__ __forceinline__ bool seg_finish(const Segs &sg, uint32_t d1, uint32_t
     return true;
 }
 
-__device__ __forceinline__ int visible_rows(const TopkArgs &a, int i) {
+// reporter: the one CTA of query i that reports a position outside the cache
+__device__ __forceinline__ int visible_rows(const TopkArgs &a, int i, bool reporter) {
     const int pos = a.q_pos[i];
     if (pos < 0 || pos >= a.L) {
-        if (threadIdx.x == 0 && blockIdx.x == 0) report_status(a.status, DSA_ERR_INVALID);
+        if (reporter && threadIdx.x == 0) report_status(a.status, DSA_ERR_INVALID);
         return 0;
     }
     return pos + 1;
@@ -501,7 +504,7 @@ __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
 #pragma unroll
         for (int j = 0; j < kBins / kT; ++j) hv[j] = __ldg(g + threadIdx.x + j * kT);
     }
-    const int n = visible_rows(a, i);
+    const int n = visible_rows(a, i, true);
     if (exact) {  // leave the histogram zero for the next indexer launch
         uint32_t *g = a.ghist + static_cast<int64_t>(i) * kBins;
 #pragma unroll
@@ -618,7 +621,7 @@ __global__ void __launch_bounds__(kT, 2) topk_hist_kernel(const TopkArgs a, int 
     __shared__ uint32_t hist[kBins];
     const int i = blockIdx.y, p = blockIdx.x;
     griddep_wait();
-    const int n = visible_rows(a, i);
+    const int n = visible_rows(a, i, p == 0);
     if (n <= a.topk) return;
     const int lo = min(n, p * chunk), hi = min(n, lo + chunk);
     if (lo >= hi) return;
@@ -662,13 +665,12 @@ struct SplitSmem {
     int last;  // 1: this CTA finishes the query; 2: the first to finish its chunk
 };
 
-// The finishing CTA's refine and write, as one function that is not inlined, so
+// The finishing CTA's refine and write, as a function that is not inlined, so
 // that a run of it on an empty candidate set executes the very instructions the
-// finish executes later.  The first chunk CTA of each query to
-// take its ticket makes that run before it exits: the finish is the only code of
-// the path that no other CTA runs first, and with its instructions fetched from
-// DRAM (the step's streams evict them from L2) its last phases took about 2 us
-// longer than with the lines cached.
+// finish executes later.  The first chunk CTA of each query to take its ticket
+// makes that run before it exits: the finish is the only code of the path that
+// no other CTA runs first, and with its instructions fetched from DRAM (the
+// step's streams evict them from L2) it ran 2-9 us slower than with them cached.
 struct StagedSegs;
 __device__ __noinline__ bool seg_finish_staged(const StagedSegs sg, uint32_t d1, uint32_t r2, uint32_t k,
                                                uint32_t *hist, uint64_t *scan, uint32_t *sel, int32_t *out);
@@ -764,7 +766,7 @@ __global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // positions that are inputs of the call are read before the wait, so the
     // chunk's score loads go out together with the histogram's
-    const int n_early = a.pos_early ? visible_rows(a, i) : 0;
+    const int n_early = a.pos_early ? visible_rows(a, i, p == 0) : 0;
     griddep_wait();
     uint32_t hv[kBins / kT];
     {
@@ -772,7 +774,7 @@ __global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a
 #pragma unroll
         for (int j = 0; j < kBins / kT; ++j) hv[j] = __ldg(g + threadIdx.x + j * kT);
     }
-    const int n = a.pos_early ? n_early : visible_rows(a, i);
+    const int n = a.pos_early ? n_early : visible_rows(a, i, p == 0);
     if (n <= a.topk) {  // every chunk of the query sees the same n
         if (p == 0) {
             write_all(a, i, n);
@@ -848,8 +850,8 @@ __global__ void __launch_bounds__(kT, kPerSm) topk_split_kernel(const TopkArgs a
     }
     __syncthreads();
     if (ss.last == 2) {
-        // the query's first chunk to finish: run the finish on no candidates (no
-        // global writes; the shared memory it reads and writes is this CTA's own)
+        // the query's first chunk to finish runs the finish on no candidates: no
+        // global writes; the shared memory it reads and writes is its own
         MergeSmem &wm = ss.u.m;
         const StagedSegs none{wm.cand, 0u};
         seg_finish_staged(none, 0u, 1u, 1u, wm.hist, wm.scan, wm.sel, nullptr);

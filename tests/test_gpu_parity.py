@@ -360,3 +360,32 @@ def test_device_detects_bad_positions(dev, L):
     B.dsa_index_scores(q, ix, scores, ws)
     assert B.dsa_check_status(ws) == B.DSA_ERR_INVALID
     assert B.dsa_check_status(ws) == B.DSA_OK      # reading clears it
+
+
+@pytest.mark.parametrize("L", [5000, 70000])
+def test_topk_reports_bad_position_of_any_query(dev, L):
+    """A position outside the cache, on a query other than the first, is reported by
+    the top-k called on its own (one CTA per query for L = 5000, chunk CTAs for L =
+    70000); every other query's selection is still the oracle's, and the bad query
+    selects nothing."""
+    n_q, topk = 4, 2048
+    s = wl.random_scores(n_q, L, seed=L, mode="normal")
+    q_pos = torch.tensor([L - 1, L // 2, L + 7, L - 3], dtype=torch.int32)
+    q = B.Queries(torch.zeros(n_q, dtype=torch.int32, device=dev), q_pos.to(dev), n_seq=1, max_ctx=L)
+    scores = B.scores_buffer(n_q, L, dev)
+    scores[:, :L] = s.to(dev)
+    ws = B.workspace(B.DSA_OP_TOPK, q, topk, device=dev)
+    idx = torch.full((n_q, topk), -7, dtype=torch.int32, device=dev)
+    cnt = torch.full((n_q,), -7, dtype=torch.int32, device=dev)
+    B.dsa_topk(q, scores, topk, idx, cnt, ws)
+    assert B.dsa_check_status(ws) == B.DSA_ERR_INVALID
+    good = [0, 1, 3]
+    ridx, rcnt = oracle.topk(s[good].double().numpy(), q_pos[good].numpy(), topk)
+    np.testing.assert_array_equal(cnt.cpu().numpy()[good], rcnt)
+    np.testing.assert_array_equal(idx.cpu().numpy()[good], ridx)
+    assert int(cnt[2]) == 0 and bool((idx[2] == -1).all())
+    # the next call on the same workspace is clean again
+    q_ok = B.Queries(torch.zeros(n_q, dtype=torch.int32, device=dev),
+                     torch.tensor([L - 1] * n_q, dtype=torch.int32, device=dev), n_seq=1, max_ctx=L)
+    B.dsa_topk(q_ok, scores, topk, idx, cnt, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
