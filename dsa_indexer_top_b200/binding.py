@@ -83,6 +83,8 @@ def lib():
         h.dsa_noalloc_check_status.argtypes = [P]
         h.dsa_indexshare_group.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Indexer),
                                            ctypes.POINTER(_Mla), I32, I32, P, P, P, SZ, P]
+        h.dsa_indexshare_group_host.argtypes = [ctypes.POINTER(_Queries), ctypes.POINTER(_Indexer),
+                                                ctypes.POINTER(_Mla), I32, I32, P, P, P, SZ, P, P, SZ, P, P, SZ, P]
         h.dsa_shard_candidates.argtypes = [ctypes.POINTER(_Queries), P, I64, P, P, I32, I32, P, P, P, SZ, P]
         h.dsa_shard_merge.argtypes = [ctypes.POINTER(_Queries), I32, P, P, I32, I32, I32, P, P, P, P, P, SZ, P]
         h.dsa_shard_combine.argtypes = [ctypes.POINTER(_Queries), I32, I32, I32, P, P, P, P, P, P]
@@ -101,7 +103,7 @@ def lib():
         h.dsa_status_str.restype = ctypes.c_char_p
         for name in ("dsa_index_scores", "dsa_topk", "dsa_sparse_mla_decode", "dsa_sparse_mla_prefill",
                      "dsa_sparse_mla_mtp", "dsa_sparse_mla_decode_noalloc", "dsa_noalloc_check_status",
-                     "dsa_indexshare_group", "dsa_workspace_init", "dsa_check_status",
+                     "dsa_indexshare_group", "dsa_indexshare_group_host", "dsa_workspace_init", "dsa_check_status",
                      "dsa_shard_candidates", "dsa_shard_merge", "dsa_shard_combine",
                      "dsa_write_cache_rows", "dsa_absorb_queries", "dsa_up_project"):
             getattr(h, name).restype = st
@@ -316,6 +318,42 @@ def dsa_indexshare_group(queries: Queries, indexer: Indexer, layers: Sequence[Ml
     _check(lib().dsa_indexshare_group(ctypes.byref(qc), ctypes.byref(ic), arr, len(layers), topk, _ptr(idx),
                                       _ptr(cnt), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "dsa_indexshare_group")
+
+
+class GroupHostCall:
+    """dsa_indexshare_group_host with its arguments converted once: a decode loop
+    whose buffers stay put (the descriptors, pinned host blocks and device blocks
+    of every step are the same) calls this each step.  h_in -> d_in is copied
+    before the group call and d_out -> h_out after it, on `stream` (default: the
+    stream current when this is made); each host buffer has its device buffer's
+    byte size and the descriptors point into the device buffers."""
+
+    def __init__(self, queries: Queries, indexer: Indexer, layers: Sequence[Mla], topk: int, idx: torch.Tensor,
+                 cnt: torch.Tensor, ws: torch.Tensor, h_in: torch.Tensor, d_in: torch.Tensor, h_out: torch.Tensor,
+                 d_out: torch.Tensor, stream=None):
+        def nbytes(t):
+            return t.numel() * t.element_size()
+        if nbytes(h_in) != nbytes(d_in) or nbytes(h_out) != nbytes(d_out):
+            raise ValueError("host and device buffers differ in size")
+        self._keep = (queries, indexer, list(layers), idx, cnt, ws, h_in, d_in, h_out, d_out)
+        self._qc, self._ic = queries.c(), indexer.c()
+        self._arr = (_Mla * len(layers))(*[m.c() for m in layers])
+        self._args = (ctypes.byref(self._qc), ctypes.byref(self._ic), self._arr, len(layers), topk, _ptr(idx),
+                      _ptr(cnt), _ptr(ws), nbytes(ws), _ptr(h_in), _ptr(d_in), nbytes(h_in), _ptr(h_out),
+                      _ptr(d_out), nbytes(h_out), _stream(stream))
+        self._fn = lib().dsa_indexshare_group_host
+
+    def __call__(self):
+        _check(self._fn(*self._args), "dsa_indexshare_group_host")
+
+
+def dsa_indexshare_group_host(queries: Queries, indexer: Indexer, layers: Sequence[Mla], topk: int,
+                              idx: torch.Tensor, cnt: torch.Tensor, ws: torch.Tensor, h_in: torch.Tensor,
+                              d_in: torch.Tensor, h_out: torch.Tensor, d_out: torch.Tensor, stream=None):
+    """The group call with its inputs copied from h_in (pinned host) to d_in before it
+    and its outputs from d_out to h_out (pinned host) after it, all enqueued on the
+    stream; the descriptors point into the device buffers."""
+    GroupHostCall(queries, indexer, layers, topk, idx, cnt, ws, h_in, d_in, h_out, d_out, stream)()
 
 
 def dsa_shard_candidates(queries: Queries, scores: torch.Tensor, idx: torch.Tensor, cnt: torch.Tensor, topk: int,

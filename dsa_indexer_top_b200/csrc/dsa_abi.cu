@@ -331,6 +331,41 @@ struct NvtxRange {
 };
 }  // namespace
 
+namespace {
+// Every argument check of the group call (nothing is enqueued before they pass).
+dsa_status group_check(const dsa_queries *queries, const dsa_indexer *indexer, const dsa_mla *layers,
+                       int32_t n_layers, int32_t topk, const int32_t *idx, const int32_t *cnt, void *ws,
+                       size_t ws_bytes) {
+    if (!valid_queries(queries)) return DSA_ERR_INVALID;
+    if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
+    dsa_status s = check_indexer(queries, indexer);
+    if (s != DSA_OK) return s;
+    s = check_mla_layers(layers, n_layers);
+    if (s != DSA_OK) return s;
+    if (!ws_ok(ws, ws_bytes, ws_group(queries->n_q, queries->max_ctx, topk, n_layers))) return DSA_ERR_WORKSPACE;
+    return DSA_OK;
+}
+
+// The group call's launches (arguments already checked, n_q > 0).
+dsa_status group_launch(const dsa_queries *queries, const dsa_indexer *indexer, const dsa_mla *layers,
+                        int32_t n_layers, int32_t topk, int32_t *idx, int32_t *cnt, void *ws, cudaStream_t st) {
+    dsa_status s;
+    uint8_t *base = static_cast<uint8_t *>(ws);
+    float *scores = reinterpret_cast<float *>(base + kStatusBytes);
+    const int64_t ld = round4(queries->max_ctx);
+    uint8_t *topk_scratch = base + kStatusBytes + ws_scores(queries->n_q, queries->max_ctx);
+    uint8_t *scratch = topk_scratch + align256(topk_scratch_bytes(queries->n_q, queries->max_ctx));
+    // the first-digit histograms of top-k come out of the indexer (ghist heads the top-k scratch)
+    s = do_index_scores(queries, indexer, scores, ld, status_word(ws), reinterpret_cast<uint32_t *>(topk_scratch), st);
+    if (s != DSA_OK) return s;
+    s = do_topk(queries, scores, ld, topk, idx, cnt, status_word(ws), topk_scratch, true, st);
+    if (s != DSA_OK) return s;
+    return do_mla(queries, layers, n_layers, idx, cnt, topk, group_uses_decode(queries->n_q), scratch,
+                  status_word(ws), st);
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *dsa_status_str(dsa_status s) {
@@ -456,31 +491,34 @@ dsa_status dsa_sparse_mla_mtp(const dsa_queries *queries, const dsa_mla *mla, co
                      draft_tokens);
 }
 
+
 dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *indexer, const dsa_mla *layers,
                                 int32_t n_layers, int32_t topk, int32_t *idx, int32_t *cnt, void *ws,
                                 size_t ws_bytes, void *stream) {
     NvtxRange range("dsa_indexshare_group");
-    if (!valid_queries(queries)) return DSA_ERR_INVALID;
-    if (topk < 1 || topk > kMaxTopk || !idx || !cnt) return DSA_ERR_INVALID;
-    dsa_status s = check_indexer(queries, indexer);
+    const dsa_status s = group_check(queries, indexer, layers, n_layers, topk, idx, cnt, ws, ws_bytes);
+    if (s != DSA_OK || queries->n_q == 0) return s;
+    return group_launch(queries, indexer, layers, n_layers, topk, idx, cnt, ws, static_cast<cudaStream_t>(stream));
+}
+
+dsa_status dsa_indexshare_group_host(const dsa_queries *queries, const dsa_indexer *indexer, const dsa_mla *layers,
+                                     int32_t n_layers, int32_t topk, int32_t *idx, int32_t *cnt, void *ws,
+                                     size_t ws_bytes, const void *h_in, void *d_in, size_t in_bytes, void *h_out,
+                                     const void *d_out, size_t out_bytes, void *stream) {
+    NvtxRange range("dsa_indexshare_group_host");
+    dsa_status s = group_check(queries, indexer, layers, n_layers, topk, idx, cnt, ws, ws_bytes);
     if (s != DSA_OK) return s;
-    s = check_mla_layers(layers, n_layers);
-    if (s != DSA_OK) return s;
-    if (!ws_ok(ws, ws_bytes, ws_group(queries->n_q, queries->max_ctx, topk, n_layers))) return DSA_ERR_WORKSPACE;
-    if (queries->n_q == 0) return DSA_OK;
+    if ((in_bytes > 0 && (!h_in || !d_in)) || (out_bytes > 0 && (!h_out || !d_out))) return DSA_ERR_INVALID;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    uint8_t *base = static_cast<uint8_t *>(ws);
-    float *scores = reinterpret_cast<float *>(base + kStatusBytes);
-    const int64_t ld = round4(queries->max_ctx);
-    uint8_t *topk_scratch = base + kStatusBytes + ws_scores(queries->n_q, queries->max_ctx);
-    uint8_t *scratch = topk_scratch + align256(topk_scratch_bytes(queries->n_q, queries->max_ctx));
-    // the first-digit histograms of top-k come out of the indexer (ghist heads the top-k scratch)
-    s = do_index_scores(queries, indexer, scores, ld, status_word(ws), reinterpret_cast<uint32_t *>(topk_scratch), st);
-    if (s != DSA_OK) return s;
-    s = do_topk(queries, scores, ld, topk, idx, cnt, status_word(ws), topk_scratch, true, st);
-    if (s != DSA_OK) return s;
-    return do_mla(queries, layers, n_layers, idx, cnt, topk, group_uses_decode(queries->n_q), scratch,
-                  status_word(ws), st);
+    if (in_bytes > 0 && cudaMemcpyAsync(d_in, h_in, in_bytes, cudaMemcpyHostToDevice, st) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    if (queries->n_q > 0) {
+        s = group_launch(queries, indexer, layers, n_layers, topk, idx, cnt, ws, st);
+        if (s != DSA_OK) return s;
+    }
+    if (out_bytes > 0 && cudaMemcpyAsync(h_out, d_out, out_bytes, cudaMemcpyDeviceToHost, st) != cudaSuccess)
+        return DSA_ERR_CUDA;
+    return DSA_OK;
 }
 
 // ------------------------------------------------------------------ key-range shards

@@ -375,6 +375,30 @@ dsa_status dsa_indexshare_group(const dsa_queries *queries, const dsa_indexer *i
                                 void *stream);
 
 /*
+ * dsa_indexshare_group with the step's inputs and outputs in host memory (the
+ * call a host-driven decode loop makes each step; the caches, the indexer keys
+ * and the workspace stay on the device).  All on `stream`, in this order:
+ *   1. in_bytes bytes from h_in (host) to d_in (device),
+ *   2. dsa_indexshare_group on the descriptors, which point into d_in and
+ *      d_out (or anywhere else on the device),
+ *   3. out_bytes bytes from d_out (device) to h_out (host).
+ * Every argument is checked before anything is enqueued (same results as
+ * dsa_indexshare_group; DSA_ERR_INVALID also for a null buffer with a
+ * non-zero size); n_q = 0 enqueues the two copies only.  The call returns once
+ * the work is enqueued: synchronise `stream` before reading h_out.  With
+ * page-locked (pinned) host buffers the copies are asynchronous; with pageable
+ * ones the driver stages them and the call may wait for them.  The caller
+ * owns all four buffers; h_in must stay unchanged and h_out unread until the
+ * stream has passed the call.
+ */
+dsa_status dsa_indexshare_group_host(const dsa_queries *queries, const dsa_indexer *indexer,
+                                     const dsa_mla *layers, int32_t n_layers, int32_t topk,
+                                     int32_t *idx, int32_t *cnt, void *ws, size_t ws_bytes,
+                                     const void *h_in, void *d_in, size_t in_bytes,
+                                     void *h_out, const void *d_out, size_t out_bytes,
+                                     void *stream);
+
+/*
  * Key-range sharding of one long sequence over several GPUs.  The pages name
  * attention data parallelism only ["GLM-5.2 -- Model techniques map",
  * inference & serving]; splitting one sequence's cache by contiguous key

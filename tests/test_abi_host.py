@@ -190,6 +190,28 @@ def test_group_rejects_layer_mismatch_and_count():
                                     _FakeWs.size, None) == B.DSA_ERR_INVALID
 
 
+def test_group_host_rejects_before_any_copy():
+    """The host-buffer group call checks everything before it enqueues a copy: the
+    group call's own argument errors, and a null host or device buffer with a
+    non-zero size (all pointers here are fake, so any copy or launch would fail)."""
+    lib = B.lib()
+    q, ix = _q(), _idx()
+
+    def call(arr, n, ws_size=_FakeWs.size, bufs=(0x20000, 0x30000, 0x40000, 0x50000)):
+        h_in, d_in, h_out, d_out = bufs
+        return lib.dsa_indexshare_group_host(ctypes.byref(q), ctypes.byref(ix), arr, n, 2048, 0xA000, 0xB000,
+                                             _FakeWs.ptr, ws_size, h_in, d_in, 4096, h_out, d_out, 4096, None)
+
+    assert call((B._Mla * 2)(_mla(), _mla(dl=256, krs=576)), 2) == B.DSA_ERR_INVALID
+    one = (B._Mla * 1)(_mla())
+    good = [0x20000, 0x30000, 0x40000, 0x50000]
+    for k in range(4):
+        bufs = list(good)
+        bufs[k] = None
+        assert call(one, 1, bufs=tuple(bufs)) == B.DSA_ERR_INVALID, k
+    assert call(one, 1, ws_size=16) == B.DSA_ERR_WORKSPACE
+
+
 def test_zero_queries_is_a_noop():
     lib = B.lib()
     q = _q(n_q=0)

@@ -287,6 +287,63 @@ def test_indexshare_group_call(dev, name):
         C.assert_lse_close(m.lse, lses[layer], w.dtype)
 
 
+def _packed(tensors, dev):
+    """One device buffer holding the tensors' bytes (256-byte aligned pieces, left
+    zero) with a view per tensor, and a pinned host buffer holding their values."""
+    offs, tot = [], 0
+    for t in tensors:
+        offs.append(tot)
+        tot += (t.numel() * t.element_size() + 255) // 256 * 256
+    d = torch.zeros(tot, dtype=torch.uint8, device=dev)
+    h = torch.zeros(tot, dtype=torch.uint8).pin_memory()
+    views = []
+    for t, o in zip(tensors, offs):
+        nb = t.numel() * t.element_size()
+        views.append(d[o:o + nb].view(t.dtype).view(t.shape))
+        h[o:o + nb].copy_(t.detach().cpu().contiguous().view(-1).view(torch.uint8))
+    return d, h, views
+
+
+@pytest.mark.parametrize("name", ["decode_edges", "indexshare_small"])
+def test_indexshare_group_host_buffers(dev, name):
+    """The group call with its per-step inputs in pinned host memory and its
+    outputs copied back to pinned host memory inside the call: the device input
+    buffer starts zero, so the results can only come from the copied inputs; the
+    host results match the oracle (indices and counts bit for bit)."""
+    w = SMALL[name]
+    xh = wl.make_inputs(w)
+    x = C.to_device(xh)
+    d_in, h_in, vin = _packed([x["q_idx"], x["w"], x["q_seq"], x["q_pos"]] + list(x["q_mla"]), dev)
+    nl = len(x["q_mla"])
+    outs = [torch.empty((w.n_q, w.mla_heads, w.d_lat), dtype=w.torch_dtype) for _ in range(nl)]
+    outs += [torch.empty((w.n_q, w.topk), dtype=torch.int32), torch.empty((w.n_q,), dtype=torch.int32)]
+    d_out, h_out, vout = _packed(outs, dev)
+    xv = dict(x, q_idx=vin[0], w=vin[1], q_seq=vin[2], q_pos=vin[3], q_mla=vin[4:])
+    q, ix, mlas = C.descriptors(w, xv, seq_run=seq_run_of(w))
+    for layer, m in enumerate(mlas):
+        m.out = vout[layer]
+    ws = B.workspace(B.DSA_OP_INDEXSHARE_GROUP, q, w.topk, w.n_layers, dev)
+    call = B.GroupHostCall(q, ix, mlas, w.topk, vout[nl], vout[nl + 1], ws, h_in, d_in, h_out, d_out)
+    for _ in range(2):  # the prepared call, twice on the same buffers
+        h_out.fill_(0xFF)
+        call()
+        torch.cuda.current_stream().synchronize()
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    # the host copy, read through views of h_out laid out like d_out
+    base = d_out.data_ptr()
+    hv = [h_out[v.data_ptr() - base:v.data_ptr() - base + v.numel() * v.element_size()].view(v.dtype).view(v.shape)
+          for v in vout]
+    ridx, rcnt, oouts, lses = oracle.indexshare_group(
+        C.host_f32(xh["q_idx"]), C.host_f32(xh["w"]), C.host_f32(xh["k_idx"]),
+        np.zeros(w.n_q, np.int32) if w.shared_cache else xh["q_seq"].numpy(), xh["q_pos"].numpy(), w.topk,
+        [C.host_f32(t) for t in xh["q_mla"]], [C.host_f32(t) for t in xh["kv"]], w.d_lat, w.scale)
+    np.testing.assert_array_equal(hv[nl].numpy(), ridx)
+    np.testing.assert_array_equal(hv[nl + 1].numpy(), rcnt)
+    for layer in range(nl):
+        C.assert_attention_close(hv[layer], oouts[layer], w.dtype, f"layer {layer}")
+        C.assert_lse_close(mlas[layer].lse, lses[layer], w.dtype)
+
+
 @pytest.mark.parametrize("mode", ["ties", "normal", "equal"])
 @pytest.mark.parametrize("L,topk", [(300, 64), (5000, 2048), (70000, 2048), (200000, 512), (700001, 2048)])
 def test_topk_alone(dev, mode, L, topk):
