@@ -363,6 +363,34 @@ def test_topk_alone(dev, mode, L, topk):
     np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
 
 
+@pytest.mark.parametrize("n_bin", [1500, 4000, 5200, 7000])
+def test_topk_split_finish_sizes(dev, n_bin):
+    """The split schedule's finish over candidate sets of every size class: 2040
+    rows far above the rest and n_bin rows inside one first-digit bin ([10, 11)),
+    so the finishing CTA stages 2040 + n_bin candidates (fewer than 9 per lane,
+    up to 15 per lane, and past that the two-pass refine and write)."""
+    n_q, L, topk = 2, 300_000, 2048
+    g = torch.Generator().manual_seed(n_bin)
+    s = torch.randn((n_q, L), generator=g) * 0.1
+    for i in range(n_q):
+        pos = torch.randperm(L // 2, generator=g)[:2040 + n_bin]  # all visible for both queries
+        s[i, pos[:2040]] = 100.0 + torch.rand(2040, generator=g)
+        s[i, pos[2040:]] = 10.0 + torch.rand(n_bin, generator=g)
+    q_pos = torch.tensor([L - 1, L // 2], dtype=torch.int32)
+    q = B.Queries(torch.zeros(n_q, dtype=torch.int32, device=dev), q_pos.to(dev), n_seq=1, max_ctx=L)
+    scores = B.scores_buffer(n_q, L, dev)
+    scores[:, :L] = s.to(dev)
+    ws = B.workspace(B.DSA_OP_TOPK, q, topk, device=dev)
+    idx = torch.full((n_q, topk), -7, dtype=torch.int32, device=dev)
+    cnt = torch.full((n_q,), -7, dtype=torch.int32, device=dev)
+    for _ in range(2):  # the second call runs on the zeroed histograms and tickets the first left
+        B.dsa_topk(q, scores, topk, idx, cnt, ws)
+        assert B.dsa_check_status(ws) == B.DSA_OK
+        ridx, rcnt = oracle.topk(s.double().numpy(), q_pos.numpy(), topk)
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
 @pytest.mark.parametrize("decode", [True, False])
 @pytest.mark.parametrize("topk,L", [(2048, 3000), (300, 1000), (100, 500), (4096, 5000)])
 def test_sparse_mla_alone(dev, decode, topk, L):
