@@ -457,18 +457,28 @@ __device__ __forceinline__ void load_warp_batch(const float *row, int base, int 
 // Append, in position order, the rows of a loaded batch whose first digit is at
 // least d_lo to a warp's (key, position) buffer of capacity cap; cnt counts every
 // such row, also past the capacity.  Groups of 128 rows without a candidate cost
-// one ballot.
-__device__ __forceinline__ void compact_batch(const float (&v)[kU][4], int base, int hi, uint32_t d_lo, uint2 *buf,
-                                              uint32_t cap, uint32_t &cnt) {
+// one ballot.  kPos (d_lo above 0x800, the digit of +0.0): only positive scores
+// qualify, and a row's first digit is at least d_lo exactly when its bits, read
+// as a signed integer, are at least tbits = the bits of the bin's smallest
+// value -- negative scores, -0.0, +0.0 and the zeros loaded past `hi` all read
+// below it -- so a row costs one integer compare and only kept rows form a key.
+template <bool kPos>
+__device__ __forceinline__ void compact_batch_t(const float (&v)[kU][4], int base, int hi, uint32_t d_lo, uint2 *buf,
+                                                uint32_t cap, uint32_t &cnt) {
     const int lane = threadIdx.x & 31;
+    const int32_t tbits = static_cast<int32_t>((d_lo << 20) & 0x7FFFFFFFu);
 #pragma unroll
     for (int j = 0; j < kU; ++j) {
         const int e0 = base + (j * 32 + lane) * 4;
         uint32_t u[4], pick = 0;
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
-            u[x] = order_key(v[j][x]);
-            if (e0 + x < hi && first_digit(u[x]) >= d_lo) pick |= 1u << x;
+            if constexpr (kPos) {
+                if (__float_as_int(v[j][x]) >= tbits) pick |= 1u << x;
+            } else {
+                u[x] = order_key(v[j][x]);
+                if (e0 + x < hi && first_digit(u[x]) >= d_lo) pick |= 1u << x;
+            }
         }
         if (__ballot_sync(0xffffffffu, pick != 0u) == 0u) continue;
         const uint32_t c = __popc(pick);
@@ -482,12 +492,20 @@ __device__ __forceinline__ void compact_batch(const float (&v)[kU][4], int base,
 #pragma unroll
         for (int x = 0; x < 4; ++x) {
             if (pick & (1u << x)) {
-                if (slot < cap) buf[slot] = make_uint2(u[x], static_cast<uint32_t>(e0 + x));
+                if (slot < cap) buf[slot] = make_uint2(kPos ? order_key(v[j][x]) : u[x], static_cast<uint32_t>(e0 + x));
                 ++slot;
             }
         }
         cnt += __shfl_sync(0xffffffffu, incl, 31);
     }
+}
+
+__device__ __forceinline__ void compact_batch(const float (&v)[kU][4], int base, int hi, uint32_t d_lo, uint2 *buf,
+                                              uint32_t cap, uint32_t &cnt) {
+    if (d_lo > 0x800u)
+        compact_batch_t<true>(v, base, hi, d_lo, buf, cap, cnt);
+    else
+        compact_batch_t<false>(v, base, hi, d_lo, buf, cap, cnt);
 }
 
 __global__ void __launch_bounds__(kT, 2) topk_row_kernel(const TopkArgs a) {
