@@ -86,7 +86,7 @@ PER_CONFIG_MAX_STEPS = 50
 NCU_TRAFFIC: dict = {
     ("decode_1m", "index_scores", False): 4 * (268_491_008 + 5_246_720),
     ("decode_1m", "index_scores", True): 4 * (138_483_712 + 4_256_768),
-    ("decode_1m", "topk", False): 4 * 4_320_512,
+    ("decode_1m", "topk", False): 4 * 4_322_816,
     ("decode_1m", "sparse_mla", False): 4 * (2_502_400 + 2_118_400),   # mla_tc + mla_combine
     ("decode_1m", "sparse_mla", True): 4 * (1_728_768 + 2_118_400),
 }
