@@ -375,6 +375,11 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
         int cur_g = -1, seq = -1, max_pos = -1;
         int qpos[kQPerWarp];   // this warp's queries of the current group
         bool qok[kQPerWarp];
+        // Several queries per tile (prefill): the head weights of the warp's first
+        // query stay in registers for the whole group, the second query's are read
+        // from shared memory per tile (both do not fit in the 96 registers a thread
+        // has at this block size: measured slower with the spills).
+        float w0[G == 1 ? 1 : 32];
         long long k_tiles = 0;
         uint32_t epi_phase = 0;
         bool hist_dirty = false;
@@ -417,6 +422,10 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
                     w_mine[e] = wv;
                 }
                 __syncwarp();
+                if constexpr (G > 1) {
+#pragma unroll
+                    for (int h = 0; h < 32; ++h) w0[h] = w_mine[qlo * 32 + h];
+                }
 #pragma unroll
                 for (int ii = 0; ii < kQPerWarp; ++ii) {
                     const int qi = q0 + qlo + ii;
@@ -445,18 +454,34 @@ __global__ void __launch_bounds__(IdxCfg<G, F8>::kThreads, IdxCfg<G, F8>::kCtasP
 #pragma unroll
             for (int ii = 0; ii < kQPerWarp; ++ii) {
                 const int i = qlo + ii;
-                uint32_t r[32];
-                tmem_ld32(taddr + i * 32, r);
-                tmem_ld_wait();
                 float score = 0.f;
-                const float4 *w4 = reinterpret_cast<const float4 *>(w_mine + i * 32);
+                if constexpr (G == 1) {
+                    uint32_t r[32];
+                    tmem_ld32(taddr + i * 32, r);
+                    tmem_ld_wait();
+                    const float4 *w4 = reinterpret_cast<const float4 *>(w_mine + i * 32);
 #pragma unroll
-                for (int h4 = 0; h4 < 8; ++h4) {
-                    const float4 wv = w4[h4];
-                    score = fmaf(wv.x, fmaxf(u2f(r[4 * h4]), 0.f), score);
-                    score = fmaf(wv.y, fmaxf(u2f(r[4 * h4 + 1]), 0.f), score);
-                    score = fmaf(wv.z, fmaxf(u2f(r[4 * h4 + 2]), 0.f), score);
-                    score = fmaf(wv.w, fmaxf(u2f(r[4 * h4 + 3]), 0.f), score);
+                    for (int h4 = 0; h4 < 8; ++h4) {
+                        const float4 wv = w4[h4];
+                        score = fmaf(wv.x, fmaxf(u2f(r[4 * h4]), 0.f), score);
+                        score = fmaf(wv.y, fmaxf(u2f(r[4 * h4 + 1]), 0.f), score);
+                        score = fmaf(wv.z, fmaxf(u2f(r[4 * h4 + 2]), 0.f), score);
+                        score = fmaf(wv.w, fmaxf(u2f(r[4 * h4 + 3]), 0.f), score);
+                    }
+                } else {
+                    // 16 heads per TMEM load (room for the weights in registers);
+                    // the same head order as above, so the same sums
+#pragma unroll
+                    for (int hh = 0; hh < 2; ++hh) {
+                        uint32_t r[16];
+                        tmem_ld16(taddr + i * 32 + 16 * hh, r);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int h = 0; h < 16; ++h) {
+                            const float wv = ii == 0 ? w0[16 * hh + h] : w_mine[i * 32 + 16 * hh + h];
+                            score = fmaf(wv, fmaxf(u2f(r[h]), 0.f), score);
+                        }
+                    }
                 }
                 if (F8) score *= ks;
                 const bool vis = qok[ii] && s <= qpos[ii];
