@@ -391,6 +391,40 @@ def test_topk_split_finish_sizes(dev, n_bin):
         np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
 
 
+@pytest.mark.parametrize("L", [5000, 70000], ids=["row", "split"])
+@pytest.mark.parametrize("topk", [100, 500, 2048], ids=["bin_of_1", "bin_of_zero", "negative"])
+def test_topk_threshold_bin_boundaries(dev, L, topk):
+    """Rows at the edges of the threshold's first-digit bin: 60 rows at 3.0, 70 at
+    exactly 1.0 (the smallest value of its bin), 300 at the float just below 1.0
+    (the previous bin), 400 zeros (half -0.0, half +0.0) and negatives, shuffled.
+    topk 100 puts the threshold in the bin of 1.0 (candidates tested as positive
+    integers), 500 in the bin of zero (-0.0 and +0.0 tie; lower positions win),
+    2048 among the negatives."""
+    n_q = 3
+    g = torch.Generator().manual_seed(L + topk)
+    below_one = float(np.nextafter(np.float32(1.0), np.float32(0.0)))
+    s = torch.empty((n_q, L))
+    for i in range(n_q):
+        vals = torch.cat([torch.full((60,), 3.0), torch.full((70,), 1.0), torch.full((300,), below_one),
+                          torch.full((200,), -0.0), torch.zeros(200),
+                          -1.0 - 4.0 * torch.rand(L - 830, generator=g)])
+        s[i] = vals[torch.randperm(L, generator=g)]
+    assert float(s[0][s[0] < 1.0].max()) == below_one
+    q_pos = torch.tensor([L - 1, L - 1 - L // 7, L // 2], dtype=torch.int32)
+    q = B.Queries(torch.zeros(n_q, dtype=torch.int32, device=dev), q_pos.to(dev), n_seq=1, max_ctx=L)
+    scores = B.scores_buffer(n_q, L, dev)
+    scores[:, :L] = s.to(dev)
+    ws = B.workspace(B.DSA_OP_TOPK, q, topk, device=dev)
+    idx = torch.full((n_q, topk), -7, dtype=torch.int32, device=dev)
+    cnt = torch.full((n_q,), -7, dtype=torch.int32, device=dev)
+    ridx, rcnt = oracle.topk(s.double().numpy(), q_pos.numpy(), topk)
+    for _ in range(2):
+        B.dsa_topk(q, scores, topk, idx, cnt, ws)
+        assert B.dsa_check_status(ws) == B.DSA_OK
+        np.testing.assert_array_equal(cnt.cpu().numpy(), rcnt)
+        np.testing.assert_array_equal(idx.cpu().numpy(), ridx)
+
+
 @pytest.mark.parametrize("decode", [True, False])
 @pytest.mark.parametrize("topk,L", [(2048, 3000), (300, 1000), (100, 500), (4096, 5000)])
 def test_sparse_mla_alone(dev, decode, topk, L):
