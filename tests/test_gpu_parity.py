@@ -249,6 +249,36 @@ def test_index_scores_bit_exact(dev, name):
         np.testing.assert_array_equal(got[i, : t + 1], ref[i, : t + 1], err_msg=f"query {i}")
 
 
+@pytest.mark.parametrize("fp8", [False, True], ids=["bf16", "fp8"])
+@pytest.mark.parametrize("seq_run", [2, 4, 6, 12])
+def test_index_scores_query_tiles(dev, seq_run, fp8):
+    """Runs of seq_run queries per sequence, so the indexer tiles gcd(seq_run, 8)
+    = 2 or 4 queries together (the 8-query tile is covered by the prefill cases):
+    three sequences, positions spread over a ragged tail, every visible score
+    equal to the oracle's."""
+    n_seq, L = 3, 3173
+    q_seq = tuple(b for b in range(n_seq) for _ in range(seq_run))
+    q_pos = tuple(L - 1 - 37 * j - 101 * b for b in range(n_seq) for j in range(seq_run))
+    w = wl.scaled(D32, n_seq=n_seq, L=L, q_pos=q_pos, q_seq=q_seq, seed=40 + seq_run)
+    xh = wl.make_inputs(w, layers=[])
+    x = C.to_device(xh)
+    q, ix, _ = C.descriptors(w, x, seq_run=seq_run)
+    if fp8:
+        f8h = wl.fp8_indexer_inputs(w, xh)
+        ix = C.fp8_indexer(w, C.to_device(f8h), x)
+        ref, _, _ = C.oracle_selection_fp8(w, f8h, xh)
+    else:
+        ref, _, _ = C.oracle_selection(w, xh)
+    ws = B.workspace(B.DSA_OP_INDEX_SCORES, q, device=dev)
+    scores = B.scores_buffer(w.n_q, w.L, dev)
+    scores.fill_(float("nan"))
+    B.dsa_index_scores(q, ix, scores, ws)
+    assert B.dsa_check_status(ws) == B.DSA_OK
+    got = scores[:, : w.L].cpu().double().numpy()
+    for i, t in enumerate(w.q_pos):
+        np.testing.assert_array_equal(got[i, : t + 1], ref[i, : t + 1], err_msg=f"query {i}")
+
+
 @pytest.mark.parametrize("name", list(SMALL))
 @pytest.mark.parametrize("decode,fused", [(True, True), (False, True), (True, False)])
 def test_chain_matches_oracle(dev, name, decode, fused):
